@@ -1,0 +1,370 @@
+#!/usr/bin/env python
+"""Benchmark of the KDA forward hot path on B200.
+
+A step is one ``kda_chunk_fwd`` call over the prefill workload: B=4 sequences
+of T=4096 tokens, H=16 heads, dk=dv=128, bf16 q/k/v, fp32 gates and state,
+S0 ~ N(0, 0.1^2). The headline value is prefill tokens/s (B*T per step over
+the whole job). The decode workload (N=256 sequences, H=32, 1024 consecutive
+``kda_decode_step`` calls captured in one CUDA graph) is measured in the same
+run and reported under "decode".
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl kda|reference]
+For N > 1 launch with torchrun (one rank per GPU, weak scaling: every rank
+runs its own batch; the only collectives are the barrier and the max-reduce
+of the timings).
+
+``--impl reference`` times the fp64 CPU oracle (the slow, obviously correct
+definition of the recurrence) on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "KDA prefill tokens/s + decode tokens/s on 1 B200; % of tensor/HBM roofline"
+PREFILL = dict(B=4, T=4096, H=16, s0_std=0.1, la_range=(0.001, 0.1), seed=20261)
+DECODE = dict(N=256, H=32, steps=1024, s0_std=0.1, la_range=(0.001, 0.1), seed=20263)
+L2_FLUSH_BYTES = 256 << 20  # larger than the 126 MB L2
+D = 128
+# algorithmic bytes (single pass) per token-head: q,k,v,o bf16 + log_alpha fp32 + beta fp32
+PREFILL_BYTES_PER_TOKEN_HEAD = 3 * D * 2 + D * 4 + 4 + D * 2  # 1540
+STATE_BYTES = D * D * 4
+PAGES_FLOPS_PER_TOKEN_HEAD = 6 * D * D + 3 * 64 * D + 64 * 64  # 6Td^2 + 3TCd + TC^2 per token
+DECODE_BYTES_PER_HEAD_STEP = 2 * STATE_BYTES + PREFILL_BYTES_PER_TOKEN_HEAD  # 132612
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """Samples nvidia-smi clocks and throttle reasons while the timed region runs."""
+
+    FIELDS = ["clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.active",
+              "clocks_event_reasons.hw_slowdown", "clocks_event_reasons.hw_thermal_slowdown",
+              "clocks_event_reasons.sw_thermal_slowdown", "clocks_event_reasons.sw_power_cap"]
+
+    def __init__(self, device_index: int):
+        self.proc = None
+        try:
+            uuid = "GPU-" + str(torch.cuda.get_device_properties(device_index).uuid)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", uuid, "--query-gpu=" + ",".join(self.FIELDS),
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, RuntimeError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        out, _ = self.proc.communicate(timeout=10)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) != len(self.FIELDS):
+                continue
+            try:
+                sm.append(float(parts[0]))
+                smax.append(float(parts[1]))
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[4:]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ helpers
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(x: float, world: int, device) -> float:
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def time_steps(fn, steps, warmup, stream, flush=None):
+    """Runs fn warmup times, then times each of `steps` calls with CUDA events
+    on `stream` (L2 flushed before each call, outside the events). Returns ms list."""
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    times = []
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(steps)]
+    with torch.cuda.stream(stream):
+        for a, b in evs:
+            if flush is not None:
+                flush()
+            a.record(stream)
+            fn()
+            b.record(stream)
+    torch.cuda.synchronize()
+    for a, b in evs:
+        times.append(a.elapsed_time(b))
+    return times
+
+
+def cpu_oracle_sample(inp, n_heads=None):
+    """Times the fp64 oracle on sequence 0 of the prefill batch (all heads)."""
+    import oracle
+
+    H = inp.q.shape[2] if n_heads is None else n_heads
+    sl = lambda x: x[0:1, :, :H]
+    q, k, v, la = sl(inp.q), sl(inp.k), sl(inp.v), sl(inp.log_alpha)
+    b = inp.beta[0:1, :, :H]
+    S0 = None if inp.S0 is None else inp.S0[0:1, :H]
+    args = [oracle._f64(t) for t in (q, k, v, la, b, S0)]
+    threads = oracle.default_threads()
+    t0 = time.perf_counter()
+    oracle.kda_fwd(*args, threads=threads)
+    dt = time.perf_counter() - t0
+    T = inp.q.shape[1]
+    full_H = inp.q.shape[2]
+    tokens = T * H / full_H  # token positions (all heads) equivalent
+    return {"value": tokens / dt, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "sample": f"1 of {inp.q.shape[0]} sequences ({T} tokens x {H} heads) of the prefill "
+                      f"batch, fp64 recurrence, {dt:.2f} s"}
+
+
+# ------------------------------------------------------------------ arms
+def run_reference(args, rank, world):
+    """The fp64 CPU oracle timed on host cores, a bounded sample per step."""
+    if rank != 0:
+        return
+    from gated_delta_rule_101_b200.inputs import prefill_inputs
+
+    inp = prefill_inputs(B=1, T=PREFILL["T"], H=PREFILL["H"], dtype=torch.bfloat16,
+                         s0_std=PREFILL["s0_std"], la_range=PREFILL["la_range"],
+                         seed=PREFILL["seed"], device="cpu")
+    import oracle
+
+    H = inp.q.shape[2]
+    args_np = [oracle._f64(t) for t in (inp.q, inp.k, inp.v, inp.log_alpha, inp.beta, inp.S0)]
+    threads = oracle.default_threads()
+    for _ in range(args.warmup):
+        oracle.kda_fwd(*args_np, threads=threads)
+    times = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        oracle.kda_fwd(*args_np, threads=threads)
+        times.append(time.perf_counter() - t0)
+    total = sum(times)
+    tokens = PREFILL["T"] * args.steps
+    value = tokens / total
+    sample = (f"one sequence of the prefill workload per step ({PREFILL['T']} tokens x {H} heads, "
+              f"bf16 inputs widened to fp64), {threads} threads")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": f"KDA prefill B=4 T=4096 H=16 d=128 C=64 (sampled: 1 sequence "
+                                   f"per step)", "l2": "n/a (CPU)"},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0},
+            "gpu_launches": 0}
+    print(json.dumps(line), flush=True)
+
+
+def run_kda(args, rank, world, local_rank):
+    import gated_delta_rule_101_b200 as kda
+    from gated_delta_rule_101_b200.inputs import decode_inputs, prefill_inputs
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    kda.lib()
+    pk, pk_kind = peaks()
+    stream = torch.cuda.Stream(device=dev)
+    flush_buf = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush = lambda: flush_buf.fill_(1)
+
+    # ---------------- prefill (the step)
+    B, T, H = PREFILL["B"], PREFILL["T"], PREFILL["H"]
+    inp = prefill_inputs(B=B, T=T, H=H, dtype=torch.bfloat16, s0_std=PREFILL["s0_std"],
+                         la_range=PREFILL["la_range"], seed=PREFILL["seed"] + 1000 * rank,
+                         device=dev)
+    o = torch.empty_like(inp.v)
+    S_T = torch.empty_like(inp.S0)
+    ws_n = kda.workspace_size(B, T, H, 0, torch.bfloat16)
+    ws = torch.empty(max(ws_n, 16), dtype=torch.uint8, device=dev)
+
+    def step():
+        kda.chunk_fwd(inp.q, inp.k, inp.v, inp.log_alpha, inp.beta, inp.S0, out=o, state_out=S_T,
+                      workspace=ws, stream=stream)
+
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    clocks = ClockSampler(dev.index)
+    times = time_steps(step, args.steps, args.warmup, stream, flush)
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    total_ms = max_over_ranks(sum(times), world, dev)
+    ms_per_step = total_ms / args.steps
+    tokens_per_step = B * T * world
+    value = tokens_per_step / (ms_per_step * 1e-3)
+    launches_per_call = 1
+    avg_kernel_s = sum(times) / len(times) * 1e-3
+    alg_bytes = PREFILL_BYTES_PER_TOKEN_HEAD * B * T * H + 2 * STATE_BYTES * B * H
+    achieved = alg_bytes / avg_kernel_s / 1e9
+    pages_flops = PAGES_FLOPS_PER_TOKEN_HEAD * B * T * H
+    tflops = pages_flops / avg_kernel_s / 1e12
+    roofline = {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / pk["hbm_gbs"], "traffic": args.traffic,
+                "peak_source": pk_kind, "kernel": "kda_chunk_fwd (prefill)",
+                "alg_bytes_per_launch": alg_bytes,
+                "tensor_pages_flops": {"achieved_tflops": tflops, "peak": pk["bf16_tflops"],
+                                       "frac": tflops / pk["bf16_tflops"],
+                                       "flops_per_launch": pages_flops}}
+
+    # ---------------- e2e through host buffers (pinned), copies inside the timed region
+    host = {n: getattr(inp, n).cpu().pin_memory() for n in ("q", "k", "v", "log_alpha", "beta", "S0")}
+    dbuf = {n: torch.empty_like(getattr(inp, n)) for n in host}
+    o_h = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+    s_h = torch.empty(S_T.shape, dtype=S_T.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = o_h.numel() * o_h.element_size() + s_h.numel() * s_h.element_size()
+
+    def e2e_step():
+        with torch.cuda.stream(stream):
+            for n, t in host.items():
+                dbuf[n].copy_(t, non_blocking=True)
+            kda.chunk_fwd(dbuf["q"], dbuf["k"], dbuf["v"], dbuf["log_alpha"], dbuf["beta"],
+                          dbuf["S0"], out=o, state_out=S_T, workspace=ws, stream=stream)
+            o_h.copy_(o, non_blocking=True)
+            s_h.copy_(S_T, non_blocking=True)
+
+    e2e_steps = max(3, min(args.steps, 10))
+    barrier(world)
+    e_times = time_steps(e2e_step, e2e_steps, max(3, args.warmup // 2), stream)
+    barrier(world)
+    e_ms = max_over_ranks(sum(e_times), world, dev) / e2e_steps
+    e2e = {"value": tokens_per_step / (e_ms * 1e-3), "unit": "tokens/s",
+           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e_ms}
+    del host, dbuf
+
+    # ---------------- decode (N=256, H=32, 1024 steps in one CUDA graph)
+    decode = None
+    if not args.no_decode:
+        N, Hd, nsteps = DECODE["N"], DECODE["H"], args.decode_steps
+        dinp = decode_inputs(steps=nsteps, N=N, H=Hd, dtype=torch.bfloat16, s0_std=DECODE["s0_std"],
+                             la_range=DECODE["la_range"], seed=DECODE["seed"] + 1000 * rank,
+                             device=dev)
+        S = dinp.S.clone()
+        od = torch.empty_like(dinp.v)
+        with torch.cuda.stream(stream):
+            kda.decode_step(dinp.q[0], dinp.k[0], dinp.v[0], dinp.log_alpha[0], dinp.beta[0],
+                            S.clone(), out=od[0], stream=stream)
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream):
+            for t in range(nsteps):
+                kda.decode_step(dinp.q[t], dinp.k[t], dinp.v[t], dinp.log_alpha[t], dinp.beta[t], S,
+                                out=od[t], stream=stream)
+        barrier(world)
+        dclk = ClockSampler(dev.index)
+        d_times = time_steps(graph.replay, 2, 1, stream, flush)
+        dclk = dclk.stop()
+        barrier(world)
+        d_ms = max_over_ranks(sum(d_times), world, dev) / len(d_times)
+        per_launch = d_ms * 1e-3 / nsteps
+        d_bytes = DECODE_BYTES_PER_HEAD_STEP * N * Hd
+        d_ach = d_bytes / per_launch / 1e9
+        decode = {"value": N * nsteps * world / (d_ms * 1e-3), "unit": "tokens/s",
+                  "ms_per_graph": d_ms, "us_per_step": per_launch * 1e6,
+                  "config": {"workload": f"KDA decode N={N} H={Hd} d=128, {nsteps} consecutive "
+                                         "steps in one CUDA graph", "l2": "state 512 MiB > L2"},
+                  "roofline": {"bound": "hbm", "achieved": d_ach, "peak": pk["hbm_gbs"],
+                               "unit": "GB/s", "frac": d_ach / pk["hbm_gbs"],
+                               "traffic": args.decode_traffic, "peak_source": pk_kind,
+                               "kernel": "kda_decode_step", "alg_bytes_per_launch": d_bytes},
+                  "gpu_launches": nsteps * len(d_times), "clocks": dclk}
+        del graph, dinp, S, od
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_oracle_sample(inp)
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+                "data": "synthetic",
+                "config": {"workload": f"KDA prefill B={B} T={T} H={H} d=128 C=64, bf16 q/k/v, fp32 "
+                                       "log_alpha/beta/state, S0~N(0,0.1^2)",
+                           "global_batch": B * world, "seq_len": T, "parallelism": f"dp{world}",
+                           "l2": "flushed before every step (256 MiB write); inputs 412 MB > L2"},
+                "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+                "gpu_launches": launches_per_call * args.steps, "clocks": clk, "decode": decode}
+        print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["kda", "reference"], default="kda")
+    ap.add_argument("--decode-steps", type=int, default=DECODE["steps"])
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--traffic", type=float, default=None,
+                    help="ncu dram bytes per prefill launch, if captured for this build")
+    ap.add_argument("--decode-traffic", type=float, default=None,
+                    help="ncu dram bytes per decode launch, if captured for this build")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1 and args.impl == "kda":
+        import datetime
+
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                             device_id=torch.device("cuda", local_rank))
+    try:
+        if args.impl == "reference":
+            run_reference(args, rank, world)
+        else:
+            run_kda(args, rank, world, local_rank)
+    finally:
+        if world > 1 and args.impl == "kda":
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

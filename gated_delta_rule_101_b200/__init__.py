@@ -1,4 +1,203 @@
-"""B200-native Kimi Delta Attention (KDA): a thin Python binding over libkda.
+"""B200-native Kimi Delta Attention (KDA) forward: a thin binding over libkda.
 
-The binding is filled in alongside the CUDA library.
+libkda (``libkda.so`` next to this file, built by ``build.py`` from
+``csrc/``) implements the two entry points of ``include/kda.h``:
+
+* ``chunk_fwd``   -> ``kda_chunk_fwd``: chunk-parallel prefill, C = 64;
+* ``decode_step`` -> ``kda_decode_step``: one recurrent decode token.
+
+This module only marshals arguments: it checks dtypes, shapes and devices,
+allocates outputs with PyTorch (device memory is PyTorch's job here), and
+passes raw device pointers and the current CUDA stream to the C ABI. Every
+step of the computation runs in libkda's CUDA kernels; there is no Python or
+CPU fallback, and a missing library is an error.
 """
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libkda.so")
+HEADER = os.path.join(os.path.dirname(_PKG), "include", "kda.h")
+
+KDA_BF16, KDA_F32 = 0, 1
+KDA_OK = 0
+STATUS = {0: "KDA_OK", -1: "KDA_ERR_INVALID_ARG", -2: "KDA_ERR_UNSUPPORTED",
+          -3: "KDA_ERR_WORKSPACE", -4: "KDA_ERR_CUDA", -5: "KDA_ERR_TIMEOUT"}
+HEAD_DIM = 128
+CHUNK = 64
+
+_lib = None
+
+
+class KDAError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where} failed: {STATUS.get(status, status)}")
+
+
+def _bind(lib: ctypes.CDLL) -> ctypes.CDLL:
+    vp, i32, i64, fp = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_void_p
+    lib.kda_strerror.restype = ctypes.c_char_p
+    lib.kda_strerror.argtypes = [i32]
+    lib.kda_version.restype = i32
+    lib.kda_version.argtypes = []
+    lib.kda_chunk_fwd_workspace_size.restype = i32
+    lib.kda_chunk_fwd_workspace_size.argtypes = [i32, i64, i32, i32, i32, i32,
+                                                 ctypes.POINTER(ctypes.c_size_t)]
+    lib.kda_chunk_fwd.restype = i32
+    lib.kda_chunk_fwd.argtypes = [vp, vp, vp, fp, fp, fp, vp, fp, i32, i64, i32, i32, vp, i32,
+                                  vp, i32, vp, ctypes.c_size_t, vp]
+    lib.kda_decode_step.restype = i32
+    lib.kda_decode_step.argtypes = [vp, vp, vp, fp, fp, fp, vp, i32, i32, i32, vp]
+    return lib
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libkda handle. Raises if the library has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"libkda is not built ({LIB_PATH} missing); "
+                               "run `python -m gated_delta_rule_101_b200.build`")
+        _lib = _bind(ctypes.CDLL(LIB_PATH))
+    return _lib
+
+
+def declared_symbols(header: str = HEADER) -> list[str]:
+    """Names of the entry points declared with KDA_API in include/kda.h."""
+    text = open(header, encoding="utf-8").read()
+    return re.findall(r"KDA_API\s+[^;(]*?\b(kda_\w+)\s*\(", text)
+
+
+def strerror(status: int) -> str:
+    return lib().kda_strerror(int(status)).decode()
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return KDA_BF16
+    if t.dtype == torch.float32:
+        return KDA_F32
+    raise TypeError(f"q/k/v must be bfloat16 or float32, got {t.dtype}")
+
+
+def _ptr(t: torch.Tensor | None):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _need(t: torch.Tensor, name: str, dtype, device) -> None:
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if t.device != device:
+        raise ValueError(f"{name} must be on {device}, got {t.device}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _stream_handle(stream: torch.cuda.Stream | None, device) -> ctypes.c_void_p:
+    s = stream if stream is not None else torch.cuda.current_stream(device)
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def workspace_size(B: int, T: int, H: int, n_seqs: int = 0, dtype=torch.bfloat16,
+                   C: int = CHUNK) -> int:
+    out = ctypes.c_size_t(0)
+    code = KDA_BF16 if dtype == torch.bfloat16 else KDA_F32
+    st = lib().kda_chunk_fwd_workspace_size(int(B), int(T), int(H), int(C), int(n_seqs), code,
+                                            ctypes.byref(out))
+    if st != KDA_OK:
+        raise KDAError(st, "kda_chunk_fwd_workspace_size")
+    return int(out.value)
+
+
+def chunk_fwd(q, k, v, log_alpha, beta, S0=None, *, cu_seqlens=None, cu_seqlens_host=None,
+              out=None, final_state=True, state_out=None, workspace=None, stream=None, C=CHUNK):
+    """KDA prefill through ``kda_chunk_fwd``; returns ``(o, S_T)`` (S_T None if not requested).
+
+    ``q, k, v, log_alpha``: ``[B, T, H, 128]`` (or packed ``[T, H, 128]`` with
+    ``cu_seqlens``, an int32 device tensor of ``n_seqs + 1`` offsets).
+    ``beta``: ``[B, T, H]``. ``S0``: fp32 ``[n_seqs, H, 128, 128]`` or None.
+    ``state_out`` may be ``S0`` itself for in-place carry.
+    """
+    dev = q.device
+    code = _dtype_code(q)
+    packed = cu_seqlens is not None
+    if packed:
+        T, H, dk = q.shape
+        B = 1
+        n_seqs = cu_seqlens.numel() - 1
+        _need(cu_seqlens, "cu_seqlens", torch.int32, dev)
+    else:
+        B, T, H, dk = q.shape
+        n_seqs = 0
+    if dk != HEAD_DIM:
+        raise ValueError(f"head dim must be {HEAD_DIM}, got {dk}")
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _need(t, name, q.dtype, dev)
+        if t.shape != q.shape:
+            raise ValueError(f"{name} shape {tuple(t.shape)} != q shape {tuple(q.shape)}")
+    _need(log_alpha, "log_alpha", torch.float32, dev)
+    _need(beta, "beta", torch.float32, dev)
+    if log_alpha.shape != q.shape or beta.shape != q.shape[:-1]:
+        raise ValueError("log_alpha must match q; beta must be q.shape[:-1]")
+    nseq = n_seqs if packed else B
+    sshape = (nseq, H, HEAD_DIM, HEAD_DIM)
+    if S0 is not None:
+        _need(S0, "S0", torch.float32, dev)
+        if tuple(S0.shape) != sshape:
+            raise ValueError(f"S0 must be {sshape}")
+    if out is None:
+        out = torch.empty_like(v)
+    _need(out, "out", q.dtype, dev)
+    S_T = None
+    if state_out is not None:
+        _need(state_out, "state_out", torch.float32, dev)
+        S_T = state_out
+    elif final_state:
+        S_T = torch.empty(sshape, dtype=torch.float32, device=dev)
+    host_cu = None
+    if cu_seqlens_host is not None:
+        host_cu = torch.as_tensor(cu_seqlens_host, dtype=torch.int32).contiguous().cpu()
+    need = workspace_size(B, T, H, n_seqs, q.dtype, C)
+    if need and workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = lib().kda_chunk_fwd(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(S0), _ptr(out), _ptr(S_T),
+        B, T, H, C, _ptr(cu_seqlens), n_seqs, _ptr(host_cu), code, _ptr(workspace), ws_bytes,
+        _stream_handle(stream, dev))
+    if st != KDA_OK:
+        raise KDAError(st, "kda_chunk_fwd")
+    return out, S_T
+
+
+def decode_step(q, k, v, log_alpha, beta, S, *, out=None, stream=None):
+    """One decode token through ``kda_decode_step``; updates ``S`` in place, returns ``o``.
+
+    ``q, k, v, log_alpha``: ``[N, H, 128]``; ``beta``: ``[N, H]``;
+    ``S``: fp32 ``[N, H, 128, 128]``.
+    """
+    dev = q.device
+    code = _dtype_code(q)
+    N, H, dk = q.shape
+    if dk != HEAD_DIM:
+        raise ValueError(f"head dim must be {HEAD_DIM}, got {dk}")
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _need(t, name, q.dtype, dev)
+    _need(log_alpha, "log_alpha", torch.float32, dev)
+    _need(beta, "beta", torch.float32, dev)
+    _need(S, "S", torch.float32, dev)
+    if tuple(S.shape) != (N, H, HEAD_DIM, HEAD_DIM):
+        raise ValueError("S must be [N, H, 128, 128]")
+    if out is None:
+        out = torch.empty_like(v)
+    st = lib().kda_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(S),
+                               _ptr(out), N, H, code, _stream_handle(stream, dev))
+    if st != KDA_OK:
+        raise KDAError(st, "kda_decode_step")
+    return out

@@ -1,0 +1,96 @@
+// libkda C ABI: argument validation and kernel dispatch.
+//
+// Every check here runs on the host before any launch, so a rejected call
+// leaves all outputs untouched. The library allocates nothing: the caller
+// provides every buffer (see include/kda.h).
+#include "kda_internal.cuh"
+
+namespace {
+
+constexpr int KDA_VERSION = 100;  // 0.1.0
+
+bool valid_dtype(int dtype) { return dtype == KDA_BF16 || dtype == KDA_F32; }
+
+// Validates the shape arguments shared by the size query and the call.
+int check_prefill_shape(int B, int64_t T, int H, int C, int n_seqs, int dtype) {
+    if (C != KDA_CHUNK) return KDA_ERR_UNSUPPORTED;
+    if (!valid_dtype(dtype)) return KDA_ERR_UNSUPPORTED;
+    if (B <= 0 || T < 0 || H <= 0 || n_seqs < 0) return KDA_ERR_INVALID_ARG;
+    if (n_seqs > 0 && B != 1) return KDA_ERR_INVALID_ARG;
+    if (n_seqs == 0 && T == 0) return KDA_ERR_INVALID_ARG;
+    // grid limits: y = H (<= 65535); x = sequences
+    if (H > 65535) return KDA_ERR_INVALID_ARG;
+    if (T > (int64_t)INT32_MAX) return KDA_ERR_INVALID_ARG;  // offsets are int32
+    return KDA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *kda_strerror(int status) {
+    switch (status) {
+    case KDA_OK: return "KDA_OK";
+    case KDA_ERR_INVALID_ARG: return "KDA_ERR_INVALID_ARG: invalid argument";
+    case KDA_ERR_UNSUPPORTED: return "KDA_ERR_UNSUPPORTED: unsupported chunk size or dtype";
+    case KDA_ERR_WORKSPACE: return "KDA_ERR_WORKSPACE: workspace missing or too small";
+    case KDA_ERR_CUDA: return "KDA_ERR_CUDA: kernel launch failed";
+    case KDA_ERR_TIMEOUT: return "KDA_ERR_TIMEOUT: bounded device wait expired";
+    default: return "unknown kda status";
+    }
+}
+
+int kda_version(void) { return KDA_VERSION; }
+
+int kda_chunk_fwd_workspace_size(int B, int64_t T, int H, int C, int n_seqs, int dtype,
+                                 size_t *bytes) {
+    if (!bytes) return KDA_ERR_INVALID_ARG;
+    const int st = check_prefill_shape(B, T, H, C, n_seqs, dtype);
+    if (st != KDA_OK) return st;
+    *bytes = 0;
+    return KDA_OK;
+}
+
+int kda_chunk_fwd(const void *q, const void *k, const void *v, const float *log_alpha,
+                  const float *beta, const float *S0, void *o, float *S_T, int B, int64_t T,
+                  int H, int C, const int32_t *cu_seqlens, int n_seqs,
+                  const int32_t *cu_seqlens_host, int dtype, void *workspace,
+                  size_t workspace_bytes, void *stream) {
+    int st = check_prefill_shape(B, T, H, C, n_seqs, dtype);
+    if (st != KDA_OK) return st;
+    const bool packed = n_seqs > 0;
+    if (packed != (cu_seqlens != nullptr)) return KDA_ERR_INVALID_ARG;
+    if (T > 0 && (!q || !k || !v || !log_alpha || !beta || !o)) return KDA_ERR_INVALID_ARG;
+    if (cu_seqlens_host) {
+        if (!packed || cu_seqlens_host[0] != 0 || cu_seqlens_host[n_seqs] != T)
+            return KDA_ERR_INVALID_ARG;
+        for (int s = 0; s < n_seqs; ++s)
+            if (cu_seqlens_host[s + 1] < cu_seqlens_host[s]) return KDA_ERR_INVALID_ARG;
+    }
+    size_t need = 0;
+    st = kda_chunk_fwd_workspace_size(B, T, H, C, n_seqs, dtype, &need);
+    if (st != KDA_OK) return st;
+    if (need > 0 && (!workspace || workspace_bytes < need)) return KDA_ERR_WORKSPACE;
+    (void)workspace;
+
+    const int nseq = packed ? n_seqs : B;
+    cudaStream_t s = (cudaStream_t)stream;
+    const cudaError_t err = kda::launch_prefill_simt(q, k, v, log_alpha, beta, S0, o, S_T, nseq,
+                                                     T, H, cu_seqlens, dtype, s);
+    return err == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+int kda_decode_step(const void *q, const void *k, const void *v, const float *log_alpha,
+                    const float *beta, float *S, void *o, int N, int H, int dtype,
+                    void *stream) {
+    if (!valid_dtype(dtype)) return KDA_ERR_UNSUPPORTED;
+    if (N <= 0 || H <= 0) return KDA_ERR_INVALID_ARG;
+    if ((int64_t)N * H > (int64_t)INT32_MAX) return KDA_ERR_INVALID_ARG;
+    if (!q || !k || !v || !log_alpha || !beta || !S || !o) return KDA_ERR_INVALID_ARG;
+    if (((uintptr_t)S & 15u) != 0) return KDA_ERR_INVALID_ARG;  // 128-bit state accesses
+    const cudaError_t err =
+        kda::launch_decode(q, k, v, log_alpha, beta, S, o, N, H, dtype, (cudaStream_t)stream);
+    return err == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+}  // extern "C"

@@ -1,0 +1,120 @@
+// KDA single-token decode step (recurrent form).
+//
+// One token of eq. (1), blog.gzher.com "Kimi K3论文：Kimi Linear" section 3,
+// for every (sequence, head); section 4 says decode runs this recurrent form
+// rather than the chunk kernel. With S' = Diag(alpha) S:
+//
+//   u = S'^T k,  p = S'^T q,  delta = beta (v - u)
+//   S_new = S' + k delta^T,   o = S_new^T q = p + (k . q) delta
+//
+// so the 64 KiB fp32 state of a head is read once and written once, and the
+// step is bound by HBM bandwidth (0.86 FLOP per byte).
+//
+// Layout: one CTA of 256 threads per (sequence, head). Warp w owns state rows
+// 16w .. 16w+15; lane l owns columns 4l .. 4l+3, so every warp access to a row
+// is one contiguous 512-byte segment (float4 per lane). All 16 row loads are
+// issued before any arithmetic to keep 64 KiB per CTA in flight.
+#include "kda_internal.cuh"
+
+namespace kda {
+namespace {
+
+constexpr int DEC_THREADS = 256;
+constexpr int DEC_WARPS = DEC_THREADS / 32;
+constexpr int ROWS_PER_WARP = D / DEC_WARPS;  // 16
+
+template <typename TIn>
+__global__ void __launch_bounds__(DEC_THREADS)
+decode_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const TIn *__restrict__ v,
+              const float *__restrict__ log_alpha, const float *__restrict__ beta,
+              float *__restrict__ S, TIn *__restrict__ o) {
+    const int64_t nh = blockIdx.x;  // sequence * H + head
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+    __shared__ float s_ka[D], s_qa[D], s_k[D], s_a[D];
+    __shared__ float4 s_red[2][DEC_WARPS][D / 4];
+    __shared__ float s_delta[D];
+    __shared__ float s_qk[4];
+
+    float4 *Sp = reinterpret_cast<float4 *>(S + nh * (int64_t)(D * D));
+    float4 st[ROWS_PER_WARP];
+#pragma unroll
+    for (int rr = 0; rr < ROWS_PER_WARP; ++rr)
+        st[rr] = __ldcs(Sp + (warp * ROWS_PER_WARP + rr) * (D / 4) + lane);
+
+    if (tid < D) {
+        const float kk = to_f32(k[nh * D + tid]);
+        const float qq = to_f32(q[nh * D + tid]);
+        const float a = expf(log_alpha[nh * D + tid]);
+        s_k[tid] = kk;
+        s_a[tid] = a;
+        s_ka[tid] = kk * a;
+        s_qa[tid] = qq * a;
+        float qk = qq * kk;
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) qk += __shfl_xor_sync(0xffffffffu, qk, off);
+        if (lane == 0) s_qk[warp] = qk;
+    }
+    __syncthreads();
+
+    float4 u = make_float4(0.f, 0.f, 0.f, 0.f), p = u;
+#pragma unroll
+    for (int rr = 0; rr < ROWS_PER_WARP; ++rr) {
+        const int i = warp * ROWS_PER_WARP + rr;
+        const float ka = s_ka[i], qa = s_qa[i];
+        u.x += ka * st[rr].x; u.y += ka * st[rr].y; u.z += ka * st[rr].z; u.w += ka * st[rr].w;
+        p.x += qa * st[rr].x; p.y += qa * st[rr].y; p.z += qa * st[rr].z; p.w += qa * st[rr].w;
+    }
+    s_red[0][warp][lane] = u;
+    s_red[1][warp][lane] = p;
+    __syncthreads();
+
+    if (tid < D) {
+        const float *ru = reinterpret_cast<const float *>(&s_red[0][0][0]);
+        const float *rp = reinterpret_cast<const float *>(&s_red[1][0][0]);
+        float uj = 0.f, pj = 0.f;
+#pragma unroll
+        for (int w = 0; w < DEC_WARPS; ++w) {
+            uj += ru[w * D + tid];
+            pj += rp[w * D + tid];
+        }
+        const float b = beta[nh];
+        const float d = b * (to_f32(v[nh * D + tid]) - uj);
+        s_delta[tid] = d;
+        const float qk = s_qk[0] + s_qk[1] + s_qk[2] + s_qk[3];
+        o[nh * D + tid] = from_f32<TIn>(pj + qk * d);
+    }
+    __syncthreads();
+
+    const float4 d4 = reinterpret_cast<const float4 *>(s_delta)[lane];
+#pragma unroll
+    for (int rr = 0; rr < ROWS_PER_WARP; ++rr) {
+        const int i = warp * ROWS_PER_WARP + rr;
+        const float a = s_a[i], kk = s_k[i];
+        float4 s = st[rr];
+        s.x = a * s.x + kk * d4.x;
+        s.y = a * s.y + kk * d4.y;
+        s.z = a * s.z + kk * d4.z;
+        s.w = a * s.w + kk * d4.w;
+        __stcs(Sp + i * (D / 4) + lane, s);
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_decode(const void *q, const void *k, const void *v, const float *log_alpha,
+                          const float *beta, float *S, void *o, int N, int H, int dtype,
+                          cudaStream_t stream) {
+    const unsigned grid = (unsigned)((int64_t)N * H);
+    if (dtype == KDA_BF16) {
+        decode_kernel<__nv_bfloat16><<<grid, DEC_THREADS, 0, stream>>>(
+            (const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k, (const __nv_bfloat16 *)v,
+            log_alpha, beta, S, (__nv_bfloat16 *)o);
+    } else {
+        decode_kernel<float><<<grid, DEC_THREADS, 0, stream>>>(
+            (const float *)q, (const float *)k, (const float *)v, log_alpha, beta, S, (float *)o);
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace kda

@@ -1,0 +1,45 @@
+// Internal declarations shared by the libkda translation units.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "kda.h"
+
+namespace kda {
+
+constexpr int D = KDA_HEAD_DIM;  // dk = dv
+constexpr int CH = KDA_CHUNK;    // chunk length
+
+__device__ __forceinline__ float to_f32(float x) { return x; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+template <typename T> __device__ __forceinline__ T from_f32(float x);
+template <> __device__ __forceinline__ float from_f32<float>(float x) { return x; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
+    return __float2bfloat16_rn(x);
+}
+
+// Where a sequence's tokens live: [start, start + len) in token rows.
+struct SeqSpan {
+    int64_t start;
+    int64_t len;
+};
+
+__device__ __forceinline__ SeqSpan seq_span(const int32_t *cu, int64_t T, int s) {
+    if (cu) return {(int64_t)cu[s], (int64_t)cu[s + 1] - (int64_t)cu[s]};
+    return {(int64_t)s * T, T};
+}
+
+// ---- launchers (host side); each returns cudaGetLastError() of its launch ----
+cudaError_t launch_decode(const void *q, const void *k, const void *v, const float *log_alpha,
+                          const float *beta, float *S, void *o, int N, int H, int dtype,
+                          cudaStream_t stream);
+
+cudaError_t launch_prefill_simt(const void *q, const void *k, const void *v,
+                                const float *log_alpha, const float *beta, const float *S0,
+                                void *o, float *S_T, int n_seqs, int64_t T, int H,
+                                const int32_t *cu_seqlens, int dtype, cudaStream_t stream);
+
+}  // namespace kda

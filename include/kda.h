@@ -1,0 +1,138 @@
+/*
+ * libkda: Kimi Delta Attention (KDA) forward on NVIDIA B200 (sm_100a).
+ *
+ * KDA is the gated delta rule with one forget rate per key channel
+ * (blog.gzher.com "Kimi K3论文：Kimi Linear", section 3, eq. (1)):
+ *
+ *     S_t = (I - beta_t k_t k_t^T) Diag(alpha_t) S_{t-1} + beta_t k_t v_t^T
+ *     o_t = S_t^T q_t                               (read after the update)
+ *
+ * with S_t a dk x dv state per (sequence, head), dk = dv = 128,
+ * alpha_t = exp(log_alpha_t) in [0,1]^dk and beta_t in [0,1]. There is no
+ * query scaling; callers that want 1/sqrt(dk) scale q themselves.
+ *
+ * Two entry points compute it: a chunk-parallel prefill over whole
+ * sequences (section 4 of the same page: chunks of C = 64, WY representation,
+ * UT transform, state passed between chunks) and a single-token recurrent
+ * decode step (section 4: decode switches to the recurrent kernel).
+ *
+ * Conventions shared by every call
+ *   - Every pointer is DEVICE memory owned by the caller. The library never
+ *     allocates, frees or synchronises; calls are asynchronous on `stream`
+ *     (a cudaStream_t, NULL = the legacy default stream).
+ *   - All tensors are contiguous, row-major, in the layouts given below.
+ *     Token-major tensors index [token][head][channel].
+ *   - q, k, v and o share one element type, `dtype` (kda_dtype). log_alpha,
+ *     beta and the state are always fp32.
+ *   - Preconditions that are not checked element by element: q and k rows
+ *     L2-normalised per head (the layer's L2Norm, section 3), log_alpha
+ *     finite and <= 0 (use a large finite negative number, not -inf, for
+ *     alpha = 0), beta in [0, 1].
+ *   - Return value: KDA_OK (0) or a negative kda_status. Argument errors are
+ *     detected on the host before anything is launched; nothing is written
+ *     in that case. KDA_ERR_CUDA means a launch failed (the CUDA error is
+ *     left for the caller to read with cudaGetLastError).
+ */
+#ifndef KDA_H_
+#define KDA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define KDA_API __attribute__((visibility("default")))
+#else
+#define KDA_API
+#endif
+
+#define KDA_HEAD_DIM 128 /* dk = dv, fixed */
+#define KDA_CHUNK 64     /* the only chunk size accepted by kda_chunk_fwd */
+
+typedef enum kda_dtype {
+    KDA_BF16 = 0, /* q, k, v, o are bfloat16 */
+    KDA_F32 = 1   /* q, k, v, o are float32 */
+} kda_dtype;
+
+typedef enum kda_status {
+    KDA_OK = 0,
+    KDA_ERR_INVALID_ARG = -1, /* null pointer, bad size, bad offsets */
+    KDA_ERR_UNSUPPORTED = -2, /* C != 64 or unknown dtype */
+    KDA_ERR_WORKSPACE = -3,   /* workspace missing or smaller than required */
+    KDA_ERR_CUDA = -4,        /* a kernel launch failed */
+    KDA_ERR_TIMEOUT = -5      /* a bounded device-side wait expired */
+} kda_status;
+
+/* Human-readable name of a status code (static string, never NULL). */
+KDA_API const char *kda_strerror(int status);
+
+/* Library version as 10000*major + 100*minor + patch. */
+KDA_API int kda_version(void);
+
+/*
+ * Bytes of device workspace kda_chunk_fwd needs for these sizes.
+ *
+ * Arguments are those of kda_chunk_fwd: B batch rows of T tokens, or, when
+ * n_seqs > 0, one packed row (B = 1) of T tokens split into n_seqs
+ * sequences. Writes the size to *bytes (0 is possible). The workspace holds
+ * per-chunk intermediates (the WY factors) between the kernels of one call;
+ * it carries nothing from one call to the next.
+ */
+KDA_API int kda_chunk_fwd_workspace_size(int B, int64_t T, int H, int C, int n_seqs, int dtype,
+                                 size_t *bytes);
+
+/*
+ * Chunk-parallel KDA prefill (blog.gzher.com section 4; chunked form of the
+ * mokono.cn explainer section 2.1: S_r = P_r S_0 + H_r within a chunk).
+ *
+ *   q, k       [B, T, H, 128]  dtype    (with cu_seqlens: [T, H, 128], B = 1)
+ *   v          [B, T, H, 128]  dtype
+ *   log_alpha  [B, T, H, 128]  fp32     log of the per-channel forget gate
+ *   beta       [B, T, H]       fp32     write strength
+ *   S0         [Nseq, H, 128, 128] fp32 initial state (dk rows, dv columns),
+ *                               or NULL for zeros
+ *   o          [B, T, H, 128]  dtype    output (written)
+ *   S_T        [Nseq, H, 128, 128] fp32 final state (written), or NULL
+ *   C          chunk length; must be 64
+ *   cu_seqlens device int32 [n_seqs + 1] token offsets of packed sequences
+ *              (cu_seqlens[0] = 0, non-decreasing, cu_seqlens[n_seqs] = T),
+ *              or NULL: then Nseq = B sequences of T tokens each.
+ *   cu_seqlens_host  optional host copy of cu_seqlens. When given it is
+ *              validated (monotone, ends at T); when NULL the device offsets
+ *              are trusted.
+ *   workspace  device buffer of at least kda_chunk_fwd_workspace_size bytes,
+ *              16-byte aligned (NULL allowed when that size is 0).
+ *
+ * Chunks start at each sequence's first token; the last chunk of a sequence
+ * may be shorter than C. A sequence of length 0 writes no output rows and
+ * S_T = S0. S0 and S_T may point to the same buffer (in-place carry, which
+ * is how a long sequence is processed as several calls). q, k, v, o must not
+ * overlap.
+ */
+KDA_API int kda_chunk_fwd(const void *q, const void *k, const void *v, const float *log_alpha,
+                  const float *beta, const float *S0, void *o, float *S_T, int B, int64_t T,
+                  int H, int C, const int32_t *cu_seqlens, int n_seqs,
+                  const int32_t *cu_seqlens_host, int dtype, void *workspace,
+                  size_t workspace_bytes, void *stream);
+
+/*
+ * One recurrent decode step for N sequences (eq. (1) applied to one token;
+ * blog.gzher.com section 4: decode uses the recurrent kernel).
+ *
+ *   q, k, v    [N, H, 128]  dtype
+ *   log_alpha  [N, H, 128]  fp32
+ *   beta       [N, H]       fp32
+ *   S          [N, H, 128, 128] fp32, read and overwritten in place with S_t
+ *   o          [N, H, 128]  dtype   output o_t = S_t^T q_t (written)
+ */
+KDA_API int kda_decode_step(const void *q, const void *k, const void *v, const float *log_alpha,
+                    const float *beta, float *S, void *o, int N, int H, int dtype, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KDA_H_ */

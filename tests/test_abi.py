@@ -1,0 +1,105 @@
+"""libkda's C ABI on the host: exports and argument validation (no GPU needed).
+
+Every rejected call below returns before any CUDA call is made, so fake
+device pointers are safe: nothing dereferences them.
+"""
+import ctypes
+
+import pytest
+
+import gated_delta_rule_101_b200 as kda
+from gated_delta_rule_101_b200 import build as kbuild
+
+BF16, F32 = kda.KDA_BF16, kda.KDA_F32
+INVALID, UNSUPPORTED, WORKSPACE = -1, -2, -3
+FAKE = ctypes.c_void_p(1 << 20)  # never dereferenced: every call here fails validation
+
+
+@pytest.fixture(scope="module")
+def lib():
+    kbuild.build()
+    return kda.lib()
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = kda.declared_symbols()
+    assert {"kda_chunk_fwd", "kda_decode_step", "kda_chunk_fwd_workspace_size",
+            "kda_strerror", "kda_version"} <= set(names)
+    for n in names:
+        assert hasattr(lib, n), f"{n} declared in include/kda.h but not exported"
+
+
+def test_strerror_and_version(lib):
+    for code, name in kda.STATUS.items():
+        assert kda.strerror(code).startswith(name)
+    assert kda.strerror(-99) == "unknown kda status"
+    assert lib.kda_version() >= 100
+
+
+def _chunk(lib, *, q=FAKE, k=FAKE, v=FAKE, la=FAKE, beta=FAKE, S0=None, o=FAKE, ST=None, B=1,
+           T=128, H=2, C=64, cu=None, n_seqs=0, cu_host=None, dtype=BF16, ws=None, ws_bytes=0):
+    return lib.kda_chunk_fwd(q, k, v, la, beta, S0, o, ST, B, T, H, C, cu, n_seqs, cu_host, dtype,
+                             ws, ws_bytes, None)
+
+
+def test_chunk_fwd_rejects_bad_arguments(lib):
+    assert _chunk(lib, C=32) == UNSUPPORTED
+    assert _chunk(lib, C=128) == UNSUPPORTED
+    assert _chunk(lib, dtype=7) == UNSUPPORTED
+    assert _chunk(lib, B=0) == INVALID
+    assert _chunk(lib, H=0) == INVALID
+    assert _chunk(lib, T=-1) == INVALID
+    assert _chunk(lib, T=0) == INVALID  # batched rows of zero tokens
+    for field in ("q", "k", "v", "la", "beta", "o"):
+        assert _chunk(lib, **{field: None}) == INVALID, field
+    # cu_seqlens without n_seqs, n_seqs without cu_seqlens, packed with B != 1
+    assert _chunk(lib, cu=FAKE) == INVALID
+    assert _chunk(lib, n_seqs=2) == INVALID
+    assert _chunk(lib, cu=FAKE, n_seqs=2, B=2) == INVALID
+
+
+@pytest.mark.parametrize("offsets", [[0, 64, 32, 128], [1, 64, 128], [0, 64, 127], [0, 64, 129]])
+def test_chunk_fwd_rejects_bad_host_offsets(lib, offsets):
+    host = (ctypes.c_int32 * len(offsets))(*offsets)
+    st = _chunk(lib, cu=FAKE, n_seqs=len(offsets) - 1, T=128, cu_host=host)
+    assert st == INVALID
+
+
+def test_workspace_size_query(lib):
+    out = ctypes.c_size_t(123)
+    assert lib.kda_chunk_fwd_workspace_size(1, 64, 2, 64, 0, BF16, None) == INVALID
+    assert lib.kda_chunk_fwd_workspace_size(1, 64, 2, 32, 0, BF16, ctypes.byref(out)) == UNSUPPORTED
+    assert lib.kda_chunk_fwd_workspace_size(4, 4096, 16, 64, 0, BF16, ctypes.byref(out)) == 0
+    assert lib.kda_chunk_fwd_workspace_size(1, 4096, 16, 64, 3, F32, ctypes.byref(out)) == 0
+
+
+def test_chunk_fwd_rejects_short_workspace(lib):
+    need = ctypes.c_size_t(0)
+    assert lib.kda_chunk_fwd_workspace_size(4, 4096, 16, 64, 0, BF16, ctypes.byref(need)) == 0
+    if need.value == 0:
+        pytest.skip("this build needs no workspace for bf16 prefill")
+    assert _chunk(lib, B=4, T=4096, H=16, ws=FAKE, ws_bytes=need.value - 1) == WORKSPACE
+    assert _chunk(lib, B=4, T=4096, H=16, ws=None, ws_bytes=need.value) == WORKSPACE
+
+
+def test_decode_rejects_bad_arguments(lib):
+    def call(**kw):
+        a = dict(q=FAKE, k=FAKE, v=FAKE, la=FAKE, beta=FAKE, S=FAKE, o=FAKE, N=4, H=2, dtype=BF16)
+        a.update(kw)
+        return lib.kda_decode_step(a["q"], a["k"], a["v"], a["la"], a["beta"], a["S"], a["o"],
+                                   a["N"], a["H"], a["dtype"], None)
+
+    assert call(dtype=3) == UNSUPPORTED
+    assert call(N=0) == INVALID
+    assert call(H=-1) == INVALID
+    for field in ("q", "k", "v", "la", "beta", "S", "o"):
+        assert call(**{field: None}) == INVALID, field
+    assert call(S=ctypes.c_void_p((1 << 20) + 4)) == INVALID  # state must be 16-byte aligned
+
+
+def test_binding_refuses_wrong_dtypes_before_calling():
+    import torch
+
+    q = torch.zeros(1, 64, 1, 128, dtype=torch.float16)
+    with pytest.raises(TypeError):
+        kda.chunk_fwd(q, q, q, q.float(), q[..., 0].float())

@@ -1,0 +1,201 @@
+"""kda_chunk_fwd on the GPU against the fp64 oracle."""
+import numpy as np
+import pytest
+import torch
+
+import gated_delta_rule_101_b200 as kda
+import oracle
+from gated_delta_rule_101_b200.inputs import cu_from_lengths, prefill_inputs, varlen_lengths
+from parity import check
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda:0"
+KIND = {torch.bfloat16: "bf16", torch.float32: "f32"}
+
+
+def run(inp, **kw):
+    o, st = kda.chunk_fwd(inp.q, inp.k, inp.v, inp.log_alpha, inp.beta, inp.S0,
+                          cu_seqlens=inp.cu_seqlens, **kw)
+    torch.cuda.synchronize()
+    return o, st
+
+
+def ref(inp):
+    return oracle.kda_fwd(inp.q, inp.k, inp.v, inp.log_alpha, inp.beta, inp.S0,
+                          cu_seqlens=None if inp.cu_seqlens is None else inp.cu_seqlens.cpu())
+
+
+def test_tiny_fp32_config_all_outputs():
+    """B=1, T=256, H=2, fp32, S0 = 0: relative L2 <= 1e-4."""
+    inp = prefill_inputs(B=1, T=256, H=2, dtype=torch.float32, seed=20260, device=DEV)
+    o, st = run(inp)
+    ro, rs = ref(inp)
+    check(o, ro, "f32", "o")
+    check(st, rs, "f32", "S_T")
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("T", [1, 63, 64, 65, 300])
+def test_batched_ragged_with_state(dtype, T):
+    inp = prefill_inputs(B=2, T=T, H=3, dtype=dtype, s0_std=0.1, seed=T, device=DEV)
+    o, st = run(inp)
+    ro, rs = ref(inp)
+    check(o, ro, KIND[dtype], f"o T={T}")
+    check(st, rs, KIND[dtype], f"S_T T={T}")
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_varlen_with_empty_and_ragged_sequences(dtype):
+    lengths = [1, 64, 65, 0, 130, 7, 0, 200]
+    cu = cu_from_lengths(lengths)
+    inp = prefill_inputs(T=int(cu[-1]), H=2, cu_seqlens=cu, dtype=dtype, s0_std=0.1, seed=9,
+                         device=DEV)
+    o, st = run(inp, cu_seqlens_host=cu)
+    ro, rs = ref(inp)
+    check(o, ro, KIND[dtype], "varlen o")
+    check(st, rs, KIND[dtype], "varlen S_T")
+    # empty sequences keep S0 exactly
+    for i, n in enumerate(lengths):
+        if n == 0:
+            assert torch.equal(st[i], inp.S0[i])
+
+
+@pytest.mark.parametrize("la_range", [(0.5, 3.0), (5.0, 20.0)])
+def test_strong_decay_uses_exact_pairwise_path(la_range):
+    """Chunk log-decay far beyond 80: the factorised exp split would overflow."""
+    inp = prefill_inputs(B=1, T=200, H=2, dtype=torch.float32, la_range=la_range, s0_std=0.1,
+                         seed=11, device=DEV)
+    o, st = run(inp)
+    ro, rs = ref(inp)
+    check(o, ro, "f32", "strong decay o")
+    check(st, rs, "f32", "strong decay S_T")
+
+
+def test_alpha_zero_and_alpha_one_tokens():
+    inp = prefill_inputs(B=1, T=160, H=2, dtype=torch.float32, s0_std=0.1, seed=12, device=DEV)
+    inp.log_alpha[:, 10:12] = -1e4   # alpha = 0: state reset inside a chunk
+    inp.log_alpha[:, 64] = -1e4      # at a chunk start
+    inp.log_alpha[:, 100:140] = 0.0  # alpha = 1 (DeltaNet)
+    inp.beta[:, 20:30] = 0.0
+    inp.beta[:, 30:40] = 1.0
+    o, st = run(inp)
+    ro, rs = ref(inp)
+    check(o, ro, "f32", "alpha 0/1 o")
+    check(st, rs, "f32", "alpha 0/1 S_T")
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_state_carry_across_calls_in_place(dtype):
+    """Processing a sequence as several calls, S0 and S_T aliased, equals one call."""
+    inp = prefill_inputs(B=2, T=333, H=2, dtype=dtype, s0_std=0.1, seed=13, device=DEV)
+    o_full, st_full = run(inp)
+    S = inp.S0.clone()
+    outs = []
+    for a, z in ((0, 64), (64, 100), (100, 101), (101, 333)):
+        o, _ = kda.chunk_fwd(inp.q[:, a:z].contiguous(), inp.k[:, a:z].contiguous(),
+                             inp.v[:, a:z].contiguous(), inp.log_alpha[:, a:z].contiguous(),
+                             inp.beta[:, a:z].contiguous(), S, state_out=S)
+        outs.append(o)
+    torch.cuda.synchronize()
+    ro, rs = ref(inp)
+    check(torch.cat(outs, dim=1), ro, KIND[dtype], "carry o")
+    check(S, rs, KIND[dtype], "carry S_T")
+    check(o_full, ro, KIND[dtype], "single call o")
+
+
+def test_decode_loop_equals_prefill():
+    inp = prefill_inputs(B=2, T=70, H=2, dtype=torch.float32, s0_std=0.1, seed=14, device=DEV)
+    o_p, st_p = run(inp)
+    S = inp.S0.clone()
+    o_d = torch.empty_like(inp.v)
+    for t in range(70):
+        o_d[:, t] = kda.decode_step(inp.q[:, t].contiguous(), inp.k[:, t].contiguous(),
+                                    inp.v[:, t].contiguous(), inp.log_alpha[:, t].contiguous(),
+                                    inp.beta[:, t].contiguous(), S)
+    torch.cuda.synchronize()
+    check(o_d, o_p.double(), "f32", "decode loop vs prefill o")
+    check(S, st_p.double(), "f32", "decode loop vs prefill S")
+
+
+def test_deterministic_bitwise():
+    inp = prefill_inputs(B=2, T=500, H=3, dtype=torch.bfloat16, s0_std=0.1, seed=15, device=DEV)
+    o1, s1 = run(inp)
+    o2, s2 = run(inp)
+    assert torch.equal(o1, o2) and torch.equal(s1, s2)
+
+
+def test_no_final_state_requested():
+    inp = prefill_inputs(B=1, T=100, H=2, dtype=torch.bfloat16, seed=16, device=DEV)
+    o, st = run(inp, final_state=False)
+    assert st is None
+    ro, _ = ref(inp)
+    check(o, ro, "bf16", "o without S_T")
+
+
+# ---------------------------------------------------------------- full sizes, sampled
+def _sample_ref(inp, seqs, heads, cols):
+    """Oracle on sampled (sequence, head) pairs and value columns, whole sequences."""
+    out = []
+    cu = None if inp.cu_seqlens is None else inp.cu_seqlens.cpu().tolist()
+    for s, h in zip(seqs, heads):
+        if cu is None:
+            sl = (slice(s, s + 1), slice(None))
+            pick = lambda x: x[sl][:, :, h:h + 1]
+        else:
+            a, z = cu[s], cu[s + 1]
+            pick = lambda x: x[a:z, h:h + 1][None]
+        q, k, la = pick(inp.q), pick(inp.k), pick(inp.log_alpha)
+        v = pick(inp.v)[..., cols]
+        b = pick(inp.beta[..., None])[..., 0]
+        S0 = None if inp.S0 is None else inp.S0[s, h][:, cols][None, None]
+        out.append(oracle.kda_fwd(q, k, v, la, b, S0))
+    return out
+
+
+def _check_sampled(inp, o, st, seqs, heads, cols, kind, what):
+    cu = None if inp.cu_seqlens is None else inp.cu_seqlens.cpu().tolist()
+    for (s, h), (ro, rs) in zip(zip(seqs, heads), _sample_ref(inp, seqs, heads, cols)):
+        got_o = o[s, :, h][:, cols] if cu is None else o[cu[s]:cu[s + 1], h][:, cols]
+        check(got_o, ro[0, :, 0], kind, f"{what} o (seq {s}, head {h})")
+        check(st[s, h][:, cols], rs[0, 0], kind, f"{what} S_T (seq {s}, head {h})")
+
+
+def test_prefill_workload_b4_t4096_h16_sampled():
+    inp = prefill_inputs(B=4, T=4096, H=16, dtype=torch.bfloat16, s0_std=0.1, seed=20261,
+                         device=DEV)
+    o, st = run(inp)
+    assert torch.isfinite(o.float()).all() and torch.isfinite(st).all()
+    cols = list(range(128))
+    _check_sampled(inp, o, st, [0, 3, 1, 2], [0, 15, 7, 9], cols, "bf16", "B4 T4096 H16")
+
+
+def test_varlen_workload_64_seqs_h32_sampled():
+    lengths = varlen_lengths(64, 512, 16384, seed=20262)
+    cu = cu_from_lengths(lengths)
+    inp = prefill_inputs(T=int(cu[-1]), H=32, cu_seqlens=cu, dtype=torch.bfloat16, seed=20262,
+                         device=DEV)
+    o, st = run(inp, cu_seqlens_host=cu)
+    assert torch.isfinite(st).all()
+    cols = list(range(0, 128, 4))
+    longest = int(np.argmax(lengths))
+    _check_sampled(inp, o, st, [0, longest, 63, 31], [0, 31, 17, 5], cols, "bf16", "varlen 64 seqs")
+
+
+def test_long_context_1m_tokens_as_16_calls_sampled():
+    """B=1, T=2^20 processed as 16 calls of 65,536 tokens with the state carried in place."""
+    H, Tc, calls, h, cols = 32, 65536, 16, 5, [0, 1, 63, 64, 126, 127]
+    S = torch.zeros(1, H, 128, 128, dtype=torch.float32, device=DEV)
+    S_ref = np.zeros((1, 1, 128, len(cols)))
+    for c in range(calls):
+        inp = prefill_inputs(B=1, T=Tc, H=H, dtype=torch.bfloat16, la_range=(0.0001, 0.05),
+                             seed=20264 * 100 + c, device=DEV)
+        o, _ = kda.chunk_fwd(inp.q, inp.k, inp.v, inp.log_alpha, inp.beta, S, state_out=S)
+        torch.cuda.synchronize()
+        # the oracle carries its own state through all calls (sampled head and columns only)
+        sl = lambda x: x[:, :, h:h + 1]
+        ro, S_ref = oracle.kda_fwd(sl(inp.q), sl(inp.k), sl(inp.v)[..., cols], sl(inp.log_alpha),
+                                   inp.beta[:, :, h:h + 1], S_ref)
+        if c in (0, 7, 15):
+            check(o[0, :, h][:, cols], ro[0, :, 0], "bf16", f"1M-token call {c} o")
+    check(S[0, h][:, cols], S_ref[0, 0], "bf16", "1M-token final S_T")
+    assert torch.isfinite(S).all()
