@@ -52,6 +52,8 @@ def _bind(lib: ctypes.CDLL) -> ctypes.CDLL:
     lib.kda_chunk_fwd.restype = i32
     lib.kda_chunk_fwd.argtypes = [vp, vp, vp, fp, fp, fp, vp, fp, i32, i64, i32, i32, vp, i32,
                                   vp, i32, vp, ctypes.c_size_t, vp]
+    lib.kda_get_device_status.restype = i32
+    lib.kda_get_device_status.argtypes = [ctypes.POINTER(ctypes.c_int)]
     lib.kda_decode_step.restype = i32
     lib.kda_decode_step.argtypes = [vp, vp, vp, fp, fp, fp, vp, i32, i32, i32, vp]
     return lib

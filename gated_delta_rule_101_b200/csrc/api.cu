@@ -47,7 +47,7 @@ int kda_chunk_fwd_workspace_size(int B, int64_t T, int H, int C, int n_seqs, int
     if (!bytes) return KDA_ERR_INVALID_ARG;
     const int st = check_prefill_shape(B, T, H, C, n_seqs, dtype);
     if (st != KDA_OK) return st;
-    *bytes = 0;
+    *bytes = dtype == KDA_BF16 ? kda::prefill_tc_workspace(B, T, H, n_seqs) : 0;
     return KDA_OK;
 }
 
@@ -71,13 +71,30 @@ int kda_chunk_fwd(const void *q, const void *k, const void *v, const float *log_
     st = kda_chunk_fwd_workspace_size(B, T, H, C, n_seqs, dtype, &need);
     if (st != KDA_OK) return st;
     if (need > 0 && (!workspace || workspace_bytes < need)) return KDA_ERR_WORKSPACE;
-    (void)workspace;
+    if (need > 0 && ((uintptr_t)workspace & 15u) != 0) return KDA_ERR_WORKSPACE;
 
     const int nseq = packed ? n_seqs : B;
     cudaStream_t s = (cudaStream_t)stream;
-    const cudaError_t err = kda::launch_prefill_simt(q, k, v, log_alpha, beta, S0, o, S_T, nseq,
-                                                     T, H, cu_seqlens, dtype, s);
+    cudaError_t err;
+    if (dtype == KDA_BF16) {
+        // TMA requires 16-byte aligned tensor bases
+        if (T > 0 && ((((uintptr_t)q | (uintptr_t)k | (uintptr_t)v | (uintptr_t)log_alpha) & 15u) != 0))
+            return KDA_ERR_INVALID_ARG;
+        if ((S0 && ((uintptr_t)S0 & 15u)) || (S_T && ((uintptr_t)S_T & 15u)) || ((uintptr_t)o & 15u))
+            return KDA_ERR_INVALID_ARG;
+        err = kda::launch_prefill_tc(q, k, v, log_alpha, beta, S0, o, S_T, B, T, H, cu_seqlens,
+                                     n_seqs, workspace, s);
+    } else {
+        err = kda::launch_prefill_simt(q, k, v, log_alpha, beta, S0, o, S_T, nseq, T, H,
+                                       cu_seqlens, dtype, s);
+    }
+    if (err == cudaErrorInvalidValue) return KDA_ERR_INVALID_ARG;
     return err == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+int kda_get_device_status(int *status) {
+    if (!status) return KDA_ERR_INVALID_ARG;
+    return kda::read_device_status(status) == 0 ? KDA_OK : KDA_ERR_CUDA;
 }
 
 int kda_decode_step(const void *q, const void *k, const void *v, const float *log_alpha,

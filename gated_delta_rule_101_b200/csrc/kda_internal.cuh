@@ -27,6 +27,12 @@ struct SeqSpan {
     int64_t len;
 };
 
+// Rows of this chunk that belong to the sequence (the chunk starts at row c0 of it).
+__device__ __forceinline__ int chunk_rows(int64_t seq_len, int64_t c0) {
+    const int64_t left = seq_len - c0;
+    return left < CH ? (int)left : CH;
+}
+
 __device__ __forceinline__ SeqSpan seq_span(const int32_t *cu, int64_t T, int s) {
     if (cu) return {(int64_t)cu[s], (int64_t)cu[s + 1] - (int64_t)cu[s]};
     return {(int64_t)s * T, T};
@@ -41,5 +47,15 @@ cudaError_t launch_prefill_simt(const void *q, const void *k, const void *v,
                                 const float *log_alpha, const float *beta, const float *S0,
                                 void *o, float *S_T, int n_seqs, int64_t T, int H,
                                 const int32_t *cu_seqlens, int dtype, cudaStream_t stream);
+
+// Tensor-core prefill (bf16 q/k/v): workspace bytes and launcher.
+size_t prefill_tc_workspace(int B, int64_t T, int H, int n_seqs);
+cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, const float *log_alpha,
+                              const float *beta, const float *S0, void *o, float *S_T, int B,
+                              int64_t T, int H, const int32_t *cu_seqlens, int n_seqs,
+                              void *workspace, cudaStream_t stream);
+
+// Reads and clears the device status word set by bounded waits (0 = no timeout).
+int read_device_status(int *status);
 
 }  // namespace kda

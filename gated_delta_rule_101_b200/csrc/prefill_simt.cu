@@ -18,7 +18,9 @@
 // The exp(g_r - g_i) factor is split as exp(g_r) * exp(-g_i) when the chunk's
 // total log-decay is at most 80 in every channel (both factors then stay far
 // from fp32 overflow); otherwise the pairwise exponentials are taken
-// directly. The triangular systems are solved by forward substitution, one
+// directly. g is accumulated as an unevaluated sum hi + lo (Knuth's two-sum),
+// so differences g_r - g_i keep full fp32 precision even when a near-zero
+// gate (log_alpha of -1e4, say) makes |g| huge. The triangular systems are solved by forward substitution, one
 // thread per right-hand-side column.
 //
 // Grid: (sequence, head, dv slice of 32 columns). Each CTA walks its
@@ -38,13 +40,15 @@ constexpr float SAFE_SPAN = 80.f; // max chunk log-decay for the factorised form
 struct SimtSmem {
     float q[CH * LD];    // q, then exp(g) * q
     float k[CH * LD];    // k, then exp(g) * k, then W (solved in place)
-    float g[CH * LD];    // log_alpha, then g, then exp(g_L - g) * k
+    float g[CH * LD];    // log_alpha, then g (high part), then exp(g_L - g) * k
+    float glo[CH * LD];  // low part of g
     float akk[CH * LDA]; // beta-scaled strict-lower Gram
     float aqk[CH * LDA]; // inclusive-lower Gram
     float vu[CH * DVS];  // v slice, then U (solved in place)
     float vn[CH * DVS];  // V_new
     float s[D * DVS];    // state slice S[c][j]
-    float gl[D];         // g_L per channel
+    float gl[D];         // g_L per channel (high part)
+    float gllo[D];       // g_L per channel (low part)
     float einv[D];       // exp(-g_L) per channel
     float beta[CH];
 };
@@ -105,14 +109,19 @@ prefill_simt_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k,
         // ---- g = chunk-local inclusive cumulative sum of log_alpha, per channel
         bool unsafe = false;
         if (tid < D) {
-            float acc = 0.f;
+            float hi = 0.f, lo = 0.f;
             for (int r = 0; r < CH; ++r) {
-                acc += sm.g[r * LD + tid];
-                sm.g[r * LD + tid] = acc;
+                const float x = sm.g[r * LD + tid];
+                const float s = hi + x, bb = s - hi;  // two-sum: s + err == hi + x exactly
+                lo += (hi - (s - bb)) + (x - bb);
+                hi = s;
+                sm.g[r * LD + tid] = hi;
+                sm.glo[r * LD + tid] = lo;
             }
-            sm.gl[tid] = acc;
-            sm.einv[tid] = expf(-acc);
-            unsafe = -acc > SAFE_SPAN;
+            sm.gl[tid] = hi;
+            sm.gllo[tid] = lo;
+            sm.einv[tid] = expf(-(hi + lo));
+            unsafe = -(hi + lo) > SAFE_SPAN;
         }
         unsafe = __syncthreads_or(unsafe);
 
@@ -129,12 +138,14 @@ prefill_simt_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k,
 #pragma unroll
                 for (int b = 0; b < 4; ++b) {
                     const int r = tu + 16 * b;
-                    const float gr = sm.g[r * LD + c], qv = sm.q[r * LD + c], kv = sm.k[r * LD + c];
+                    const float gr = sm.g[r * LD + c], grl = sm.glo[r * LD + c];
+                    const float qv = sm.q[r * LD + c], kv = sm.k[r * LD + c];
 #pragma unroll
                     for (int a = 0; a < 4; ++a) {
                         const int i = tt + 16 * a;
                         if (i <= r) {
-                            const float f = sm.k[i * LD + c] * expf(gr - sm.g[i * LD + c]);
+                            const float d = (gr - sm.g[i * LD + c]) + (grl - sm.glo[i * LD + c]);
+                            const float f = sm.k[i * LD + c] * expf(d);
                             accq[b][a] += qv * f;
                             acck[b][a] += kv * f;
                         }
@@ -147,11 +158,11 @@ prefill_simt_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k,
         // ---- rescale in place: q <- exp(g) q; k <- exp(g) k; g <- exp(g_L - g) k
         for (int e = tid; e < CH * D; e += NT) {
             const int r = e / D, c = e % D;
-            const float g = sm.g[r * LD + c], kv = sm.k[r * LD + c];
-            const float eg = expf(g);
+            const float g = sm.g[r * LD + c], glo = sm.glo[r * LD + c], kv = sm.k[r * LD + c];
+            const float eg = expf(g + glo);
             sm.q[r * LD + c] *= eg;
             sm.k[r * LD + c] = kv * eg;
-            sm.g[r * LD + c] = kv * expf(sm.gl[c] - g);
+            sm.g[r * LD + c] = kv * expf((sm.gl[c] - g) + (sm.gllo[c] - glo));
         }
         __syncthreads();
 
@@ -230,7 +241,7 @@ prefill_simt_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k,
 #pragma unroll 4
         for (int m = 0; m < D / 8; ++m) {
             const int c = rb + 8 * m;
-            float acc = expf(sm.gl[c]) * sm.s[c * DVS + j];
+            float acc = expf(sm.gl[c] + sm.gllo[c]) * sm.s[c * DVS + j];
             for (int i = 0; i < L; ++i) acc += sm.g[i * LD + c] * sm.vn[i * DVS + j];
             sm.s[c * DVS + j] = acc;
         }

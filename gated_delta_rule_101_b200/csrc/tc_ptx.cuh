@@ -1,0 +1,221 @@
+// Thin inline-PTX wrappers for the sm_100a features the tensor-core path uses:
+// mbarriers, TMA (tiled tensor and 1-D bulk copies), and tcgen05 (TMEM
+// allocation, MMA issue/commit, TMEM loads). Written from the PTX ISA.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+namespace kda {
+namespace ptx {
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// ------------------------------------------------------------------ mbarrier
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count)
+                 : "memory");
+}
+__device__ __forceinline__ void fence_mbar_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+                 "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+__device__ __forceinline__ uint64_t global_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+constexpr uint64_t WAIT_LIMIT_NS = 1000000000ull;  // give up a wait after one second
+
+// Waits for `parity` on `bar`. Gives up after WAIT_LIMIT_NS, or as soon as any
+// CTA has recorded a timeout in *status (so one failure does not make every
+// other CTA wait its full limit in turn). On giving up it sets *status to 1
+// and `dead`; once `dead` is set every later wait returns at once, so the
+// kernel unwinds instead of hanging.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, bool &dead, int *status) {
+    if (dead) return false;
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_ns();
+    for (uint32_t i = 1;; ++i) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((i & 255u) == 0) {
+            if (*reinterpret_cast<volatile int *>(status) != 0 || global_ns() - t0 > WAIT_LIMIT_NS)
+                break;
+        }
+    }
+    dead = true;
+    atomicExch(status, 1);
+    return false;
+}
+
+// ------------------------------------------------------------------ async proxy / TMA
+__device__ __forceinline__ void fence_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// 1-D bulk copy global -> shared, completing `bytes` on `bar`. Addresses and
+// size must be multiples of 16 bytes.
+__device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+            "r"(smem_u32(dst)),
+        "l"(src), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
+}
+// 1-D bulk copy shared -> global (bulk-group completion).
+__device__ __forceinline__ void bulk_s2g(void *dst, const void *src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst),
+                 "r"(smem_u32(src)), "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
+// 2-D tiled tensor load (no multicast). x is the innermost coordinate.
+__device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, int x, int y,
+                                            uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
+        : "memory");
+}
+
+// ------------------------------------------------------------------ tcgen05
+// TMEM allocation (whole warp). ncols: power of two >= 32.
+__device__ __forceinline__ void tmem_alloc(uint32_t *dst_smem, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(dst_smem)),
+                 "r"(ncols)
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+                 : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// D[tmem] (+)= A[smem] * B[smem], kind::f16 (bf16 inputs, fp32 accumulate).
+__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                         uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n\t}" ::"r"(
+            d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(0), "r"(0), "r"(0), "r"(0)
+        : "memory");
+}
+// Arrive once on `bar` when every MMA issued so far by this thread has completed.
+__device__ __forceinline__ void mma_commit(uint64_t *bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                     smem_u32(bar))
+                 : "memory");
+}
+
+// Loads 32 consecutive 32-bit TMEM columns of this thread's lane
+// (lane = 32 * (warp % 4) + lane id) starting at taddr, and waits for them:
+// the wait sits in the same asm statement so no use of the registers can be
+// scheduled before the data has arrived.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float *v) {
+    uint32_t r[32];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+        "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+          "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+          "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+          "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr)
+        : "memory");
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// ------------------------------------------------------------------ operand layouts
+// K-major bf16 operand tiles with the 128-byte swizzle: `rows` rows (a
+// multiple of 8), K a multiple of 64. Each group of 64 K-elements is an
+// "atom column" of rows x 128 bytes; inside it row r sits at r * 128 and its
+// 16-byte chunk q is stored at chunk position q ^ (r % 8). Tiles start on a
+// 1024-byte boundary so the swizzle phase matches the hardware's.
+__device__ __forceinline__ uint32_t sw128_chunk_off(uint32_t row, uint32_t chunk, uint32_t rows) {
+    // chunk: 16-byte chunk index along K (0 .. K/8 - 1)
+    const uint32_t kb = chunk >> 3, q = chunk & 7;
+    return kb * rows * 128u + row * 128u + ((q ^ (row & 7u)) << 4);
+}
+__device__ __forceinline__ uint32_t sw128_elem_off(uint32_t row, uint32_t k, uint32_t rows) {
+    return sw128_chunk_off(row, k >> 3, rows) + ((k & 7u) << 1);
+}
+
+// Shared-memory matrix descriptor for a K-major SWIZZLE_128B tile whose
+// 8-row groups are 1024 bytes apart.
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t smem_addr) {
+    uint64_t d = 0;
+    d |= (uint64_t)((smem_addr & 0x3FFFFu) >> 4);  // start address, 16-byte units
+    d |= (uint64_t)1u << 16;                       // leading byte offset (unused when swizzled)
+    d |= (uint64_t)(1024u >> 4) << 32;             // stride byte offset: 8-row group pitch
+    d |= (uint64_t)1u << 46;                       // descriptor version for sm_100
+    d |= (uint64_t)2u << 61;                       // layout: 128-byte swizzle
+    return d;
+}
+
+// Instruction descriptor: bf16 A and B, fp32 accumulator, both K-major, M x N.
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N) {
+    return (1u << 4)    // D format: f32
+           | (1u << 7)  // A format: bf16
+           | (1u << 10) // B format: bf16
+           | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+// Issues the K/16 MMAs of D (+)= A * B^T where A is an `a_rows` x K tile and
+// B an `b_rows` x K tile (both K-major, swizzled as above). M = a_rows.
+__device__ __forceinline__ void mma_tiles(uint32_t d_tmem, uint32_t a_base, uint32_t a_rows,
+                                          uint32_t b_base, uint32_t b_rows, int K, uint32_t idesc,
+                                          bool accumulate) {
+#pragma unroll 1
+    for (int kk = 0; kk < K / 16; ++kk) {
+        const uint32_t kb = (uint32_t)kk >> 2, in = ((uint32_t)kk & 3u) * 32u;
+        const uint64_t ad = sw128_desc(a_base + kb * a_rows * 128u + in);
+        const uint64_t bd = sw128_desc(b_base + kb * b_rows * 128u + in);
+        mma_bf16(d_tmem, ad, bd, idesc, (accumulate || kk > 0) ? 1u : 0u);
+    }
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    __nv_bfloat162 p = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&p);
+}
+
+}  // namespace ptx
+}  // namespace kda

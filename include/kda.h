@@ -131,6 +131,15 @@ KDA_API int kda_chunk_fwd(const void *q, const void *k, const void *v, const flo
 KDA_API int kda_decode_step(const void *q, const void *k, const void *v, const float *log_alpha,
                     const float *beta, float *S, void *o, int N, int H, int dtype, void *stream);
 
+/*
+ * Reads and clears the library's device status word. *status is 0 when no
+ * kernel has given up on a bounded wait since the last read, 1 otherwise
+ * (the affected call's outputs are then invalid; KDA_ERR_TIMEOUT describes
+ * it). Synchronises with the device (a blocking symbol copy on the legacy
+ * stream); do not call it inside stream capture.
+ */
+KDA_API int kda_get_device_status(int *status);
+
 #ifdef __cplusplus
 }
 #endif

@@ -60,19 +60,34 @@ def test_varlen_with_empty_and_ragged_sequences(dtype):
             assert torch.equal(st[i], inp.S0[i])
 
 
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
 @pytest.mark.parametrize("la_range", [(0.5, 3.0), (5.0, 20.0)])
-def test_strong_decay_uses_exact_pairwise_path(la_range):
+def test_strong_decay_uses_exact_pairwise_path(la_range, dtype):
     """Chunk log-decay far beyond 80: the factorised exp split would overflow."""
-    inp = prefill_inputs(B=1, T=200, H=2, dtype=torch.float32, la_range=la_range, s0_std=0.1,
+    inp = prefill_inputs(B=1, T=200, H=2, dtype=dtype, la_range=la_range, s0_std=0.1,
                          seed=11, device=DEV)
     o, st = run(inp)
     ro, rs = ref(inp)
-    check(o, ro, "f32", "strong decay o")
-    check(st, rs, "f32", "strong decay S_T")
+    check(o, ro, KIND[dtype], "strong decay o")
+    check(st, rs, KIND[dtype], "strong decay S_T")
 
 
-def test_alpha_zero_and_alpha_one_tokens():
-    inp = prefill_inputs(B=1, T=160, H=2, dtype=torch.float32, s0_std=0.1, seed=12, device=DEV)
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_some_channels_strongly_decayed(dtype):
+    """Only a few key channels exceed the factorised range; the rest use the MMA."""
+    inp = prefill_inputs(B=2, T=190, H=2, dtype=dtype, s0_std=0.1, seed=21, device=DEV)
+    inp.log_alpha[..., 5] = -3.0
+    inp.log_alpha[..., 77] = -40.0
+    inp.log_alpha[0, 70:80, 1, 100] = -1e4
+    o, st = run(inp)
+    ro, rs = ref(inp)
+    check(o, ro, KIND[dtype], "mixed decay o")
+    check(st, rs, KIND[dtype], "mixed decay S_T")
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_alpha_zero_and_alpha_one_tokens(dtype):
+    inp = prefill_inputs(B=1, T=160, H=2, dtype=dtype, s0_std=0.1, seed=12, device=DEV)
     inp.log_alpha[:, 10:12] = -1e4   # alpha = 0: state reset inside a chunk
     inp.log_alpha[:, 64] = -1e4      # at a chunk start
     inp.log_alpha[:, 100:140] = 0.0  # alpha = 1 (DeltaNet)
@@ -80,8 +95,8 @@ def test_alpha_zero_and_alpha_one_tokens():
     inp.beta[:, 30:40] = 1.0
     o, st = run(inp)
     ro, rs = ref(inp)
-    check(o, ro, "f32", "alpha 0/1 o")
-    check(st, rs, "f32", "alpha 0/1 S_T")
+    check(o, ro, KIND[dtype], "alpha 0/1 o")
+    check(st, rs, KIND[dtype], "alpha 0/1 S_T")
 
 
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
@@ -199,3 +214,12 @@ def test_long_context_1m_tokens_as_16_calls_sampled():
             check(o[0, :, h][:, cols], ro[0, :, 0], "bf16", f"1M-token call {c} o")
     check(S[0, h][:, cols], S_ref[0, 0], "bf16", "1M-token final S_T")
     assert torch.isfinite(S).all()
+
+
+def test_no_bounded_wait_timed_out():
+    """Every tensor-core kernel run so far finished without a wait giving up."""
+    import ctypes
+
+    st = ctypes.c_int(-1)
+    assert kda.lib().kda_get_device_status(ctypes.byref(st)) == 0
+    assert st.value == 0
