@@ -265,13 +265,15 @@ def run_kda(args, rank, world, local_rank):
             o_h.copy_(o, non_blocking=True)
             s_h.copy_(S_T, non_blocking=True)
 
-    e2e_steps = max(3, min(args.steps, 10))
-    barrier(world)
-    e_times = time_steps(e2e_step, e2e_steps, max(3, args.warmup // 2), stream)
-    barrier(world)
-    e_ms = max_over_ranks(sum(e_times), world, dev) / e2e_steps
-    e2e = {"value": tokens_per_step / (e_ms * 1e-3), "unit": "tokens/s",
-           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e_ms}
+    e2e = None
+    if not args.no_e2e:
+        e2e_steps = max(3, min(args.steps, 10))
+        barrier(world)
+        e_times = time_steps(e2e_step, e2e_steps, max(3, args.warmup // 2), stream)
+        barrier(world)
+        e_ms = max_over_ranks(sum(e_times), world, dev) / e2e_steps
+        e2e = {"value": tokens_per_step / (e_ms * 1e-3), "unit": "tokens/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e_ms}
     del host, dbuf
 
     # ---------------- decode (N=256, H=32, 1024 steps in one CUDA graph)
@@ -339,6 +341,8 @@ def main():
     ap.add_argument("--decode-steps", type=int, default=DECODE["steps"])
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true",
+                    help="skip the host-buffer end-to-end leg (for short profiling runs)")
     ap.add_argument("--traffic", type=float, default=None,
                     help="ncu dram bytes per prefill launch, if captured for this build")
     ap.add_argument("--decode-traffic", type=float, default=None,
