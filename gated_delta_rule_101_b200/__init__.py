@@ -27,7 +27,8 @@ HEADER = os.path.join(os.path.dirname(_PKG), "include", "kda.h")
 KDA_BF16, KDA_F32 = 0, 1
 KDA_OK = 0
 STATUS = {0: "KDA_OK", -1: "KDA_ERR_INVALID_ARG", -2: "KDA_ERR_UNSUPPORTED",
-          -3: "KDA_ERR_WORKSPACE", -4: "KDA_ERR_CUDA", -5: "KDA_ERR_TIMEOUT"}
+          -3: "KDA_ERR_WORKSPACE", -4: "KDA_ERR_CUDA", -5: "KDA_ERR_TIMEOUT",
+          -6: "KDA_ERR_SCRATCH_LIMIT"}
 HEAD_DIM = 128
 CHUNK = 64
 
@@ -52,6 +53,11 @@ def _bind(lib: ctypes.CDLL) -> ctypes.CDLL:
     lib.kda_chunk_fwd.restype = i32
     lib.kda_chunk_fwd.argtypes = [vp, vp, vp, fp, fp, fp, vp, fp, i32, i64, i32, i32, vp, i32,
                                   vp, i32, vp, ctypes.c_size_t, vp]
+    lib.kda_chunk_fwd_noalloc.restype = i32
+    lib.kda_chunk_fwd_noalloc.argtypes = [vp, vp, vp, fp, fp, fp, vp, fp, i32, i64, i32, i32, vp,
+                                          i32, vp, i32, vp]
+    lib.kda_noalloc_scratch_bytes.restype = ctypes.c_size_t
+    lib.kda_noalloc_scratch_bytes.argtypes = []
     lib.kda_get_device_status.restype = i32
     lib.kda_get_device_status.argtypes = [ctypes.POINTER(ctypes.c_int)]
     lib.kda_decode_step.restype = i32
@@ -203,3 +209,34 @@ def decode_step(q, k, v, log_alpha, beta, S, *, out=None, stream=None):
     if st != KDA_OK:
         raise KDAError(st, "kda_decode_step")
     return out
+
+
+def chunk_fwd_noalloc(q, k, v, log_alpha, beta, S0=None, *, out, state_out=None,
+                      cu_seqlens=None, cu_seqlens_host=None, stream=None, C=CHUNK):
+    """KDA prefill through ``kda_chunk_fwd_noalloc``: no workspace, no allocation.
+
+    For callers that cannot allocate device memory (a plugin whose host framework
+    owns all GPU memory, or a loop that must not call cudaMalloc). The caller
+    passes the output tensors; the library uses its fixed scratch buffer (see
+    include/kda.h for its size limit and the rule that calls sharing it must not
+    overlap on the GPU). Returns ``(out, state_out)``.
+    """
+    dev = q.device
+    code = _dtype_code(q)
+    packed = cu_seqlens is not None
+    if packed:
+        T, H, _ = q.shape
+        B, n_seqs = 1, cu_seqlens.numel() - 1
+    else:
+        B, T, H, _ = q.shape
+        n_seqs = 0
+    host_cu = None
+    if cu_seqlens_host is not None:
+        host_cu = torch.as_tensor(cu_seqlens_host, dtype=torch.int32).contiguous().cpu()
+    st = lib().kda_chunk_fwd_noalloc(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(S0), _ptr(out),
+        _ptr(state_out), B, T, H, C, _ptr(cu_seqlens), n_seqs, _ptr(host_cu), code,
+        _stream_handle(stream, dev))
+    if st != KDA_OK:
+        raise KDAError(st, "kda_chunk_fwd_noalloc")
+    return out, state_out

@@ -36,6 +36,9 @@ const char *kda_strerror(int status) {
     case KDA_ERR_WORKSPACE: return "KDA_ERR_WORKSPACE: workspace missing or too small";
     case KDA_ERR_CUDA: return "KDA_ERR_CUDA: kernel launch failed";
     case KDA_ERR_TIMEOUT: return "KDA_ERR_TIMEOUT: bounded device wait expired";
+    case KDA_ERR_SCRATCH_LIMIT:
+        return "KDA_ERR_SCRATCH_LIMIT: problem needs more than the fixed scratch of "
+               "kda_chunk_fwd_noalloc";
     default: return "unknown kda status";
     }
 }

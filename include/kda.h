@@ -63,7 +63,8 @@ typedef enum kda_status {
     KDA_ERR_UNSUPPORTED = -2, /* C != 64 or unknown dtype */
     KDA_ERR_WORKSPACE = -3,   /* workspace missing or smaller than required */
     KDA_ERR_CUDA = -4,        /* a kernel launch failed */
-    KDA_ERR_TIMEOUT = -5      /* a bounded device-side wait expired */
+    KDA_ERR_TIMEOUT = -5,     /* a bounded device-side wait expired */
+    KDA_ERR_SCRATCH_LIMIT = -6 /* kda_chunk_fwd_noalloc: problem needs more than its fixed scratch */
 } kda_status;
 
 /* Human-readable name of a status code (static string, never NULL). */
@@ -130,6 +131,40 @@ KDA_API int kda_chunk_fwd(const void *q, const void *k, const void *v, const flo
  */
 KDA_API int kda_decode_step(const void *q, const void *k, const void *v, const float *log_alpha,
                     const float *beta, float *S, void *o, int N, int H, int dtype, void *stream);
+
+/*
+ * kda_chunk_fwd for callers that cannot allocate device memory. The pages
+ * describe no counterpart: this is a library-integration entry point, not
+ * part of the method.
+ *
+ * Who needs it: code that may not call cudaMalloc, for example a plugin inside
+ * a host framework that owns all device memory through its own pool and gives
+ * plugins no allocation hook, or a latency-critical loop where cudaMalloc's
+ * possible device-wide synchronisation is not acceptable. Such a caller still
+ * passes its inputs and outputs, exactly as for kda_chunk_fwd (same argument
+ * meaning, layouts and ownership), but no workspace.
+ *
+ * Instead of a workspace the call uses one fixed scratch buffer of
+ * kda_noalloc_scratch_bytes() bytes (64 MiB) that lives in the library's
+ * device image: every GPU that loads the library holds it until the process
+ * exits. A problem whose kda_chunk_fwd_workspace_size exceeds it is rejected
+ * with KDA_ERR_SCRATCH_LIMIT before anything is launched (roughly 900
+ * chunk-head pairs for bf16, i.e. B * ceil(T/64) * H <= 903 for unpacked
+ * input; fp32 input needs no scratch). All calls on a GPU share the buffer and
+ * it keeps the previous call's contents; nothing in it has to start at zero.
+ * Calls that may overlap on the GPU (different streams, no ordering between
+ * them) race on the buffer: issue them on one stream. The first call on each
+ * GPU looks up the buffer's device address with that GPU current; make it
+ * before any stream capture begins. The function itself allocates nothing.
+ */
+KDA_API int kda_chunk_fwd_noalloc(const void *q, const void *k, const void *v,
+                                  const float *log_alpha, const float *beta, const float *S0,
+                                  void *o, float *S_T, int B, int64_t T, int H, int C,
+                                  const int32_t *cu_seqlens, int n_seqs,
+                                  const int32_t *cu_seqlens_host, int dtype, void *stream);
+
+/* Size in bytes of the fixed scratch used by kda_chunk_fwd_noalloc. */
+KDA_API size_t kda_noalloc_scratch_bytes(void);
 
 /*
  * Reads and clears the library's device status word. *status is 0 when no
