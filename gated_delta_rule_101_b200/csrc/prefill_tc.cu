@@ -62,40 +62,57 @@ constexpr uint32_t BLOB_U = 57344;     // U:       64 x 128 bf16 (two 64-column 
 constexpr uint32_t BLOB_GAM = 73728;   // exp(g_L): 128 fp32
 constexpr uint32_t BLOB_BYTES = 74240;
 
-// ---- prep kernel shared memory (offsets from a 1024-byte aligned base)
-constexpr uint32_t P_A1 = 0;          // 32768: Gram A = [Q e^g; K e^g], later [Q~; W]
-constexpr uint32_t P_KINV = 32768;    // 16384: Gram B = K e^-g (64 x 128); later solve scratch
-constexpr uint32_t P_KTT = 49152;     // 16384: K~^T (128 x 64)
-constexpr uint32_t P_XWT = 65536;     // 16384: (beta e^g K)^T (128 x 64)
-constexpr uint32_t P_XUT = 81920;     // 16384: (beta V)^T (128 x 64)
-constexpr uint32_t P_RAW = 98304;     // 81920: raw TMA tiles, reused after the gates are built
-constexpr uint32_t R_Q = 0, R_K = 16384, R_V = 32768, R_G = 49152;  // q, k, v bf16; log_alpha fp32
-constexpr uint32_t P_AQK = P_RAW + 0;       // 8192: A_qk image (64 x 64)
-constexpr uint32_t P_TB = P_RAW + 8192;     // 8192: T image (64 x 64), B operand of the W/U MMAs
-constexpr uint32_t P_UIMG = P_RAW + 16384;  // 16384: U image
-constexpr uint32_t P_AKK = P_RAW + 32768;   // 64 x 65 fp32
-constexpr uint32_t P_TF = P_RAW + 49408;    // 64 x 65 fp32
-constexpr uint32_t P_GAM = 180224;          // 512
-constexpr uint32_t P_BETA = 180736;         // 256
-constexpr uint32_t P_BADL = 180992;         // 512: list of key channels needing the exact path
-constexpr uint32_t P_BAR = 181504;          // 2 mbarriers
-constexpr uint32_t P_TMEM = 181520;         // TMEM base address
-constexpr uint32_t PREP_SMEM = 181536 + 1024;
-constexpr uint32_t PREP_TMEM_COLS = 256;  // Gram 64 + W^T 64 + U^T 64
-constexpr int LDA = 65;
+// ---- prep kernel shared memory (offsets from a 1024-byte aligned base). Every
+// operand image is a 128-byte-swizzled tile of 128-byte rows (see tc_ptx.cuh).
+//   A1   K-major, rows r' = 0..127, K = key channel c (two 64-channel blocks of 16 KiB).
+//        TMA puts q in rows 0..63 and k in rows 64..127; they are scaled in place
+//        to Q e^g and K e^g. Rows 64..127 are later replaced by W.
+//   V    rows = token i, two 64-column blocks (TMA); later overwritten by U.
+//   LAG  log_alpha [64][128] fp32 (TMA, unswizzled), turned into g in place;
+//        after the gates are built it holds KT and KINV:
+//   KT   rows = token i, two 64-channel blocks: (exp(g_L - g) K)[i][c]. The chain's
+//        MN-major A operand K~^T.
+//   KINV rows = token i, two 64-channel blocks: (K e^-g)[i][c]; the Gram's K-major B.
+//   AKK  64 x 64 fp32 (XOR-swizzled columns): A_kk, then T in place; over KINV.
+constexpr int PREP_NT = 256;
+constexpr uint32_t P_A1 = 0;          // 32768
+constexpr uint32_t P_V = 32768;       // 16384 (V, then U)
+constexpr uint32_t P_LAG = 49152;     // 32768 (log_alpha -> g), then KT | KINV
+constexpr uint32_t P_KT = 49152;      // 16384
+constexpr uint32_t P_KINV = 65536;    // 16384 (dead after the Gram MMA)
+constexpr uint32_t P_AKK = 65536;     // 16384: A_kk / T (after the Gram MMA)
+constexpr uint32_t P_PBUF = 81920;    // 16 x 48 fp32 solve scratch
+constexpr uint32_t P_AQK = 86016;     // 8192: A_qk image, rows r, columns i
+constexpr uint32_t P_TB = 94208;      // 8192: T Diag(beta) image, rows r, columns i
+constexpr uint32_t P_BADB = 86016;    // 8 x 3 x 64 fp32 bad-channel batch (before A_qk / T exist)
+constexpr uint32_t P_GAM = 102400;    // 128 fp32: exp(g_L)
+constexpr uint32_t P_GL = 102912;     // 128 fp32: g_L
+constexpr uint32_t P_TOT = 103424;    // 128 fp32: first-half log-decay totals
+constexpr uint32_t P_BETA = 103936;   // 64 fp32
+constexpr uint32_t P_BADL = 104192;   // 128 int
+constexpr uint32_t P_BAR = 104704;    // 2 mbarriers
+constexpr uint32_t P_TMEM = 104720;
+constexpr uint32_t P_NBAD = 104724;   // number of listed bad channels
+constexpr uint32_t PREP_SMEM = 104736 + 1024;
+constexpr uint32_t PREP_TMEM_COLS = 256;  // Gram 64 (then W 128) | U 128
+constexpr uint32_t PREP_TMA_BYTES = 32768 + 16384 + 32768;  // q, k | v | log_alpha
+
+// A_kk / T element (r, i): rows of 64 floats, columns XOR-swizzled by the row so
+// that both row-wise and column-wise accesses of a warp hit distinct banks.
+__device__ __forceinline__ int akk_idx(int r, int i) { return r * 64 + (i ^ (r & 31)); }
 
 // ---- chain kernel shared memory
 template <int N>
 struct ChainLayout {
-    static constexpr uint32_t A1 = 0;                 // 32768
-    static constexpr uint32_t A2 = 32768;             // 16384: [A_qk; zeros]
-    static constexpr uint32_t KTT = 49152;            // 16384
+    static constexpr uint32_t A1 = 0;                 // 32768 (K-major [Q~; W])
+    static constexpr uint32_t A2 = 32768;             // 16384: [A_qk; zeros] (K-major)
+    static constexpr uint32_t KTT = 49152;            // 16384 (MN-major K~^T: rows i, channels)
     static constexpr uint32_t U = 65536;              // N == 128 ? 16384 : 8192
     static constexpr uint32_t U_BYTES = N == 128 ? 16384 : 8192;
     static constexpr uint32_t GAM = U + U_BYTES;      // 512
     static constexpr uint32_t STAGE = ((GAM + 512 + 1023) / 1024) * 1024;
-    static constexpr uint32_t SIMG = 2 * STAGE;       // N x 128 bf16
-    static constexpr uint32_t VIMG = SIMG + N * 256;  // N x 64 bf16
+    static constexpr uint32_t SIMG = 2 * STAGE;       // S bf16, MN-major: rows c (128), N columns
+    static constexpr uint32_t VIMG = SIMG + N * 256;  // V_new bf16, MN-major: rows r (64), N columns
     static constexpr uint32_t BAR = VIMG + N * 128;   // 3 mbarriers
     static constexpr uint32_t TMEM = BAR + 24;
     static constexpr uint32_t BYTES = TMEM + 8 + 1024;
@@ -106,10 +123,6 @@ struct ChainLayout {
 __device__ __forceinline__ unsigned char *aligned_smem(unsigned char *raw) {
     return reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(raw) + 1023) &
                                              ~uintptr_t(1023));
-}
-
-__device__ __forceinline__ void st_bf16(unsigned char *base, uint32_t off, float x) {
-    *reinterpret_cast<__nv_bfloat16 *>(base + off) = __float2bfloat16_rn(x);
 }
 
 // Resolves a chunk slot into (sequence, chunk index). Returns false for slots past the end.
@@ -162,12 +175,24 @@ chunk_offsets_kernel(const int32_t *__restrict__ cu, int n_seqs, int32_t *__rest
 // =====================================================================================
 // prep: per (chunk, head) gates, Grams, UT inverse, W, U -> workspace blob
 // =====================================================================================
-__global__ void __launch_bounds__(NT, 1)
+__device__ __forceinline__ void st_chunk(unsigned char *p, const float (&v)[8]) {
+    *reinterpret_cast<uint4 *>(p) = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]),
+                                               pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
+}
+__device__ __forceinline__ void ld_chunk(const unsigned char *p, float (&v)[8]) {
+    const uint4 u = *reinterpret_cast<const uint4 *>(p);
+    const __nv_bfloat16 *b = reinterpret_cast<const __nv_bfloat16 *>(&u);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) v[e] = __bfloat162float(b[e]);
+}
+
+__global__ void __launch_bounds__(PREP_NT, 2)
 kda_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_la,
-                const float *__restrict__ beta, unsigned char *__restrict__ ws_blobs,
-                const int32_t *__restrict__ chunk_off, const int32_t *__restrict__ cu, int64_t T,
-                int H, int n_seqs, int nck) {
+                const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
+                const float *__restrict__ log_alpha, const float *__restrict__ beta,
+                unsigned char *__restrict__ ws_blobs, const int32_t *__restrict__ chunk_off,
+                const int32_t *__restrict__ cu, int64_t T, int H, int n_seqs, int nck) {
     extern __shared__ unsigned char smem_raw[];
     unsigned char *sm = aligned_smem(smem_raw);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -183,7 +208,10 @@ kda_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     uint64_t *bar_mma = bar_tma + 1;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + P_TMEM);
     float *sgam = reinterpret_cast<float *>(sm + P_GAM);
+    float *sgl = reinterpret_cast<float *>(sm + P_GL);
+    float *stot = reinterpret_cast<float *>(sm + P_TOT);
     float *sbeta = reinterpret_cast<float *>(sm + P_BETA);
+    float *lag = reinterpret_cast<float *>(sm + P_LAG);
     int *badl = reinterpret_cast<int *>(sm + P_BADL);
     bool dead = false;
 
@@ -191,12 +219,15 @@ kda_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         mbar_init(bar_tma, 1);
         mbar_init(bar_mma, 1);
         fence_mbar_init();
-        mbar_arrive_expect_tx(bar_tma, 3 * 16384 + 32768);
+        mbar_arrive_expect_tx(bar_tma, PREP_TMA_BYTES);
         const int x = h * D, y = (int)tok0;
-        tma_load_2d(sm + P_RAW + R_Q, &tm_q, x, y, bar_tma);
-        tma_load_2d(sm + P_RAW + R_K, &tm_k, x, y, bar_tma);
-        tma_load_2d(sm + P_RAW + R_V, &tm_v, x, y, bar_tma);
-        tma_load_2d(sm + P_RAW + R_G, &tm_la, x, y, bar_tma);
+        tma_load_2d(sm + P_A1, &tm_q, x, y, bar_tma);                  // q, channels 0..63
+        tma_load_2d(sm + P_A1 + 16384, &tm_q, x + 64, y, bar_tma);     // q, channels 64..127
+        tma_load_2d(sm + P_A1 + 8192, &tm_k, x, y, bar_tma);           // k -> rows 64..127
+        tma_load_2d(sm + P_A1 + 16384 + 8192, &tm_k, x + 64, y, bar_tma);
+        tma_load_2d(sm + P_V, &tm_v, x, y, bar_tma);
+        tma_load_2d(sm + P_V + 8192, &tm_v, x + 64, y, bar_tma);
+        tma_load_2d(sm + P_LAG, &tm_la, x, y, bar_tma);
     }
     if (warp == 0) {
         tmem_alloc(tmem_slot, PREP_TMEM_COLS);
@@ -208,179 +239,224 @@ kda_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     const uint32_t sm_base = smem_u32(sm);
-
     mbar_wait(bar_tma, 0, dead, &g_kda_device_status);
 
-    // ---- gates: thread c owns key channel c (and value column c)
-    const int c = tid;
-    const __nv_bfloat16 *rq = reinterpret_cast<const __nv_bfloat16 *>(sm + P_RAW + R_Q);
-    const __nv_bfloat16 *rk = reinterpret_cast<const __nv_bfloat16 *>(sm + P_RAW + R_K);
-    const __nv_bfloat16 *rv = reinterpret_cast<const __nv_bfloat16 *>(sm + P_RAW + R_V);
-    float *rg = reinterpret_cast<float *>(sm + P_RAW + R_G);  // log_alpha, overwritten by g
-    float gl = 0.f;
-    for (int r = 0; r < CH; ++r) {
-        gl += r < L ? rg[r * D + c] : 0.f;
-        rg[r * D + c] = gl;
-    }
-    const bool bad = -gl > SAFE_SPAN;
-    sgam[c] = expf(gl);
-
-    // ---- operand images (rows >= L are zero)
-#pragma unroll 1
-    for (int qc = 0; qc < CH / 8; ++qc) {
-        uint32_t kt[4], xw[4], xu[4];
-#pragma unroll
-        for (int e = 0; e < 8; e += 2) {
-            float ktv[2], xwv[2], xuv[2];
-#pragma unroll
-            for (int u = 0; u < 2; ++u) {
-                const int r = qc * 8 + e + u;
-                const bool live = r < L;
-                const float g = rg[r * D + c];
-                const float qv = live ? __bfloat162float(rq[r * D + c]) : 0.f;
-                const float kv = live ? __bfloat162float(rk[r * D + c]) : 0.f;
-                const float vv = live ? __bfloat162float(rv[r * D + c]) : 0.f;
-                const float eg = expf(g);
-                const float ke = kv * eg;
-                st_bf16(sm, P_A1 + sw128_elem_off(r, c, 128), qv * eg);
-                st_bf16(sm, P_A1 + sw128_elem_off(64 + r, c, 128), ke);
-                st_bf16(sm, P_KINV + sw128_elem_off(r, c, 64), bad ? 0.f : kv * expf(-g));
-                ktv[u] = kv * expf(gl - g);
-                xwv[u] = sbeta[r] * ke;
-                xuv[u] = sbeta[r] * vv;
-            }
-            kt[e / 2] = pack_bf16x2(ktv[0], ktv[1]);
-            xw[e / 2] = pack_bf16x2(xwv[0], xwv[1]);
-            xu[e / 2] = pack_bf16x2(xuv[0], xuv[1]);
+    // ---- g = chunk-local cumulative sum of log_alpha (rows >= L count as 0), in place.
+    //      Thread t: channel c = t % 128, rows 32*(t/128) .. +31.
+    {
+        const int c = tid & (D - 1), half = tid >> 7, r0 = half * 32;
+        float acc = 0.f;
+#pragma unroll 8
+        for (int e = 0; e < 32; ++e) {
+            const int r = r0 + e;
+            acc += r < L ? lag[r * D + c] : 0.f;
+            lag[r * D + c] = acc;
         }
-        *reinterpret_cast<uint4 *>(sm + P_KTT + sw128_chunk_off(c, qc, 128)) = make_uint4(kt[0], kt[1], kt[2], kt[3]);
-        *reinterpret_cast<uint4 *>(sm + P_XWT + sw128_chunk_off(c, qc, 128)) = make_uint4(xw[0], xw[1], xw[2], xw[3]);
-        *reinterpret_cast<uint4 *>(sm + P_XUT + sw128_chunk_off(c, qc, 128)) = make_uint4(xu[0], xu[1], xu[2], xu[3]);
+        if (half == 0) stot[c] = acc;
+        __syncthreads();
+        if (half == 1) {
+            const float off = stot[c];
+#pragma unroll 8
+            for (int e = 0; e < 32; ++e) lag[(r0 + e) * D + c] += off;
+            sgl[c] = acc + off;
+            sgam[c] = expf(acc + off);
+        }
     }
-    fence_async_smem();
-    tc_fence_before();
-    const int n_bad = __syncthreads_count(bad);
+    __syncthreads();
 
-    // ---- Gram MMA: rows 0..63 = (Q e^g)(K e^-g)^T, rows 64..127 = (K e^g)(K e^-g)^T
+    // ---- gates and operand images. Thread t: row r = t / 4, channel chunks
+    //      cq = 4*(t%4) .. +3 (8 channels each). Read everything, sync, then write.
+    const int gr = tid >> 2, cq0 = (tid & 3) * 4;
+    const bool live = gr < L;
+    float qv[4][8], kv[4][8], gv[4][8];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+        const int cq = cq0 + u;
+        const uint32_t blk = (uint32_t)(cq >> 3) * 16384u;
+        ld_chunk(sm + P_A1 + blk + sw128_chunk_off(gr, cq & 7, 128), qv[u]);
+        ld_chunk(sm + P_A1 + blk + sw128_chunk_off(64 + gr, cq & 7, 128), kv[u]);
+        const float4 g0 = *reinterpret_cast<const float4 *>(lag + gr * D + cq * 8);
+        const float4 g1 = *reinterpret_cast<const float4 *>(lag + gr * D + cq * 8 + 4);
+        gv[u][0] = g0.x; gv[u][1] = g0.y; gv[u][2] = g0.z; gv[u][3] = g0.w;
+        gv[u][4] = g1.x; gv[u][5] = g1.y; gv[u][6] = g1.z; gv[u][7] = g1.w;
+    }
+    __syncthreads();  // log_alpha/g tile fully read: its space becomes KT | KINV
+    int n_bad = 0;
+    {
+        bool any_bad = false;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int cq = cq0 + u;
+            const uint32_t blk = (uint32_t)(cq >> 3) * 16384u;
+            float qe[8], ke[8], kin[8], kt[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const int c = cq * 8 + e;
+                const float g = gv[u][e], gl = sgl[c];
+                const float x = live ? qv[u][e] : 0.f, kk = live ? kv[u][e] : 0.f;
+                const float eg = __expf(g);
+                qe[e] = x * eg;
+                ke[e] = kk * eg;
+                const bool bad = -gl > SAFE_SPAN;
+                any_bad |= bad;
+                kin[e] = bad ? 0.f : kk * __expf(-g);
+                kt[e] = kk * __expf(gl - g);
+            }
+            st_chunk(sm + P_A1 + blk + sw128_chunk_off(gr, cq & 7, 128), qe);
+            st_chunk(sm + P_A1 + blk + sw128_chunk_off(64 + gr, cq & 7, 128), ke);
+            st_chunk(sm + P_KT + (cq >> 3) * 8192 + sw128_chunk_off(gr, cq & 7, 64), kt);
+            st_chunk(sm + P_KINV + (cq >> 3) * 8192 + sw128_chunk_off(gr, cq & 7, 64), kin);
+        }
+        fence_async_smem();
+        tc_fence_before();
+        n_bad = __syncthreads_or(any_bad) ? 1 : 0;
+    }
+
+    // ---- Gram MMA: D[m][i] = sum_c A1[m][c] KINV[i][c]; rows 0..63 Q-rows, 64..127 K-rows
     if (tid == 0) {
         tc_fence_after();
-        mma_tiles(tmem, sm_base + P_A1, 128, sm_base + P_KINV, 64, D, idesc_bf16(128, 64), false);
+        mma_run(tmem, kmajor(sm_base + P_A1, 128), kmajor(sm_base + P_KINV, 64), D,
+                idesc_bf16(128, 64), false);
         mma_commit(bar_mma);
     }
 
-    // ---- exact contribution of channels left out of the MMA (pairwise exponentials)
-    float acc_bad[CH];
+    // Readout mapping: warp w reads TMEM lanes 32*(w%4) .. +31 (Gram rows m),
+    // columns 32*(w/4) .. +31.
+    const int m = 32 * (warp & 3) + lane, cb = 32 * (warp >> 2);
+    const int r_own = m & 63;
+    const bool kk_row = m >= 64;
+    float acc_bad[32];
 #pragma unroll
-    for (int i = 0; i < CH; ++i) acc_bad[i] = 0.f;
-    const int r_own = tid & 63;
-    const bool kk_row = tid >= 64;
-    if (n_bad > 0) {
+    for (int e = 0; e < 32; ++e) acc_bad[e] = 0.f;
+    if (n_bad) {  // exact pairwise terms of the channels left out of the MMA
+        int *nbad = reinterpret_cast<int *>(sm + P_NBAD);
         if (tid == 0) {
-            int m = 0;
+            int cnt = 0;
             for (int cc = 0; cc < D; ++cc)
-                if (-reinterpret_cast<float *>(sm + P_RAW + R_G)[(CH - 1) * D + cc] > SAFE_SPAN)
-                    badl[m++] = cc;
+                if (-sgl[cc] > SAFE_SPAN) badl[cnt++] = cc;
+            *nbad = cnt;
         }
         __syncthreads();
-        if (r_own < L) {
-            for (int b = 0; b < n_bad; ++b) {
-                const int cc = badl[b];
-                const float xr = __bfloat162float((kk_row ? rk : rq)[r_own * D + cc]);
-                const float gr = rg[r_own * D + cc];
+        const int nb_total = *nbad;
+        float *bb = reinterpret_cast<float *>(sm + P_BADB);  // [8][3][64]: q, k, g per row
+        for (int b0 = 0; b0 < nb_total; b0 += 8) {
+            for (int e = tid; e < 8 * 64; e += PREP_NT) {  // gather the batch's columns
+                const int bi = e >> 6, r = e & 63;
+                float qx = 0.f, kx = 0.f, gx = 0.f;
+                if (b0 + bi < nb_total) {
+                    const int64_t ccol = (int64_t)h * D + badl[b0 + bi];
+                    float a = 0.f;
+                    for (int j = 0; j <= r; ++j)
+                        a += j < L ? log_alpha[(tok0 + j) * H * D + ccol] : 0.f;
+                    gx = a;
+                    if (r < L) {
+                        qx = __bfloat162float(q[(tok0 + r) * H * D + ccol]);
+                        kx = __bfloat162float(k[(tok0 + r) * H * D + ccol]);
+                    }
+                }
+                bb[(bi * 3 + 0) * 64 + r] = qx;
+                bb[(bi * 3 + 1) * 64 + r] = kx;
+                bb[(bi * 3 + 2) * 64 + r] = gx;
+            }
+            __syncthreads();
+            const int nb = min(8, nb_total - b0);
+            for (int bi = 0; bi < nb; ++bi) {
+                const float xr = bb[(bi * 3 + (kk_row ? 1 : 0)) * 64 + r_own];
+                const float grr = bb[(bi * 3 + 2) * 64 + r_own];
 #pragma unroll
-                for (int i = 0; i < CH; ++i) {
-                    const bool use = i <= r_own;  // (i < L follows from i <= r_own < L)
-                    const float f = use ? __bfloat162float(rk[i * D + cc]) *
-                                              expf(fminf(gr - rg[i * D + cc], 0.f))
-                                        : 0.f;
-                    acc_bad[i] += xr * f;
+                for (int e = 0; e < 32; ++e) {
+                    const int i = cb + e;
+                    const float f = i <= r_own ? bb[(bi * 3 + 1) * 64 + i] *
+                                                     expf(fminf(grr - bb[(bi * 3 + 2) * 64 + i], 0.f))
+                                               : 0.f;
+                    acc_bad[e] += xr * f;
                 }
             }
+            __syncthreads();
         }
     }
 
     mbar_wait(bar_mma, 0, dead, &g_kda_device_status);
     tc_fence_after();
-    __syncthreads();  // raw tiles are dead from here on: their space is reused below
-
     {
-        float G[CH];
-        tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + 0, G);
-        tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + 32, G + 32);
+        float G[32];
+        tmem_ld32(tmem + ((uint32_t)(32 * (warp & 3)) << 16) + cb, G);
         const int r = r_own;
-        if (!kk_row) {
-            // A_qk row r (inclusive lower), bf16 image for the chain kernel
+        if (!kk_row) {  // A_qk (inclusive lower) -> bf16 image, rows r, columns i
 #pragma unroll
-            for (int qq = 0; qq < 8; ++qq) {
-                uint32_t p[4];
+            for (int cq = 0; cq < 4; ++cq) {
+                float v[8];
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int i0 = qq * 8 + 2 * e, i1 = i0 + 1;
-                    const float a0 = (i0 <= r && r < L) ? G[i0] + acc_bad[i0] : 0.f;
-                    const float a1 = (i1 <= r && r < L) ? G[i1] + acc_bad[i1] : 0.f;
-                    p[e] = pack_bf16x2(a0, a1);
+                for (int e = 0; e < 8; ++e) {
+                    const int i = cb + cq * 8 + e;
+                    v[e] = (i <= r && r < L) ? G[cq * 8 + e] + acc_bad[cq * 8 + e] : 0.f;
                 }
-                *reinterpret_cast<uint4 *>(sm + P_AQK + sw128_chunk_off(r, qq, 64)) = make_uint4(p[0], p[1], p[2], p[3]);
+                st_chunk(sm + P_AQK + sw128_chunk_off(r, (cb >> 3) + cq, 64), v);
             }
-        } else {
+        } else {  // A_kk (strict lower, times beta_r) -> fp32 for the solve (over KINV)
             float *akk = reinterpret_cast<float *>(sm + P_AKK);
             const float b = sbeta[r];
 #pragma unroll
-            for (int i = 0; i < CH; ++i) akk[r * LDA + i] = (i < r) ? b * (G[i] + acc_bad[i]) : 0.f;
+            for (int e = 0; e < 32; ++e) {
+                const int i = cb + e;
+                akk[akk_idx(r, i)] = i < r ? b * (G[e] + acc_bad[e]) : 0.f;
+            }
         }
     }
     __syncthreads();
 
-    // ---- T = (I + A_kk)^-1 by blocked forward substitution (16 x 16 blocks), fp32
+    // ---- T = (I + A_kk)^-1 in place by blocked forward substitution (16 x 16 blocks)
     {
-        const float *akk = reinterpret_cast<const float *>(sm + P_AKK);
-        float *tf = reinterpret_cast<float *>(sm + P_TF);
-        float *pbuf = reinterpret_cast<float *>(sm + P_KINV);  // 16 x 48 scratch
-        if (lane < 16) {  // warp b inverts diagonal block b; lane l -> column l
-            const int o = warp * 16, l = lane;
+        float *at = reinterpret_cast<float *>(sm + P_AKK);  // A_kk, becoming T
+        float *pbuf = reinterpret_cast<float *>(sm + P_PBUF);
+        if (warp < 4) {  // warp b inverts diagonal block b; lane l -> column l
+            const int o = warp * 16, l = lane & 15;
             float t[16];
 #pragma unroll
             for (int r = 0; r < 16; ++r) {
                 float x = (r == l) ? 1.f : 0.f;
 #pragma unroll
-                for (int m = 0; m < r; ++m) x -= akk[(o + r) * LDA + o + m] * t[m];
+                for (int mm = 0; mm < r; ++mm) x -= at[akk_idx(o + r, o + mm)] * t[mm];
                 t[r] = x;
             }
+            __syncwarp();
+            if (lane < 16) {
 #pragma unroll
-            for (int r = 0; r < 16; ++r) tf[(o + r) * LDA + o + l] = t[r];
+                for (int r = 0; r < 16; ++r) at[akk_idx(o + r, o + l)] = t[r];
+            }
         }
         __syncthreads();
-        for (int bi = 1; bi < 4; ++bi) {  // block row bi: T_bj = -T_bb sum_{k=j}^{b-1} A_bk T_kj
+        for (int bi = 1; bi < 4; ++bi) {  // block row bi: T_bj = -T_bb sum_{kb=j}^{bi-1} A_b,kb T_kb,j
             const int nent = bi * 256;
-            for (int e = tid; e < nent; e += NT) {
-                const int bj = e >> 8, a = (e >> 4) & 15, col = bj * 16 + (e & 15);
+            for (int e = tid; e < nent; e += PREP_NT) {
+                const int bj = e >> 8, a = (e >> 4) & 15, cc = bj * 16 + (e & 15);
                 const int row = bi * 16 + a;
-                float s = 0.f;
-                for (int m = bj * 16; m < bi * 16; ++m) s += akk[row * LDA + m] * tf[m * LDA + col];
-                pbuf[a * 48 + col] = s;
+                float sacc = 0.f;
+                for (int mm = bj * 16; mm < bi * 16; ++mm) sacc += at[akk_idx(row, mm)] * at[akk_idx(mm, cc)];
+                pbuf[a * 48 + cc] = sacc;
             }
             __syncthreads();
-            for (int e = tid; e < nent; e += NT) {
-                const int bj = e >> 8, a = (e >> 4) & 15, col = bj * 16 + (e & 15);
-                float s = 0.f;
+            for (int e = tid; e < nent; e += PREP_NT) {
+                const int bj = e >> 8, a = (e >> 4) & 15, cc = bj * 16 + (e & 15);
+                float sacc = 0.f;
 #pragma unroll
-                for (int m = 0; m < 16; ++m) s += tf[(bi * 16 + a) * LDA + bi * 16 + m] * pbuf[m * 48 + col];
-                tf[(bi * 16 + a) * LDA + col] = -s;
+                for (int mm = 0; mm < 16; ++mm) sacc += at[akk_idx(bi * 16 + a, bi * 16 + mm)] * pbuf[mm * 48 + cc];
+                at[akk_idx(bi * 16 + a, cc)] = -sacc;
             }
             __syncthreads();
         }
-        // bf16 image of T (rows r, K = i), zero above the diagonal
+        // image of T Diag(beta): rows r, columns i, zero above the diagonal
         {
-            const int r = tid >> 1, half = tid & 1;
+            const int r = tid >> 2, qd = tid & 3;
 #pragma unroll
-            for (int cc = 0; cc < 4; ++cc) {
-                uint32_t p[4];
+            for (int cq = 0; cq < 2; ++cq) {
+                float v[8];
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int i0 = half * 32 + cc * 8 + 2 * e, i1 = i0 + 1;
-                    p[e] = pack_bf16x2(i0 <= r ? tf[r * LDA + i0] : 0.f, i1 <= r ? tf[r * LDA + i1] : 0.f);
+                for (int e = 0; e < 8; ++e) {
+                    const int i = qd * 16 + cq * 8 + e;
+                    v[e] = i <= r ? at[akk_idx(r, i)] * sbeta[i] : 0.f;
                 }
-                *reinterpret_cast<uint4 *>(sm + P_TB + sw128_chunk_off(r, half * 4 + cc, 64)) = make_uint4(p[0], p[1], p[2], p[3]);
+                st_chunk(sm + P_TB + sw128_chunk_off(r, qd * 2 + cq, 64), v);
             }
         }
     }
@@ -388,25 +464,49 @@ kda_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     tc_fence_before();
     __syncthreads();
 
-    // ---- W^T = (beta e^g K)^T T^T and U^T = (beta V)^T T^T
+    // ---- W = (T Diag(beta)) (K e^g) and U = (T Diag(beta)) V, both M = 64, N = 128.
+    //      K e^g sits in rows 64..127 of A1, read here as an MN-major B (K = token i).
     if (tid == 0) {
         tc_fence_after();
-        mma_tiles(tmem + 64, sm_base + P_XWT, 128, sm_base + P_TB, 64, CH, idesc_bf16(128, 64), false);
-        mma_tiles(tmem + 128, sm_base + P_XUT, 128, sm_base + P_TB, 64, CH, idesc_bf16(128, 64), false);
+        mma_run(tmem, kmajor(sm_base + P_TB, 64), mnmajor(sm_base + P_A1 + 8192, 16384), CH,
+                idesc_bf16(64, 128, 0, 1), false);
+        mma_run(tmem + 128, kmajor(sm_base + P_TB, 64), mnmajor(sm_base + P_V, 8192), CH,
+                idesc_bf16(64, 128, 0, 1), false);
         mma_commit(bar_mma);
     }
     mbar_wait(bar_mma, 1, dead, &g_kda_device_status);
     tc_fence_after();
     {
-        float w[CH];
-        tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + 64, w);
-        tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + 96, w + 32);
+        // M = 64 accumulators: row r sits in lane 16*(w%4) + (lane < 16) of quarter w%4.
+        // Warp half w/4 takes columns 64*(w/4) .. +63 of W and of U.
+        float a0[32], a1[32];
+        const uint32_t lanes = (uint32_t)(32 * (warp & 3)) << 16;
+        const uint32_t cofs = 64u * (uint32_t)(warp >> 2);
+        const int r = 16 * (warp & 3) + lane;
+        tmem_ld32(tmem + lanes + cofs, a0);
+        tmem_ld32(tmem + lanes + cofs + 32, a1);
+        if (lane < 16) {  // W row r -> A1 row 64 + r, channel block w/4
+            unsigned char *wb = sm + P_A1 + (warp >> 2) * 16384;
 #pragma unroll
-        for (int r = 0; r < CH; ++r) st_bf16(sm, P_A1 + sw128_elem_off(64 + r, c, 128), w[r]);
-        tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + 128, w);
-        tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + 160, w + 32);
+            for (int cq = 0; cq < 8; ++cq) {
+                float v[8];
 #pragma unroll
-        for (int r = 0; r < CH; ++r) st_bf16(sm, P_UIMG + sw128_elem_off(r, c, 64), w[r]);
+                for (int e = 0; e < 8; ++e) v[e] = cq < 4 ? a0[cq * 8 + e] : a1[(cq - 4) * 8 + e];
+                st_chunk(wb + sw128_chunk_off(64 + r, cq, 128), v);
+            }
+        }
+        tmem_ld32(tmem + lanes + 128 + cofs, a0);
+        tmem_ld32(tmem + lanes + 128 + cofs + 32, a1);
+        if (lane < 16) {  // U row r -> U image (over V), value-column block w/4
+            unsigned char *ub = sm + P_V + (warp >> 2) * 8192;
+#pragma unroll
+            for (int cq = 0; cq < 8; ++cq) {
+                float v[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) v[e] = cq < 4 ? a0[cq * 8 + e] : a1[(cq - 4) * 8 + e];
+                st_chunk(ub + sw128_chunk_off(r, cq, 64), v);
+            }
+        }
     }
     fence_async_smem();
     tc_fence_before();
@@ -416,8 +516,8 @@ kda_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         unsigned char *blob = ws_blobs + ((size_t)slot * H + h) * BLOB_BYTES;
         bulk_s2g(blob + BLOB_A1, sm + P_A1, 32768);
         bulk_s2g(blob + BLOB_AQK, sm + P_AQK, 8192);
-        bulk_s2g(blob + BLOB_KTT, sm + P_KTT, 16384);
-        bulk_s2g(blob + BLOB_U, sm + P_UIMG, 16384);
+        bulk_s2g(blob + BLOB_KTT, sm + P_KT, 16384);
+        bulk_s2g(blob + BLOB_U, sm + P_V, 16384);
         bulk_s2g(blob + BLOB_GAM, sm + P_GAM, 512);
         bulk_commit();
         bulk_wait_all();
@@ -487,7 +587,12 @@ kda_chain_kernel(const unsigned char *__restrict__ ws_blobs, const int32_t *__re
         s_reg[j] = v4.x; s_reg[j + 1] = v4.y; s_reg[j + 2] = v4.z; s_reg[j + 3] = v4.w;
     }
 #pragma unroll
-    for (int j = 0; j < N; ++j) st_bf16(sm, Lay::SIMG + sw128_elem_off(j, c, N), s_reg[j]);
+    for (int jc = 0; jc < N / 8; ++jc) {  // row c of the MN-major S image
+        float v[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) v[e] = s_reg[jc * 8 + e];
+        st_chunk(sm + Lay::SIMG + sw128_chunk_off(c, jc, 128), v);
+    }
     fence_async_smem();
     tc_fence_before();
     __syncthreads();
@@ -515,7 +620,8 @@ kda_chain_kernel(const unsigned char *__restrict__ ws_blobs, const int32_t *__re
         // D1 = [Q~; W] S
         if (tid == 0) {
             tc_fence_after();
-            mma_tiles(d1, st_base + Lay::A1, 128, sm_base + Lay::SIMG, N, D, idesc_bf16(128, N), false);
+            mma_run(d1, kmajor(st_base + Lay::A1, 128), mnmajor(sm_base + Lay::SIMG, 16384), D,
+                    idesc_bf16(128, N, 0, 1), false);
             mma_commit(bar_mma);
         }
         mbar_wait(bar_mma, mma_phase, dead, &g_kda_device_status);
@@ -532,11 +638,10 @@ kda_chain_kernel(const unsigned char *__restrict__ ws_blobs, const int32_t *__re
                 const int jg = (N == 128 ? 0 : (j0 & 63)) + jc * 8;  // column inside the U image
                 const uint4 u4 = *reinterpret_cast<const uint4 *>(st + Lay::U + sw128_chunk_off(r, jg >> 3, 64));
                 const __nv_bfloat16 *ub = reinterpret_cast<const __nv_bfloat16 *>(&u4);
+                float v[8];
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const int j = jc * 8 + e;
-                    st_bf16(sm, Lay::VIMG + sw128_elem_off(j, r, N), __bfloat162float(ub[e]) - ws[j]);
-                }
+                for (int e = 0; e < 8; ++e) v[e] = __bfloat162float(ub[e]) - ws[jc * 8 + e];
+                st_chunk(sm + Lay::VIMG + sw128_chunk_off(r, jc, 64), v);  // row r, MN-major
             }
         }
         fence_async_smem();
@@ -545,8 +650,10 @@ kda_chain_kernel(const unsigned char *__restrict__ ws_blobs, const int32_t *__re
         // D1 += [A_qk; 0] V_new ; D3 = K~^T V_new
         if (tid == 0) {
             tc_fence_after();
-            mma_tiles(d1, st_base + Lay::A2, 128, sm_base + Lay::VIMG, N, CH, idesc_bf16(128, N), true);
-            mma_tiles(d3, st_base + Lay::KTT, 128, sm_base + Lay::VIMG, N, CH, idesc_bf16(128, N), false);
+            mma_run(d1, kmajor(st_base + Lay::A2, 128), mnmajor(sm_base + Lay::VIMG, 8192), CH,
+                    idesc_bf16(128, N, 0, 1), true);
+            mma_run(d3, mnmajor(st_base + Lay::KTT, 8192), mnmajor(sm_base + Lay::VIMG, 8192), CH,
+                    idesc_bf16(128, N, 1, 1), false);
             mma_commit(bar_mma);
         }
         mbar_wait(bar_mma, mma_phase, dead, &g_kda_device_status);
@@ -575,9 +682,14 @@ kda_chain_kernel(const unsigned char *__restrict__ ws_blobs, const int32_t *__re
                 tmem_ld32(d3 + lane_off + j, dv + j);
             const float gam = reinterpret_cast<const float *>(st + Lay::GAM)[c];
 #pragma unroll
-            for (int j = 0; j < N; ++j) {
-                s_reg[j] = gam * s_reg[j] + dv[j];
-                st_bf16(sm, Lay::SIMG + sw128_elem_off(j, c, N), s_reg[j]);
+            for (int jc = 0; jc < N / 8; ++jc) {
+                float v[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    s_reg[jc * 8 + e] = gam * s_reg[jc * 8 + e] + dv[jc * 8 + e];
+                    v[e] = s_reg[jc * 8 + e];
+                }
+                st_chunk(sm + Lay::SIMG + sw128_chunk_off(c, jc, 128), v);
             }
         }
         fence_async_smem();
@@ -613,17 +725,20 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     return fn;
 }
 
-// [n_tok, H*128] row-major tensor, box of 64 rows x 128 columns starting at (h*128, tok0).
-bool make_map(CUtensorMap *m, const void *ptr, CUtensorMapDataType dt, int esize, int64_t n_tok,
-              int H) {
+// [n_tok, H*128] row-major tensor; boxes of 64 rows x `box_cols` columns. bf16
+// boxes use the 128-byte swizzle (64 columns), so a box lands in shared memory
+// as one swizzled operand block; the fp32 log_alpha box (128 columns) is plain.
+bool make_map(CUtensorMap *m, const void *ptr, bool bf16, int64_t n_tok, int H) {
     auto fn = encode_fn();
     if (!fn) return false;
+    const int esize = bf16 ? 2 : 4;
     cuuint64_t dims[2] = {(cuuint64_t)H * D, (cuuint64_t)n_tok};
     cuuint64_t strides[1] = {(cuuint64_t)H * D * esize};
-    cuuint32_t box[2] = {D, CH};
+    cuuint32_t box[2] = {bf16 ? 64u : (cuuint32_t)D, (cuuint32_t)CH};
     cuuint32_t estr[2] = {1, 1};
-    return fn(m, dt, 2, const_cast<void *>(ptr), dims, strides, box, estr,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+    return fn(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2,
+              const_cast<void *>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+              bf16 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -662,16 +777,15 @@ cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, const
     cudaError_t err;
     if (n_tok > 0 && slots > 0) {
         CUtensorMap mq, mk, mv, mla;
-        if (!make_map(&mq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, n_tok, H) ||
-            !make_map(&mk, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, n_tok, H) ||
-            !make_map(&mv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, n_tok, H) ||
-            !make_map(&mla, log_alpha, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, n_tok, H))
+        if (!make_map(&mq, q, true, n_tok, H) || !make_map(&mk, k, true, n_tok, H) ||
+            !make_map(&mv, v, true, n_tok, H) || !make_map(&mla, log_alpha, false, n_tok, H))
             return cudaErrorInvalidValue;
         err = cudaFuncSetAttribute(kda_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                    (int)PREP_SMEM);
         if (err != cudaSuccess) return err;
-        kda_prep_kernel<<<dim3((unsigned)slots, (unsigned)H), NT, PREP_SMEM, stream>>>(
-            mq, mk, mv, mla, beta, blobs, chunk_off, cu_seqlens, T, H, n_seqs, nck);
+        kda_prep_kernel<<<dim3((unsigned)slots, (unsigned)H), PREP_NT, PREP_SMEM, stream>>>(
+            mq, mk, mv, mla, (const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k, log_alpha, beta,
+            blobs, chunk_off, cu_seqlens, T, H, n_seqs, nck);
         err = cudaGetLastError();
         if (err != cudaSuccess) return err;
     }

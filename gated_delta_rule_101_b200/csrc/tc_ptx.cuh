@@ -178,38 +178,55 @@ __device__ __forceinline__ uint32_t sw128_elem_off(uint32_t row, uint32_t k, uin
     return sw128_chunk_off(row, k >> 3, rows) + ((k & 7u) << 1);
 }
 
-// Shared-memory matrix descriptor for a K-major SWIZZLE_128B tile whose
-// 8-row groups are 1024 bytes apart.
-__device__ __forceinline__ uint64_t sw128_desc(uint32_t smem_addr) {
+// Shared-memory matrix descriptor for a SWIZZLE_128B operand tile. The tile is
+// made of 128-byte rows (64 bf16 elements each, 16-byte chunks XOR-swizzled
+// by row % 8), 8-row groups 1024 bytes apart (the stride byte offset).
+// K-major operands: rows are M (or N) rows, the 64 elements run along K.
+// MN-major operands: rows are K rows, the 64 elements run along M (or N);
+// further blocks of 64 M/N elements sit `lbo` bytes apart (leading byte offset).
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t smem_addr, uint32_t lbo = 16) {
     uint64_t d = 0;
-    d |= (uint64_t)((smem_addr & 0x3FFFFu) >> 4);  // start address, 16-byte units
-    d |= (uint64_t)1u << 16;                       // leading byte offset (unused when swizzled)
-    d |= (uint64_t)(1024u >> 4) << 32;             // stride byte offset: 8-row group pitch
-    d |= (uint64_t)1u << 46;                       // descriptor version for sm_100
-    d |= (uint64_t)2u << 61;                       // layout: 128-byte swizzle
+    d |= (uint64_t)((smem_addr & 0x3FFFFu) >> 4);   // start address, 16-byte units
+    d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;     // leading byte offset
+    d |= (uint64_t)(1024u >> 4) << 32;               // stride byte offset: 8-row group pitch
+    d |= (uint64_t)1u << 46;                         // descriptor version for sm_100
+    d |= (uint64_t)2u << 61;                         // layout: 128-byte swizzle
     return d;
 }
 
-// Instruction descriptor: bf16 A and B, fp32 accumulator, both K-major, M x N.
-__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N) {
+// Instruction descriptor: bf16 A and B, fp32 accumulator, M x N; a_mn / b_mn
+// select MN-major (1) or K-major (0) operands.
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int a_mn = 0, int b_mn = 0) {
     return (1u << 4)    // D format: f32
            | (1u << 7)  // A format: bf16
            | (1u << 10) // B format: bf16
-           | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+           | ((uint32_t)a_mn << 15) | ((uint32_t)b_mn << 16) | ((uint32_t)(N >> 3) << 17) |
+           ((uint32_t)(M >> 4) << 24);
 }
 
-// Issues the K/16 MMAs of D (+)= A * B^T where A is an `a_rows` x K tile and
-// B an `b_rows` x K tile (both K-major, swizzled as above). M = a_rows.
-__device__ __forceinline__ void mma_tiles(uint32_t d_tmem, uint32_t a_base, uint32_t a_rows,
-                                          uint32_t b_base, uint32_t b_rows, int K, uint32_t idesc,
-                                          bool accumulate) {
-#pragma unroll 1
-    for (int kk = 0; kk < K / 16; ++kk) {
+// One MMA operand in shared memory.
+//   K-major:  `rows` rows of the tile; 64-element K blocks are rows*128 bytes apart.
+//   MN-major: K runs down the rows; `lbo` = bytes between 64-element M/N blocks.
+struct Operand {
+    uint32_t base;
+    uint32_t rows_or_lbo;
+    bool mn;
+    __device__ __forceinline__ uint64_t desc(int kk) const {  // kk-th K step of 16 elements
+        if (mn) return sw128_desc(base + (uint32_t)kk * 2048u, rows_or_lbo);
         const uint32_t kb = (uint32_t)kk >> 2, in = ((uint32_t)kk & 3u) * 32u;
-        const uint64_t ad = sw128_desc(a_base + kb * a_rows * 128u + in);
-        const uint64_t bd = sw128_desc(b_base + kb * b_rows * 128u + in);
-        mma_bf16(d_tmem, ad, bd, idesc, (accumulate || kk > 0) ? 1u : 0u);
+        return sw128_desc(base + kb * rows_or_lbo * 128u + in);
     }
+};
+__device__ __forceinline__ Operand kmajor(uint32_t base, uint32_t rows) { return {base, rows, false}; }
+__device__ __forceinline__ Operand mnmajor(uint32_t base, uint32_t lbo) { return {base, lbo, true}; }
+
+// Issues the K/16 MMAs of D (+)= A * B (A: M x K, B: K x N as described by
+// the operands; the instruction descriptor must carry the same majorness).
+__device__ __forceinline__ void mma_run(uint32_t d_tmem, Operand a, Operand b, int K, uint32_t idesc,
+                                        bool accumulate) {
+#pragma unroll 1
+    for (int kk = 0; kk < K / 16; ++kk)
+        mma_bf16(d_tmem, a.desc(kk), b.desc(kk), idesc, (accumulate || kk > 0) ? 1u : 0u);
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
