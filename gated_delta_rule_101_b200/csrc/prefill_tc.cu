@@ -51,7 +51,6 @@ namespace {
 
 using namespace ptx;
 
-constexpr int NT = 128;            // threads per CTA in both kernels (4 warps)
 constexpr float SAFE_SPAN = 80.f;  // largest chunk log-decay the factorised Gram accepts
 
 // ---- one workspace blob per (chunk, head): operand images for the chain kernel
@@ -73,15 +72,15 @@ constexpr uint32_t BLOB_BYTES = 74240;
 //   KT   rows = token i, two 64-channel blocks: (exp(g_L - g) K)[i][c]. The chain's
 //        MN-major A operand K~^T.
 //   KINV rows = token i, two 64-channel blocks: (K e^-g)[i][c]; the Gram's K-major B.
-//   AKK  64 x 64 fp32 (XOR-swizzled columns): A_kk, then T in place; over KINV.
+//   AKK  64 x 68 fp32 (rows padded to 68 floats): A_kk, then T in place; over KINV.
 constexpr int PREP_NT = 256;
 constexpr uint32_t P_A1 = 0;          // 32768
 constexpr uint32_t P_V = 32768;       // 16384 (V, then U)
 constexpr uint32_t P_LAG = 49152;     // 32768 (log_alpha -> g), then KT | KINV
 constexpr uint32_t P_KT = 49152;      // 16384
 constexpr uint32_t P_KINV = 65536;    // 16384 (dead after the Gram MMA)
-constexpr uint32_t P_AKK = 65536;     // 16384: A_kk / T (after the Gram MMA)
-constexpr uint32_t P_PBUF = 81920;    // 16 x 48 fp32 solve scratch
+constexpr uint32_t P_AKK = 65536;     // 64 x 68 fp32: A_kk / T (after the Gram MMA)
+constexpr uint32_t P_PBUF = 82944;    // 16 x 48 fp32 solve scratch
 constexpr uint32_t P_AQK = 86016;     // 8192: A_qk image, rows r, columns i
 constexpr uint32_t P_TB = 94208;      // 8192: T Diag(beta) image, rows r, columns i
 constexpr uint32_t P_BADB = 86016;    // 8 x 3 x 64 fp32 bad-channel batch (before A_qk / T exist)
@@ -97,9 +96,9 @@ constexpr uint32_t PREP_SMEM = 104736 + 1024;
 constexpr uint32_t PREP_TMEM_COLS = 256;  // Gram 64 (then W 128) | U 128
 constexpr uint32_t PREP_TMA_BYTES = 32768 + 16384 + 32768;  // q, k | v | log_alpha
 
-// A_kk / T element (r, i): rows of 64 floats, columns XOR-swizzled by the row so
-// that both row-wise and column-wise accesses of a warp hit distinct banks.
-__device__ __forceinline__ int akk_idx(int r, int i) { return r * 64 + (i ^ (r & 31)); }
+// A_kk / T rows are padded to 68 floats: float4 row segments stay aligned, and
+// 8 consecutive rows at the same column fall on distinct bank quads.
+constexpr int LDT = 68;
 
 // ---- chain kernel shared memory
 template <int N>
@@ -113,8 +112,8 @@ struct ChainLayout {
     static constexpr uint32_t STAGE = ((GAM + 512 + 1023) / 1024) * 1024;
     static constexpr uint32_t SIMG = 2 * STAGE;       // S bf16, MN-major: rows c (128), N columns
     static constexpr uint32_t VIMG = SIMG + N * 256;  // V_new bf16, MN-major: rows r (64), N columns
-    static constexpr uint32_t BAR = VIMG + N * 128;   // 3 mbarriers
-    static constexpr uint32_t TMEM = BAR + 24;
+    static constexpr uint32_t BAR = VIMG + N * 128;   // 5 mbarriers
+    static constexpr uint32_t TMEM = BAR + 40;
     static constexpr uint32_t BYTES = TMEM + 8 + 1024;
     static constexpr uint32_t TMEM_COLS = 2 * N < 32 ? 32 : 2 * N;
     static constexpr uint32_t LOAD_BYTES = 32768 + 8192 + 16384 + U_BYTES + 512;
@@ -264,53 +263,67 @@ kda_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     }
     __syncthreads();
 
-    // ---- gates and operand images. Thread t: row r = t / 4, channel chunks
-    //      cq = 4*(t%4) .. +3 (8 channels each). Read everything, sync, then write.
-    const int gr = tid >> 2, cq0 = (tid & 3) * 4;
-    const bool live = gr < L;
-    float qv[4][8], kv[4][8], gv[4][8];
+    // ---- gates and operand images. Warp w handles rows r = w + 8v; lane f handles
+    //      channels 4f .. 4f+3 (8-byte pieces of the swizzled rows). Read all, sync, write.
+    const int f = lane, fblk = f >> 4, fchunk = (f & 15) >> 1, fhalf = (f & 1) * 8;
+    uint2 qraw[8], kraw[8];
+    float4 graw[8];
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-        const int cq = cq0 + u;
-        const uint32_t blk = (uint32_t)(cq >> 3) * 16384u;
-        ld_chunk(sm + P_A1 + blk + sw128_chunk_off(gr, cq & 7, 128), qv[u]);
-        ld_chunk(sm + P_A1 + blk + sw128_chunk_off(64 + gr, cq & 7, 128), kv[u]);
-        const float4 g0 = *reinterpret_cast<const float4 *>(lag + gr * D + cq * 8);
-        const float4 g1 = *reinterpret_cast<const float4 *>(lag + gr * D + cq * 8 + 4);
-        gv[u][0] = g0.x; gv[u][1] = g0.y; gv[u][2] = g0.z; gv[u][3] = g0.w;
-        gv[u][4] = g1.x; gv[u][5] = g1.y; gv[u][6] = g1.z; gv[u][7] = g1.w;
+    for (int v8 = 0; v8 < 8; ++v8) {
+        const int r = warp + 8 * v8;
+        const unsigned char *blk = sm + P_A1 + fblk * 16384;
+        qraw[v8] = *reinterpret_cast<const uint2 *>(blk + sw128_chunk_off(r, fchunk, 128) + fhalf);
+        kraw[v8] = *reinterpret_cast<const uint2 *>(blk + sw128_chunk_off(64 + r, fchunk, 128) + fhalf);
+        graw[v8] = *reinterpret_cast<const float4 *>(lag + r * D + 4 * f);
+    }
+    const float4 gl4 = *reinterpret_cast<const float4 *>(sgl + 4 * f);
+    const float gls[4] = {gl4.x, gl4.y, gl4.z, gl4.w};
+    const float4 ga4 = *reinterpret_cast<const float4 *>(sgam + 4 * f);
+    const float gams[4] = {ga4.x, ga4.y, ga4.z, ga4.w};
+    bool badc[4], any_bad = false;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        badc[e] = -gls[e] > SAFE_SPAN;
+        any_bad |= badc[e];
     }
     __syncthreads();  // log_alpha/g tile fully read: its space becomes KT | KINV
-    int n_bad = 0;
-    {
-        bool any_bad = false;
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const int cq = cq0 + u;
-            const uint32_t blk = (uint32_t)(cq >> 3) * 16384u;
-            float qe[8], ke[8], kin[8], kt[8];
+    for (int v8 = 0; v8 < 8; ++v8) {
+        const int r = warp + 8 * v8;
+        const bool live = r < L;
+        const __nv_bfloat16 *qb = reinterpret_cast<const __nv_bfloat16 *>(&qraw[v8]);
+        const __nv_bfloat16 *kb = reinterpret_cast<const __nv_bfloat16 *>(&kraw[v8]);
+        const float gs[4] = {graw[v8].x, graw[v8].y, graw[v8].z, graw[v8].w};
+        float qe[4], ke[4], kin[4], kt[4];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                const int c = cq * 8 + e;
-                const float g = gv[u][e], gl = sgl[c];
-                const float x = live ? qv[u][e] : 0.f, kk = live ? kv[u][e] : 0.f;
-                const float eg = __expf(g);
-                qe[e] = x * eg;
-                ke[e] = kk * eg;
-                const bool bad = -gl > SAFE_SPAN;
-                any_bad |= bad;
-                kin[e] = bad ? 0.f : kk * __expf(-g);
-                kt[e] = kk * __expf(gl - g);
+        for (int e = 0; e < 4; ++e) {
+            const float x = live ? __bfloat162float(qb[e]) : 0.f;
+            const float kk = live ? __bfloat162float(kb[e]) : 0.f;
+            const float eg = __expf(gs[e]);
+            qe[e] = x * eg;
+            ke[e] = kk * eg;
+            if (!badc[e]) {  // exp(-g) <= exp(80): finite, and exp(g_L - g) = exp(g_L) exp(-g)
+                const float kin_ = kk * __expf(-gs[e]);
+                kin[e] = kin_;
+                kt[e] = kin_ * gams[e];
+            } else {
+                kin[e] = 0.f;
+                kt[e] = kk * __expf(gls[e] - gs[e]);
             }
-            st_chunk(sm + P_A1 + blk + sw128_chunk_off(gr, cq & 7, 128), qe);
-            st_chunk(sm + P_A1 + blk + sw128_chunk_off(64 + gr, cq & 7, 128), ke);
-            st_chunk(sm + P_KT + (cq >> 3) * 8192 + sw128_chunk_off(gr, cq & 7, 64), kt);
-            st_chunk(sm + P_KINV + (cq >> 3) * 8192 + sw128_chunk_off(gr, cq & 7, 64), kin);
         }
-        fence_async_smem();
-        tc_fence_before();
-        n_bad = __syncthreads_or(any_bad) ? 1 : 0;
+        unsigned char *blk = sm + P_A1 + fblk * 16384;
+        *reinterpret_cast<uint2 *>(blk + sw128_chunk_off(r, fchunk, 128) + fhalf) =
+            make_uint2(pack_bf16x2(qe[0], qe[1]), pack_bf16x2(qe[2], qe[3]));
+        *reinterpret_cast<uint2 *>(blk + sw128_chunk_off(64 + r, fchunk, 128) + fhalf) =
+            make_uint2(pack_bf16x2(ke[0], ke[1]), pack_bf16x2(ke[2], ke[3]));
+        *reinterpret_cast<uint2 *>(sm + P_KT + fblk * 8192 + sw128_chunk_off(r, fchunk, 64) + fhalf) =
+            make_uint2(pack_bf16x2(kt[0], kt[1]), pack_bf16x2(kt[2], kt[3]));
+        *reinterpret_cast<uint2 *>(sm + P_KINV + fblk * 8192 + sw128_chunk_off(r, fchunk, 64) + fhalf) =
+            make_uint2(pack_bf16x2(kin[0], kin[1]), pack_bf16x2(kin[2], kin[3]));
     }
+    fence_async_smem();
+    tc_fence_before();
+    const int n_bad = __syncthreads_or(any_bad) ? 1 : 0;
 
     // ---- Gram MMA: D[m][i] = sum_c A1[m][c] KINV[i][c]; rows 0..63 Q-rows, 64..127 K-rows
     if (tid == 0) {
@@ -397,65 +410,129 @@ kda_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             float *akk = reinterpret_cast<float *>(sm + P_AKK);
             const float b = sbeta[r];
 #pragma unroll
-            for (int e = 0; e < 32; ++e) {
-                const int i = cb + e;
-                akk[akk_idx(r, i)] = i < r ? b * (G[e] + acc_bad[e]) : 0.f;
+            for (int e4 = 0; e4 < 32; e4 += 4) {
+                float v[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int i = cb + e4 + e;
+                    v[e] = i < r ? b * (G[e4 + e] + acc_bad[e4 + e]) : 0.f;
+                }
+                *reinterpret_cast<float4 *>(akk + r * LDT + cb + e4) = make_float4(v[0], v[1], v[2], v[3]);
             }
         }
     }
     __syncthreads();
 
-    // ---- T = (I + A_kk)^-1 in place by blocked forward substitution (16 x 16 blocks)
+    // ---- T = (I + A_kk)^-1 in place, by blocks: invert the four 16 x 16 diagonal
+    //      blocks, then merge 16 -> 32 -> 64 with [[X, 0], [Y, Z]]^-1 =
+    //      [[X^-1, 0], [-Z^-1 Y X^-1, Z^-1]] (each level two small products).
     {
-        float *at = reinterpret_cast<float *>(sm + P_AKK);  // A_kk, becoming T
-        float *pbuf = reinterpret_cast<float *>(sm + P_PBUF);
+        float *at = reinterpret_cast<float *>(sm + P_AKK);  // A_kk, becoming T (row stride LDT)
+        float *pb = reinterpret_cast<float *>(sm + P_PBUF);  // 2 x [16][20] level-1 products
+        float *qb = reinterpret_cast<float *>(sm + P_TB);    // [32][36] level-2 product (TB is free)
         if (warp < 4) {  // warp b inverts diagonal block b; lane l -> column l
             const int o = warp * 16, l = lane & 15;
             float t[16];
 #pragma unroll
             for (int r = 0; r < 16; ++r) {
+                float arow[16];
+#pragma unroll
+                for (int m4 = 0; m4 < 16; m4 += 4) {
+                    const float4 a4 = *reinterpret_cast<const float4 *>(at + (o + r) * LDT + o + m4);
+                    arow[m4] = a4.x; arow[m4 + 1] = a4.y; arow[m4 + 2] = a4.z; arow[m4 + 3] = a4.w;
+                }
                 float x = (r == l) ? 1.f : 0.f;
 #pragma unroll
-                for (int mm = 0; mm < r; ++mm) x -= at[akk_idx(o + r, o + mm)] * t[mm];
+                for (int mm = 0; mm < r; ++mm) x -= arow[mm] * t[mm];
                 t[r] = x;
             }
             __syncwarp();
             if (lane < 16) {
 #pragma unroll
-                for (int r = 0; r < 16; ++r) at[akk_idx(o + r, o + l)] = t[r];
+                for (int r = 0; r < 16; ++r) at[(o + r) * LDT + o + l] = t[r];
             }
         }
         __syncthreads();
-        for (int bi = 1; bi < 4; ++bi) {  // block row bi: T_bj = -T_bb sum_{kb=j}^{bi-1} A_b,kb T_kb,j
-            const int nent = bi * 256;
-            for (int e = tid; e < nent; e += PREP_NT) {
-                const int bj = e >> 8, a = (e >> 4) & 15, cc = bj * 16 + (e & 15);
-                const int row = bi * 16 + a;
-                float sacc = 0.f;
-                for (int mm = bj * 16; mm < bi * 16; ++mm) sacc += at[akk_idx(row, mm)] * at[akk_idx(mm, cc)];
-                pbuf[a * 48 + cc] = sacc;
-            }
-            __syncthreads();
-            for (int e = tid; e < nent; e += PREP_NT) {
-                const int bj = e >> 8, a = (e >> 4) & 15, cc = bj * 16 + (e & 15);
-                float sacc = 0.f;
+        // level 1: blocks (16..31, 0..15) and (48..63, 32..47); thread -> 1 x 4 tile
+        const int l1b = tid >> 6, l1a = (tid >> 2) & 15, l1c = (tid & 3) * 4, l1o = 32 * l1b;
+        if (tid < 128) {  // P = A_lo-hi-block X^-1
+            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-                for (int mm = 0; mm < 16; ++mm) sacc += at[akk_idx(bi * 16 + a, bi * 16 + mm)] * pbuf[mm * 48 + cc];
-                at[akk_idx(bi * 16 + a, cc)] = -sacc;
+            for (int m4 = 0; m4 < 16; m4 += 4) {
+                const float4 a4 = *reinterpret_cast<const float4 *>(at + (l1o + 16 + l1a) * LDT + l1o + m4);
+                const float av[4] = {a4.x, a4.y, a4.z, a4.w};
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const float4 b4 = *reinterpret_cast<const float4 *>(at + (l1o + m4 + u) * LDT + l1o + l1c);
+                    acc.x += av[u] * b4.x; acc.y += av[u] * b4.y; acc.z += av[u] * b4.z; acc.w += av[u] * b4.w;
+                }
             }
-            __syncthreads();
+            *reinterpret_cast<float4 *>(pb + (l1b * 16 + l1a) * 20 + l1c) = acc;
         }
+        __syncthreads();
+        if (tid < 128) {  // T = -Z^-1 P
+            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+            for (int m4 = 0; m4 < 16; m4 += 4) {
+                const float4 d4 = *reinterpret_cast<const float4 *>(at + (l1o + 16 + l1a) * LDT + l1o + 16 + m4);
+                const float dv[4] = {d4.x, d4.y, d4.z, d4.w};
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const float4 p4 = *reinterpret_cast<const float4 *>(pb + (l1b * 16 + m4 + u) * 20 + l1c);
+                    acc.x += dv[u] * p4.x; acc.y += dv[u] * p4.y; acc.z += dv[u] * p4.z; acc.w += dv[u] * p4.w;
+                }
+            }
+            *reinterpret_cast<float4 *>(at + (l1o + 16 + l1a) * LDT + l1o + l1c) =
+                make_float4(-acc.x, -acc.y, -acc.z, -acc.w);
+        }
+        __syncthreads();
+        // level 2: block (32..63, 0..31); thread -> 1 x 4 tile of the 32 x 32 block
+        const int l2a = tid >> 3, l2c = (tid & 7) * 4;
+        {  // Q = A[32.., 0..31] T[0..31, 0..31]
+            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+            for (int m4 = 0; m4 < 32; m4 += 4) {
+                const float4 a4 = *reinterpret_cast<const float4 *>(at + (32 + l2a) * LDT + m4);
+                const float av[4] = {a4.x, a4.y, a4.z, a4.w};
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const float4 b4 = *reinterpret_cast<const float4 *>(at + (m4 + u) * LDT + l2c);
+                    acc.x += av[u] * b4.x; acc.y += av[u] * b4.y; acc.z += av[u] * b4.z; acc.w += av[u] * b4.w;
+                }
+            }
+            *reinterpret_cast<float4 *>(qb + l2a * 36 + l2c) = acc;
+        }
+        __syncthreads();
+        {  // T[32.., 0..31] = -T[32.., 32..] Q
+            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+            for (int m4 = 0; m4 < 32; m4 += 4) {
+                const float4 d4 = *reinterpret_cast<const float4 *>(at + (32 + l2a) * LDT + 32 + m4);
+                const float dv[4] = {d4.x, d4.y, d4.z, d4.w};
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const float4 p4 = *reinterpret_cast<const float4 *>(qb + (m4 + u) * 36 + l2c);
+                    acc.x += dv[u] * p4.x; acc.y += dv[u] * p4.y; acc.z += dv[u] * p4.z; acc.w += dv[u] * p4.w;
+                }
+            }
+            *reinterpret_cast<float4 *>(at + (32 + l2a) * LDT + l2c) = make_float4(-acc.x, -acc.y, -acc.z, -acc.w);
+        }
+        __syncthreads();
         // image of T Diag(beta): rows r, columns i, zero above the diagonal
         {
             const int r = tid >> 2, qd = tid & 3;
 #pragma unroll
             for (int cq = 0; cq < 2; ++cq) {
+                const int i0 = qd * 16 + cq * 8;
+                const float4 t0 = *reinterpret_cast<const float4 *>(at + r * LDT + i0);
+                const float4 t1 = *reinterpret_cast<const float4 *>(at + r * LDT + i0 + 4);
+                const float4 b0 = *reinterpret_cast<const float4 *>(sbeta + i0);
+                const float4 b1 = *reinterpret_cast<const float4 *>(sbeta + i0 + 4);
+                const float tv[8] = {t0.x, t0.y, t0.z, t0.w, t1.x, t1.y, t1.z, t1.w};
+                const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
                 float v[8];
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const int i = qd * 16 + cq * 8 + e;
-                    v[e] = i <= r ? at[akk_idx(r, i)] * sbeta[i] : 0.f;
-                }
+                for (int e = 0; e < 8; ++e) v[e] = (i0 + e) <= r ? tv[e] * bv[e] : 0.f;
                 st_chunk(sm + P_TB + sw128_chunk_off(r, qd * 2 + cq, 64), v);
             }
         }
@@ -479,31 +556,29 @@ kda_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     {
         // M = 64 accumulators: row r sits in lane 16*(w%4) + (lane < 16) of quarter w%4.
         // Warp half w/4 takes columns 64*(w/4) .. +63 of W and of U.
-        float a0[32], a1[32];
+        float a[64];
         const uint32_t lanes = (uint32_t)(32 * (warp & 3)) << 16;
         const uint32_t cofs = 64u * (uint32_t)(warp >> 2);
         const int r = 16 * (warp & 3) + lane;
-        tmem_ld32(tmem + lanes + cofs, a0);
-        tmem_ld32(tmem + lanes + cofs + 32, a1);
+        tmem_ld64(tmem + lanes + cofs, a);
         if (lane < 16) {  // W row r -> A1 row 64 + r, channel block w/4
             unsigned char *wb = sm + P_A1 + (warp >> 2) * 16384;
 #pragma unroll
             for (int cq = 0; cq < 8; ++cq) {
                 float v[8];
 #pragma unroll
-                for (int e = 0; e < 8; ++e) v[e] = cq < 4 ? a0[cq * 8 + e] : a1[(cq - 4) * 8 + e];
+                for (int e = 0; e < 8; ++e) v[e] = a[cq * 8 + e];
                 st_chunk(wb + sw128_chunk_off(64 + r, cq, 128), v);
             }
         }
-        tmem_ld32(tmem + lanes + 128 + cofs, a0);
-        tmem_ld32(tmem + lanes + 128 + cofs + 32, a1);
+        tmem_ld64(tmem + lanes + 128 + cofs, a);
         if (lane < 16) {  // U row r -> U image (over V), value-column block w/4
             unsigned char *ub = sm + P_V + (warp >> 2) * 8192;
 #pragma unroll
             for (int cq = 0; cq < 8; ++cq) {
                 float v[8];
 #pragma unroll
-                for (int e = 0; e < 8; ++e) v[e] = cq < 4 ? a0[cq * 8 + e] : a1[(cq - 4) * 8 + e];
+                for (int e = 0; e < 8; ++e) v[e] = a[cq * 8 + e];
                 st_chunk(ub + sw128_chunk_off(r, cq, 64), v);
             }
         }
@@ -520,7 +595,7 @@ kda_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         bulk_s2g(blob + BLOB_U, sm + P_V, 16384);
         bulk_s2g(blob + BLOB_GAM, sm + P_GAM, 512);
         bulk_commit();
-        bulk_wait_all();
+        bulk_wait_read();  // shared memory may be released; the writes complete with the grid
     }
     __syncthreads();
     if (warp == 0) tmem_dealloc(tmem, PREP_TMEM_COLS);
@@ -529,16 +604,23 @@ kda_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 // =====================================================================================
 // chain: per (sequence, head, value slice) state recurrence over the chunks
 // =====================================================================================
+// 256 threads. Warp w reads TMEM lane quarter q = w % 4 and handles value columns
+// 32*(w/4) .. +31 of the slice, so every epilogue is split over two warps per quarter.
+// Thread (q, lane, w/4) keeps state row c = 32q + lane, those 32 columns, in registers.
+constexpr int CHAIN_NT = 256;
+
 template <int N>
-__global__ void __launch_bounds__(NT, 1)
+__global__ void __launch_bounds__(CHAIN_NT, 1)
 kda_chain_kernel(const unsigned char *__restrict__ ws_blobs, const int32_t *__restrict__ chunk_off,
                  const float *__restrict__ S0, __nv_bfloat16 *__restrict__ o,
                  float *__restrict__ S_T, const int32_t *__restrict__ cu, int64_t T, int H,
                  int nck) {
+    static_assert(N == 64, "the chain kernel is written for 64-column value slices");
     using Lay = ChainLayout<N>;
     extern __shared__ unsigned char smem_raw[];
     unsigned char *sm = aligned_smem(smem_raw);
-    const int tid = threadIdx.x, warp = tid >> 5;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int q4 = warp & 3, hf = warp >> 2;
     const int seq = blockIdx.x, h = blockIdx.y, j0 = blockIdx.z * N;
     const SeqSpan span = seq_span(cu, T, seq);
     const int nchunks = (int)((span.len + CH - 1) / CH);
@@ -546,7 +628,9 @@ kda_chain_kernel(const unsigned char *__restrict__ ws_blobs, const int32_t *__re
     const int64_t state_off = ((int64_t)seq * H + h) * (int64_t)(D * D);
 
     uint64_t *bar_ld = reinterpret_cast<uint64_t *>(sm + Lay::BAR);  // [2]
-    uint64_t *bar_mma = bar_ld + 2;
+    uint64_t *bar_a = bar_ld + 2;  // MMA1 done
+    uint64_t *bar_b = bar_ld + 3;  // state MMA done
+    uint64_t *bar_c = bar_ld + 4;  // output MMA done
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + Lay::TMEM);
     bool dead = false;
 
@@ -557,15 +641,12 @@ kda_chain_kernel(const unsigned char *__restrict__ ws_blobs, const int32_t *__re
         bulk_g2s(st + Lay::A1, blob + BLOB_A1, 32768, &bar_ld[stage]);
         bulk_g2s(st + Lay::A2, blob + BLOB_AQK, 8192, &bar_ld[stage]);
         bulk_g2s(st + Lay::KTT, blob + BLOB_KTT, 16384, &bar_ld[stage]);
-        bulk_g2s(st + Lay::U, blob + BLOB_U + (N == 128 ? 0 : (uint32_t)(j0 / 64) * 8192),
-                 Lay::U_BYTES, &bar_ld[stage]);
+        bulk_g2s(st + Lay::U, blob + BLOB_U + (uint32_t)(j0 / 64) * 8192, Lay::U_BYTES, &bar_ld[stage]);
         bulk_g2s(st + Lay::GAM, blob + BLOB_GAM, 512, &bar_ld[stage]);
     };
 
     if (tid == 0) {
-        mbar_init(&bar_ld[0], 1);
-        mbar_init(&bar_ld[1], 1);
-        mbar_init(bar_mma, 1);
+        for (int b = 0; b < 5; ++b) mbar_init(&bar_ld[b], 1);
         fence_mbar_init();
     }
     if (warp == 0) {
@@ -573,25 +654,25 @@ kda_chain_kernel(const unsigned char *__restrict__ ws_blobs, const int32_t *__re
         tmem_relinquish();
     }
     // zero rows 64..127 of both A2 stage buffers (A2 = [A_qk; 0])
-    for (int e = tid; e < 2 * 512; e += NT) {
+    for (int e = tid; e < 2 * 512; e += CHAIN_NT) {
         const int stage = e >> 9, w16 = e & 511;
         reinterpret_cast<uint4 *>(sm + stage * Lay::STAGE + Lay::A2 + 8192)[w16] = make_uint4(0, 0, 0, 0);
     }
-    // state slice: thread c owns key row c, columns j0 .. j0+N-1
-    const int c = tid;
-    float s_reg[N];
+    const int c = 32 * q4 + lane;    // state row owned by this thread
+    const int jh = 32 * hf;          // first of its 32 value columns (inside the slice)
+    float s_reg[32];
 #pragma unroll
-    for (int j = 0; j < N; j += 4) {
-        float4 v4 = S0 ? *reinterpret_cast<const float4 *>(S0 + state_off + (int64_t)c * D + j0 + j)
+    for (int j = 0; j < 32; j += 4) {
+        float4 v4 = S0 ? *reinterpret_cast<const float4 *>(S0 + state_off + (int64_t)c * D + j0 + jh + j)
                        : make_float4(0.f, 0.f, 0.f, 0.f);
         s_reg[j] = v4.x; s_reg[j + 1] = v4.y; s_reg[j + 2] = v4.z; s_reg[j + 3] = v4.w;
     }
 #pragma unroll
-    for (int jc = 0; jc < N / 8; ++jc) {  // row c of the MN-major S image
+    for (int jc = 0; jc < 4; ++jc) {  // row c of the MN-major S image, this thread's 4 chunks
         float v[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) v[e] = s_reg[jc * 8 + e];
-        st_chunk(sm + Lay::SIMG + sw128_chunk_off(c, jc, 128), v);
+        st_chunk(sm + Lay::SIMG + sw128_chunk_off(c, hf * 4 + jc, 128), v);
     }
     fence_async_smem();
     tc_fence_before();
@@ -600,17 +681,17 @@ kda_chain_kernel(const unsigned char *__restrict__ ws_blobs, const int32_t *__re
     const uint32_t tmem = *tmem_slot;
     const uint32_t d1 = tmem, d3 = tmem + N;
     const uint32_t sm_base = smem_u32(sm);
-    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
 
     if (tid == 0) {
         if (nchunks > 0) issue_load(0, 0);
         if (nchunks > 1) issue_load(1, 1);
     }
-    uint32_t mma_phase = 0;
 
 #pragma unroll 1
     for (int n = 0; n < nchunks && !dead; ++n) {
         const int stage = n & 1;
+        const uint32_t ph = (uint32_t)n & 1u;
         unsigned char *st = sm + stage * Lay::STAGE;
         const uint32_t st_base = sm_base + stage * Lay::STAGE;
         const int64_t tok0 = span.start + (int64_t)n * CH;
@@ -622,75 +703,72 @@ kda_chain_kernel(const unsigned char *__restrict__ ws_blobs, const int32_t *__re
             tc_fence_after();
             mma_run(d1, kmajor(st_base + Lay::A1, 128), mnmajor(sm_base + Lay::SIMG, 16384), D,
                     idesc_bf16(128, N, 0, 1), false);
-            mma_commit(bar_mma);
+            mma_commit(bar_a);
         }
-        mbar_wait(bar_mma, mma_phase, dead, &g_kda_device_status);
-        mma_phase ^= 1u;
+        mbar_wait(bar_a, ph, dead, &g_kda_device_status);
         tc_fence_after();
-        if (warp >= 2) {  // rows 64..127 of D1 hold (W S)[r]; V_new = U - W S
-            const int r = tid - 64;
-            float ws[N];
+        if (q4 >= 2) {  // rows 64..127 of D1 hold (W S)[r]; V_new = U - W S
+            const int r = c - 64;
+            float ws[32];
+            tmem_ld32(d1 + lane_off + jh, ws);
 #pragma unroll
-            for (int j = 0; j < N; j += 32)
-                tmem_ld32(d1 + lane_off + j, ws + j);
-#pragma unroll
-            for (int jc = 0; jc < N / 8; ++jc) {
-                const int jg = (N == 128 ? 0 : (j0 & 63)) + jc * 8;  // column inside the U image
-                const uint4 u4 = *reinterpret_cast<const uint4 *>(st + Lay::U + sw128_chunk_off(r, jg >> 3, 64));
+            for (int jc = 0; jc < 4; ++jc) {
+                const uint4 u4 = *reinterpret_cast<const uint4 *>(
+                    st + Lay::U + sw128_chunk_off(r, hf * 4 + jc, 64));
                 const __nv_bfloat16 *ub = reinterpret_cast<const __nv_bfloat16 *>(&u4);
                 float v[8];
 #pragma unroll
                 for (int e = 0; e < 8; ++e) v[e] = __bfloat162float(ub[e]) - ws[jc * 8 + e];
-                st_chunk(sm + Lay::VIMG + sw128_chunk_off(r, jc, 64), v);  // row r, MN-major
+                st_chunk(sm + Lay::VIMG + sw128_chunk_off(r, hf * 4 + jc, 64), v);  // row r, MN-major
             }
         }
         fence_async_smem();
         tc_fence_before();
         __syncthreads();
-        // D1 += [A_qk; 0] V_new ; D3 = K~^T V_new
+        // D3 = K~^T V_new (the state path first), then D1 += [A_qk; 0] V_new
         if (tid == 0) {
             tc_fence_after();
-            mma_run(d1, kmajor(st_base + Lay::A2, 128), mnmajor(sm_base + Lay::VIMG, 8192), CH,
-                    idesc_bf16(128, N, 0, 1), true);
             mma_run(d3, mnmajor(st_base + Lay::KTT, 8192), mnmajor(sm_base + Lay::VIMG, 8192), CH,
                     idesc_bf16(128, N, 1, 1), false);
-            mma_commit(bar_mma);
+            mma_commit(bar_b);
+            mma_run(d1, kmajor(st_base + Lay::A2, 128), mnmajor(sm_base + Lay::VIMG, 8192), CH,
+                    idesc_bf16(128, N, 0, 1), true);
+            mma_commit(bar_c);
         }
-        mbar_wait(bar_mma, mma_phase, dead, &g_kda_device_status);
-        mma_phase ^= 1u;
-        tc_fence_after();
-        if (warp < 2) {  // rows 0..63 of D1: the chunk's output
-            const int r = tid;
-            float ov[N];
-#pragma unroll
-            for (int j = 0; j < N; j += 32)
-                tmem_ld32(d1 + lane_off + j, ov + j);
-            if (r < L) {
-                __nv_bfloat16 *dst = o + ((tok0 + r) * H + h) * (int64_t)D + j0;
-#pragma unroll
-                for (int j = 0; j < N; j += 8) {
-                    uint4 pk = make_uint4(pack_bf16x2(ov[j], ov[j + 1]), pack_bf16x2(ov[j + 2], ov[j + 3]),
-                                          pack_bf16x2(ov[j + 4], ov[j + 5]), pack_bf16x2(ov[j + 6], ov[j + 7]));
-                    *reinterpret_cast<uint4 *>(dst + j) = pk;
-                }
-            }
-        }
-        {  // S <- Diag(exp(g_L)) S + K~^T V_new; thread c = key row c
-            float dv[N];
-#pragma unroll
-            for (int j = 0; j < N; j += 32)
-                tmem_ld32(d3 + lane_off + j, dv + j);
+        {  // S <- Diag(exp(g_L)) S + K~^T V_new
+            mbar_wait(bar_b, ph, dead, &g_kda_device_status);
+            tc_fence_after();
+            float dv[32];
+            tmem_ld32(d3 + lane_off + jh, dv);
             const float gam = reinterpret_cast<const float *>(st + Lay::GAM)[c];
 #pragma unroll
-            for (int jc = 0; jc < N / 8; ++jc) {
+            for (int jc = 0; jc < 4; ++jc) {
                 float v[8];
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
                     s_reg[jc * 8 + e] = gam * s_reg[jc * 8 + e] + dv[jc * 8 + e];
                     v[e] = s_reg[jc * 8 + e];
                 }
-                st_chunk(sm + Lay::SIMG + sw128_chunk_off(c, jc, 128), v);
+                st_chunk(sm + Lay::SIMG + sw128_chunk_off(c, hf * 4 + jc, 128), v);
             }
+        }
+        if (q4 < 2) {  // rows 0..63 of D1: the chunk's output
+            mbar_wait(bar_c, ph, dead, &g_kda_device_status);
+            tc_fence_after();
+            const int r = c;
+            float ov[32];
+            tmem_ld32(d1 + lane_off + jh, ov);
+            if (r < L) {
+                __nv_bfloat16 *dst = o + ((tok0 + r) * H + h) * (int64_t)D + j0 + jh;
+#pragma unroll
+                for (int j = 0; j < 32; j += 8) {
+                    uint4 pk = make_uint4(pack_bf16x2(ov[j], ov[j + 1]), pack_bf16x2(ov[j + 2], ov[j + 3]),
+                                          pack_bf16x2(ov[j + 4], ov[j + 5]), pack_bf16x2(ov[j + 6], ov[j + 7]));
+                    *reinterpret_cast<uint4 *>(dst + j) = pk;
+                }
+            }
+        } else {
+            mbar_wait(bar_c, ph, dead, &g_kda_device_status);  // keep every thread's phase in step
         }
         fence_async_smem();
         tc_fence_before();
@@ -700,8 +778,8 @@ kda_chain_kernel(const unsigned char *__restrict__ ws_blobs, const int32_t *__re
 
     if (S_T) {
 #pragma unroll
-        for (int j = 0; j < N; j += 4)
-            *reinterpret_cast<float4 *>(S_T + state_off + (int64_t)c * D + j0 + j) =
+        for (int j = 0; j < 32; j += 4)
+            *reinterpret_cast<float4 *>(S_T + state_off + (int64_t)c * D + j0 + jh + j) =
                 make_float4(s_reg[j], s_reg[j + 1], s_reg[j + 2], s_reg[j + 3]);
     }
     tc_fence_before();
@@ -793,7 +871,7 @@ cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, const
     err = cudaFuncSetAttribute(kda_chain_kernel<CHAIN_N>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Lay::BYTES);
     if (err != cudaSuccess) return err;
-    kda_chain_kernel<CHAIN_N><<<dim3((unsigned)nseq, (unsigned)H, D / CHAIN_N), NT, Lay::BYTES, stream>>>(
+    kda_chain_kernel<CHAIN_N><<<dim3((unsigned)nseq, (unsigned)H, D / CHAIN_N), CHAIN_NT, Lay::BYTES, stream>>>(
         blobs, chunk_off, S0, (__nv_bfloat16 *)o, S_T, cu_seqlens, T, H, nck);
     return cudaGetLastError();
 }
