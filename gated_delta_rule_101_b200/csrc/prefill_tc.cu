@@ -112,10 +112,10 @@ struct ChainLayout {
     static constexpr uint32_t STAGE = ((GAM + 512 + 1023) / 1024) * 1024;
     static constexpr uint32_t SIMG = 2 * STAGE;       // S bf16, MN-major: rows c (128), N columns
     static constexpr uint32_t VIMG = SIMG + N * 256;  // V_new bf16, MN-major: rows r (64), N columns
-    static constexpr uint32_t BAR = VIMG + N * 128;   // 5 mbarriers
-    static constexpr uint32_t TMEM = BAR + 40;
+    static constexpr uint32_t BAR = VIMG + N * 128;   // 6 mbarriers
+    static constexpr uint32_t TMEM = BAR + 48;
     static constexpr uint32_t BYTES = TMEM + 8 + 1024;
-    static constexpr uint32_t TMEM_COLS = 2 * N < 32 ? 32 : 2 * N;
+    static constexpr uint32_t TMEM_COLS = 4 * N;      // D1 (two buffers) and D3
     static constexpr uint32_t LOAD_BYTES = 32768 + 8192 + 16384 + U_BYTES + 512;
 };
 
@@ -328,8 +328,7 @@ kda_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     // ---- Gram MMA: D[m][i] = sum_c A1[m][c] KINV[i][c]; rows 0..63 Q-rows, 64..127 K-rows
     if (tid == 0) {
         tc_fence_after();
-        mma_run(tmem, kmajor(sm_base + P_A1, 128), kmajor(sm_base + P_KINV, 64), D,
-                idesc_bf16(128, 64), false);
+        mma_run<D>(tmem, kmajor(sm_base + P_A1, 128), kmajor(sm_base + P_KINV, 64), idesc_bf16(128, 64), false);
         mma_commit(bar_mma);
     }
 
@@ -545,10 +544,8 @@ kda_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     //      K e^g sits in rows 64..127 of A1, read here as an MN-major B (K = token i).
     if (tid == 0) {
         tc_fence_after();
-        mma_run(tmem, kmajor(sm_base + P_TB, 64), mnmajor(sm_base + P_A1 + 8192, 16384), CH,
-                idesc_bf16(64, 128, 0, 1), false);
-        mma_run(tmem + 128, kmajor(sm_base + P_TB, 64), mnmajor(sm_base + P_V, 8192), CH,
-                idesc_bf16(64, 128, 0, 1), false);
+        mma_run<CH>(tmem, kmajor(sm_base + P_TB, 64), mnmajor(sm_base + P_A1 + 8192, 16384), idesc_bf16(64, 128, 0, 1), false);
+        mma_run<CH>(tmem + 128, kmajor(sm_base + P_TB, 64), mnmajor(sm_base + P_V, 8192), idesc_bf16(64, 128, 0, 1), false);
         mma_commit(bar_mma);
     }
     mbar_wait(bar_mma, 1, dead, &g_kda_device_status);
@@ -627,10 +624,10 @@ kda_chain_kernel(const unsigned char *__restrict__ ws_blobs, const int32_t *__re
     const int64_t slot0 = chunk_off ? (int64_t)chunk_off[seq] : (int64_t)seq * nck;
     const int64_t state_off = ((int64_t)seq * H + h) * (int64_t)(D * D);
 
-    uint64_t *bar_ld = reinterpret_cast<uint64_t *>(sm + Lay::BAR);  // [2]
+    uint64_t *bar_ld = reinterpret_cast<uint64_t *>(sm + Lay::BAR);  // [2] chunk loads
     uint64_t *bar_a = bar_ld + 2;  // MMA1 done
     uint64_t *bar_b = bar_ld + 3;  // state MMA done
-    uint64_t *bar_c = bar_ld + 4;  // output MMA done
+    uint64_t *bar_c = bar_ld + 4;  // [2] output MMA done, per D1 buffer
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + Lay::TMEM);
     bool dead = false;
 
@@ -646,7 +643,7 @@ kda_chain_kernel(const unsigned char *__restrict__ ws_blobs, const int32_t *__re
     };
 
     if (tid == 0) {
-        for (int b = 0; b < 5; ++b) mbar_init(&bar_ld[b], 1);
+        for (int b = 0; b < 6; ++b) mbar_init(&bar_ld[b], 1);
         fence_mbar_init();
     }
     if (warp == 0) {
@@ -679,7 +676,7 @@ kda_chain_kernel(const unsigned char *__restrict__ ws_blobs, const int32_t *__re
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t d1 = tmem, d3 = tmem + N;
+    const uint32_t d3 = tmem + 2 * N;  // D1 buffers at columns 0 and N
     const uint32_t sm_base = smem_u32(sm);
     const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
 
@@ -688,23 +685,46 @@ kda_chain_kernel(const unsigned char *__restrict__ ws_blobs, const int32_t *__re
         if (nchunks > 1) issue_load(1, 1);
     }
 
+    // Output of chunk m: rows 0..63 of D1 buffer m % 2, read by the warps of lane
+    // quarters 0 and 1 once the output MMA of chunk m has completed. It runs while
+    // the next chunk's first MMA executes, off the state recurrence's path.
+    auto store_output = [&](int m) {
+        if (q4 < 2) {
+            mbar_wait(&bar_c[m & 1], (uint32_t)(m >> 1) & 1u, dead, &g_kda_device_status);
+            tc_fence_after();
+            const int r = c;
+            float ov[32];
+            tmem_ld32(tmem + (uint32_t)((m & 1) * N) + lane_off + jh, ov);
+            const int64_t tok = span.start + (int64_t)m * CH + r;
+            if (r < chunk_rows(span.len, (int64_t)m * CH)) {
+                __nv_bfloat16 *dst = o + (tok * H + h) * (int64_t)D + j0 + jh;
+#pragma unroll
+                for (int j = 0; j < 32; j += 8) {
+                    uint4 pk = make_uint4(pack_bf16x2(ov[j], ov[j + 1]), pack_bf16x2(ov[j + 2], ov[j + 3]),
+                                          pack_bf16x2(ov[j + 4], ov[j + 5]), pack_bf16x2(ov[j + 6], ov[j + 7]));
+                    *reinterpret_cast<uint4 *>(dst + j) = pk;
+                }
+            }
+        }
+    };
+
 #pragma unroll 1
     for (int n = 0; n < nchunks && !dead; ++n) {
         const int stage = n & 1;
         const uint32_t ph = (uint32_t)n & 1u;
         unsigned char *st = sm + stage * Lay::STAGE;
         const uint32_t st_base = sm_base + stage * Lay::STAGE;
-        const int64_t tok0 = span.start + (int64_t)n * CH;
-        const int L = chunk_rows(span.len, (int64_t)n * CH);
+        const uint32_t d1 = tmem + (uint32_t)((n & 1) * N);
 
         mbar_wait(&bar_ld[stage], (uint32_t)(n >> 1) & 1u, dead, &g_kda_device_status);
         // D1 = [Q~; W] S
         if (tid == 0) {
             tc_fence_after();
-            mma_run(d1, kmajor(st_base + Lay::A1, 128), mnmajor(sm_base + Lay::SIMG, 16384), D,
-                    idesc_bf16(128, N, 0, 1), false);
+            mma_run<D>(d1, kmajor(st_base + Lay::A1, 128), mnmajor(sm_base + Lay::SIMG, 16384),
+                       idesc_bf16(128, N, 0, 1), false);
             mma_commit(bar_a);
         }
+        if (n > 0) store_output(n - 1);
         mbar_wait(bar_a, ph, dead, &g_kda_device_status);
         tc_fence_after();
         if (q4 >= 2) {  // rows 64..127 of D1 hold (W S)[r]; V_new = U - W S
@@ -728,12 +748,12 @@ kda_chain_kernel(const unsigned char *__restrict__ ws_blobs, const int32_t *__re
         // D3 = K~^T V_new (the state path first), then D1 += [A_qk; 0] V_new
         if (tid == 0) {
             tc_fence_after();
-            mma_run(d3, mnmajor(st_base + Lay::KTT, 8192), mnmajor(sm_base + Lay::VIMG, 8192), CH,
-                    idesc_bf16(128, N, 1, 1), false);
+            mma_run<CH>(d3, mnmajor(st_base + Lay::KTT, 8192), mnmajor(sm_base + Lay::VIMG, 8192),
+                        idesc_bf16(128, N, 1, 1), false);
             mma_commit(bar_b);
-            mma_run(d1, kmajor(st_base + Lay::A2, 128), mnmajor(sm_base + Lay::VIMG, 8192), CH,
-                    idesc_bf16(128, N, 0, 1), true);
-            mma_commit(bar_c);
+            mma_run<CH>(d1, kmajor(st_base + Lay::A2, 128), mnmajor(sm_base + Lay::VIMG, 8192),
+                        idesc_bf16(128, N, 0, 1), true);
+            mma_commit(&bar_c[n & 1]);
         }
         {  // S <- Diag(exp(g_L)) S + K~^T V_new
             mbar_wait(bar_b, ph, dead, &g_kda_device_status);
@@ -752,29 +772,17 @@ kda_chain_kernel(const unsigned char *__restrict__ ws_blobs, const int32_t *__re
                 st_chunk(sm + Lay::SIMG + sw128_chunk_off(c, hf * 4 + jc, 128), v);
             }
         }
-        if (q4 < 2) {  // rows 0..63 of D1: the chunk's output
-            mbar_wait(bar_c, ph, dead, &g_kda_device_status);
-            tc_fence_after();
-            const int r = c;
-            float ov[32];
-            tmem_ld32(d1 + lane_off + jh, ov);
-            if (r < L) {
-                __nv_bfloat16 *dst = o + ((tok0 + r) * H + h) * (int64_t)D + j0 + jh;
-#pragma unroll
-                for (int j = 0; j < 32; j += 8) {
-                    uint4 pk = make_uint4(pack_bf16x2(ov[j], ov[j + 1]), pack_bf16x2(ov[j + 2], ov[j + 3]),
-                                          pack_bf16x2(ov[j + 4], ov[j + 5]), pack_bf16x2(ov[j + 6], ov[j + 7]));
-                    *reinterpret_cast<uint4 *>(dst + j) = pk;
-                }
-            }
-        } else {
-            mbar_wait(bar_c, ph, dead, &g_kda_device_status);  // keep every thread's phase in step
-        }
         fence_async_smem();
         tc_fence_before();
         __syncthreads();
-        if (tid == 0 && n + 2 < nchunks) issue_load(n + 2, stage);
+        // The stage is free once the output MMA (which reads A2) has completed; the
+        // next load into it is issued after that MMA's barrier.
+        if (tid == 0 && n + 2 < nchunks) {
+            mbar_wait(&bar_c[n & 1], (uint32_t)(n >> 1) & 1u, dead, &g_kda_device_status);
+            issue_load(n + 2, stage);
+        }
     }
+    if (nchunks > 0 && !dead) store_output(nchunks - 1);
 
     if (S_T) {
 #pragma unroll

@@ -223,24 +223,31 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int a_mn = 0, in
 // One MMA operand in shared memory.
 //   K-major:  `rows` rows of the tile; 64-element K blocks are rows*128 bytes apart.
 //   MN-major: K runs down the rows; `lbo` = bytes between 64-element M/N blocks.
+// The descriptor of the kk-th K step (16 elements) is the base descriptor plus
+// the step's byte offset in 16-byte units (shared addresses stay below 256 KiB,
+// so the 14-bit start-address field never carries).
 struct Operand {
-    uint32_t base;
-    uint32_t rows_or_lbo;
-    bool mn;
-    __device__ __forceinline__ uint64_t desc(int kk) const {  // kk-th K step of 16 elements
-        if (mn) return sw128_desc(base + (uint32_t)kk * 2048u, rows_or_lbo);
-        const uint32_t kb = (uint32_t)kk >> 2, in = ((uint32_t)kk & 3u) * 32u;
-        return sw128_desc(base + kb * rows_or_lbo * 128u + in);
+    uint64_t base_desc;
+    uint32_t rows;  // K-major row count (0 for MN-major)
+    __device__ __forceinline__ uint64_t desc(int kk) const {
+        const uint32_t off = rows ? ((uint32_t)kk >> 2) * rows * 128u + ((uint32_t)kk & 3u) * 32u
+                                  : (uint32_t)kk * 2048u;
+        return base_desc + (uint64_t)(off >> 4);
     }
 };
-__device__ __forceinline__ Operand kmajor(uint32_t base, uint32_t rows) { return {base, rows, false}; }
-__device__ __forceinline__ Operand mnmajor(uint32_t base, uint32_t lbo) { return {base, lbo, true}; }
+__device__ __forceinline__ Operand kmajor(uint32_t base, uint32_t rows) {
+    return {sw128_desc(base), rows};
+}
+__device__ __forceinline__ Operand mnmajor(uint32_t base, uint32_t lbo) {
+    return {sw128_desc(base, lbo), 0u};
+}
 
 // Issues the K/16 MMAs of D (+)= A * B (A: M x K, B: K x N as described by
 // the operands; the instruction descriptor must carry the same majorness).
-__device__ __forceinline__ void mma_run(uint32_t d_tmem, Operand a, Operand b, int K, uint32_t idesc,
+template <int K>
+__device__ __forceinline__ void mma_run(uint32_t d_tmem, Operand a, Operand b, uint32_t idesc,
                                         bool accumulate) {
-#pragma unroll 1
+#pragma unroll
     for (int kk = 0; kk < K / 16; ++kk)
         mma_bf16(d_tmem, a.desc(kk), b.desc(kk), idesc, (accumulate || kk > 0) ? 1u : 0u);
 }
