@@ -55,45 +55,101 @@ def peaks():
 
 # ------------------------------------------------------------------ clocks
 class ClockSampler:
-    """Samples nvidia-smi clocks and throttle reasons while the timed region runs."""
+    """Samples SM clocks and throttle reasons while the timed region runs.
 
-    FIELDS = ["clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.active",
-              "clocks_event_reasons.hw_slowdown", "clocks_event_reasons.hw_thermal_slowdown",
-              "clocks_event_reasons.sw_thermal_slowdown", "clocks_event_reasons.sw_power_cap"]
+    Uses NVML from a background thread every 5 ms (the timed regions are tens
+    of milliseconds); falls back to `nvidia-smi -lms 200` when NVML is absent.
+    """
 
-    def __init__(self, device_index: int):
-        self.proc = None
+    REASONS = {"hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+               "sw_power_cap": 0x4}
+
+    def __init__(self, device_index: int, period_s: float = 0.005):
+        import threading
+
+        self.samples, self.reasons, self.smax = [], set(), None
+        self.proc = self.thread = None
+        uuid = "GPU-" + str(torch.cuda.get_device_properties(device_index).uuid)
         try:
-            uuid = "GPU-" + str(torch.cuda.get_device_properties(device_index).uuid)
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", uuid, "--query-gpu=" + ",".join(self.FIELDS),
-                 "--format=csv,noheader,nounits", "-lms", "200"],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-        except (OSError, RuntimeError):
-            self.proc = None
+            import pynvml
+
+            pynvml.nvmlInit()
+            handle = pynvml.nvmlDeviceGetHandleByUUID(uuid)
+            self.smax = float(pynvml.nvmlDeviceGetMaxClockInfo(handle, pynvml.NVML_CLOCK_SM))
+            self.stop_evt = threading.Event()
+
+            def run():
+                while not self.stop_evt.is_set():
+                    self.samples.append(float(pynvml.nvmlDeviceGetClockInfo(handle, pynvml.NVML_CLOCK_SM)))
+                    mask = pynvml.nvmlDeviceGetCurrentClocksEventReasons(handle)
+                    for name, bit in self.REASONS.items():
+                        if mask & bit:
+                            self.reasons.add(name)
+                    self.stop_evt.wait(period_s)
+
+            self.thread = threading.Thread(target=run, daemon=True)
+            self.thread.start()
+        except Exception:  # NVML unavailable: nvidia-smi loop
+            fields = "clocks.sm,clocks.max.sm,clocks_event_reasons.hw_slowdown," \
+                     "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown," \
+                     "clocks_event_reasons.sw_power_cap"
+            try:
+                self.proc = subprocess.Popen(
+                    ["nvidia-smi", "-i", uuid, "--query-gpu=" + fields, "--format=csv,noheader,nounits",
+                     "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            except OSError:
+                self.proc = None
 
     def stop(self):
-        if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        self.proc.terminate()
-        out, _ = self.proc.communicate(timeout=10)
-        sm, smax, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in out.strip().splitlines():
-            parts = [x.strip() for x in line.split(",")]
-            if len(parts) != len(self.FIELDS):
-                continue
-            try:
-                sm.append(float(parts[0]))
-                smax.append(float(parts[1]))
-            except ValueError:
-                continue
-            for name, val in zip(names, parts[4:]):
-                if val.lower() == "active":
-                    reasons.add(name)
-        return {"sm_mhz": statistics.median(sm) if sm else None,
-                "sm_max_mhz": max(smax) if smax else None, "reasons": sorted(reasons),
-                "samples": len(sm)}
+        if self.thread is not None:
+            self.stop_evt.set()
+            self.thread.join(timeout=5)
+        elif self.proc is not None:
+            self.proc.terminate()
+            out, _ = self.proc.communicate(timeout=10)
+            names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+            for line in out.strip().splitlines():
+                parts = [x.strip() for x in line.split(",")]
+                try:
+                    self.samples.append(float(parts[0]))
+                    self.smax = float(parts[1])
+                except (ValueError, IndexError):
+                    continue
+                for name, val in zip(names, parts[2:]):
+                    if val.lower() == "active":
+                        self.reasons.add(name)
+        else:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["clock sampling unavailable"]}
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.smax, "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------------ ncu traffic
+# DRAM bytes (read + write) per launch from one ncu capture of the B=4, T=4096,
+# H=16 step and of one N=256, H=32 decode step (profiles/). They are reported
+# only while the CUDA sources hash to the build they were taken from.
+TRAFFIC = {"source_hash": "353fc00f9f230e47",
+           "prefill": 338424064 + 257215232 + 308346880 + 58567936,  # prep + chain
+           "decode": 547402496 + 480379392}
+
+
+def source_hash() -> str:
+    import glob
+    import hashlib
+
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "gated_delta_rule_101_b200", "csrc")
+    for p in sorted(glob.glob(os.path.join(csrc, "*.cu")) + glob.glob(os.path.join(csrc, "*.cuh"))):
+        h.update(os.path.basename(p).encode())
+        with open(p, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def traffic(kind: str, override):
+    if override is not None:
+        return override
+    return TRAFFIC[kind] if source_hash() == TRAFFIC["source_hash"] else None
 
 
 # ------------------------------------------------------------------ helpers
@@ -241,8 +297,9 @@ def run_kda(args, rank, world, local_rank):
     pages_flops = PAGES_FLOPS_PER_TOKEN_HEAD * B * T * H
     tflops = pages_flops / avg_kernel_s / 1e12
     roofline = {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
-                "frac": achieved / pk["hbm_gbs"], "traffic": args.traffic,
-                "peak_source": pk_kind, "kernel": "kda_chunk_fwd (prefill)",
+                "frac": achieved / pk["hbm_gbs"], "traffic": traffic("prefill", args.traffic),
+                "peak_source": pk_kind,
+                "kernel": "kda_chunk_fwd: kda_prep_kernel + kda_chain_kernel (one call, timed together)",
                 "alg_bytes_per_launch": alg_bytes,
                 "tensor_pages_flops": {"achieved_tflops": tflops, "peak": pk["bf16_tflops"],
                                        "frac": tflops / pk["bf16_tflops"],
@@ -309,7 +366,7 @@ def run_kda(args, rank, world, local_rank):
                                          "steps in one CUDA graph", "l2": "state 512 MiB > L2"},
                   "roofline": {"bound": "hbm", "achieved": d_ach, "peak": pk["hbm_gbs"],
                                "unit": "GB/s", "frac": d_ach / pk["hbm_gbs"],
-                               "traffic": args.decode_traffic, "peak_source": pk_kind,
+                               "traffic": traffic("decode", args.decode_traffic), "peak_source": pk_kind,
                                "kernel": "kda_decode_step", "alg_bytes_per_launch": d_bytes},
                   "gpu_launches": nsteps * len(d_times), "clocks": dclk}
         del graph, dinp, S, od
