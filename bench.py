@@ -210,6 +210,14 @@ def cpu_oracle_sample(inp, n_heads=None):
                       f"batch, fp64 recurrence, {dt:.2f} s"}
 
 
+def prefill_config(world: int) -> dict:
+    B, T, H = PREFILL["B"], PREFILL["T"], PREFILL["H"]
+    return {"workload": f"KDA prefill B={B} T={T} H={H} d=128 C=64, bf16 q/k/v, fp32 log_alpha/beta/"
+                        "state, S0~N(0,0.1^2)",
+            "global_batch": B * world, "seq_len": T, "parallelism": f"dp{world}",
+            "l2": "flushed before every step (256 MiB write); inputs 412 MB > L2"}
+
+
 # ------------------------------------------------------------------ arms
 def run_reference(args, rank, world):
     """The fp64 CPU oracle timed on host cores, a bounded sample per step."""
@@ -235,14 +243,14 @@ def run_reference(args, rank, world):
     total = sum(times)
     tokens = PREFILL["T"] * args.steps
     value = tokens / total
-    sample = (f"one sequence of the prefill workload per step ({PREFILL['T']} tokens x {H} heads, "
-              f"bf16 inputs widened to fp64), {threads} threads")
+    sample = (f"one of the {PREFILL['B']} sequences of the prefill workload per step "
+              f"({PREFILL['T']} tokens x {H} heads, bf16 inputs widened to fp64), {threads} threads; "
+              f"value = tokens of that sequence / CPU time")
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": f"KDA prefill B=4 T=4096 H=16 d=128 C=64 (sampled: 1 sequence "
-                                   f"per step)", "l2": "n/a (CPU)"},
+            "config": prefill_config(world),
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
@@ -380,10 +388,7 @@ def run_kda(args, rank, world, local_rank):
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
                 "data": "synthetic",
-                "config": {"workload": f"KDA prefill B={B} T={T} H={H} d=128 C=64, bf16 q/k/v, fp32 "
-                                       "log_alpha/beta/state, S0~N(0,0.1^2)",
-                           "global_batch": B * world, "seq_len": T, "parallelism": f"dp{world}",
-                           "l2": "flushed before every step (256 MiB write); inputs 412 MB > L2"},
+                "config": prefill_config(world),
                 "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
                 "gpu_launches": launches_per_call * args.steps, "clocks": clk, "decode": decode}
         print(json.dumps(line), flush=True)
