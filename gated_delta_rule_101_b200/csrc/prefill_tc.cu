@@ -241,24 +241,22 @@ kda_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     mbar_wait(bar_tma, 0, dead, &g_kda_device_status);
 
     // ---- g = chunk-local cumulative sum of log_alpha (rows >= L count as 0), in place.
-    //      Thread t: channel c = t % 128, rows 32*(t/128) .. +31.
+    //      Thread t: channel c = t % 128, rows 32*(t/128) .. +31, summed in registers.
     {
         const int c = tid & (D - 1), half = tid >> 7, r0 = half * 32;
-        float acc = 0.f;
-#pragma unroll 8
-        for (int e = 0; e < 32; ++e) {
-            const int r = r0 + e;
-            acc += r < L ? lag[r * D + c] : 0.f;
-            lag[r * D + c] = acc;
-        }
-        if (half == 0) stot[c] = acc;
+        float gg[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) gg[e] = (r0 + e) < L ? lag[(r0 + e) * D + c] : 0.f;
+#pragma unroll
+        for (int e = 1; e < 32; ++e) gg[e] += gg[e - 1];
+        if (half == 0) stot[c] = gg[31];
         __syncthreads();
+        const float off = half ? stot[c] : 0.f;
+#pragma unroll
+        for (int e = 0; e < 32; ++e) lag[(r0 + e) * D + c] = gg[e] + off;
         if (half == 1) {
-            const float off = stot[c];
-#pragma unroll 8
-            for (int e = 0; e < 32; ++e) lag[(r0 + e) * D + c] += off;
-            sgl[c] = acc + off;
-            sgam[c] = expf(acc + off);
+            sgl[c] = gg[31] + off;
+            sgam[c] = expf(gg[31] + off);
         }
     }
     __syncthreads();
@@ -286,7 +284,8 @@ kda_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         badc[e] = -gls[e] > SAFE_SPAN;
         any_bad |= badc[e];
     }
-    __syncthreads();  // log_alpha/g tile fully read: its space becomes KT | KINV
+    // log_alpha/g tile fully read: its space becomes KT | KINV
+    const int n_bad = __syncthreads_or(any_bad) ? 1 : 0;
 #pragma unroll
     for (int v8 = 0; v8 < 8; ++v8) {
         const int r = warp + 8 * v8;
@@ -302,7 +301,7 @@ kda_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             const float eg = __expf(gs[e]);
             qe[e] = x * eg;
             ke[e] = kk * eg;
-            if (!badc[e]) {  // exp(-g) <= exp(80): finite, and exp(g_L - g) = exp(g_L) exp(-g)
+            if (!n_bad || !badc[e]) {  // exp(-g) <= exp(80): finite; exp(g_L - g) = exp(g_L) exp(-g)
                 const float kin_ = kk * __expf(-gs[e]);
                 kin[e] = kin_;
                 kt[e] = kin_ * gams[e];
@@ -323,7 +322,7 @@ kda_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     }
     fence_async_smem();
     tc_fence_before();
-    const int n_bad = __syncthreads_or(any_bad) ? 1 : 0;
+    __syncthreads();
 
     // ---- Gram MMA: D[m][i] = sum_c A1[m][c] KINV[i][c]; rows 0..63 Q-rows, 64..127 K-rows
     if (tid == 0) {
@@ -440,10 +439,13 @@ kda_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     const float4 a4 = *reinterpret_cast<const float4 *>(at + (o + r) * LDT + o + m4);
                     arow[m4] = a4.x; arow[m4 + 1] = a4.y; arow[m4 + 2] = a4.z; arow[m4 + 3] = a4.w;
                 }
-                float x = (r == l) ? 1.f : 0.f;
+                float x0 = (r == l) ? 1.f : 0.f, x1 = 0.f;
 #pragma unroll
-                for (int mm = 0; mm < r; ++mm) x -= arow[mm] * t[mm];
-                t[r] = x;
+                for (int mm = 0; mm < r; mm += 2) {
+                    x0 -= arow[mm] * t[mm];
+                    if (mm + 1 < r) x1 -= arow[mm + 1] * t[mm + 1];
+                }
+                t[r] = x0 + x1;
             }
             __syncwarp();
             if (lane < 16) {
@@ -452,37 +454,36 @@ kda_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             }
         }
         __syncthreads();
-        // level 1: blocks (16..31, 0..15) and (48..63, 32..47); thread -> 1 x 4 tile
-        const int l1b = tid >> 6, l1a = (tid >> 2) & 15, l1c = (tid & 3) * 4, l1o = 32 * l1b;
-        if (tid < 128) {  // P = A_lo-hi-block X^-1
-            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        // level 1: blocks (16..31, 0..15) and (48..63, 32..47); thread -> 1 x 2 tile
+        const int l1b = tid >> 7, l1a = (tid >> 3) & 15, l1c = (tid & 7) * 2, l1o = 32 * l1b;
+        {  // P = A_lo-hi-block X^-1
+            float2 acc = make_float2(0.f, 0.f);
 #pragma unroll
             for (int m4 = 0; m4 < 16; m4 += 4) {
                 const float4 a4 = *reinterpret_cast<const float4 *>(at + (l1o + 16 + l1a) * LDT + l1o + m4);
                 const float av[4] = {a4.x, a4.y, a4.z, a4.w};
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
-                    const float4 b4 = *reinterpret_cast<const float4 *>(at + (l1o + m4 + u) * LDT + l1o + l1c);
-                    acc.x += av[u] * b4.x; acc.y += av[u] * b4.y; acc.z += av[u] * b4.z; acc.w += av[u] * b4.w;
+                    const float2 b2 = *reinterpret_cast<const float2 *>(at + (l1o + m4 + u) * LDT + l1o + l1c);
+                    acc.x += av[u] * b2.x; acc.y += av[u] * b2.y;
                 }
             }
-            *reinterpret_cast<float4 *>(pb + (l1b * 16 + l1a) * 20 + l1c) = acc;
+            *reinterpret_cast<float2 *>(pb + (l1b * 16 + l1a) * 20 + l1c) = acc;
         }
         __syncthreads();
-        if (tid < 128) {  // T = -Z^-1 P
-            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        {  // T = -Z^-1 P
+            float2 acc = make_float2(0.f, 0.f);
 #pragma unroll
             for (int m4 = 0; m4 < 16; m4 += 4) {
                 const float4 d4 = *reinterpret_cast<const float4 *>(at + (l1o + 16 + l1a) * LDT + l1o + 16 + m4);
                 const float dv[4] = {d4.x, d4.y, d4.z, d4.w};
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
-                    const float4 p4 = *reinterpret_cast<const float4 *>(pb + (l1b * 16 + m4 + u) * 20 + l1c);
-                    acc.x += dv[u] * p4.x; acc.y += dv[u] * p4.y; acc.z += dv[u] * p4.z; acc.w += dv[u] * p4.w;
+                    const float2 p2 = *reinterpret_cast<const float2 *>(pb + (l1b * 16 + m4 + u) * 20 + l1c);
+                    acc.x += dv[u] * p2.x; acc.y += dv[u] * p2.y;
                 }
             }
-            *reinterpret_cast<float4 *>(at + (l1o + 16 + l1a) * LDT + l1o + l1c) =
-                make_float4(-acc.x, -acc.y, -acc.z, -acc.w);
+            *reinterpret_cast<float2 *>(at + (l1o + 16 + l1a) * LDT + l1o + l1c) = make_float2(-acc.x, -acc.y);
         }
         __syncthreads();
         // level 2: block (32..63, 0..31); thread -> 1 x 4 tile of the 32 x 32 block
