@@ -56,10 +56,10 @@ constexpr float SAFE_SPAN = 80.f;  // largest chunk log-decay the factorised Gra
 // ---- one workspace blob per (chunk, head): operand images for the chain kernel
 constexpr uint32_t BLOB_A1 = 0;        // [Q~; W]: 128 x 128 bf16, K-major swizzled   (32 KiB)
 constexpr uint32_t BLOB_AQK = 32768;   // A_qk:    64 x 64 bf16                        (8 KiB)
-constexpr uint32_t BLOB_KTT = 40960;   // K~^T:    128 x 64 bf16                       (16 KiB)
-constexpr uint32_t BLOB_U = 57344;     // U:       64 x 128 bf16 (two 64-column atoms) (16 KiB)
-constexpr uint32_t BLOB_GAM = 73728;   // exp(g_L): 128 fp32
-constexpr uint32_t BLOB_BYTES = 74240;
+constexpr uint32_t BLOB_KTT = 40960;   // K~:      64 x 128 bf16 (rows = token)        (16 KiB)
+constexpr uint32_t BLOB_TB = 57344;    // T Diag(beta): 64 x 64 bf16                  (8 KiB)
+constexpr uint32_t BLOB_GAM = 65536;   // exp(g_L): 128 fp32
+constexpr uint32_t BLOB_BYTES = 66048;
 
 // ---- prep kernel shared memory (offsets from a 1024-byte aligned base). Every
 // operand image is a 128-byte-swizzled tile of 128-byte rows (see tc_ptx.cuh).
@@ -75,7 +75,7 @@ constexpr uint32_t BLOB_BYTES = 74240;
 //   AKK  64 x 68 fp32 (rows padded to 68 floats): A_kk, then T in place; over KINV.
 constexpr int PREP_NT = 256;
 constexpr uint32_t P_A1 = 0;          // 32768
-constexpr uint32_t P_V = 32768;       // 16384 (V, then U)
+constexpr uint32_t P_V = 32768;       // 16384 (unused)
 constexpr uint32_t P_LAG = 49152;     // 32768 (log_alpha -> g), then KT | KINV
 constexpr uint32_t P_KT = 49152;      // 16384
 constexpr uint32_t P_KINV = 65536;    // 16384 (dead after the Gram MMA)
@@ -94,7 +94,7 @@ constexpr uint32_t P_TMEM = 104720;
 constexpr uint32_t P_NBAD = 104724;   // number of listed bad channels
 constexpr uint32_t PREP_SMEM = 104736 + 1024;
 constexpr uint32_t PREP_TMEM_COLS = 256;  // Gram 64 (then W 128) | U 128
-constexpr uint32_t PREP_TMA_BYTES = 32768 + 16384 + 32768;  // q, k | v | log_alpha
+constexpr uint32_t PREP_TMA_BYTES = 32768 + 32768;  // q, k | log_alpha
 
 // A_kk / T rows are padded to 68 floats: float4 row segments stay aligned, and
 // 8 consecutive rows at the same column fall on distinct bank quads.
@@ -103,20 +103,23 @@ constexpr int LDT = 68;
 // ---- chain kernel shared memory
 template <int N>
 struct ChainLayout {
+    // One stage holds a chunk's blob and its value slice. The M = 128 operands that
+    // only have 64 meaningful rows read the 64 rows stored just before or after
+    // them as filler: those rows only reach accumulator rows that are dead by then.
     static constexpr uint32_t A1 = 0;                 // 32768 (K-major [Q~; W])
-    static constexpr uint32_t A2 = 32768;             // 16384: [A_qk; zeros] (K-major)
-    static constexpr uint32_t KTT = 49152;            // 16384 (MN-major K~^T: rows i, channels)
-    static constexpr uint32_t U = 65536;              // N == 128 ? 16384 : 8192
-    static constexpr uint32_t U_BYTES = N == 128 ? 16384 : 8192;
-    static constexpr uint32_t GAM = U + U_BYTES;      // 512
+    static constexpr uint32_t A2 = 32768;             // A_qk (8192); rows 64..127 = start of KTT
+    static constexpr uint32_t KTT = 40960;            // 16384 (MN-major K~^T: rows i, channels)
+    static constexpr uint32_t TB = 57344;             // 8192: T Diag(beta); the U MMA starts 8192 earlier
+    static constexpr uint32_t V = 65536;              // 8192: value slice, 64 rows x 64 columns (TMA)
+    static constexpr uint32_t GAM = 73728;            // 512
     static constexpr uint32_t STAGE = ((GAM + 512 + 1023) / 1024) * 1024;
     static constexpr uint32_t SIMG = 2 * STAGE;       // S bf16, MN-major: rows c (128), N columns
     static constexpr uint32_t VIMG = SIMG + N * 256;  // V_new bf16, MN-major: rows r (64), N columns
     static constexpr uint32_t BAR = VIMG + N * 128;   // 6 mbarriers
     static constexpr uint32_t TMEM = BAR + 48;
     static constexpr uint32_t BYTES = TMEM + 8 + 1024;
-    static constexpr uint32_t TMEM_COLS = 4 * N;      // D1 (two buffers) and D3
-    static constexpr uint32_t LOAD_BYTES = 32768 + 8192 + 16384 + U_BYTES + 512;
+    static constexpr uint32_t TMEM_COLS = 4 * N;      // D1 (two buffers), D3, U
+    static constexpr uint32_t LOAD_BYTES = 32768 + 8192 + 16384 + 8192 + 512 + 8192;
 };
 
 __device__ __forceinline__ unsigned char *aligned_smem(unsigned char *raw) {
@@ -224,8 +227,6 @@ kda_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         tma_load_2d(sm + P_A1 + 16384, &tm_q, x + 64, y, bar_tma);     // q, channels 64..127
         tma_load_2d(sm + P_A1 + 8192, &tm_k, x, y, bar_tma);           // k -> rows 64..127
         tma_load_2d(sm + P_A1 + 16384 + 8192, &tm_k, x + 64, y, bar_tma);
-        tma_load_2d(sm + P_V, &tm_v, x, y, bar_tma);
-        tma_load_2d(sm + P_V + 8192, &tm_v, x + 64, y, bar_tma);
         tma_load_2d(sm + P_LAG, &tm_la, x, y, bar_tma);
     }
     if (warp == 0) {
@@ -541,19 +542,19 @@ kda_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     tc_fence_before();
     __syncthreads();
 
-    // ---- W = (T Diag(beta)) (K e^g) and U = (T Diag(beta)) V, both M = 64, N = 128.
-    //      K e^g sits in rows 64..127 of A1, read here as an MN-major B (K = token i).
+    // ---- W = (T Diag(beta)) (K e^g), M = 64, N = 128. K e^g sits in rows 64..127 of A1,
+    //      read here as an MN-major B (K = token i). (U = T Diag(beta) V is formed by the
+    //      chain kernel from the blob's T Diag(beta) and its own slice of V.)
     if (tid == 0) {
         tc_fence_after();
         mma_run<CH>(tmem, kmajor(sm_base + P_TB, 64), mnmajor(sm_base + P_A1 + 8192, 16384), idesc_bf16(64, 128, 0, 1), false);
-        mma_run<CH>(tmem + 128, kmajor(sm_base + P_TB, 64), mnmajor(sm_base + P_V, 8192), idesc_bf16(64, 128, 0, 1), false);
         mma_commit(bar_mma);
     }
     mbar_wait(bar_mma, 1, dead, &g_kda_device_status);
     tc_fence_after();
     {
-        // M = 64 accumulators: row r sits in lane 16*(w%4) + (lane < 16) of quarter w%4.
-        // Warp half w/4 takes columns 64*(w/4) .. +63 of W and of U.
+        // M = 64 accumulator: row r sits in lane 16*(w%4) + (lane < 16) of quarter w%4.
+        // Warp half w/4 takes columns 64*(w/4) .. +63.
         float a[64];
         const uint32_t lanes = (uint32_t)(32 * (warp & 3)) << 16;
         const uint32_t cofs = 64u * (uint32_t)(warp >> 2);
@@ -569,17 +570,6 @@ kda_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 st_chunk(wb + sw128_chunk_off(64 + r, cq, 128), v);
             }
         }
-        tmem_ld64(tmem + lanes + 128 + cofs, a);
-        if (lane < 16) {  // U row r -> U image (over V), value-column block w/4
-            unsigned char *ub = sm + P_V + (warp >> 2) * 8192;
-#pragma unroll
-            for (int cq = 0; cq < 8; ++cq) {
-                float v[8];
-#pragma unroll
-                for (int e = 0; e < 8; ++e) v[e] = a[cq * 8 + e];
-                st_chunk(ub + sw128_chunk_off(r, cq, 64), v);
-            }
-        }
     }
     fence_async_smem();
     tc_fence_before();
@@ -590,7 +580,7 @@ kda_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         bulk_s2g(blob + BLOB_A1, sm + P_A1, 32768);
         bulk_s2g(blob + BLOB_AQK, sm + P_AQK, 8192);
         bulk_s2g(blob + BLOB_KTT, sm + P_KT, 16384);
-        bulk_s2g(blob + BLOB_U, sm + P_V, 16384);
+        bulk_s2g(blob + BLOB_TB, sm + P_TB, 8192);
         bulk_s2g(blob + BLOB_GAM, sm + P_GAM, 512);
         bulk_commit();
         bulk_wait_read();  // shared memory may be released; the writes complete with the grid
@@ -609,7 +599,8 @@ constexpr int CHAIN_NT = 256;
 
 template <int N>
 __global__ void __launch_bounds__(CHAIN_NT, 1)
-kda_chain_kernel(const unsigned char *__restrict__ ws_blobs, const int32_t *__restrict__ chunk_off,
+kda_chain_kernel(const __grid_constant__ CUtensorMap tm_v,
+                 const unsigned char *__restrict__ ws_blobs, const int32_t *__restrict__ chunk_off,
                  const float *__restrict__ S0, __nv_bfloat16 *__restrict__ o,
                  float *__restrict__ S_T, const int32_t *__restrict__ cu, int64_t T, int H,
                  int nck) {
@@ -639,8 +630,10 @@ kda_chain_kernel(const unsigned char *__restrict__ ws_blobs, const int32_t *__re
         bulk_g2s(st + Lay::A1, blob + BLOB_A1, 32768, &bar_ld[stage]);
         bulk_g2s(st + Lay::A2, blob + BLOB_AQK, 8192, &bar_ld[stage]);
         bulk_g2s(st + Lay::KTT, blob + BLOB_KTT, 16384, &bar_ld[stage]);
-        bulk_g2s(st + Lay::U, blob + BLOB_U + (uint32_t)(j0 / 64) * 8192, Lay::U_BYTES, &bar_ld[stage]);
+        bulk_g2s(st + Lay::TB, blob + BLOB_TB, 8192, &bar_ld[stage]);
         bulk_g2s(st + Lay::GAM, blob + BLOB_GAM, 512, &bar_ld[stage]);
+        tma_load_2d(st + Lay::V, &tm_v, h * D + j0, (int)(span.start + (int64_t)chunk * CH),
+                    &bar_ld[stage]);
     };
 
     if (tid == 0) {
@@ -650,11 +643,6 @@ kda_chain_kernel(const unsigned char *__restrict__ ws_blobs, const int32_t *__re
     if (warp == 0) {
         tmem_alloc(tmem_slot, Lay::TMEM_COLS);
         tmem_relinquish();
-    }
-    // zero rows 64..127 of both A2 stage buffers (A2 = [A_qk; 0])
-    for (int e = tid; e < 2 * 512; e += CHAIN_NT) {
-        const int stage = e >> 9, w16 = e & 511;
-        reinterpret_cast<uint4 *>(sm + stage * Lay::STAGE + Lay::A2 + 8192)[w16] = make_uint4(0, 0, 0, 0);
     }
     const int c = 32 * q4 + lane;    // state row owned by this thread
     const int jh = 32 * hf;          // first of its 32 value columns (inside the slice)
@@ -678,6 +666,7 @@ kda_chain_kernel(const unsigned char *__restrict__ ws_blobs, const int32_t *__re
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     const uint32_t d3 = tmem + 2 * N;  // D1 buffers at columns 0 and N
+    const uint32_t du = tmem + 3 * N;  // U = T Diag(beta) V (rows 64..127)
     const uint32_t sm_base = smem_u32(sm);
     const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
 
@@ -723,23 +712,23 @@ kda_chain_kernel(const unsigned char *__restrict__ ws_blobs, const int32_t *__re
             tc_fence_after();
             mma_run<D>(d1, kmajor(st_base + Lay::A1, 128), mnmajor(sm_base + Lay::SIMG, 16384),
                        idesc_bf16(128, N, 0, 1), false);
+            mma_run<CH>(du, kmajor(st_base + Lay::TB - 8192, 128), mnmajor(st_base + Lay::V, 8192),
+                        idesc_bf16(128, N, 0, 1), false);
             mma_commit(bar_a);
         }
         if (n > 0) store_output(n - 1);
         mbar_wait(bar_a, ph, dead, &g_kda_device_status);
         tc_fence_after();
-        if (q4 >= 2) {  // rows 64..127 of D1 hold (W S)[r]; V_new = U - W S
+        if (q4 >= 2) {  // rows 64..127 hold (W S)[r] in D1 and U[r] in DU; V_new = U - W S
             const int r = c - 64;
-            float ws[32];
+            float ws[32], us[32];
             tmem_ld32(d1 + lane_off + jh, ws);
+            tmem_ld32(du + lane_off + jh, us);
 #pragma unroll
             for (int jc = 0; jc < 4; ++jc) {
-                const uint4 u4 = *reinterpret_cast<const uint4 *>(
-                    st + Lay::U + sw128_chunk_off(r, hf * 4 + jc, 64));
-                const __nv_bfloat16 *ub = reinterpret_cast<const __nv_bfloat16 *>(&u4);
                 float v[8];
 #pragma unroll
-                for (int e = 0; e < 8; ++e) v[e] = __bfloat162float(ub[e]) - ws[jc * 8 + e];
+                for (int e = 0; e < 8; ++e) v[e] = us[jc * 8 + e] - ws[jc * 8 + e];
                 st_chunk(sm + Lay::VIMG + sw128_chunk_off(r, hf * 4 + jc, 64), v);  // row r, MN-major
             }
         }
@@ -880,8 +869,10 @@ cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, const
     err = cudaFuncSetAttribute(kda_chain_kernel<CHAIN_N>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Lay::BYTES);
     if (err != cudaSuccess) return err;
+    CUtensorMap mv;
+    if (n_tok > 0 && !make_map(&mv, v, true, n_tok, H)) return cudaErrorInvalidValue;
     kda_chain_kernel<CHAIN_N><<<dim3((unsigned)nseq, (unsigned)H, D / CHAIN_N), CHAIN_NT, Lay::BYTES, stream>>>(
-        blobs, chunk_off, S0, (__nv_bfloat16 *)o, S_T, cu_seqlens, T, H, nck);
+        mv, blobs, chunk_off, S0, (__nv_bfloat16 *)o, S_T, cu_seqlens, T, H, nck);
     return cudaGetLastError();
 }
 
