@@ -110,8 +110,8 @@ struct ChainLayout {
     static constexpr uint32_t A2 = 32768;             // A_qk (8192); rows 64..127 = start of KTT
     static constexpr uint32_t KTT = 40960;            // 16384 (MN-major K~^T: rows i, channels)
     static constexpr uint32_t TB = 57344;             // 8192: T Diag(beta); the U MMA starts 8192 earlier
-    static constexpr uint32_t V = 65536;              // 8192: value slice, 64 rows x 64 columns (TMA)
-    static constexpr uint32_t GAM = 73728;            // 512
+    static constexpr uint32_t V = 65536;              // value slice: 64 rows x N columns (TMA, 64-column blocks)
+    static constexpr uint32_t GAM = V + N * 128;      // 512
     static constexpr uint32_t STAGE = ((GAM + 512 + 1023) / 1024) * 1024;
     static constexpr uint32_t SIMG = 2 * STAGE;       // S bf16, MN-major: rows c (128), N columns
     static constexpr uint32_t VIMG = SIMG + N * 256;  // V_new bf16, MN-major: rows r (64), N columns
@@ -119,8 +119,15 @@ struct ChainLayout {
     static constexpr uint32_t TMEM = BAR + 48;
     static constexpr uint32_t BYTES = TMEM + 8 + 1024;
     static constexpr uint32_t TMEM_COLS = 4 * N;      // D1 (two buffers), D3, U
-    static constexpr uint32_t LOAD_BYTES = 32768 + 8192 + 16384 + 8192 + 512 + 8192;
+    static constexpr uint32_t LOAD_BYTES = 32768 + 8192 + 16384 + 8192 + 512 + N * 128;
 };
+
+// TMEM load of this thread's lane, N/2 consecutive columns.
+template <int NH>
+__device__ __forceinline__ void tmem_ld_half(uint32_t taddr, float *v) {
+    if constexpr (NH == 32) tmem_ld32(taddr, v);
+    else tmem_ld64(taddr, v);
+}
 
 __device__ __forceinline__ unsigned char *aligned_smem(unsigned char *raw) {
     return reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(raw) + 1023) &
@@ -593,8 +600,9 @@ kda_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 // chain: per (sequence, head, value slice) state recurrence over the chunks
 // =====================================================================================
 // 256 threads. Warp w reads TMEM lane quarter q = w % 4 and handles value columns
-// 32*(w/4) .. +31 of the slice, so every epilogue is split over two warps per quarter.
-// Thread (q, lane, w/4) keeps state row c = 32q + lane, those 32 columns, in registers.
+// (N/2)*(w/4) .. +N/2-1 of the slice, so every epilogue is split over two warps per
+// quarter. Thread (q, lane, w/4) keeps state row c = 32q + lane, those columns, in
+// registers. N = 64 gives two CTAs per (sequence, head), N = 128 one.
 constexpr int CHAIN_NT = 256;
 
 template <int N>
@@ -604,7 +612,8 @@ kda_chain_kernel(const __grid_constant__ CUtensorMap tm_v,
                  const float *__restrict__ S0, __nv_bfloat16 *__restrict__ o,
                  float *__restrict__ S_T, const int32_t *__restrict__ cu, int64_t T, int H,
                  int nck) {
-    static_assert(N == 64, "the chain kernel is written for 64-column value slices");
+    static_assert(N == 64 || N == 128, "value slices of 64 or 128 columns");
+    constexpr int NH = N / 2;  // columns per thread
     using Lay = ChainLayout<N>;
     extern __shared__ unsigned char smem_raw[];
     unsigned char *sm = aligned_smem(smem_raw);
@@ -632,8 +641,10 @@ kda_chain_kernel(const __grid_constant__ CUtensorMap tm_v,
         bulk_g2s(st + Lay::KTT, blob + BLOB_KTT, 16384, &bar_ld[stage]);
         bulk_g2s(st + Lay::TB, blob + BLOB_TB, 8192, &bar_ld[stage]);
         bulk_g2s(st + Lay::GAM, blob + BLOB_GAM, 512, &bar_ld[stage]);
-        tma_load_2d(st + Lay::V, &tm_v, h * D + j0, (int)(span.start + (int64_t)chunk * CH),
-                    &bar_ld[stage]);
+#pragma unroll
+        for (int b = 0; b < N / 64; ++b)
+            tma_load_2d(st + Lay::V + b * 8192, &tm_v, h * D + j0 + 64 * b,
+                        (int)(span.start + (int64_t)chunk * CH), &bar_ld[stage]);
     };
 
     if (tid == 0) {
@@ -645,20 +656,20 @@ kda_chain_kernel(const __grid_constant__ CUtensorMap tm_v,
         tmem_relinquish();
     }
     const int c = 32 * q4 + lane;    // state row owned by this thread
-    const int jh = 32 * hf;          // first of its 32 value columns (inside the slice)
-    float s_reg[32];
+    const int jh = NH * hf;          // first of its NH value columns (inside the slice)
+    float s_reg[NH];
 #pragma unroll
-    for (int j = 0; j < 32; j += 4) {
+    for (int j = 0; j < NH; j += 4) {
         float4 v4 = S0 ? *reinterpret_cast<const float4 *>(S0 + state_off + (int64_t)c * D + j0 + jh + j)
                        : make_float4(0.f, 0.f, 0.f, 0.f);
         s_reg[j] = v4.x; s_reg[j + 1] = v4.y; s_reg[j + 2] = v4.z; s_reg[j + 3] = v4.w;
     }
 #pragma unroll
-    for (int jc = 0; jc < 4; ++jc) {  // row c of the MN-major S image, this thread's 4 chunks
+    for (int jc = 0; jc < NH / 8; ++jc) {  // row c of the MN-major S image, this thread's chunks
         float v[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) v[e] = s_reg[jc * 8 + e];
-        st_chunk(sm + Lay::SIMG + sw128_chunk_off(c, hf * 4 + jc, 128), v);
+        st_chunk(sm + Lay::SIMG + sw128_chunk_off(c, (jh >> 3) + jc, 128), v);
     }
     fence_async_smem();
     tc_fence_before();
@@ -683,13 +694,13 @@ kda_chain_kernel(const __grid_constant__ CUtensorMap tm_v,
             mbar_wait(&bar_c[m & 1], (uint32_t)(m >> 1) & 1u, dead, &g_kda_device_status);
             tc_fence_after();
             const int r = c;
-            float ov[32];
-            tmem_ld32(tmem + (uint32_t)((m & 1) * N) + lane_off + jh, ov);
+            float ov[NH];
+            tmem_ld_half<NH>(tmem + (uint32_t)((m & 1) * N) + lane_off + jh, ov);
             const int64_t tok = span.start + (int64_t)m * CH + r;
             if (r < chunk_rows(span.len, (int64_t)m * CH)) {
                 __nv_bfloat16 *dst = o + (tok * H + h) * (int64_t)D + j0 + jh;
 #pragma unroll
-                for (int j = 0; j < 32; j += 8) {
+                for (int j = 0; j < NH; j += 8) {
                     uint4 pk = make_uint4(pack_bf16x2(ov[j], ov[j + 1]), pack_bf16x2(ov[j + 2], ov[j + 3]),
                                           pack_bf16x2(ov[j + 4], ov[j + 5]), pack_bf16x2(ov[j + 6], ov[j + 7]));
                     *reinterpret_cast<uint4 *>(dst + j) = pk;
@@ -721,15 +732,15 @@ kda_chain_kernel(const __grid_constant__ CUtensorMap tm_v,
         tc_fence_after();
         if (q4 >= 2) {  // rows 64..127 hold (W S)[r] in D1 and U[r] in DU; V_new = U - W S
             const int r = c - 64;
-            float ws[32], us[32];
-            tmem_ld32(d1 + lane_off + jh, ws);
-            tmem_ld32(du + lane_off + jh, us);
+            float ws[NH], us[NH];
+            tmem_ld_half<NH>(d1 + lane_off + jh, ws);
+            tmem_ld_half<NH>(du + lane_off + jh, us);
 #pragma unroll
-            for (int jc = 0; jc < 4; ++jc) {
+            for (int jc = 0; jc < NH / 8; ++jc) {
                 float v[8];
 #pragma unroll
                 for (int e = 0; e < 8; ++e) v[e] = us[jc * 8 + e] - ws[jc * 8 + e];
-                st_chunk(sm + Lay::VIMG + sw128_chunk_off(r, hf * 4 + jc, 64), v);  // row r, MN-major
+                st_chunk(sm + Lay::VIMG + sw128_chunk_off(r, (jh >> 3) + jc, 64), v);  // row r, MN-major
             }
         }
         fence_async_smem();
@@ -748,18 +759,18 @@ kda_chain_kernel(const __grid_constant__ CUtensorMap tm_v,
         {  // S <- Diag(exp(g_L)) S + K~^T V_new
             mbar_wait(bar_b, ph, dead, &g_kda_device_status);
             tc_fence_after();
-            float dv[32];
-            tmem_ld32(d3 + lane_off + jh, dv);
+            float dv[NH];
+            tmem_ld_half<NH>(d3 + lane_off + jh, dv);
             const float gam = reinterpret_cast<const float *>(st + Lay::GAM)[c];
 #pragma unroll
-            for (int jc = 0; jc < 4; ++jc) {
+            for (int jc = 0; jc < NH / 8; ++jc) {
                 float v[8];
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
                     s_reg[jc * 8 + e] = gam * s_reg[jc * 8 + e] + dv[jc * 8 + e];
                     v[e] = s_reg[jc * 8 + e];
                 }
-                st_chunk(sm + Lay::SIMG + sw128_chunk_off(c, hf * 4 + jc, 128), v);
+                st_chunk(sm + Lay::SIMG + sw128_chunk_off(c, (jh >> 3) + jc, 128), v);
             }
         }
         fence_async_smem();
@@ -776,7 +787,7 @@ kda_chain_kernel(const __grid_constant__ CUtensorMap tm_v,
 
     if (S_T) {
 #pragma unroll
-        for (int j = 0; j < 32; j += 4)
+        for (int j = 0; j < NH; j += 4)
             *reinterpret_cast<float4 *>(S_T + state_off + (int64_t)c * D + j0 + jh + j) =
                 make_float4(s_reg[j], s_reg[j + 1], s_reg[j + 2], s_reg[j + 3]);
     }
@@ -818,7 +829,18 @@ bool make_map(CUtensorMap *m, const void *ptr, bool bf16, int64_t n_tok, int H) 
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-constexpr int CHAIN_N = 64;
+template <int N>
+cudaError_t launch_chain(const CUtensorMap &mv, const unsigned char *blobs, const int32_t *chunk_off,
+                         const float *S0, void *o, float *S_T, const int32_t *cu, int64_t T, int H,
+                         int nck, int nseq, cudaStream_t stream) {
+    using Lay = ChainLayout<N>;
+    cudaError_t err = cudaFuncSetAttribute(kda_chain_kernel<N>,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Lay::BYTES);
+    if (err != cudaSuccess) return err;
+    kda_chain_kernel<N><<<dim3((unsigned)nseq, (unsigned)H, D / N), CHAIN_NT, Lay::BYTES, stream>>>(
+        mv, blobs, chunk_off, S0, (__nv_bfloat16 *)o, S_T, cu, T, H, nck);
+    return cudaGetLastError();
+}
 
 }  // namespace
 
@@ -865,15 +887,15 @@ cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, const
         err = cudaGetLastError();
         if (err != cudaSuccess) return err;
     }
-    using Lay = ChainLayout<CHAIN_N>;
-    err = cudaFuncSetAttribute(kda_chain_kernel<CHAIN_N>,
-                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Lay::BYTES);
-    if (err != cudaSuccess) return err;
     CUtensorMap mv;
     if (n_tok > 0 && !make_map(&mv, v, true, n_tok, H)) return cudaErrorInvalidValue;
-    kda_chain_kernel<CHAIN_N><<<dim3((unsigned)nseq, (unsigned)H, D / CHAIN_N), CHAIN_NT, Lay::BYTES, stream>>>(
-        mv, blobs, chunk_off, S0, (__nv_bfloat16 *)o, S_T, cu_seqlens, T, H, nck);
-    return cudaGetLastError();
+    // 128-column slices (one CTA per sequence-head) when there are enough pairs to fill
+    // the GPU; otherwise 64-column slices for twice the parallelism.
+    int dev = 0, n_sm = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess)
+        cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
+    if ((int64_t)nseq * H >= n_sm) return launch_chain<128>(mv, blobs, chunk_off, S0, o, S_T, cu_seqlens, T, H, nck, nseq, stream);
+    return launch_chain<64>(mv, blobs, chunk_off, S0, o, S_T, cu_seqlens, T, H, nck, nseq, stream);
 }
 
 int read_device_status(int *status) {

@@ -216,6 +216,15 @@ def test_long_context_1m_tokens_as_16_calls_sampled():
     assert torch.isfinite(S).all()
 
 
+def test_many_sequence_heads_take_full_width_chain():
+    """B*H >= the SM count selects one 128-column chain CTA per (sequence, head)."""
+    inp = prefill_inputs(B=2, T=130, H=80, dtype=torch.bfloat16, s0_std=0.1, seed=22, device=DEV)
+    o, st = run(inp)
+    ro, rs = ref(inp)
+    check(o, ro, "bf16", "128-column chain o")
+    check(st, rs, "bf16", "128-column chain S_T")
+
+
 def test_no_bounded_wait_timed_out():
     """Every tensor-core kernel run so far finished without a wait giving up."""
     import ctypes
