@@ -38,6 +38,8 @@
 // exponentials, on CUDA cores.
 #include <cudaTypedefs.h>
 
+#include <type_traits>
+
 #include "kda_internal.cuh"
 #include "tc_ptx.cuh"
 
@@ -246,7 +248,7 @@ kda_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     const uint32_t sm_base = smem_u32(sm);
-    mbar_wait(bar_tma, 0, dead, &g_kda_device_status);
+    cta_wait(bar_tma, 0, dead, &g_kda_device_status);
 
     // ---- g = chunk-local cumulative sum of log_alpha (rows >= L count as 0), in place.
     //      Thread t: channel c = t % 128, rows 32*(t/128) .. +31, summed in registers.
@@ -294,43 +296,60 @@ kda_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     }
     // log_alpha/g tile fully read: its space becomes KT | KINV
     const int n_bad = __syncthreads_or(any_bad) ? 1 : 0;
+    // One pass over this thread's 8 rows. BAD selects the exact handling of key
+    // channels whose chunk log-decay exceeds SAFE_SPAN (kept out of the unrolled
+    // common path so that it stays branch-free).
+    auto gate_rows = [&](auto bad_tag) {
+        constexpr bool BAD = decltype(bad_tag)::value;
 #pragma unroll
-    for (int v8 = 0; v8 < 8; ++v8) {
-        const int r = warp + 8 * v8;
-        const bool live = r < L;
-        const __nv_bfloat16 *qb = reinterpret_cast<const __nv_bfloat16 *>(&qraw[v8]);
-        const __nv_bfloat16 *kb = reinterpret_cast<const __nv_bfloat16 *>(&kraw[v8]);
-        const float gs[4] = {graw[v8].x, graw[v8].y, graw[v8].z, graw[v8].w};
-        float qe[4], ke[4], kin[4], kt[4];
+        for (int v8 = 0; v8 < 8; ++v8) {
+            const int r = warp + 8 * v8;
+            const bool live = r < L;
+            const __nv_bfloat16 *qb = reinterpret_cast<const __nv_bfloat16 *>(&qraw[v8]);
+            const __nv_bfloat16 *kb = reinterpret_cast<const __nv_bfloat16 *>(&kraw[v8]);
+            const float gs[4] = {graw[v8].x, graw[v8].y, graw[v8].z, graw[v8].w};
+            float qe[4], ke[4], kin[4], kt[4];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const float x = live ? __bfloat162float(qb[e]) : 0.f;
-            const float kk = live ? __bfloat162float(kb[e]) : 0.f;
-            const float eg = __expf(gs[e]);
-            qe[e] = x * eg;
-            ke[e] = kk * eg;
-            if (!n_bad || !badc[e]) {  // exp(-g) <= exp(80): finite; exp(g_L - g) = exp(g_L) exp(-g)
-                const float kin_ = kk * __expf(-gs[e]);
-                kin[e] = kin_;
-                kt[e] = kin_ * gams[e];
-            } else {
-                kin[e] = 0.f;
-                kt[e] = kk * __expf(gls[e] - gs[e]);
+            for (int e = 0; e < 4; ++e) {
+                const float x = live ? __bfloat162float(qb[e]) : 0.f;
+                const float kk = live ? __bfloat162float(kb[e]) : 0.f;
+                const float eg = __expf(gs[e]);
+                qe[e] = x * eg;
+                ke[e] = kk * eg;
+                const float kin_ = kk * __expf(-gs[e]);  // exp(-g) <= exp(80) for good channels
+                if constexpr (BAD) {
+                    kin[e] = badc[e] ? 0.f : kin_;
+                    kt[e] = badc[e] ? kk * __expf(gls[e] - gs[e]) : kin_ * gams[e];
+                } else {
+                    kin[e] = kin_;
+                    kt[e] = kin_ * gams[e];  // exp(g_L - g) = exp(g_L) exp(-g)
+                }
             }
+            unsigned char *blk = sm + P_A1 + fblk * 16384;
+            *reinterpret_cast<uint2 *>(blk + sw128_chunk_off(r, fchunk, 128) + fhalf) =
+                make_uint2(pack_bf16x2(qe[0], qe[1]), pack_bf16x2(qe[2], qe[3]));
+            *reinterpret_cast<uint2 *>(blk + sw128_chunk_off(64 + r, fchunk, 128) + fhalf) =
+                make_uint2(pack_bf16x2(ke[0], ke[1]), pack_bf16x2(ke[2], ke[3]));
+            *reinterpret_cast<uint2 *>(sm + P_KT + fblk * 8192 + sw128_chunk_off(r, fchunk, 64) + fhalf) =
+                make_uint2(pack_bf16x2(kt[0], kt[1]), pack_bf16x2(kt[2], kt[3]));
+            *reinterpret_cast<uint2 *>(sm + P_KINV + fblk * 8192 + sw128_chunk_off(r, fchunk, 64) + fhalf) =
+                make_uint2(pack_bf16x2(kin[0], kin[1]), pack_bf16x2(kin[2], kin[3]));
         }
-        unsigned char *blk = sm + P_A1 + fblk * 16384;
-        *reinterpret_cast<uint2 *>(blk + sw128_chunk_off(r, fchunk, 128) + fhalf) =
-            make_uint2(pack_bf16x2(qe[0], qe[1]), pack_bf16x2(qe[2], qe[3]));
-        *reinterpret_cast<uint2 *>(blk + sw128_chunk_off(64 + r, fchunk, 128) + fhalf) =
-            make_uint2(pack_bf16x2(ke[0], ke[1]), pack_bf16x2(ke[2], ke[3]));
-        *reinterpret_cast<uint2 *>(sm + P_KT + fblk * 8192 + sw128_chunk_off(r, fchunk, 64) + fhalf) =
-            make_uint2(pack_bf16x2(kt[0], kt[1]), pack_bf16x2(kt[2], kt[3]));
-        *reinterpret_cast<uint2 *>(sm + P_KINV + fblk * 8192 + sw128_chunk_off(r, fchunk, 64) + fhalf) =
-            make_uint2(pack_bf16x2(kin[0], kin[1]), pack_bf16x2(kin[2], kin[3]));
-    }
+    };
+    if (n_bad) gate_rows(std::true_type{});
+    else gate_rows(std::false_type{});
     fence_async_smem();
     tc_fence_before();
     __syncthreads();
+
+    // Each blob image is stored as soon as it is final (bulk copies drain while the CTA
+    // keeps computing); K~ and exp(g_L) are final now.
+    unsigned char *blob = ws_blobs + ((size_t)slot * H + h) * BLOB_BYTES;
+    if (tid == 0) {
+        bulk_s2g(blob + BLOB_KTT, sm + P_KT, 16384);
+        bulk_s2g(blob + BLOB_GAM, sm + P_GAM, 512);
+        bulk_commit();
+    }
 
     // ---- Gram MMA: D[m][i] = sum_c A1[m][c] KINV[i][c]; rows 0..63 Q-rows, 64..127 K-rows
     if (tid == 0) {
@@ -395,7 +414,7 @@ kda_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         }
     }
 
-    mbar_wait(bar_mma, 0, dead, &g_kda_device_status);
+    cta_wait(bar_mma, 0, dead, &g_kda_device_status);
     tc_fence_after();
     {
         float G[32];
@@ -427,7 +446,12 @@ kda_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             }
         }
     }
+    fence_async_smem();
     __syncthreads();
+    if (tid == 0) {  // A_qk is final
+        bulk_s2g(blob + BLOB_AQK, sm + P_AQK, 8192);
+        bulk_commit();
+    }
 
     // ---- T = (I + A_kk)^-1 in place, by blocks: invert the four 16 x 16 diagonal
     //      blocks, then merge 16 -> 32 -> 64 with [[X, 0], [Y, Z]]^-1 =
@@ -462,68 +486,36 @@ kda_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             }
         }
         __syncthreads();
-        // level 1: blocks (16..31, 0..15) and (48..63, 32..47); thread -> 1 x 2 tile
-        const int l1b = tid >> 7, l1a = (tid >> 3) & 15, l1c = (tid & 7) * 2, l1o = 32 * l1b;
-        {  // P = A_lo-hi-block X^-1
-            float2 acc = make_float2(0.f, 0.f);
-#pragma unroll
-            for (int m4 = 0; m4 < 16; m4 += 4) {
-                const float4 a4 = *reinterpret_cast<const float4 *>(at + (l1o + 16 + l1a) * LDT + l1o + m4);
-                const float av[4] = {a4.x, a4.y, a4.z, a4.w};
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const float2 b2 = *reinterpret_cast<const float2 *>(at + (l1o + m4 + u) * LDT + l1o + l1c);
-                    acc.x += av[u] * b2.x; acc.y += av[u] * b2.y;
-                }
-            }
-            *reinterpret_cast<float2 *>(pb + (l1b * 16 + l1a) * 20 + l1c) = acc;
+        // Merges, as 16 x 8 warp-level tf32 MMA tiles.
+        // level 1: blocks (16..31, 0..15) and (48..63, 32..47); warps 0-3 take one 16 x 8
+        // tile each (block w/2, columns 8*(w%2) ..).
+        if (warp < 4) {  // P = A[o+16.., o..o+15] X^-1
+            const int o = 32 * (warp >> 1), n0 = 8 * (warp & 1);
+            float d[4] = {0.f, 0.f, 0.f, 0.f};
+            warp_gemm_16x8<16>(d, at + (o + 16) * LDT + o, LDT, at + o * LDT + o + n0, LDT);
+            warp_store_16x8(d, pb + (warp >> 1) * 16 * 20 + n0, 20, 1.f);
         }
         __syncthreads();
-        {  // T = -Z^-1 P
-            float2 acc = make_float2(0.f, 0.f);
-#pragma unroll
-            for (int m4 = 0; m4 < 16; m4 += 4) {
-                const float4 d4 = *reinterpret_cast<const float4 *>(at + (l1o + 16 + l1a) * LDT + l1o + 16 + m4);
-                const float dv[4] = {d4.x, d4.y, d4.z, d4.w};
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const float2 p2 = *reinterpret_cast<const float2 *>(pb + (l1b * 16 + m4 + u) * 20 + l1c);
-                    acc.x += dv[u] * p2.x; acc.y += dv[u] * p2.y;
-                }
-            }
-            *reinterpret_cast<float2 *>(at + (l1o + 16 + l1a) * LDT + l1o + l1c) = make_float2(-acc.x, -acc.y);
+        if (warp < 4) {  // T = -Z^-1 P
+            const int o = 32 * (warp >> 1), n0 = 8 * (warp & 1);
+            float d[4] = {0.f, 0.f, 0.f, 0.f};
+            warp_gemm_16x8<16>(d, at + (o + 16) * LDT + o + 16, LDT, pb + (warp >> 1) * 16 * 20 + n0, 20);
+            warp_store_16x8(d, at + (o + 16) * LDT + o + n0, LDT, -1.f);
         }
         __syncthreads();
-        // level 2: block (32..63, 0..31); thread -> 1 x 4 tile of the 32 x 32 block
-        const int l2a = tid >> 3, l2c = (tid & 7) * 4;
+        // level 2: block (32..63, 0..31); warp w takes the 16 x 8 tile (rows 16*(w/4), cols 8*(w%4)).
         {  // Q = A[32.., 0..31] T[0..31, 0..31]
-            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-            for (int m4 = 0; m4 < 32; m4 += 4) {
-                const float4 a4 = *reinterpret_cast<const float4 *>(at + (32 + l2a) * LDT + m4);
-                const float av[4] = {a4.x, a4.y, a4.z, a4.w};
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const float4 b4 = *reinterpret_cast<const float4 *>(at + (m4 + u) * LDT + l2c);
-                    acc.x += av[u] * b4.x; acc.y += av[u] * b4.y; acc.z += av[u] * b4.z; acc.w += av[u] * b4.w;
-                }
-            }
-            *reinterpret_cast<float4 *>(qb + l2a * 36 + l2c) = acc;
+            const int m0 = 16 * (warp >> 2), n0 = 8 * (warp & 3);
+            float d[4] = {0.f, 0.f, 0.f, 0.f};
+            warp_gemm_16x8<32>(d, at + (32 + m0) * LDT, LDT, at + n0, LDT);
+            warp_store_16x8(d, qb + m0 * 36 + n0, 36, 1.f);
         }
         __syncthreads();
         {  // T[32.., 0..31] = -T[32.., 32..] Q
-            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-            for (int m4 = 0; m4 < 32; m4 += 4) {
-                const float4 d4 = *reinterpret_cast<const float4 *>(at + (32 + l2a) * LDT + 32 + m4);
-                const float dv[4] = {d4.x, d4.y, d4.z, d4.w};
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const float4 p4 = *reinterpret_cast<const float4 *>(qb + (m4 + u) * 36 + l2c);
-                    acc.x += dv[u] * p4.x; acc.y += dv[u] * p4.y; acc.z += dv[u] * p4.z; acc.w += dv[u] * p4.w;
-                }
-            }
-            *reinterpret_cast<float4 *>(at + (32 + l2a) * LDT + l2c) = make_float4(-acc.x, -acc.y, -acc.z, -acc.w);
+            const int m0 = 16 * (warp >> 2), n0 = 8 * (warp & 3);
+            float d[4] = {0.f, 0.f, 0.f, 0.f};
+            warp_gemm_16x8<32>(d, at + (32 + m0) * LDT + 32, LDT, qb + n0, 36);
+            warp_store_16x8(d, at + (32 + m0) * LDT + n0, LDT, -1.f);
         }
         __syncthreads();
         // image of T Diag(beta): rows r, columns i, zero above the diagonal
@@ -553,11 +545,13 @@ kda_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     //      read here as an MN-major B (K = token i). (U = T Diag(beta) V is formed by the
     //      chain kernel from the blob's T Diag(beta) and its own slice of V.)
     if (tid == 0) {
+        bulk_s2g(blob + BLOB_TB, sm + P_TB, 8192);  // T Diag(beta) is final
+        bulk_commit();
         tc_fence_after();
         mma_run<CH>(tmem, kmajor(sm_base + P_TB, 64), mnmajor(sm_base + P_A1 + 8192, 16384), idesc_bf16(64, 128, 0, 1), false);
         mma_commit(bar_mma);
     }
-    mbar_wait(bar_mma, 1, dead, &g_kda_device_status);
+    cta_wait(bar_mma, 1, dead, &g_kda_device_status);
     tc_fence_after();
     {
         // M = 64 accumulator: row r sits in lane 16*(w%4) + (lane < 16) of quarter w%4.
@@ -583,12 +577,7 @@ kda_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     __syncthreads();
 
     if (tid == 0) {
-        unsigned char *blob = ws_blobs + ((size_t)slot * H + h) * BLOB_BYTES;
         bulk_s2g(blob + BLOB_A1, sm + P_A1, 32768);
-        bulk_s2g(blob + BLOB_AQK, sm + P_AQK, 8192);
-        bulk_s2g(blob + BLOB_KTT, sm + P_KT, 16384);
-        bulk_s2g(blob + BLOB_TB, sm + P_TB, 8192);
-        bulk_s2g(blob + BLOB_GAM, sm + P_GAM, 512);
         bulk_commit();
         bulk_wait_read();  // shared memory may be released; the writes complete with the grid
     }

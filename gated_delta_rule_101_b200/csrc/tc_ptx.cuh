@@ -68,6 +68,15 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, bool &
     return false;
 }
 
+// CTA-wide wait: thread 0 polls the barrier while every other thread sleeps at
+// the CTA barrier (polling threads would take issue slots from co-resident
+// CTAs). All threads leave with the same `dead` value.
+__device__ __forceinline__ void cta_wait(uint64_t *bar, uint32_t parity, bool &dead, int *status) {
+    bool ok = true;
+    if (threadIdx.x == 0) ok = mbar_wait(bar, parity, dead, status);
+    dead = __syncthreads_or(!ok || dead) != 0;
+}
+
 // ------------------------------------------------------------------ async proxy / TMA
 __device__ __forceinline__ void fence_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -177,6 +186,48 @@ __device__ __forceinline__ void tmem_ld64(uint32_t taddr, float *v) {
         : "memory");
 #pragma unroll
     for (int i = 0; i < 64; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// ------------------------------------------------------------------ warp-level MMA
+// D (16x8, fp32) += A (16x8) * B (8x8), tf32 inputs. Used only for the 16- and
+// 32-wide block products inside the 64 x 64 triangular inverse, which are far
+// below tcgen05's 64-row minimum. Fragments (g = lane / 4, t = lane % 4):
+//   A: a0 (g, t), a1 (g+8, t), a2 (g, t+4), a3 (g+8, t+4)
+//   B: b0 (t, g), b1 (t+4, g)
+//   D: d0 (g, 2t), d1 (g, 2t+1), d2 (g+8, 2t), d3 (g+8, 2t+1)
+__device__ __forceinline__ uint32_t to_tf32(float x) {
+    uint32_t r;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+    return r;
+}
+__device__ __forceinline__ void mma_tf32_16x8x8(float (&d)[4], const uint32_t (&a)[4], const uint32_t (&b)[2]) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+        "{%8, %9}, {%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+// One 16 x 8 tile of D = A * B over K (multiple of 8), with A and B read from
+// shared memory: A(i, k) = a[i * lda + k], B(k, j) = b[k * ldb + j].
+template <int K>
+__device__ __forceinline__ void warp_gemm_16x8(float (&d)[4], const float *a, int lda, const float *b,
+                                               int ldb) {
+    const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+#pragma unroll
+    for (int k0 = 0; k0 < K; k0 += 8) {
+        const uint32_t af[4] = {to_tf32(a[g * lda + k0 + t]), to_tf32(a[(g + 8) * lda + k0 + t]),
+                                to_tf32(a[g * lda + k0 + t + 4]), to_tf32(a[(g + 8) * lda + k0 + t + 4])};
+        const uint32_t bf[2] = {to_tf32(b[(k0 + t) * ldb + g]), to_tf32(b[(k0 + t + 4) * ldb + g])};
+        mma_tf32_16x8x8(d, af, bf);
+    }
+}
+// Stores a D tile (scaled by s) to c[i * ldc + j].
+__device__ __forceinline__ void warp_store_16x8(const float (&d)[4], float *c, int ldc, float s) {
+    const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+    c[g * ldc + 2 * t] = s * d[0];
+    c[g * ldc + 2 * t + 1] = s * d[1];
+    c[(g + 8) * ldc + 2 * t] = s * d[2];
+    c[(g + 8) * ldc + 2 * t + 1] = s * d[3];
 }
 
 // ------------------------------------------------------------------ operand layouts
