@@ -65,38 +65,41 @@ constexpr uint32_t BLOB_BYTES = 66048;
 
 // ---- prep kernel shared memory (offsets from a 1024-byte aligned base). Every
 // operand image is a 128-byte-swizzled tile of 128-byte rows (see tc_ptx.cuh).
+// The layout keeps a CTA under 68 KB so that three run on each SM.
 //   A1   K-major, rows r' = 0..127, K = key channel c (two 64-channel blocks of 16 KiB).
 //        TMA puts q in rows 0..63 and k in rows 64..127; they are scaled in place
 //        to Q e^g and K e^g. Rows 64..127 are later replaced by W.
-//   V    rows = token i, two 64-column blocks (TMA); later overwritten by U.
-//   LAG  log_alpha [64][128] fp32 (TMA, unswizzled), turned into g in place;
-//        after the gates are built it holds KT and KINV:
 //   KT   rows = token i, two 64-channel blocks: (exp(g_L - g) K)[i][c]. The chain's
-//        MN-major A operand K~^T.
+//        MN-major A operand K~^T. Stored to the blob as soon as it is built.
 //   KINV rows = token i, two 64-channel blocks: (K e^-g)[i][c]; the Gram's K-major B.
-//   AKK  64 x 68 fp32 (rows padded to 68 floats): A_kk, then T in place; over KINV.
+// Once the Gram MMA has completed and K~ has been stored, the 32 KiB of KT | KINV
+// take A_kk / T (fp32, rows padded to LDT floats), the solve's scratch and the
+// A_qk image, whose space then takes the T Diag(beta) image.
 constexpr int PREP_NT = 256;
 constexpr uint32_t P_A1 = 0;          // 32768
-constexpr uint32_t P_V = 32768;       // 16384 (unused)
-constexpr uint32_t P_LAG = 49152;     // 32768 (log_alpha -> g), then KT | KINV
-constexpr uint32_t P_KT = 49152;      // 16384
-constexpr uint32_t P_KINV = 65536;    // 16384 (dead after the Gram MMA)
-constexpr uint32_t P_AKK = 65536;     // 64 x 68 fp32: A_kk / T (after the Gram MMA)
-constexpr uint32_t P_PBUF = 82944;    // 16 x 48 fp32 solve scratch
-constexpr uint32_t P_AQK = 86016;     // 8192: A_qk image, rows r, columns i
-constexpr uint32_t P_TB = 94208;      // 8192: T Diag(beta) image, rows r, columns i
-constexpr uint32_t P_BADB = 86016;    // 8 x 3 x 64 fp32 bad-channel batch (before A_qk / T exist)
-constexpr uint32_t P_GAM = 102400;    // 128 fp32: exp(g_L)
-constexpr uint32_t P_GL = 102912;     // 128 fp32: g_L
-constexpr uint32_t P_TOT = 103424;    // 128 fp32: first-half log-decay totals
-constexpr uint32_t P_BETA = 103936;   // 64 fp32
-constexpr uint32_t P_BADL = 104192;   // 128 int
-constexpr uint32_t P_BAR = 104704;    // 2 mbarriers
-constexpr uint32_t P_TMEM = 104720;
-constexpr uint32_t P_NBAD = 104724;   // number of listed bad channels
-constexpr uint32_t PREP_SMEM = 104736 + 1024;
-constexpr uint32_t PREP_TMEM_COLS = 256;  // Gram 64 (then W 128) | U 128
-constexpr uint32_t PREP_TMA_BYTES = 32768 + 32768;  // q, k | log_alpha
+constexpr uint32_t P_KT = 32768;      // 16384
+constexpr uint32_t P_KINV = 49152;    // 16384 (dead after the Gram MMA)
+constexpr uint32_t P_GTOT = 49152;    // 8 x 128 fp32 per-warp log-decay totals (before KINV)
+constexpr uint32_t P_BADB = 49152;    // 8 x 3 x 64 fp32 bad-channel batch (after the Gram MMA)
+constexpr uint32_t P_AKK = 32768;     // 64 x 68 fp32 (17408): A_kk, then T in place
+constexpr uint32_t P_PBUF = 50176;    // 4608: solve scratch (2 x [16][20], then [32][36])
+constexpr uint32_t P_AQK = 55296;     // 8192: A_qk image, rows r, columns i
+constexpr uint32_t P_TB = 55296;      // 8192: T Diag(beta) image (after A_qk has been stored)
+constexpr uint32_t P_GAM = 65536;     // 128 fp32: exp(g_L)
+constexpr uint32_t P_GL = 66048;      // 128 fp32: g_L
+constexpr uint32_t P_BETA = 66560;    // 64 fp32
+constexpr uint32_t P_BADL = 66816;    // 128 int
+constexpr uint32_t P_BAR = 67328;     // 2 mbarriers
+constexpr uint32_t P_TMEM = 67344;
+constexpr uint32_t P_NBAD = 67348;    // number of listed bad channels
+constexpr uint32_t PREP_SMEM = 67352 + 1024;
+constexpr uint32_t PREP_TMEM_COLS = 128;  // Gram 64, then W 128
+constexpr uint32_t PREP_TMA_BYTES = 32768;  // q, k
+static_assert(P_AKK + 64 * 68 * 4 <= P_PBUF && P_PBUF + 4608 <= P_AQK && P_AQK + 8192 <= P_GAM,
+              "prep layout: A_kk, scratch and A_qk must fit in KT | KINV");
+static_assert(P_GTOT + 8 * 128 * 4 <= P_KINV + 16384 && P_BADB + 8 * 3 * 64 * 4 <= P_AQK + 8192,
+              "prep layout: scratch regions");
+static_assert(3 * (PREP_SMEM + 1024) <= 233472, "three prep CTAs per SM");
 
 // A_kk / T rows are padded to 68 floats: float4 row segments stay aligned, and
 // 8 consecutive rows at the same column fall on distinct bank quads.
@@ -197,9 +200,8 @@ __device__ __forceinline__ void ld_chunk(const unsigned char *p, float (&v)[8]) 
     for (int e = 0; e < 8; ++e) v[e] = __bfloat162float(b[e]);
 }
 
-__global__ void __launch_bounds__(PREP_NT, 2)
+__global__ void __launch_bounds__(PREP_NT, 3)
 kda_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_la,
                 const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
                 const float *__restrict__ log_alpha, const float *__restrict__ beta,
                 unsigned char *__restrict__ ws_blobs, const int32_t *__restrict__ chunk_off,
@@ -220,9 +222,7 @@ kda_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + P_TMEM);
     float *sgam = reinterpret_cast<float *>(sm + P_GAM);
     float *sgl = reinterpret_cast<float *>(sm + P_GL);
-    float *stot = reinterpret_cast<float *>(sm + P_TOT);
     float *sbeta = reinterpret_cast<float *>(sm + P_BETA);
-    float *lag = reinterpret_cast<float *>(sm + P_LAG);
     int *badl = reinterpret_cast<int *>(sm + P_BADL);
     bool dead = false;
 
@@ -236,78 +236,84 @@ kda_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         tma_load_2d(sm + P_A1 + 16384, &tm_q, x + 64, y, bar_tma);     // q, channels 64..127
         tma_load_2d(sm + P_A1 + 8192, &tm_k, x, y, bar_tma);           // k -> rows 64..127
         tma_load_2d(sm + P_A1 + 16384 + 8192, &tm_k, x + 64, y, bar_tma);
-        tma_load_2d(sm + P_LAG, &tm_la, x, y, bar_tma);
     }
     if (warp == 0) {
         tmem_alloc(tmem_slot, PREP_TMEM_COLS);
         tmem_relinquish();
     }
     if (tid < CH) sbeta[tid] = tid < L ? beta[(tok0 + tid) * H + h] : 0.f;
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem = *tmem_slot;
-    const uint32_t sm_base = smem_u32(sm);
-    cta_wait(bar_tma, 0, dead, &g_kda_device_status);
+    tc_fence_before();  // the TMEM address is read after the next CTA barrier
 
-    // ---- g = chunk-local cumulative sum of log_alpha (rows >= L count as 0), in place.
-    //      Thread t: channel c = t % 128, rows 32*(t/128) .. +31, summed in registers.
+    // ---- g = chunk-local cumulative sum of log_alpha (rows >= L count as 0), while
+    //      the q / k tiles are in flight. Thread (w, f) loads rows 8w .. 8w+7, channels
+    //      4f .. 4f+3 straight into registers, sums down its rows, and adds the totals
+    //      of the warps before it; g_L is the sum of all eight totals.
+    const int f = lane, fblk = f >> 4, fchunk = (f & 15) >> 1, fhalf = (f & 1) * 8;
+    float4 g4[8];
+    float gls[4], gams[4];
     {
-        const int c = tid & (D - 1), half = tid >> 7, r0 = half * 32;
-        float gg[32];
+        const float *la = log_alpha + (tok0 * H + h) * (int64_t)D + 4 * f;
 #pragma unroll
-        for (int e = 0; e < 32; ++e) gg[e] = (r0 + e) < L ? lag[(r0 + e) * D + c] : 0.f;
+        for (int v = 0; v < 8; ++v) {
+            const int r = 8 * warp + v;
+            g4[v] = r < L ? __ldcs(reinterpret_cast<const float4 *>(la + (int64_t)r * H * D))
+                          : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
 #pragma unroll
-        for (int e = 1; e < 32; ++e) gg[e] += gg[e - 1];
-        if (half == 0) stot[c] = gg[31];
+        for (int v = 1; v < 8; ++v) {
+            g4[v].x += g4[v - 1].x; g4[v].y += g4[v - 1].y;
+            g4[v].z += g4[v - 1].z; g4[v].w += g4[v - 1].w;
+        }
+        float *gtot = reinterpret_cast<float *>(sm + P_GTOT);
+        *reinterpret_cast<float4 *>(gtot + warp * D + 4 * f) = g4[7];
         __syncthreads();
-        const float off = half ? stot[c] : 0.f;
+        float4 off = make_float4(0.f, 0.f, 0.f, 0.f), tot = off;
 #pragma unroll
-        for (int e = 0; e < 32; ++e) lag[(r0 + e) * D + c] = gg[e] + off;
-        if (half == 1) {
-            sgl[c] = gg[31] + off;
-            sgam[c] = expf(gg[31] + off);
+        for (int w2 = 0; w2 < 8; ++w2) {
+            const float4 t = *reinterpret_cast<const float4 *>(gtot + w2 * D + 4 * f);
+            if (w2 < warp) { off.x += t.x; off.y += t.y; off.z += t.z; off.w += t.w; }
+            tot.x += t.x; tot.y += t.y; tot.z += t.z; tot.w += t.w;
+        }
+#pragma unroll
+        for (int v = 0; v < 8; ++v) {
+            g4[v].x += off.x; g4[v].y += off.y; g4[v].z += off.z; g4[v].w += off.w;
+        }
+        gls[0] = tot.x; gls[1] = tot.y; gls[2] = tot.z; gls[3] = tot.w;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) gams[e] = expf(gls[e]);
+        if (warp == 0) {
+            *reinterpret_cast<float4 *>(sgl + 4 * f) = tot;
+            *reinterpret_cast<float4 *>(sgam + 4 * f) = make_float4(gams[0], gams[1], gams[2], gams[3]);
         }
     }
-    __syncthreads();
-
-    // ---- gates and operand images. Warp w handles rows r = w + 8v; lane f handles
-    //      channels 4f .. 4f+3 (8-byte pieces of the swizzled rows). Read all, sync, write.
-    const int f = lane, fblk = f >> 4, fchunk = (f & 15) >> 1, fhalf = (f & 1) * 8;
-    uint2 qraw[8], kraw[8];
-    float4 graw[8];
-#pragma unroll
-    for (int v8 = 0; v8 < 8; ++v8) {
-        const int r = warp + 8 * v8;
-        const unsigned char *blk = sm + P_A1 + fblk * 16384;
-        qraw[v8] = *reinterpret_cast<const uint2 *>(blk + sw128_chunk_off(r, fchunk, 128) + fhalf);
-        kraw[v8] = *reinterpret_cast<const uint2 *>(blk + sw128_chunk_off(64 + r, fchunk, 128) + fhalf);
-        graw[v8] = *reinterpret_cast<const float4 *>(lag + r * D + 4 * f);
-    }
-    const float4 gl4 = *reinterpret_cast<const float4 *>(sgl + 4 * f);
-    const float gls[4] = {gl4.x, gl4.y, gl4.z, gl4.w};
-    const float4 ga4 = *reinterpret_cast<const float4 *>(sgam + 4 * f);
-    const float gams[4] = {ga4.x, ga4.y, ga4.z, ga4.w};
     bool badc[4], any_bad = false;
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
         badc[e] = -gls[e] > SAFE_SPAN;
         any_bad |= badc[e];
     }
-    // log_alpha/g tile fully read: its space becomes KT | KINV
+    // (this barrier also ends the reads of the warp totals, whose space becomes KINV)
     const int n_bad = __syncthreads_or(any_bad) ? 1 : 0;
-    // One pass over this thread's 8 rows. BAD selects the exact handling of key
-    // channels whose chunk log-decay exceeds SAFE_SPAN (kept out of the unrolled
-    // common path so that it stays branch-free).
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t sm_base = smem_u32(sm);
+    cta_wait(bar_tma, 0, dead, &g_kda_device_status);
+
+    // ---- gates and operand images, row by row. BAD selects the exact handling of key
+    //      channels whose chunk log-decay exceeds SAFE_SPAN (kept out of the unrolled
+    //      common path so that it stays branch-free).
     auto gate_rows = [&](auto bad_tag) {
         constexpr bool BAD = decltype(bad_tag)::value;
+        unsigned char *blk = sm + P_A1 + fblk * 16384;
 #pragma unroll
-        for (int v8 = 0; v8 < 8; ++v8) {
-            const int r = warp + 8 * v8;
+        for (int v = 0; v < 8; ++v) {
+            const int r = 8 * warp + v;
             const bool live = r < L;
-            const __nv_bfloat16 *qb = reinterpret_cast<const __nv_bfloat16 *>(&qraw[v8]);
-            const __nv_bfloat16 *kb = reinterpret_cast<const __nv_bfloat16 *>(&kraw[v8]);
-            const float gs[4] = {graw[v8].x, graw[v8].y, graw[v8].z, graw[v8].w};
+            const uint2 qraw = *reinterpret_cast<const uint2 *>(blk + sw128_chunk_off(r, fchunk, 128) + fhalf);
+            const uint2 kraw = *reinterpret_cast<const uint2 *>(blk + sw128_chunk_off(64 + r, fchunk, 128) + fhalf);
+            const __nv_bfloat16 *qb = reinterpret_cast<const __nv_bfloat16 *>(&qraw);
+            const __nv_bfloat16 *kb = reinterpret_cast<const __nv_bfloat16 *>(&kraw);
+            const float gs[4] = {g4[v].x, g4[v].y, g4[v].z, g4[v].w};
             float qe[4], ke[4], kin[4], kt[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
@@ -325,7 +331,6 @@ kda_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     kt[e] = kin_ * gams[e];  // exp(g_L - g) = exp(g_L) exp(-g)
                 }
             }
-            unsigned char *blk = sm + P_A1 + fblk * 16384;
             *reinterpret_cast<uint2 *>(blk + sw128_chunk_off(r, fchunk, 128) + fhalf) =
                 make_uint2(pack_bf16x2(qe[0], qe[1]), pack_bf16x2(qe[2], qe[3]));
             *reinterpret_cast<uint2 *>(blk + sw128_chunk_off(64 + r, fchunk, 128) + fhalf) =
@@ -343,11 +348,13 @@ kda_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     __syncthreads();
 
     // Each blob image is stored as soon as it is final (bulk copies drain while the CTA
-    // keeps computing); K~ and exp(g_L) are final now.
+    // keeps computing): K~, exp(g_L) and the Q~ rows of A1 are final now.
     unsigned char *blob = ws_blobs + ((size_t)slot * H + h) * BLOB_BYTES;
     if (tid == 0) {
         bulk_s2g(blob + BLOB_KTT, sm + P_KT, 16384);
         bulk_s2g(blob + BLOB_GAM, sm + P_GAM, 512);
+        bulk_s2g(blob + BLOB_A1, sm + P_A1, 8192);                   // Q~, channels 0..63
+        bulk_s2g(blob + BLOB_A1 + 16384, sm + P_A1 + 16384, 8192);   // Q~, channels 64..127
         bulk_commit();
     }
 
@@ -356,69 +363,74 @@ kda_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         tc_fence_after();
         mma_run<D>(tmem, kmajor(sm_base + P_A1, 128), kmajor(sm_base + P_KINV, 64), idesc_bf16(128, 64), false);
         mma_commit(bar_mma);
+        bulk_wait_read();  // K~ has left shared memory: its space takes A_kk after the MMA
     }
+    cta_wait(bar_mma, 0, dead, &g_kda_device_status);
+    tc_fence_after();
 
     // Readout mapping: warp w reads TMEM lanes 32*(w%4) .. +31 (Gram rows m),
     // columns 32*(w/4) .. +31.
     const int m = 32 * (warp & 3) + lane, cb = 32 * (warp >> 2);
     const int r_own = m & 63;
     const bool kk_row = m >= 64;
-    float acc_bad[32];
+    auto gram_readout = [&](auto bad_tag) {
+        constexpr bool BAD = decltype(bad_tag)::value;
+        float G[32];
+        if constexpr (BAD) {  // exact pairwise terms of the channels left out of the MMA
+            float acc[32];
 #pragma unroll
-    for (int e = 0; e < 32; ++e) acc_bad[e] = 0.f;
-    if (n_bad) {  // exact pairwise terms of the channels left out of the MMA
-        int *nbad = reinterpret_cast<int *>(sm + P_NBAD);
-        if (tid == 0) {
-            int cnt = 0;
-            for (int cc = 0; cc < D; ++cc)
-                if (-sgl[cc] > SAFE_SPAN) badl[cnt++] = cc;
-            *nbad = cnt;
-        }
-        __syncthreads();
-        const int nb_total = *nbad;
-        float *bb = reinterpret_cast<float *>(sm + P_BADB);  // [8][3][64]: q, k, g per row
-        for (int b0 = 0; b0 < nb_total; b0 += 8) {
-            for (int e = tid; e < 8 * 64; e += PREP_NT) {  // gather the batch's columns
-                const int bi = e >> 6, r = e & 63;
-                float qx = 0.f, kx = 0.f, gx = 0.f;
-                if (b0 + bi < nb_total) {
-                    const int64_t ccol = (int64_t)h * D + badl[b0 + bi];
-                    float a = 0.f;
-                    for (int j = 0; j <= r; ++j)
-                        a += j < L ? log_alpha[(tok0 + j) * H * D + ccol] : 0.f;
-                    gx = a;
-                    if (r < L) {
-                        qx = __bfloat162float(q[(tok0 + r) * H * D + ccol]);
-                        kx = __bfloat162float(k[(tok0 + r) * H * D + ccol]);
+            for (int e = 0; e < 32; ++e) acc[e] = 0.f;
+            int *nbad = reinterpret_cast<int *>(sm + P_NBAD);
+            if (tid == 0) {
+                int cnt = 0;
+                for (int cc = 0; cc < D; ++cc)
+                    if (-sgl[cc] > SAFE_SPAN) badl[cnt++] = cc;
+                *nbad = cnt;
+            }
+            __syncthreads();
+            const int nb_total = *nbad;
+            float *bb = reinterpret_cast<float *>(sm + P_BADB);  // [8][3][64]: q, k, g per row
+            for (int b0 = 0; b0 < nb_total; b0 += 8) {
+                for (int e = tid; e < 8 * 64; e += PREP_NT) {  // gather the batch's columns
+                    const int bi = e >> 6, r = e & 63;
+                    float qx = 0.f, kx = 0.f, gx = 0.f;
+                    if (b0 + bi < nb_total) {
+                        const int64_t ccol = (int64_t)h * D + badl[b0 + bi];
+                        float a = 0.f;
+                        for (int j = 0; j <= r; ++j)
+                            a += j < L ? log_alpha[(tok0 + j) * H * D + ccol] : 0.f;
+                        gx = a;
+                        if (r < L) {
+                            qx = __bfloat162float(q[(tok0 + r) * H * D + ccol]);
+                            kx = __bfloat162float(k[(tok0 + r) * H * D + ccol]);
+                        }
+                    }
+                    bb[(bi * 3 + 0) * 64 + r] = qx;
+                    bb[(bi * 3 + 1) * 64 + r] = kx;
+                    bb[(bi * 3 + 2) * 64 + r] = gx;
+                }
+                __syncthreads();
+                const int nb = min(8, nb_total - b0);
+                for (int bi = 0; bi < nb; ++bi) {
+                    const float xr = bb[(bi * 3 + (kk_row ? 1 : 0)) * 64 + r_own];
+                    const float grr = bb[(bi * 3 + 2) * 64 + r_own];
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) {
+                        const int i = cb + e;
+                        const float fi = i <= r_own ? bb[(bi * 3 + 1) * 64 + i] *
+                                                          expf(fminf(grr - bb[(bi * 3 + 2) * 64 + i], 0.f))
+                                                    : 0.f;
+                        acc[e] += xr * fi;
                     }
                 }
-                bb[(bi * 3 + 0) * 64 + r] = qx;
-                bb[(bi * 3 + 1) * 64 + r] = kx;
-                bb[(bi * 3 + 2) * 64 + r] = gx;
+                __syncthreads();
             }
-            __syncthreads();
-            const int nb = min(8, nb_total - b0);
-            for (int bi = 0; bi < nb; ++bi) {
-                const float xr = bb[(bi * 3 + (kk_row ? 1 : 0)) * 64 + r_own];
-                const float grr = bb[(bi * 3 + 2) * 64 + r_own];
+            tmem_ld32(tmem + ((uint32_t)(32 * (warp & 3)) << 16) + cb, G);
 #pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    const int i = cb + e;
-                    const float f = i <= r_own ? bb[(bi * 3 + 1) * 64 + i] *
-                                                     expf(fminf(grr - bb[(bi * 3 + 2) * 64 + i], 0.f))
-                                               : 0.f;
-                    acc_bad[e] += xr * f;
-                }
-            }
-            __syncthreads();
+            for (int e = 0; e < 32; ++e) G[e] += acc[e];
+        } else {
+            tmem_ld32(tmem + ((uint32_t)(32 * (warp & 3)) << 16) + cb, G);
         }
-    }
-
-    cta_wait(bar_mma, 0, dead, &g_kda_device_status);
-    tc_fence_after();
-    {
-        float G[32];
-        tmem_ld32(tmem + ((uint32_t)(32 * (warp & 3)) << 16) + cb, G);
         const int r = r_own;
         if (!kk_row) {  // A_qk (inclusive lower) -> bf16 image, rows r, columns i
 #pragma unroll
@@ -427,11 +439,11 @@ kda_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
                     const int i = cb + cq * 8 + e;
-                    v[e] = (i <= r && r < L) ? G[cq * 8 + e] + acc_bad[cq * 8 + e] : 0.f;
+                    v[e] = (i <= r && r < L) ? G[cq * 8 + e] : 0.f;
                 }
                 st_chunk(sm + P_AQK + sw128_chunk_off(r, (cb >> 3) + cq, 64), v);
             }
-        } else {  // A_kk (strict lower, times beta_r) -> fp32 for the solve (over KINV)
+        } else {  // A_kk (strict lower, times beta_r) -> fp32 for the solve
             float *akk = reinterpret_cast<float *>(sm + P_AKK);
             const float b = sbeta[r];
 #pragma unroll
@@ -440,13 +452,16 @@ kda_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     const int i = cb + e4 + e;
-                    v[e] = i < r ? b * (G[e4 + e] + acc_bad[e4 + e]) : 0.f;
+                    v[e] = i < r ? b * G[e4 + e] : 0.f;
                 }
                 *reinterpret_cast<float4 *>(akk + r * LDT + cb + e4) = make_float4(v[0], v[1], v[2], v[3]);
             }
         }
-    }
+    };
+    if (n_bad) gram_readout(std::true_type{});
+    else gram_readout(std::false_type{});
     fence_async_smem();
+    tc_fence_before();
     __syncthreads();
     if (tid == 0) {  // A_qk is final
         bulk_s2g(blob + BLOB_AQK, sm + P_AQK, 8192);
@@ -457,9 +472,9 @@ kda_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     //      blocks, then merge 16 -> 32 -> 64 with [[X, 0], [Y, Z]]^-1 =
     //      [[X^-1, 0], [-Z^-1 Y X^-1, Z^-1]] (each level two small products).
     {
-        float *at = reinterpret_cast<float *>(sm + P_AKK);  // A_kk, becoming T (row stride LDT)
+        float *at = reinterpret_cast<float *>(sm + P_AKK);   // A_kk, becoming T (row stride LDT)
         float *pb = reinterpret_cast<float *>(sm + P_PBUF);  // 2 x [16][20] level-1 products
-        float *qb = reinterpret_cast<float *>(sm + P_TB);    // [32][36] level-2 product (TB is free)
+        float *qb = reinterpret_cast<float *>(sm + P_PBUF);  // [32][36] level-2 product
         if (warp < 4) {  // warp b inverts diagonal block b; lane l -> column l
             const int o = warp * 16, l = lane & 15;
             float t[16];
@@ -517,6 +532,7 @@ kda_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             warp_gemm_16x8<32>(d, at + (32 + m0) * LDT + 32, LDT, qb + n0, 36);
             warp_store_16x8(d, at + (32 + m0) * LDT + n0, LDT, -1.f);
         }
+        if (tid == 0) bulk_wait_read();  // A_qk has left shared memory: its space takes T Diag(beta)
         __syncthreads();
         // image of T Diag(beta): rows r, columns i, zero above the diagonal
         {
@@ -555,20 +571,22 @@ kda_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     tc_fence_after();
     {
         // M = 64 accumulator: row r sits in lane 16*(w%4) + (lane < 16) of quarter w%4.
-        // Warp half w/4 takes columns 64*(w/4) .. +63.
-        float a[64];
+        // Warp half w/4 takes columns 64*(w/4) .. +63, in two loads of 32.
         const uint32_t lanes = (uint32_t)(32 * (warp & 3)) << 16;
-        const uint32_t cofs = 64u * (uint32_t)(warp >> 2);
         const int r = 16 * (warp & 3) + lane;
-        tmem_ld64(tmem + lanes + cofs, a);
-        if (lane < 16) {  // W row r -> A1 row 64 + r, channel block w/4
-            unsigned char *wb = sm + P_A1 + (warp >> 2) * 16384;
+        unsigned char *wb = sm + P_A1 + (warp >> 2) * 16384;
 #pragma unroll
-            for (int cq = 0; cq < 8; ++cq) {
-                float v[8];
+        for (int hq = 0; hq < 2; ++hq) {
+            float a[32];
+            tmem_ld32(tmem + lanes + 64u * (uint32_t)(warp >> 2) + 32u * hq, a);
+            if (lane < 16) {  // W row r -> A1 row 64 + r, channel block w/4
 #pragma unroll
-                for (int e = 0; e < 8; ++e) v[e] = a[cq * 8 + e];
-                st_chunk(wb + sw128_chunk_off(64 + r, cq, 128), v);
+                for (int cq = 0; cq < 4; ++cq) {
+                    float v[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) v[e] = a[cq * 8 + e];
+                    st_chunk(wb + sw128_chunk_off(64 + r, 4 * hq + cq, 128), v);
+                }
             }
         }
     }
@@ -576,8 +594,9 @@ kda_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     tc_fence_before();
     __syncthreads();
 
-    if (tid == 0) {
-        bulk_s2g(blob + BLOB_A1, sm + P_A1, 32768);
+    if (tid == 0) {  // the W rows of A1
+        bulk_s2g(blob + BLOB_A1 + 8192, sm + P_A1 + 8192, 8192);
+        bulk_s2g(blob + BLOB_A1 + 16384 + 8192, sm + P_A1 + 16384 + 8192, 8192);
         bulk_commit();
         bulk_wait_read();  // shared memory may be released; the writes complete with the grid
     }
@@ -675,28 +694,33 @@ kda_chain_kernel(const __grid_constant__ CUtensorMap tm_v,
         if (nchunks > 1) issue_load(1, 1);
     }
 
-    // Output of chunk m: rows 0..63 of D1 buffer m % 2, read by the warps of lane
-    // quarters 0 and 1 once the output MMA of chunk m has completed. It runs while
-    // the next chunk's first MMA executes, off the state recurrence's path.
+    // Output of chunk m: rows 0..63 of D1 buffer m % 2, all N columns, read by warps
+    // 4 and 5 (lane quarters 0 and 1) once the output MMA of chunk m has completed.
+    // It runs during the next chunk, on warps that neither issue MMAs nor form
+    // V_new, so it never delays the state recurrence.
     auto store_output = [&](int m) {
-        if (q4 < 2) {
-            mbar_wait(&bar_c[m & 1], (uint32_t)(m >> 1) & 1u, dead, &g_kda_device_status);
-            tc_fence_after();
-            const int r = c;
-            float ov[NH];
-            tmem_ld_half<NH>(tmem + (uint32_t)((m & 1) * N) + lane_off + jh, ov);
-            const int64_t tok = span.start + (int64_t)m * CH + r;
-            if (r < chunk_rows(span.len, (int64_t)m * CH)) {
-                __nv_bfloat16 *dst = o + (tok * H + h) * (int64_t)D + j0 + jh;
+        mbar_wait(&bar_c[m & 1], (uint32_t)(m >> 1) & 1u, dead, &g_kda_device_status);
+        tc_fence_after();
+        const int r = c;
+        const bool live = r < chunk_rows(span.len, (int64_t)m * CH);
+        __nv_bfloat16 *dst = o + ((span.start + (int64_t)m * CH + r) * H + h) * (int64_t)D + j0;
 #pragma unroll
-                for (int j = 0; j < NH; j += 8) {
+        for (int b = 0; b < N / 64; ++b) {
+            float ov[64];
+            tmem_ld64(tmem + (uint32_t)((m & 1) * N + 64 * b) + lane_off, ov);
+            if (live) {
+#pragma unroll
+                for (int j = 0; j < 64; j += 8) {
                     uint4 pk = make_uint4(pack_bf16x2(ov[j], ov[j + 1]), pack_bf16x2(ov[j + 2], ov[j + 3]),
                                           pack_bf16x2(ov[j + 4], ov[j + 5]), pack_bf16x2(ov[j + 6], ov[j + 7]));
-                    *reinterpret_cast<uint4 *>(dst + j) = pk;
+                    *reinterpret_cast<uint4 *>(dst + 64 * b + j) = pk;
                 }
             }
         }
     };
+    // Named barrier 1: the V_new warps (lane quarters 2, 3) arrive once their rows of
+    // the V_new image are in shared memory; warp 0, which issues the MMAs, waits.
+    constexpr uint32_t BAR_VNEW = 1, BAR_VNEW_COUNT = 5 * 32;
 
 #pragma unroll 1
     for (int n = 0; n < nchunks && !dead; ++n) {
@@ -708,7 +732,7 @@ kda_chain_kernel(const __grid_constant__ CUtensorMap tm_v,
 
         mbar_wait(&bar_ld[stage], (uint32_t)(n >> 1) & 1u, dead, &g_kda_device_status);
         // D1 = [Q~; W] S
-        if (tid == 0) {
+        if (tid == 0 && !dead) {
             tc_fence_after();
             mma_run<D>(d1, kmajor(st_base + Lay::A1, 128), mnmajor(sm_base + Lay::SIMG, 16384),
                        idesc_bf16(128, N, 0, 1), false);
@@ -716,10 +740,9 @@ kda_chain_kernel(const __grid_constant__ CUtensorMap tm_v,
                         idesc_bf16(128, N, 0, 1), false);
             mma_commit(bar_a);
         }
-        if (n > 0) store_output(n - 1);
-        mbar_wait(bar_a, ph, dead, &g_kda_device_status);
-        tc_fence_after();
         if (q4 >= 2) {  // rows 64..127 hold (W S)[r] in D1 and U[r] in DU; V_new = U - W S
+            mbar_wait(bar_a, ph, dead, &g_kda_device_status);
+            tc_fence_after();
             const int r = c - 64;
             float ws[NH], us[NH];
             tmem_ld_half<NH>(d1 + lane_off + jh, ws);
@@ -731,19 +754,23 @@ kda_chain_kernel(const __grid_constant__ CUtensorMap tm_v,
                 for (int e = 0; e < 8; ++e) v[e] = us[jc * 8 + e] - ws[jc * 8 + e];
                 st_chunk(sm + Lay::VIMG + sw128_chunk_off(r, (jh >> 3) + jc, 64), v);  // row r, MN-major
             }
-        }
-        fence_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        // D3 = K~^T V_new (the state path first), then D1 += [A_qk; 0] V_new
-        if (tid == 0) {
-            tc_fence_after();
-            mma_run<CH>(d3, mnmajor(st_base + Lay::KTT, 8192), mnmajor(sm_base + Lay::VIMG, 8192),
-                        idesc_bf16(128, N, 1, 1), false);
-            mma_commit(bar_b);
-            mma_run<CH>(d1, kmajor(st_base + Lay::A2, 128), mnmajor(sm_base + Lay::VIMG, 8192),
-                        idesc_bf16(128, N, 0, 1), true);
-            mma_commit(&bar_c[n & 1]);
+            fence_async_smem();
+            tc_fence_before();
+            named_bar_arrive(BAR_VNEW, BAR_VNEW_COUNT);
+        } else if (warp == 0) {
+            named_bar_sync(BAR_VNEW, BAR_VNEW_COUNT);
+            // D3 = K~^T V_new (the state path first), then D1 += [A_qk; 0] V_new
+            if (tid == 0 && !dead) {
+                tc_fence_after();
+                mma_run<CH>(d3, mnmajor(st_base + Lay::KTT, 8192), mnmajor(sm_base + Lay::VIMG, 8192),
+                            idesc_bf16(128, N, 1, 1), false);
+                mma_commit(bar_b);
+                mma_run<CH>(d1, kmajor(st_base + Lay::A2, 128), mnmajor(sm_base + Lay::VIMG, 8192),
+                            idesc_bf16(128, N, 0, 1), true);
+                mma_commit(&bar_c[n & 1]);
+            }
+        } else if (hf == 1 && n > 0) {
+            store_output(n - 1);
         }
         {  // S <- Diag(exp(g_L)) S + K~^T V_new
             mbar_wait(bar_b, ph, dead, &g_kda_device_status);
@@ -764,15 +791,18 @@ kda_chain_kernel(const __grid_constant__ CUtensorMap tm_v,
         }
         fence_async_smem();
         tc_fence_before();
-        __syncthreads();
-        // The stage is free once the output MMA (which reads A2) has completed; the
-        // next load into it is issued after that MMA's barrier.
-        if (tid == 0 && n + 2 < nchunks) {
+        // every thread leaves the loop at the same chunk, so the named barrier's
+        // participants always meet
+        dead = __syncthreads_or(dead) != 0;
+        // The stage is free once the output MMA (which reads A2) has completed. Warp 1
+        // waits for that and refills it, so the MMA issuer goes straight on to the
+        // next chunk.
+        if (tid == 32 && n + 2 < nchunks) {
             mbar_wait(&bar_c[n & 1], (uint32_t)(n >> 1) & 1u, dead, &g_kda_device_status);
-            issue_load(n + 2, stage);
+            if (!dead) issue_load(n + 2, stage);
         }
     }
-    if (nchunks > 0 && !dead) store_output(nchunks - 1);
+    if (nchunks > 0 && !dead && q4 < 2 && hf == 1) store_output(nchunks - 1);
 
     if (S_T) {
 #pragma unroll
@@ -863,15 +893,17 @@ cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, const
     }
     cudaError_t err;
     if (n_tok > 0 && slots > 0) {
-        CUtensorMap mq, mk, mv, mla;
-        if (!make_map(&mq, q, true, n_tok, H) || !make_map(&mk, k, true, n_tok, H) ||
-            !make_map(&mv, v, true, n_tok, H) || !make_map(&mla, log_alpha, false, n_tok, H))
+        CUtensorMap mq, mk;
+        if (!make_map(&mq, q, true, n_tok, H) || !make_map(&mk, k, true, n_tok, H))
             return cudaErrorInvalidValue;
         err = cudaFuncSetAttribute(kda_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                    (int)PREP_SMEM);
+        if (err == cudaSuccess)  // three CTAs per SM need the largest shared-memory carveout
+            err = cudaFuncSetAttribute(kda_prep_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                       (int)cudaSharedmemCarveoutMaxShared);
         if (err != cudaSuccess) return err;
         kda_prep_kernel<<<dim3((unsigned)slots, (unsigned)H), PREP_NT, PREP_SMEM, stream>>>(
-            mq, mk, mv, mla, (const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k, log_alpha, beta,
+            mq, mk, (const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k, log_alpha, beta,
             blobs, chunk_off, cu_seqlens, T, H, n_seqs, nck);
         err = cudaGetLastError();
         if (err != cudaSuccess) return err;

@@ -77,6 +77,17 @@ __device__ __forceinline__ void cta_wait(uint64_t *bar, uint32_t parity, bool &d
     dead = __syncthreads_or(!ok || dead) != 0;
 }
 
+// Named CTA barriers (ids 1..15; id 0 belongs to __syncthreads). `count` is the
+// number of threads taking part, a multiple of 32. bar.arrive does not wait; like
+// bar.sync it makes the arriving thread's earlier memory accesses visible to the
+// threads that wait on the barrier.
+__device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t count) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+__device__ __forceinline__ void named_bar_arrive(uint32_t id, uint32_t count) {
+    asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
 // ------------------------------------------------------------------ async proxy / TMA
 __device__ __forceinline__ void fence_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
