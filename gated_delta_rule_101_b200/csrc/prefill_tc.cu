@@ -120,11 +120,14 @@ struct ChainLayout {
     static constexpr uint32_t STAGE = ((GAM + 512 + 1023) / 1024) * 1024;
     static constexpr uint32_t SIMG = 2 * STAGE;       // S bf16, MN-major: rows c (128), N columns
     static constexpr uint32_t VIMG = SIMG + N * 256;  // V_new bf16, MN-major: rows r (64), N columns
-    static constexpr uint32_t BAR = VIMG + N * 128;   // 6 mbarriers
-    static constexpr uint32_t TMEM = BAR + 48;
+    static constexpr uint32_t BAR = VIMG + N * 128;   // 8 mbarriers
+    static constexpr uint32_t TMEM = BAR + 64;
     static constexpr uint32_t BYTES = TMEM + 8 + 1024;
     static constexpr uint32_t TMEM_COLS = 4 * N;      // D1 (two buffers), D3, U
-    static constexpr uint32_t LOAD_BYTES = 32768 + 8192 + 16384 + 8192 + 512 + N * 128;
+    // A stage is filled in two parts, each released as soon as its readers are done:
+    // part 1 (A1, TB, V) feeds the chunk's first MMAs, part 2 (A2, KTT, GAM) the rest.
+    static constexpr uint32_t LOAD1_BYTES = 32768 + 8192 + N * 128;
+    static constexpr uint32_t LOAD2_BYTES = 8192 + 16384 + 512;
 };
 
 // TMEM load of this thread's lane, N/2 consecutive columns.
@@ -607,11 +610,23 @@ kda_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 // =====================================================================================
 // chain: per (sequence, head, value slice) state recurrence over the chunks
 // =====================================================================================
-// 256 threads. Warp w reads TMEM lane quarter q = w % 4 and handles value columns
-// (N/2)*(w/4) .. +N/2-1 of the slice, so every epilogue is split over two warps per
-// quarter. Thread (q, lane, w/4) keeps state row c = 32q + lane, those columns, in
-// registers. N = 64 gives two CTAs per (sequence, head), N = 128 one.
-constexpr int CHAIN_NT = 256;
+// 288 threads, warp-specialised. Warps 0-7 are the epilogue warps: warp w reads TMEM
+// lane quarter q = w % 4 and handles value columns (N/2)*(w/4) .. +N/2-1 of the slice,
+// and thread (q, lane, w/4) keeps state row c = 32q + lane, those columns, in
+// registers. Warp 8 issues every MMA and bulk load; a tcgen05.mma issue can stall
+// while the tensor pipe is busy, and on its own warp that stall delays no epilogue.
+// N = 64 gives two CTAs per (sequence, head), N = 128 one.
+constexpr int CHAIN_EPI_WARPS = 8;
+constexpr int CHAIN_NT = 32 * (CHAIN_EPI_WARPS + 1);
+// Named barriers (id 0 is __syncthreads):
+//   BAR_VNEW: the V_new warps (lane quarters 2, 3) arrive once their rows of the V_new
+//             image are written; the issuer waits before the MMAs that read it.
+//   BAR_END:  every thread, at the end of each chunk: the state image is written and
+//             the chunk's TMEM reads are done. It also ORs the threads' `dead` flags,
+//             so all warps leave the loop at the same chunk and the barriers' arrivals
+//             always pair up, even after a bounded wait has given up.
+constexpr uint32_t BAR_VNEW = 1, BAR_VNEW_COUNT = 32 * 5;
+constexpr uint32_t BAR_END = 2;
 
 template <int N>
 __global__ void __launch_bounds__(CHAIN_NT, 1)
@@ -621,63 +636,75 @@ kda_chain_kernel(const __grid_constant__ CUtensorMap tm_v,
                  float *__restrict__ S_T, const int32_t *__restrict__ cu, int64_t T, int H,
                  int nck) {
     static_assert(N == 64 || N == 128, "value slices of 64 or 128 columns");
-    constexpr int NH = N / 2;  // columns per thread
+    constexpr int NH = N / 2;  // columns per epilogue thread
     using Lay = ChainLayout<N>;
     extern __shared__ unsigned char smem_raw[];
     unsigned char *sm = aligned_smem(smem_raw);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int q4 = warp & 3, hf = warp >> 2;
+    const bool issuer = warp == CHAIN_EPI_WARPS;
+    const int q4 = warp & 3, hf = (warp >> 2) & 1;
     const int seq = blockIdx.x, h = blockIdx.y, j0 = blockIdx.z * N;
     const SeqSpan span = seq_span(cu, T, seq);
     const int nchunks = (int)((span.len + CH - 1) / CH);
     const int64_t slot0 = chunk_off ? (int64_t)chunk_off[seq] : (int64_t)seq * nck;
     const int64_t state_off = ((int64_t)seq * H + h) * (int64_t)(D * D);
 
-    uint64_t *bar_ld = reinterpret_cast<uint64_t *>(sm + Lay::BAR);  // [2] chunk loads
-    uint64_t *bar_a = bar_ld + 2;  // MMA1 done
-    uint64_t *bar_b = bar_ld + 3;  // state MMA done
-    uint64_t *bar_c = bar_ld + 4;  // [2] output MMA done, per D1 buffer
+    uint64_t *bar_ld1 = reinterpret_cast<uint64_t *>(sm + Lay::BAR);  // [2] load part 1, per stage
+    uint64_t *bar_ld2 = bar_ld1 + 2;  // [2] load part 2, per stage
+    uint64_t *bar_a = bar_ld1 + 4;    // first MMAs done
+    uint64_t *bar_b = bar_ld1 + 5;    // state MMA done
+    uint64_t *bar_c = bar_ld1 + 6;    // [2] output MMA done, per D1 buffer
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + Lay::TMEM);
     bool dead = false;
 
-    auto issue_load = [&](int chunk, int stage) {
-        const unsigned char *blob = ws_blobs + ((size_t)(slot0 + chunk) * H + h) * BLOB_BYTES;
+    auto blob_of = [&](int chunk) {
+        return ws_blobs + ((size_t)(slot0 + chunk) * H + h) * BLOB_BYTES;
+    };
+    auto issue_load1 = [&](int chunk, int stage) {
+        const unsigned char *blob = blob_of(chunk);
         unsigned char *st = sm + stage * Lay::STAGE;
-        mbar_arrive_expect_tx(&bar_ld[stage], Lay::LOAD_BYTES);
-        bulk_g2s(st + Lay::A1, blob + BLOB_A1, 32768, &bar_ld[stage]);
-        bulk_g2s(st + Lay::A2, blob + BLOB_AQK, 8192, &bar_ld[stage]);
-        bulk_g2s(st + Lay::KTT, blob + BLOB_KTT, 16384, &bar_ld[stage]);
-        bulk_g2s(st + Lay::TB, blob + BLOB_TB, 8192, &bar_ld[stage]);
-        bulk_g2s(st + Lay::GAM, blob + BLOB_GAM, 512, &bar_ld[stage]);
+        mbar_arrive_expect_tx(&bar_ld1[stage], Lay::LOAD1_BYTES);
+        bulk_g2s(st + Lay::A1, blob + BLOB_A1, 32768, &bar_ld1[stage]);
+        bulk_g2s(st + Lay::TB, blob + BLOB_TB, 8192, &bar_ld1[stage]);
 #pragma unroll
         for (int b = 0; b < N / 64; ++b)
             tma_load_2d(st + Lay::V + b * 8192, &tm_v, h * D + j0 + 64 * b,
-                        (int)(span.start + (int64_t)chunk * CH), &bar_ld[stage]);
+                        (int)(span.start + (int64_t)chunk * CH), &bar_ld1[stage]);
+    };
+    auto issue_load2 = [&](int chunk, int stage) {
+        const unsigned char *blob = blob_of(chunk);
+        unsigned char *st = sm + stage * Lay::STAGE;
+        mbar_arrive_expect_tx(&bar_ld2[stage], Lay::LOAD2_BYTES);
+        bulk_g2s(st + Lay::A2, blob + BLOB_AQK, 8192, &bar_ld2[stage]);
+        bulk_g2s(st + Lay::KTT, blob + BLOB_KTT, 16384, &bar_ld2[stage]);
+        bulk_g2s(st + Lay::GAM, blob + BLOB_GAM, 512, &bar_ld2[stage]);
     };
 
     if (tid == 0) {
-        for (int b = 0; b < 6; ++b) mbar_init(&bar_ld[b], 1);
+        for (int b = 0; b < 8; ++b) mbar_init(&bar_ld1[b], 1);
         fence_mbar_init();
     }
     if (warp == 0) {
         tmem_alloc(tmem_slot, Lay::TMEM_COLS);
         tmem_relinquish();
     }
-    const int c = 32 * q4 + lane;    // state row owned by this thread
+    const int c = 32 * q4 + lane;    // state row owned by an epilogue thread
     const int jh = NH * hf;          // first of its NH value columns (inside the slice)
     float s_reg[NH];
+    if (!issuer) {
 #pragma unroll
-    for (int j = 0; j < NH; j += 4) {
-        float4 v4 = S0 ? *reinterpret_cast<const float4 *>(S0 + state_off + (int64_t)c * D + j0 + jh + j)
-                       : make_float4(0.f, 0.f, 0.f, 0.f);
-        s_reg[j] = v4.x; s_reg[j + 1] = v4.y; s_reg[j + 2] = v4.z; s_reg[j + 3] = v4.w;
-    }
+        for (int j = 0; j < NH; j += 4) {
+            float4 v4 = S0 ? *reinterpret_cast<const float4 *>(S0 + state_off + (int64_t)c * D + j0 + jh + j)
+                           : make_float4(0.f, 0.f, 0.f, 0.f);
+            s_reg[j] = v4.x; s_reg[j + 1] = v4.y; s_reg[j + 2] = v4.z; s_reg[j + 3] = v4.w;
+        }
 #pragma unroll
-    for (int jc = 0; jc < NH / 8; ++jc) {  // row c of the MN-major S image, this thread's chunks
-        float v[8];
+        for (int jc = 0; jc < NH / 8; ++jc) {  // row c of the MN-major S image, this thread's chunks
+            float v[8];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) v[e] = s_reg[jc * 8 + e];
-        st_chunk(sm + Lay::SIMG + sw128_chunk_off(c, (jh >> 3) + jc, 128), v);
+            for (int e = 0; e < 8; ++e) v[e] = s_reg[jc * 8 + e];
+            st_chunk(sm + Lay::SIMG + sw128_chunk_off(c, (jh >> 3) + jc, 128), v);
+        }
     }
     fence_async_smem();
     tc_fence_before();
@@ -689,78 +716,36 @@ kda_chain_kernel(const __grid_constant__ CUtensorMap tm_v,
     const uint32_t sm_base = smem_u32(sm);
     const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
 
-    if (tid == 0) {
-        if (nchunks > 0) issue_load(0, 0);
-        if (nchunks > 1) issue_load(1, 1);
-    }
-
-    // Output of chunk m: rows 0..63 of D1 buffer m % 2, all N columns, read by warps
-    // 4 and 5 (lane quarters 0 and 1) once the output MMA of chunk m has completed.
-    // It runs during the next chunk, on warps that neither issue MMAs nor form
-    // V_new, so it never delays the state recurrence.
-    auto store_output = [&](int m) {
-        mbar_wait(&bar_c[m & 1], (uint32_t)(m >> 1) & 1u, dead, &g_kda_device_status);
-        tc_fence_after();
-        const int r = c;
-        const bool live = r < chunk_rows(span.len, (int64_t)m * CH);
-        __nv_bfloat16 *dst = o + ((span.start + (int64_t)m * CH + r) * H + h) * (int64_t)D + j0;
-#pragma unroll
-        for (int b = 0; b < N / 64; ++b) {
-            float ov[64];
-            tmem_ld64(tmem + (uint32_t)((m & 1) * N + 64 * b) + lane_off, ov);
-            if (live) {
-#pragma unroll
-                for (int j = 0; j < 64; j += 8) {
-                    uint4 pk = make_uint4(pack_bf16x2(ov[j], ov[j + 1]), pack_bf16x2(ov[j + 2], ov[j + 3]),
-                                          pack_bf16x2(ov[j + 4], ov[j + 5]), pack_bf16x2(ov[j + 6], ov[j + 7]));
-                    *reinterpret_cast<uint4 *>(dst + 64 * b + j) = pk;
+    if (issuer) {
+        // ------------------------------------------------------------ MMA / load warp
+        if (lane == 0) {
+            for (int m = 0; m < 2 && m < nchunks; ++m) {
+                issue_load1(m, m);
+                issue_load2(m, m);
+            }
+        }
+#pragma unroll 1
+        for (int n = 0; n < nchunks; ++n) {
+            const int stage = n & 1;
+            const uint32_t st_base = sm_base + stage * Lay::STAGE;
+            const uint32_t d1 = tmem + (uint32_t)((n & 1) * N);
+            const uint32_t lph = (uint32_t)(n >> 1) & 1u;
+            if (lane == 0) {
+                mbar_wait(&bar_ld1[stage], lph, dead, &g_kda_device_status);
+                if (!dead) {  // D1 = [Q~; W] S, DU = [.; T Diag(beta)] V
+                    tc_fence_after();
+                    mma_run<D>(d1, kmajor(st_base + Lay::A1, 128), mnmajor(sm_base + Lay::SIMG, 16384),
+                               idesc_bf16(128, N, 0, 1), false);
+                    mma_run<CH>(du, kmajor(st_base + Lay::TB - 8192, 128), mnmajor(st_base + Lay::V, 8192),
+                                idesc_bf16(128, N, 0, 1), false);
+                    mma_commit(bar_a);
                 }
             }
-        }
-    };
-    // Named barrier 1: the V_new warps (lane quarters 2, 3) arrive once their rows of
-    // the V_new image are in shared memory; warp 0, which issues the MMAs, waits.
-    constexpr uint32_t BAR_VNEW = 1, BAR_VNEW_COUNT = 5 * 32;
-
-#pragma unroll 1
-    for (int n = 0; n < nchunks && !dead; ++n) {
-        const int stage = n & 1;
-        const uint32_t ph = (uint32_t)n & 1u;
-        unsigned char *st = sm + stage * Lay::STAGE;
-        const uint32_t st_base = sm_base + stage * Lay::STAGE;
-        const uint32_t d1 = tmem + (uint32_t)((n & 1) * N);
-
-        mbar_wait(&bar_ld[stage], (uint32_t)(n >> 1) & 1u, dead, &g_kda_device_status);
-        // D1 = [Q~; W] S
-        if (tid == 0 && !dead) {
-            tc_fence_after();
-            mma_run<D>(d1, kmajor(st_base + Lay::A1, 128), mnmajor(sm_base + Lay::SIMG, 16384),
-                       idesc_bf16(128, N, 0, 1), false);
-            mma_run<CH>(du, kmajor(st_base + Lay::TB - 8192, 128), mnmajor(st_base + Lay::V, 8192),
-                        idesc_bf16(128, N, 0, 1), false);
-            mma_commit(bar_a);
-        }
-        if (q4 >= 2) {  // rows 64..127 hold (W S)[r] in D1 and U[r] in DU; V_new = U - W S
-            mbar_wait(bar_a, ph, dead, &g_kda_device_status);
-            tc_fence_after();
-            const int r = c - 64;
-            float ws[NH], us[NH];
-            tmem_ld_half<NH>(d1 + lane_off + jh, ws);
-            tmem_ld_half<NH>(du + lane_off + jh, us);
-#pragma unroll
-            for (int jc = 0; jc < NH / 8; ++jc) {
-                float v[8];
-#pragma unroll
-                for (int e = 0; e < 8; ++e) v[e] = us[jc * 8 + e] - ws[jc * 8 + e];
-                st_chunk(sm + Lay::VIMG + sw128_chunk_off(r, (jh >> 3) + jc, 64), v);  // row r, MN-major
-            }
-            fence_async_smem();
-            tc_fence_before();
-            named_bar_arrive(BAR_VNEW, BAR_VNEW_COUNT);
-        } else if (warp == 0) {
-            named_bar_sync(BAR_VNEW, BAR_VNEW_COUNT);
-            // D3 = K~^T V_new (the state path first), then D1 += [A_qk; 0] V_new
-            if (tid == 0 && !dead) {
+            __syncwarp();
+            named_bar_sync(BAR_VNEW, BAR_VNEW_COUNT);  // V_new image of chunk n written
+            if (lane == 0) mbar_wait(&bar_ld2[stage], lph, dead, &g_kda_device_status);
+            if (lane == 0 && !dead) {
+                // D3 = K~^T V_new (the state path first), then D1 += [A_qk; 0] V_new
                 tc_fence_after();
                 mma_run<CH>(d3, mnmajor(st_base + Lay::KTT, 8192), mnmajor(sm_base + Lay::VIMG, 8192),
                             idesc_bf16(128, N, 1, 1), false);
@@ -769,46 +754,117 @@ kda_chain_kernel(const __grid_constant__ CUtensorMap tm_v,
                             idesc_bf16(128, N, 0, 1), true);
                 mma_commit(&bar_c[n & 1]);
             }
-        } else if (hf == 1 && n > 0) {
-            store_output(n - 1);
-        }
-        {  // S <- Diag(exp(g_L)) S + K~^T V_new
-            mbar_wait(bar_b, ph, dead, &g_kda_device_status);
-            tc_fence_after();
-            float dv[NH];
-            tmem_ld_half<NH>(d3 + lane_off + jh, dv);
-            const float gam = reinterpret_cast<const float *>(st + Lay::GAM)[c];
-#pragma unroll
-            for (int jc = 0; jc < NH / 8; ++jc) {
-                float v[8];
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    s_reg[jc * 8 + e] = gam * s_reg[jc * 8 + e] + dv[jc * 8 + e];
-                    v[e] = s_reg[jc * 8 + e];
-                }
-                st_chunk(sm + Lay::SIMG + sw128_chunk_off(c, (jh >> 3) + jc, 128), v);
+            __syncwarp();
+            if (named_bar_or(BAR_END, CHAIN_NT, dead)) {
+                dead = true;
+                break;
             }
         }
-        fence_async_smem();
-        tc_fence_before();
-        // every thread leaves the loop at the same chunk, so the named barrier's
-        // participants always meet
-        dead = __syncthreads_or(dead) != 0;
-        // The stage is free once the output MMA (which reads A2) has completed. Warp 1
-        // waits for that and refills it, so the MMA issuer goes straight on to the
-        // next chunk.
-        if (tid == 32 && n + 2 < nchunks) {
-            mbar_wait(&bar_c[n & 1], (uint32_t)(n >> 1) & 1u, dead, &g_kda_device_status);
-            if (!dead) issue_load(n + 2, stage);
-        }
-    }
-    if (nchunks > 0 && !dead && q4 < 2 && hf == 1) store_output(nchunks - 1);
-
-    if (S_T) {
+    } else {
+        // ------------------------------------------------------------ epilogue warps
+        // Output of chunk m: rows 0..63 of D1 buffer m % 2, all N columns, read by warps
+        // 4 and 5 (lane quarters 0 and 1) once the output MMA of chunk m has completed,
+        // while the next chunk's first MMAs run.
+        auto store_output = [&](int m) {
+            mbar_wait(&bar_c[m & 1], (uint32_t)(m >> 1) & 1u, dead, &g_kda_device_status);
+            tc_fence_after();
+            const int r = c;
+            const bool live = r < chunk_rows(span.len, (int64_t)m * CH);
+            __nv_bfloat16 *dst = o + ((span.start + (int64_t)m * CH + r) * H + h) * (int64_t)D + j0;
 #pragma unroll
-        for (int j = 0; j < NH; j += 4)
-            *reinterpret_cast<float4 *>(S_T + state_off + (int64_t)c * D + j0 + jh + j) =
-                make_float4(s_reg[j], s_reg[j + 1], s_reg[j + 2], s_reg[j + 3]);
+            for (int b = 0; b < N / 32; ++b) {
+                float ov[32];
+                tmem_ld32(tmem + (uint32_t)((m & 1) * N + 32 * b) + lane_off, ov);
+                if (live) {
+#pragma unroll
+                    for (int j = 0; j < 32; j += 8) {
+                        uint4 pk = make_uint4(pack_bf16x2(ov[j], ov[j + 1]), pack_bf16x2(ov[j + 2], ov[j + 3]),
+                                              pack_bf16x2(ov[j + 4], ov[j + 5]), pack_bf16x2(ov[j + 6], ov[j + 7]));
+                        *reinterpret_cast<uint4 *>(dst + 32 * b + j) = pk;
+                    }
+                }
+            }
+        };
+#pragma unroll 1
+        for (int n = 0; n < nchunks; ++n) {
+            const int stage = n & 1;
+            const uint32_t ph = (uint32_t)n & 1u;
+            const unsigned char *st = sm + stage * Lay::STAGE;
+            const uint32_t d1 = tmem + (uint32_t)((n & 1) * N);
+            const uint32_t lph = (uint32_t)(n >> 1) & 1u;
+            if (q4 >= 2) {  // rows 64..127 hold (W S)[r] in D1 and U[r] in DU; V_new = U - W S
+                mbar_wait(bar_a, ph, dead, &g_kda_device_status);
+                tc_fence_after();
+                const int r = c - 64;
+#pragma unroll
+                for (int p = 0; p < NH / 32; ++p) {
+                    float ws[32], us[32];
+                    tmem_ld32(d1 + lane_off + jh + 32 * p, ws);
+                    tmem_ld32(du + lane_off + jh + 32 * p, us);
+#pragma unroll
+                    for (int jc = 0; jc < 4; ++jc) {
+                        float v[8];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) v[e] = us[jc * 8 + e] - ws[jc * 8 + e];
+                        st_chunk(sm + Lay::VIMG + sw128_chunk_off(r, ((jh + 32 * p) >> 3) + jc, 64), v);
+                    }
+                }
+                fence_async_smem();
+                tc_fence_before();
+                named_bar_arrive(BAR_VNEW, BAR_VNEW_COUNT);
+            } else if (hf == 1) {
+                if (n > 0) store_output(n - 1);
+            } else if (warp == 1) {
+                // Part 1 of the stage is free once the first MMAs have completed: refill it
+                // with chunk n + 2 while this chunk is still being processed.
+                if (lane == 0 && n + 2 < nchunks) {
+                    mbar_wait(bar_a, ph, dead, &g_kda_device_status);
+                    if (!dead) issue_load1(n + 2, stage);
+                }
+                __syncwarp();
+            }
+            {  // S <- Diag(exp(g_L)) S + K~^T V_new
+                mbar_wait(&bar_ld2[stage], lph, dead, &g_kda_device_status);  // GAM
+                mbar_wait(bar_b, ph, dead, &g_kda_device_status);
+                tc_fence_after();
+                const float gam = reinterpret_cast<const float *>(st + Lay::GAM)[c];
+#pragma unroll
+                for (int p = 0; p < NH / 32; ++p) {
+                    float dv[32];
+                    tmem_ld32(d3 + lane_off + jh + 32 * p, dv);
+#pragma unroll
+                    for (int jc = 0; jc < 4; ++jc) {
+                        float v[8];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) {
+                            float &s = s_reg[32 * p + jc * 8 + e];
+                            s = gam * s + dv[jc * 8 + e];
+                            v[e] = s;
+                        }
+                        st_chunk(sm + Lay::SIMG + sw128_chunk_off(c, ((jh + 32 * p) >> 3) + jc, 128), v);
+                    }
+                }
+            }
+            fence_async_smem();
+            tc_fence_before();
+            if (named_bar_or(BAR_END, CHAIN_NT, dead)) {
+                dead = true;
+                break;
+            }
+            // Part 2 is free once the output MMA (the last reader of A2 and KTT) has
+            // completed and the state update (the reader of GAM) has passed BAR_END.
+            if (tid == 32 && n + 2 < nchunks) {
+                mbar_wait(&bar_c[stage], lph, dead, &g_kda_device_status);
+                if (!dead) issue_load2(n + 2, stage);
+            }
+        }
+        if (nchunks > 0 && !dead && q4 < 2 && hf == 1) store_output(nchunks - 1);
+        if (S_T) {
+#pragma unroll
+            for (int j = 0; j < NH; j += 4)
+                *reinterpret_cast<float4 *>(S_T + state_off + (int64_t)c * D + j0 + jh + j) =
+                    make_float4(s_reg[j], s_reg[j + 1], s_reg[j + 2], s_reg[j + 3]);
+        }
     }
     tc_fence_before();
     __syncthreads();
