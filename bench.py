@@ -126,22 +126,24 @@ class ClockSampler:
 
 # ------------------------------------------------------------------ ncu traffic
 # DRAM bytes (read + write) per launch from one ncu capture of the B=4, T=4096,
-# H=16 step and of one N=256, H=32 decode step (profiles/). They are reported
-# only while the CUDA sources hash to the build they were taken from.
-TRAFFIC = {"source_hash": "353fc00f9f230e47",
-           "prefill": 338424064 + 257215232 + 308346880 + 58567936,  # prep + chain
-           "decode": 547402496 + 480379392}
+# H=16 step and of one N=256, H=32 decode step (profiles/). Each figure is
+# reported only while the sources of its kernels hash to the build it was taken
+# from; otherwise the roofline's traffic is null.
+TRAFFIC_SOURCES = {"prefill": ("prefill_tc.cu", "tc_ptx.cuh", "kda_internal.cuh"),
+                   "decode": ("decode.cu", "kda_internal.cuh")}
+TRAFFIC = {"prefill": {"source_hash": "ad83ac7aec4312e9",  # prep + chain
+                       "bytes": 270749696 + 215545856 + 341876992 + 56629504},
+           "decode": {"source_hash": "bfbc16685498d103", "bytes": 547402496 + 480379392}}
 
 
-def source_hash() -> str:
-    import glob
+def source_hash(kind: str) -> str:
     import hashlib
 
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "gated_delta_rule_101_b200", "csrc")
-    for p in sorted(glob.glob(os.path.join(csrc, "*.cu")) + glob.glob(os.path.join(csrc, "*.cuh"))):
-        h.update(os.path.basename(p).encode())
-        with open(p, "rb") as f:
+    for name in TRAFFIC_SOURCES[kind]:
+        h.update(name.encode())
+        with open(os.path.join(csrc, name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
 
@@ -149,7 +151,8 @@ def source_hash() -> str:
 def traffic(kind: str, override):
     if override is not None:
         return override
-    return TRAFFIC[kind] if source_hash() == TRAFFIC["source_hash"] else None
+    t = TRAFFIC[kind]
+    return t["bytes"] if t["source_hash"] == source_hash(kind) else None
 
 
 # ------------------------------------------------------------------ helpers
