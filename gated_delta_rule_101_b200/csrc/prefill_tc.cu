@@ -205,6 +205,7 @@ __device__ __forceinline__ void ld_chunk(const unsigned char *p, float (&v)[8]) 
 
 __global__ void __launch_bounds__(PREP_NT, 3)
 kda_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                const __grid_constant__ CUtensorMap tm_la, int pf_dist,
                 const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
                 const float *__restrict__ log_alpha, const float *__restrict__ beta,
                 unsigned char *__restrict__ ws_blobs, const int32_t *__restrict__ chunk_off,
@@ -239,6 +240,22 @@ kda_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         tma_load_2d(sm + P_A1 + 16384, &tm_q, x + 64, y, bar_tma);     // q, channels 64..127
         tma_load_2d(sm + P_A1 + 8192, &tm_k, x, y, bar_tma);           // k -> rows 64..127
         tma_load_2d(sm + P_A1 + 16384 + 8192, &tm_k, x + 64, y, bar_tma);
+        // Warm L2 for the CTA that starts pf_dist launches after this one (about one
+        // full residency later): its q, k and log_alpha tiles, so that its own loads
+        // find them in L2 instead of waiting on DRAM.
+        const int64_t lin = blockIdx.x + (int64_t)blockIdx.y * gridDim.x + pf_dist;
+        if (pf_dist > 0 && lin < (int64_t)gridDim.x * gridDim.y) {
+            const int pslot = (int)(lin % gridDim.x), ph = (int)(lin / gridDim.x);
+            int pseq, pn;
+            if (resolve_slot(pslot, chunk_off, n_seqs, nck, pseq, pn)) {
+                const int py = (int)(seq_span(cu, T, pseq).start + (int64_t)pn * CH), px = ph * D;
+                tma_prefetch_l2_2d(&tm_q, px, py);
+                tma_prefetch_l2_2d(&tm_q, px + 64, py);
+                tma_prefetch_l2_2d(&tm_k, px, py);
+                tma_prefetch_l2_2d(&tm_k, px + 64, py);
+                tma_prefetch_l2_2d(&tm_la, px, py);
+            }
+        }
     }
     if (warp == 0) {
         tmem_alloc(tmem_slot, PREP_TMEM_COLS);
@@ -917,6 +934,18 @@ cudaError_t launch_chain(const CUtensorMap &mv, const unsigned char *blobs, cons
     return cudaGetLastError();
 }
 
+// CTAs of the prep kernel resident on the whole GPU at once (its L2 prefetch
+// distance); 0 if it cannot be determined.
+int prep_residency() {
+    int dev = 0, n_sm = 0, per_sm = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kda_prep_kernel, PREP_NT, PREP_SMEM) !=
+            cudaSuccess)
+        return 0;
+    return n_sm * per_sm;
+}
+
 }  // namespace
 
 size_t prefill_tc_workspace(int B, int64_t T, int H, int n_seqs) {
@@ -949,8 +978,9 @@ cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, const
     }
     cudaError_t err;
     if (n_tok > 0 && slots > 0) {
-        CUtensorMap mq, mk;
-        if (!make_map(&mq, q, true, n_tok, H) || !make_map(&mk, k, true, n_tok, H))
+        CUtensorMap mq, mk, mla;
+        if (!make_map(&mq, q, true, n_tok, H) || !make_map(&mk, k, true, n_tok, H) ||
+            !make_map(&mla, log_alpha, false, n_tok, H))
             return cudaErrorInvalidValue;
         err = cudaFuncSetAttribute(kda_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                    (int)PREP_SMEM);
@@ -959,7 +989,7 @@ cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, const
                                        (int)cudaSharedmemCarveoutMaxShared);
         if (err != cudaSuccess) return err;
         kda_prep_kernel<<<dim3((unsigned)slots, (unsigned)H), PREP_NT, PREP_SMEM, stream>>>(
-            mq, mk, (const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k, log_alpha, beta,
+            mq, mk, mla, prep_residency(), (const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k, log_alpha, beta,
             blobs, chunk_off, cu_seqlens, T, H, n_seqs, nck);
         err = cudaGetLastError();
         if (err != cudaSuccess) return err;
