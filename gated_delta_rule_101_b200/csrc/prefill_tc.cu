@@ -92,7 +92,8 @@ constexpr uint32_t P_BADL = 66816;    // 128 int
 constexpr uint32_t P_BAR = 67328;     // 2 mbarriers
 constexpr uint32_t P_TMEM = 67344;
 constexpr uint32_t P_NBAD = 67348;    // number of listed bad channels
-constexpr uint32_t PREP_SMEM = 67352 + 1024;
+constexpr uint32_t P_CLAIM = 67352;   // item index handed to the worker's threads
+constexpr uint32_t PREP_SMEM = 67360 + 1024;
 constexpr uint32_t PREP_TMEM_COLS = 128;  // Gram 64, then W 128
 constexpr uint32_t PREP_TMA_BYTES = 32768;  // q, k
 static_assert(P_AKK + 64 * 68 * 4 <= P_PBUF && P_PBUF + 4608 <= P_AQK && P_AQK + 8192 <= P_GAM,
@@ -122,6 +123,7 @@ struct ChainLayout {
     static constexpr uint32_t VIMG = SIMG + N * 256;  // V_new bf16, MN-major: rows r (64), N columns
     static constexpr uint32_t BAR = VIMG + N * 128;   // 8 mbarriers
     static constexpr uint32_t TMEM = BAR + 64;
+    static constexpr uint32_t READY = TMEM + 4;       // chunks whose blobs are known ready
     static constexpr uint32_t BYTES = TMEM + 8 + 1024;
     static constexpr uint32_t TMEM_COLS = 4 * N;      // D1 (two buffers), D3, U
     // A stage is filled in two parts, each released as soon as its readers are done:
@@ -203,66 +205,134 @@ __device__ __forceinline__ void ld_chunk(const unsigned char *p, float (&v)[8]) 
     for (int e = 0; e < 8; ++e) v[e] = __bfloat162float(b[e]);
 }
 
-__global__ void __launch_bounds__(PREP_NT, 3)
-kda_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                const __grid_constant__ CUtensorMap tm_la, int pf_dist,
-                const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
-                const float *__restrict__ log_alpha, const float *__restrict__ beta,
-                unsigned char *__restrict__ ws_blobs, const int32_t *__restrict__ chunk_off,
-                const int32_t *__restrict__ cu, int64_t T, int H, int n_seqs, int nck) {
-    extern __shared__ unsigned char smem_raw[];
-    unsigned char *sm = aligned_smem(smem_raw);
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int slot = blockIdx.x, h = blockIdx.y;
+// Shared-memory stride between the prep workers of one CTA.
+constexpr uint32_t PREP_PART = ((PREP_SMEM - 1024 + 1023) / 1024) * 1024;
 
-    int seq, n;
-    if (!resolve_slot(slot, chunk_off, n_seqs, nck, seq, n)) return;
-    const SeqSpan span = seq_span(cu, T, seq);
+// Arguments of the prep work that are fixed for a launch.
+struct PrepArgs {
+    const CUtensorMap *tm_q, *tm_k, *tm_la;
+    const __nv_bfloat16 *q, *k;
+    const float *log_alpha, *beta;
+    unsigned char *ws_blobs;
+    int64_t T;
+    int H;
+};
+
+// One prep worker: 256 threads with their own shared-memory partition (PREP_SMEM
+// bytes, 1024-aligned), PREP_TMEM_COLS TMEM columns, two mbarriers and one named
+// barrier. A CTA of kda_prep_kernel is one worker; a CTA of the fused kernel runs three.
+template <bool SINGLE>
+struct PrepWorker {
+    // Everything that identifies the worker is recomputed from threadIdx (its threads
+    // are PREP_NT consecutive ones, worker g = threadIdx.x / PREP_NT), so that a loop
+    // over items keeps few values live across the item's code. SINGLE: the worker is
+    // the whole CTA (of PREP_NT threads).
+    uint32_t tma_phase;  // parity of the TMA barrier's next completion
+    bool dead;
+    // Thread 0: ready-flag index of the worker's last blob, not yet published (or -1).
+    // It is published once that blob's stores have completed, which the worker checks
+    // after issuing its next item's loads, so that the wait overlaps them.
+    int pending;
+    __device__ __forceinline__ static int g() { return SINGLE ? 0 : (int)(threadIdx.x / PREP_NT); }
+    __device__ __forceinline__ static int tid() { return SINGLE ? (int)threadIdx.x : (int)(threadIdx.x % PREP_NT); }
+    __device__ __forceinline__ static uint32_t bar_id() { return 1u + (uint32_t)g(); }
+    __device__ __forceinline__ static unsigned char *sm() {
+        extern __shared__ unsigned char smem_raw[];
+        return aligned_smem(smem_raw) + g() * PREP_PART;
+    }
+    __device__ __forceinline__ void publish_pending(int32_t *ready) {
+        if (pending >= 0) {
+            bulk_wait_all();
+            flag_publish(ready + pending);
+            pending = -1;
+        }
+    }
+    __device__ __forceinline__ static void sync() { named_bar_sync(bar_id(), PREP_NT); }
+    __device__ __forceinline__ static bool sync_or(bool p) { return named_bar_or(bar_id(), PREP_NT, p); }
+    // Worker-wide wait: thread 0 polls, the others sleep at the worker's barrier.
+    __device__ __forceinline__ void wait(uint64_t *bar, uint32_t parity) {
+        bool ok = true;
+        if (tid() == 0) ok = mbar_wait(bar, parity, dead, &g_kda_device_status);
+        dead = sync_or(!ok || dead);
+    }
+    // Barriers and TMEM; every thread of the worker calls this once, before any item.
+    // No barrier here: the first item issues its loads at once, and reads the TMEM
+    // address after its first worker barrier. `last_alloc`: no other TMEM allocation
+    // follows in this CTA, so the CTA gives up its right to allocate (a CTA that has
+    // done so may not allocate again).
+    __device__ __forceinline__ void init(bool last_alloc) {
+        tma_phase = 0;
+        dead = false;
+        pending = -1;
+        unsigned char *s = sm();
+        uint64_t *bars = reinterpret_cast<uint64_t *>(s + P_BAR);
+        if (tid() == 0) {
+            mbar_init(bars, 1);
+            mbar_init(bars + 1, 1);
+            fence_mbar_init();
+        }
+        if (tid() >> 5 == 1) {  // warp 1, so that thread 0 goes on to issue the first loads
+            tmem_alloc(reinterpret_cast<uint32_t *>(s + P_TMEM), PREP_TMEM_COLS);
+            if (last_alloc) tmem_relinquish();
+        }
+        tc_fence_before();
+    }
+    // Frees the worker's TMEM and ends its mbarriers, so that its shared memory and
+    // columns can serve another role.
+    __device__ __forceinline__ void release(int32_t *ready) {
+        tc_fence_before();
+        sync();
+        tc_fence_after();
+        unsigned char *s = sm();
+        if (tid() >> 5 == 1) tmem_dealloc(*reinterpret_cast<volatile uint32_t *>(s + P_TMEM), PREP_TMEM_COLS);
+        if (tid() == 0) {
+            publish_pending(ready);
+            uint64_t *bars = reinterpret_cast<uint64_t *>(s + P_BAR);
+            mbar_inval(bars);
+            mbar_inval(bars + 1);
+        }
+    }
+};
+
+// Prep of one (chunk, head): the chunk's gates, Grams, inverse and W, written to the
+// chunk's workspace blob. pf(x, y) is called by thread 0 after it has issued the
+// item's loads; it returns false or the coordinates of a later item's tiles, which are
+// then warmed in L2. ready != null: publish the blob's ready flag.
+template <class Worker, class Prefetch>
+__device__ __forceinline__ void prep_item(Worker &w, const PrepArgs &a, int slot, int h,
+                                          SeqSpan span, int n, Prefetch pf,
+                                          int32_t *__restrict__ ready) {
+    unsigned char *sm = Worker::sm();
+    const int tid = Worker::tid(), warp = tid >> 5, lane = tid & 31;
+    const int H = a.H;
     const int64_t tok0 = span.start + (int64_t)n * CH;
     const int L = chunk_rows(span.len, (int64_t)n * CH);
 
     uint64_t *bar_tma = reinterpret_cast<uint64_t *>(sm + P_BAR);
     uint64_t *bar_mma = bar_tma + 1;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + P_TMEM);
     float *sgam = reinterpret_cast<float *>(sm + P_GAM);
     float *sgl = reinterpret_cast<float *>(sm + P_GL);
     float *sbeta = reinterpret_cast<float *>(sm + P_BETA);
     int *badl = reinterpret_cast<int *>(sm + P_BADL);
-    bool dead = false;
 
     if (tid == 0) {
-        mbar_init(bar_tma, 1);
-        mbar_init(bar_mma, 1);
-        fence_mbar_init();
         mbar_arrive_expect_tx(bar_tma, PREP_TMA_BYTES);
         const int x = h * D, y = (int)tok0;
-        tma_load_2d(sm + P_A1, &tm_q, x, y, bar_tma);                  // q, channels 0..63
-        tma_load_2d(sm + P_A1 + 16384, &tm_q, x + 64, y, bar_tma);     // q, channels 64..127
-        tma_load_2d(sm + P_A1 + 8192, &tm_k, x, y, bar_tma);           // k -> rows 64..127
-        tma_load_2d(sm + P_A1 + 16384 + 8192, &tm_k, x + 64, y, bar_tma);
-        // Warm L2 for the CTA that starts pf_dist launches after this one (about one
-        // full residency later): its q, k and log_alpha tiles, so that its own loads
-        // find them in L2 instead of waiting on DRAM.
-        const int64_t lin = blockIdx.x + (int64_t)blockIdx.y * gridDim.x + pf_dist;
-        if (pf_dist > 0 && lin < (int64_t)gridDim.x * gridDim.y) {
-            const int pslot = (int)(lin % gridDim.x), ph = (int)(lin / gridDim.x);
-            int pseq, pn;
-            if (resolve_slot(pslot, chunk_off, n_seqs, nck, pseq, pn)) {
-                const int py = (int)(seq_span(cu, T, pseq).start + (int64_t)pn * CH), px = ph * D;
-                tma_prefetch_l2_2d(&tm_q, px, py);
-                tma_prefetch_l2_2d(&tm_q, px + 64, py);
-                tma_prefetch_l2_2d(&tm_k, px, py);
-                tma_prefetch_l2_2d(&tm_k, px + 64, py);
-                tma_prefetch_l2_2d(&tm_la, px, py);
-            }
+        tma_load_2d(sm + P_A1, a.tm_q, x, y, bar_tma);                  // q, channels 0..63
+        tma_load_2d(sm + P_A1 + 16384, a.tm_q, x + 64, y, bar_tma);     // q, channels 64..127
+        tma_load_2d(sm + P_A1 + 8192, a.tm_k, x, y, bar_tma);           // k -> rows 64..127
+        tma_load_2d(sm + P_A1 + 16384 + 8192, a.tm_k, x + 64, y, bar_tma);
+        int pf_x, pf_y;
+        if (pf(pf_x, pf_y)) {
+            tma_prefetch_l2_2d(a.tm_q, pf_x, pf_y);
+            tma_prefetch_l2_2d(a.tm_q, pf_x + 64, pf_y);
+            tma_prefetch_l2_2d(a.tm_k, pf_x, pf_y);
+            tma_prefetch_l2_2d(a.tm_k, pf_x + 64, pf_y);
+            tma_prefetch_l2_2d(a.tm_la, pf_x, pf_y);
         }
+        w.publish_pending(ready);  // the previous item's stores are the only ones in flight
     }
-    if (warp == 0) {
-        tmem_alloc(tmem_slot, PREP_TMEM_COLS);
-        tmem_relinquish();
-    }
-    if (tid < CH) sbeta[tid] = tid < L ? beta[(tok0 + tid) * H + h] : 0.f;
-    tc_fence_before();  // the TMEM address is read after the next CTA barrier
+    if (tid < CH) sbeta[tid] = tid < L ? a.beta[(tok0 + tid) * H + h] : 0.f;
 
     // ---- g = chunk-local cumulative sum of log_alpha (rows >= L count as 0), while
     //      the q / k tiles are in flight. Thread (w, f) loads rows 8w .. 8w+7, channels
@@ -272,7 +342,7 @@ kda_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     float4 g4[8];
     float gls[4], gams[4];
     {
-        const float *la = log_alpha + (tok0 * H + h) * (int64_t)D + 4 * f;
+        const float *la = a.log_alpha + (tok0 * H + h) * (int64_t)D + 4 * f;
 #pragma unroll
         for (int v = 0; v < 8; ++v) {
             const int r = 8 * warp + v;
@@ -286,7 +356,7 @@ kda_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         }
         float *gtot = reinterpret_cast<float *>(sm + P_GTOT);
         *reinterpret_cast<float4 *>(gtot + warp * D + 4 * f) = g4[7];
-        __syncthreads();
+        w.sync();
         float4 off = make_float4(0.f, 0.f, 0.f, 0.f), tot = off;
 #pragma unroll
         for (int w2 = 0; w2 < 8; ++w2) {
@@ -313,11 +383,12 @@ kda_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         any_bad |= badc[e];
     }
     // (this barrier also ends the reads of the warp totals, whose space becomes KINV)
-    const int n_bad = __syncthreads_or(any_bad) ? 1 : 0;
+    const int n_bad = w.sync_or(any_bad) ? 1 : 0;
     tc_fence_after();
-    const uint32_t tmem = *tmem_slot;
+    const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(sm + P_TMEM);
     const uint32_t sm_base = smem_u32(sm);
-    cta_wait(bar_tma, 0, dead, &g_kda_device_status);
+    w.wait(bar_tma, w.tma_phase);
+    w.tma_phase ^= 1u;
 
     // ---- gates and operand images, row by row. BAD selects the exact handling of key
     //      channels whose chunk log-decay exceeds SAFE_SPAN (kept out of the unrolled
@@ -365,11 +436,11 @@ kda_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     else gate_rows(std::false_type{});
     fence_async_smem();
     tc_fence_before();
-    __syncthreads();
+    w.sync();
 
     // Each blob image is stored as soon as it is final (bulk copies drain while the CTA
     // keeps computing): K~, exp(g_L) and the Q~ rows of A1 are final now.
-    unsigned char *blob = ws_blobs + ((size_t)slot * H + h) * BLOB_BYTES;
+    unsigned char *blob = a.ws_blobs + ((size_t)slot * H + h) * BLOB_BYTES;
     if (tid == 0) {
         bulk_s2g(blob + BLOB_KTT, sm + P_KT, 16384);
         bulk_s2g(blob + BLOB_GAM, sm + P_GAM, 512);
@@ -385,7 +456,7 @@ kda_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         mma_commit(bar_mma);
         bulk_wait_read();  // K~ has left shared memory: its space takes A_kk after the MMA
     }
-    cta_wait(bar_mma, 0, dead, &g_kda_device_status);
+    w.wait(bar_mma, 0);
     tc_fence_after();
 
     // Readout mapping: warp w reads TMEM lanes 32*(w%4) .. +31 (Gram rows m),
@@ -407,7 +478,7 @@ kda_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     if (-sgl[cc] > SAFE_SPAN) badl[cnt++] = cc;
                 *nbad = cnt;
             }
-            __syncthreads();
+            w.sync();
             const int nb_total = *nbad;
             float *bb = reinterpret_cast<float *>(sm + P_BADB);  // [8][3][64]: q, k, g per row
             for (int b0 = 0; b0 < nb_total; b0 += 8) {
@@ -416,20 +487,20 @@ kda_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     float qx = 0.f, kx = 0.f, gx = 0.f;
                     if (b0 + bi < nb_total) {
                         const int64_t ccol = (int64_t)h * D + badl[b0 + bi];
-                        float a = 0.f;
+                        float gsum = 0.f;
                         for (int j = 0; j <= r; ++j)
-                            a += j < L ? log_alpha[(tok0 + j) * H * D + ccol] : 0.f;
-                        gx = a;
+                            gsum += j < L ? a.log_alpha[(tok0 + j) * H * D + ccol] : 0.f;
+                        gx = gsum;
                         if (r < L) {
-                            qx = __bfloat162float(q[(tok0 + r) * H * D + ccol]);
-                            kx = __bfloat162float(k[(tok0 + r) * H * D + ccol]);
+                            qx = __bfloat162float(a.q[(tok0 + r) * H * D + ccol]);
+                            kx = __bfloat162float(a.k[(tok0 + r) * H * D + ccol]);
                         }
                     }
                     bb[(bi * 3 + 0) * 64 + r] = qx;
                     bb[(bi * 3 + 1) * 64 + r] = kx;
                     bb[(bi * 3 + 2) * 64 + r] = gx;
                 }
-                __syncthreads();
+                w.sync();
                 const int nb = min(8, nb_total - b0);
                 for (int bi = 0; bi < nb; ++bi) {
                     const float xr = bb[(bi * 3 + (kk_row ? 1 : 0)) * 64 + r_own];
@@ -443,7 +514,7 @@ kda_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                         acc[e] += xr * fi;
                     }
                 }
-                __syncthreads();
+                w.sync();
             }
             tmem_ld32(tmem + ((uint32_t)(32 * (warp & 3)) << 16) + cb, G);
 #pragma unroll
@@ -482,7 +553,7 @@ kda_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     else gram_readout(std::false_type{});
     fence_async_smem();
     tc_fence_before();
-    __syncthreads();
+    w.sync();
     if (tid == 0) {  // A_qk is final
         bulk_s2g(blob + BLOB_AQK, sm + P_AQK, 8192);
         bulk_commit();
@@ -520,7 +591,7 @@ kda_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 for (int r = 0; r < 16; ++r) at[(o + r) * LDT + o + l] = t[r];
             }
         }
-        __syncthreads();
+        w.sync();
         // Merges, as 16 x 8 warp-level tf32 MMA tiles.
         // level 1: blocks (16..31, 0..15) and (48..63, 32..47); warps 0-3 take one 16 x 8
         // tile each (block w/2, columns 8*(w%2) ..).
@@ -530,14 +601,14 @@ kda_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             warp_gemm_16x8<16>(d, at + (o + 16) * LDT + o, LDT, at + o * LDT + o + n0, LDT);
             warp_store_16x8(d, pb + (warp >> 1) * 16 * 20 + n0, 20, 1.f);
         }
-        __syncthreads();
+        w.sync();
         if (warp < 4) {  // T = -Z^-1 P
             const int o = 32 * (warp >> 1), n0 = 8 * (warp & 1);
             float d[4] = {0.f, 0.f, 0.f, 0.f};
             warp_gemm_16x8<16>(d, at + (o + 16) * LDT + o + 16, LDT, pb + (warp >> 1) * 16 * 20 + n0, 20);
             warp_store_16x8(d, at + (o + 16) * LDT + o + n0, LDT, -1.f);
         }
-        __syncthreads();
+        w.sync();
         // level 2: block (32..63, 0..31); warp w takes the 16 x 8 tile (rows 16*(w/4), cols 8*(w%4)).
         {  // Q = A[32.., 0..31] T[0..31, 0..31]
             const int m0 = 16 * (warp >> 2), n0 = 8 * (warp & 3);
@@ -545,7 +616,7 @@ kda_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             warp_gemm_16x8<32>(d, at + (32 + m0) * LDT, LDT, at + n0, LDT);
             warp_store_16x8(d, qb + m0 * 36 + n0, 36, 1.f);
         }
-        __syncthreads();
+        w.sync();
         {  // T[32.., 0..31] = -T[32.., 32..] Q
             const int m0 = 16 * (warp >> 2), n0 = 8 * (warp & 3);
             float d[4] = {0.f, 0.f, 0.f, 0.f};
@@ -553,7 +624,7 @@ kda_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             warp_store_16x8(d, at + (32 + m0) * LDT + n0, LDT, -1.f);
         }
         if (tid == 0) bulk_wait_read();  // A_qk has left shared memory: its space takes T Diag(beta)
-        __syncthreads();
+        w.sync();
         // image of T Diag(beta): rows r, columns i, zero above the diagonal
         {
             const int r = tid >> 2, qd = tid & 3;
@@ -575,7 +646,7 @@ kda_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     }
     fence_async_smem();
     tc_fence_before();
-    __syncthreads();
+    w.sync();
 
     // ---- W = (T Diag(beta)) (K e^g), M = 64, N = 128. K e^g sits in rows 64..127 of A1,
     //      read here as an MN-major B (K = token i). (U = T Diag(beta) V is formed by the
@@ -587,7 +658,7 @@ kda_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         mma_run<CH>(tmem, kmajor(sm_base + P_TB, 64), mnmajor(sm_base + P_A1 + 8192, 16384), idesc_bf16(64, 128, 0, 1), false);
         mma_commit(bar_mma);
     }
-    cta_wait(bar_mma, 1, dead, &g_kda_device_status);
+    w.wait(bar_mma, 1);
     tc_fence_after();
     {
         // M = 64 accumulator: row r sits in lane 16*(w%4) + (lane < 16) of quarter w%4.
@@ -612,16 +683,49 @@ kda_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     }
     fence_async_smem();
     tc_fence_before();
-    __syncthreads();
+    w.sync();
 
     if (tid == 0) {  // the W rows of A1
         bulk_s2g(blob + BLOB_A1 + 8192, sm + P_A1 + 8192, 8192);
         bulk_s2g(blob + BLOB_A1 + 16384 + 8192, sm + P_A1 + 16384 + 8192, 8192);
         bulk_commit();
-        bulk_wait_read();  // shared memory may be released; the writes complete with the grid
+        bulk_wait_read();  // shared memory may be reused; the writes complete with the grid
+        if (ready) w.pending = slot * H + h;  // a chain in the same grid waits for it
+
     }
-    __syncthreads();
-    if (warp == 0) tmem_dealloc(tmem, PREP_TMEM_COLS);
+    w.sync();  // the worker's shared memory and TMEM are free for its next item
+}
+
+
+__global__ void __launch_bounds__(PREP_NT, 3)
+kda_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                const __grid_constant__ CUtensorMap tm_la, int pf_dist,
+                const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
+                const float *__restrict__ log_alpha, const float *__restrict__ beta,
+                unsigned char *__restrict__ ws_blobs, const int32_t *__restrict__ chunk_off,
+                const int32_t *__restrict__ cu, int64_t T, int H, int n_seqs, int nck) {
+    extern __shared__ unsigned char smem_raw[];
+    const int slot = blockIdx.x, h = blockIdx.y;
+    int seq, n;
+    if (!resolve_slot(slot, chunk_off, n_seqs, nck, seq, n)) return;
+    // Warm L2 for the CTA that starts pf_dist launches after this one (about one full
+    // residency later): its q, k and log_alpha tiles, so that its own loads find them
+    // in L2 instead of waiting on DRAM.
+    auto pf = [&](int &x, int &y) {
+        const int64_t lin = blockIdx.x + (int64_t)blockIdx.y * gridDim.x + pf_dist;
+        int pseq, pn;
+        if (pf_dist <= 0 || lin >= (int64_t)gridDim.x * gridDim.y ||
+            !resolve_slot((int)(lin % gridDim.x), chunk_off, n_seqs, nck, pseq, pn))
+            return false;
+        x = (int)(lin / gridDim.x) * D;
+        y = (int)(seq_span(cu, T, pseq).start + (int64_t)pn * CH);
+        return true;
+    };
+    const PrepArgs a{&tm_q, &tm_k, &tm_la, q, k, log_alpha, beta, ws_blobs, T, H};
+    PrepWorker<true> w;
+    w.init(true);
+    prep_item(w, a, slot, h, seq_span(cu, T, seq), n, pf, nullptr);
+    w.release(nullptr);
 }
 
 // =====================================================================================
@@ -642,26 +746,54 @@ constexpr int CHAIN_NT = 32 * (CHAIN_EPI_WARPS + 1);
 //             the chunk's TMEM reads are done. It also ORs the threads' `dead` flags,
 //             so all warps leave the loop at the same chunk and the barriers' arrivals
 //             always pair up, even after a bounded wait has given up.
+//   BAR_CHAIN: all 288 threads, around the prologue and the epilogue.
 constexpr uint32_t BAR_VNEW = 1, BAR_VNEW_COUNT = 32 * 5;
 constexpr uint32_t BAR_END = 2;
+constexpr uint32_t BAR_CHAIN = 3;
 
-template <int N>
-__global__ void __launch_bounds__(CHAIN_NT, 1)
-kda_chain_kernel(const __grid_constant__ CUtensorMap tm_v,
-                 const unsigned char *__restrict__ ws_blobs, const int32_t *__restrict__ chunk_off,
-                 const float *__restrict__ S0, __nv_bfloat16 *__restrict__ o,
-                 float *__restrict__ S_T, const int32_t *__restrict__ cu, int64_t T, int H,
-                 int nck) {
+// Arguments of the chain work that are fixed for a launch.
+struct ChainArgs {
+    const CUtensorMap *tm_v;
+    const unsigned char *ws_blobs;
+    const int32_t *chunk_off;
+    const float *S0;
+    __nv_bfloat16 *o;
+    float *S_T;
+    const int32_t *cu;
+    int64_t T;
+    int H;
+    int nck;
+    const int32_t *ready;  // non-null: wait for each blob's ready flag before reading it
+};
+
+// The state recurrence of one (sequence, head, N-column value slice), run by threads
+// 0 .. CHAIN_NT-1 of the CTA (tid) on shared memory `sm` (1024-aligned,
+// ChainLayout<N>::BYTES - 1024 bytes). ROLE 0: the calling thread's warp decides its
+// part. ROLE 1 / 2: compiled for the epilogue warps / the MMA warp only, so that each
+// can run under its own register budget. With a.ready set (blobs produced by prep
+// workers of the same grid), a watcher warp (ROLE 3, threads CHAIN_NT .. +31) reads
+// the blobs' ready flags in chunk order and raises a shared counter, so the threads
+// that issue the loads only poll shared memory.
+template <int N, int ROLE = 0>
+__device__ __forceinline__ void chain_task(unsigned char *sm, const int tid, const ChainArgs &a,
+                                           const int seq, const int h, const int j0) {
     static_assert(N == 64 || N == 128, "value slices of 64 or 128 columns");
     constexpr int NH = N / 2;  // columns per epilogue thread
     using Lay = ChainLayout<N>;
-    extern __shared__ unsigned char smem_raw[];
-    unsigned char *sm = aligned_smem(smem_raw);
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const bool issuer = warp == CHAIN_EPI_WARPS;
+    const int warp = tid >> 5, lane = tid & 31;
+    const bool issuer = ROLE == 0 ? warp == CHAIN_EPI_WARPS : ROLE == 2;
+    const bool epi = ROLE == 0 ? warp < CHAIN_EPI_WARPS : ROLE == 1;
+    const uint32_t bar_chain_count = a.ready ? CHAIN_NT + 32 : CHAIN_NT;  // + the watcher
     const int q4 = warp & 3, hf = (warp >> 2) & 1;
-    const int seq = blockIdx.x, h = blockIdx.y, j0 = blockIdx.z * N;
-    const SeqSpan span = seq_span(cu, T, seq);
+    const CUtensorMap &tm_v = *a.tm_v;
+    const unsigned char *ws_blobs = a.ws_blobs;
+    const int32_t *chunk_off = a.chunk_off;
+    const float *S0 = a.S0;
+    __nv_bfloat16 *o = a.o;
+    float *S_T = a.S_T;
+    const int64_t T = a.T;
+    const int H = a.H, nck = a.nck;
+    const SeqSpan span = seq_span(a.cu, T, seq);
     const int nchunks = (int)((span.len + CH - 1) / CH);
     const int64_t slot0 = chunk_off ? (int64_t)chunk_off[seq] : (int64_t)seq * nck;
     const int64_t state_off = ((int64_t)seq * H + h) * (int64_t)(D * D);
@@ -672,9 +804,11 @@ kda_chain_kernel(const __grid_constant__ CUtensorMap tm_v,
     uint64_t *bar_b = bar_ld1 + 5;    // state MMA done
     uint64_t *bar_c = bar_ld1 + 6;    // [2] output MMA done, per D1 buffer
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + Lay::TMEM);
+    int32_t *ready_upto = reinterpret_cast<int32_t *>(sm + Lay::READY);
     bool dead = false;
 
     auto blob_of = [&](int chunk) {
+        if (a.ready) counter_wait_gt(ready_upto, chunk, dead, &g_kda_device_status);
         return ws_blobs + ((size_t)(slot0 + chunk) * H + h) * BLOB_BYTES;
     };
     auto issue_load1 = [&](int chunk, int stage) {
@@ -699,6 +833,7 @@ kda_chain_kernel(const __grid_constant__ CUtensorMap tm_v,
 
     if (tid == 0) {
         for (int b = 0; b < 8; ++b) mbar_init(&bar_ld1[b], 1);
+        *ready_upto = 0;
         fence_mbar_init();
     }
     if (warp == 0) {
@@ -708,7 +843,7 @@ kda_chain_kernel(const __grid_constant__ CUtensorMap tm_v,
     const int c = 32 * q4 + lane;    // state row owned by an epilogue thread
     const int jh = NH * hf;          // first of its NH value columns (inside the slice)
     float s_reg[NH];
-    if (!issuer) {
+    if (epi) {
 #pragma unroll
         for (int j = 0; j < NH; j += 4) {
             float4 v4 = S0 ? *reinterpret_cast<const float4 *>(S0 + state_off + (int64_t)c * D + j0 + jh + j)
@@ -725,15 +860,24 @@ kda_chain_kernel(const __grid_constant__ CUtensorMap tm_v,
     }
     fence_async_smem();
     tc_fence_before();
-    __syncthreads();
+    named_bar_sync(BAR_CHAIN, bar_chain_count);
     tc_fence_after();
-    const uint32_t tmem = *tmem_slot;
+    const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(tmem_slot);
     const uint32_t d3 = tmem + 2 * N;  // D1 buffers at columns 0 and N
     const uint32_t du = tmem + 3 * N;  // U = T Diag(beta) V (rows 64..127)
     const uint32_t sm_base = smem_u32(sm);
     const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
 
-    if (issuer) {
+    if (ROLE == 3) {
+        // ------------------------------------------------------------ flag watcher
+        if (lane == 0) {
+            for (int m = 0; m < nchunks; ++m) {
+                if (!flag_wait(a.ready + (size_t)(slot0 + m) * H + h, dead, &g_kda_device_status)) break;
+                st_release_cta(ready_upto, m + 1);
+            }
+        }
+        __syncwarp();
+    } else if (issuer) {
         // ------------------------------------------------------------ MMA / load warp
         if (lane == 0) {
             for (int m = 0; m < 2 && m < nchunks; ++m) {
@@ -884,8 +1028,116 @@ kda_chain_kernel(const __grid_constant__ CUtensorMap tm_v,
         }
     }
     tc_fence_before();
-    __syncthreads();
+    named_bar_sync(BAR_CHAIN, bar_chain_count);
     if (warp == 0) tmem_dealloc(tmem, Lay::TMEM_COLS);
+}
+
+template <int N>
+__global__ void __launch_bounds__(CHAIN_NT, 1)
+kda_chain_kernel(const __grid_constant__ CUtensorMap tm_v,
+                 const unsigned char *__restrict__ ws_blobs, const int32_t *__restrict__ chunk_off,
+                 const float *__restrict__ S0, __nv_bfloat16 *__restrict__ o,
+                 float *__restrict__ S_T, const int32_t *__restrict__ cu, int64_t T, int H,
+                 int nck) {
+    extern __shared__ unsigned char smem_raw[];
+    const ChainArgs a{&tm_v, ws_blobs, chunk_off, S0, o, S_T, cu, T, H, nck, nullptr};
+    chain_task<N>(aligned_smem(smem_raw), threadIdx.x, a, blockIdx.x, blockIdx.y, blockIdx.z * N);
+}
+
+// =====================================================================================
+// fused: prep and chain in one cooperative grid (batched inputs)
+// =====================================================================================
+// One CTA of FUSED_NT threads per SM, all resident at once (cooperative launch). Each
+// CTA starts as three prep workers that take (chunk, head) items from a queue in
+// chunk order: items of the first n_first chunks are shared by all CTAs, the rest go
+// only to CTAs that never run a chain. Once the shared items are all claimed, CTA
+// b < n_chain finishes its items and becomes the chain of task b = (seq H + h) D/N +
+// slice; a watcher warp of that CTA follows the blobs' ready flags. Prep workers never
+// wait on a chain, so every flag a chain waits for is eventually set. n_first is chosen
+// so that the CTAs left on prep finish the remaining items about when the chains need
+// them.
+constexpr int FUSED_NT = 3 * PREP_NT;
+template <int N>
+constexpr uint32_t fused_smem() {
+    return (3 * PREP_PART > ChainLayout<N>::BYTES - 1024 ? 3 * PREP_PART : ChainLayout<N>::BYTES - 1024) + 1024;
+}
+static_assert(fused_smem<128>() <= 232448, "fused CTA exceeds the shared memory of an SM");
+// Registers per thread in the chain role: epilogue warpgroups 0-1 get FUSED_REG_EPI,
+// warpgroup 2 (the MMA warp, the watcher and two idle warps) 72, idle warpgroups 3-5
+// drop to 24. Their sum must stay within the launch's 80 per thread.
+template <int N>
+__host__ __device__ constexpr int fused_reg_epi() { return N == 64 ? 144 : 168; }
+constexpr int FUSED_REG_MMA = 72, FUSED_REG_IDLE = 24;
+static_assert(256 * 168 + 128 * FUSED_REG_MMA + 384 * FUSED_REG_IDLE <= FUSED_NT * 80,
+              "register split exceeds the launch's registers");
+
+struct FusedQueue {
+    int32_t next_shared;  // items of the first n_first chunks, claimed by every CTA
+    int32_t next_rest;    // the other items, claimed by prep-only CTAs
+};
+
+template <int N>
+__global__ void __launch_bounds__(FUSED_NT, 1)
+kda_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                 const __grid_constant__ CUtensorMap tm_la, const __grid_constant__ CUtensorMap tm_v,
+                 const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
+                 const float *__restrict__ log_alpha, const float *__restrict__ beta,
+                 unsigned char *__restrict__ ws_blobs, int32_t *__restrict__ ready,
+                 FusedQueue *__restrict__ queue, const float *__restrict__ S0,
+                 __nv_bfloat16 *__restrict__ o, float *__restrict__ S_T, int64_t T, int H, int B,
+                 int nck, int n_first, int n_chain) {
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char *sm = aligned_smem(smem_raw);
+    const int tid = threadIdx.x, g = tid / PREP_NT;
+    const int P = B * H;
+    const int n_shared = n_first * P, n_total = nck * P;
+    const bool chain_cta = (int)blockIdx.x < n_chain;
+    {
+        const PrepArgs pa{&tm_q, &tm_k, &tm_la, q, k, log_alpha, beta, ws_blobs, T, H};
+        using Worker = PrepWorker<false>;
+        Worker w;
+        w.init(false);
+        volatile int32_t *claim = reinterpret_cast<volatile int32_t *>(Worker::sm() + P_CLAIM);
+        for (;;) {
+            if (Worker::tid() == 0) {
+                int it = atomicAdd(&queue->next_shared, 1);
+                if (it >= n_shared) it = chain_cta ? -1 : n_shared + atomicAdd(&queue->next_rest, 1);
+                *claim = it < n_total ? it : -1;
+            }
+            Worker::sync();
+            const int it = *claim;  // read before the item's first barrier; rewritten after it
+            if (it < 0 || w.dead) break;
+            const int n = it / P, p = it % P, seq = p / H, h = p % H;
+            // warm L2 for the item about one round of all workers later
+            auto pf = [&](int &x, int &y) {
+                const int pit = it + 3 * (int)gridDim.x;
+                if (pit >= n_total) return false;
+                const int pp = pit % P;
+                x = (pp % H) * D;
+                y = (int)((int64_t)(pp / H) * T + (int64_t)(pit / P) * CH);
+                return true;
+            };
+            prep_item(w, pa, seq * nck + n, h, SeqSpan{(int64_t)seq * T, T}, n, pf, ready);
+        }
+        w.release(ready);
+    }
+    __syncthreads();  // every worker is done: shared memory and TMEM pass to the chain
+    if (!chain_cta) return;
+    const int wg = tid >> 7;
+    const ChainArgs ca{&tm_v, ws_blobs, nullptr, S0, o, S_T, nullptr, T, H, nck, ready};
+    constexpr int SLICES = D / N;
+    const int task = blockIdx.x, pair = task / SLICES, seq = pair / H, h = pair % H;
+    const int j0 = (task % SLICES) * N;
+    if (wg < 2) {
+        setmaxnreg_inc<fused_reg_epi<N>()>();
+        chain_task<N, 1>(sm, tid, ca, seq, h, j0);
+    } else if (wg == 2) {
+        setmaxnreg_dec<FUSED_REG_MMA>();
+        if (tid < CHAIN_NT) chain_task<N, 2>(sm, tid, ca, seq, h, j0);
+        else if (tid < CHAIN_NT + 32) chain_task<N, 3>(sm, tid, ca, seq, h, j0);
+    } else {
+        setmaxnreg_dec<FUSED_REG_IDLE>();
+    }
 }
 
 // =====================================================================================
@@ -948,14 +1200,79 @@ int prep_residency() {
 
 }  // namespace
 
+// Workspace of batched inputs: one ready flag per blob and the fused kernel's queue,
+// then the blobs.
+size_t batched_head_bytes(int B, int nck, int H) {
+    return (((size_t)B * nck * H * 4 + sizeof(FusedQueue) + 255) / 256) * 256;
+}
+
+// Plan of the fused kernel for batched inputs. The model (B200 measurements): a prep
+// worker finishes an item about every PREP_US, three per SM; a chain takes about
+// CHAIN_US[N] per chunk. With n_chain chain CTAs, the other SMs produce the items of
+// the last chunks while the chains run; the split puts the end of that production at
+// about the end of the chains. The two-kernel path (prep on every SM, then the
+// chains) is kept when the model gives the fused kernel no clear gain.
+struct FusedPlan {
+    int n;        // value columns per chain CTA (64 or 128); 0: do not fuse
+    int n_first;  // chunks whose items every CTA shares
+};
+bool fused_supported() {
+    static int ok = -1;  // device capabilities, queried once
+    if (ok < 0) {
+        int dev = 0, coop = 0, per64 = 0, per128 = 0;
+        ok = cudaGetDevice(&dev) == cudaSuccess &&
+             cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev) == cudaSuccess && coop &&
+             cudaFuncSetAttribute(kda_fused_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)fused_smem<64>()) == cudaSuccess &&
+             cudaFuncSetAttribute(kda_fused_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)fused_smem<128>()) == cudaSuccess &&
+             cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per64, kda_fused_kernel<64>, FUSED_NT,
+                                                           fused_smem<64>()) == cudaSuccess &&
+             cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per128, kda_fused_kernel<128>, FUSED_NT,
+                                                           fused_smem<128>()) == cudaSuccess &&
+             per64 >= 1 && per128 >= 1;
+    }
+    return ok == 1;
+}
+FusedPlan fused_plan(int B, int H, int nck, int n_sm) {
+    constexpr double PREP_US = 16.5, CHAIN_US_64 = 1.45, CHAIN_US_128 = 2.3;
+    constexpr int MIN_PREP_CTAS = 8;
+    const int P = B * H;
+    const double r = 3.0 / PREP_US;  // items per microsecond per SM
+    if ((int64_t)nck * P >= (1ll << 30) || !fused_supported()) return {0, 0};
+    // the two-kernel path: prep on every SM, then the chains in waves
+    const int n2 = P >= n_sm ? 128 : 64;
+    const double waves = (double)((P * (D / n2) + n_sm - 1) / n_sm);
+    const double t_two = nck * (double)P / (n_sm * r) + waves * nck * (n2 == 64 ? CHAIN_US_64 : CHAIN_US_128);
+    FusedPlan best{0, 0};
+    double t_best = 0.95 * t_two;
+    for (int n : {64}) {  // 128-column chains run about 2.3 us per chunk here: no gain
+        const int n_chain = P * (D / n);
+        if (n_chain + MIN_PREP_CTAS > n_sm) continue;
+        const double tau = n == 64 ? CHAIN_US_64 : CHAIN_US_128;
+        const int n_prep = n_sm - n_chain;
+        int n_first = nck - (int)((double)nck * tau * n_prep * r / P);
+        const int lo = nck < 2 ? nck : 2;
+        n_first = n_first < lo ? lo : (n_first > nck ? nck : n_first);
+        const double t_a = (double)n_first * P / (n_sm * r);
+        const double t_b = (double)(nck - n_first) * P / (n_prep * r);
+        const double t = t_a + (nck * tau > t_b ? nck * tau : t_b);
+        if (t < t_best) {
+            t_best = t;
+            best = {n, n_first};
+        }
+    }
+    return best;
+}
+
 size_t prefill_tc_workspace(int B, int64_t T, int H, int n_seqs) {
     if (n_seqs > 0) {
         const size_t head = (((size_t)(n_seqs + 1) * 4 + 255) / 256) * 256;
         const size_t slots = (size_t)(T / CH) + (size_t)n_seqs;
         return head + slots * (size_t)H * BLOB_BYTES;
     }
-    const size_t nck = (size_t)((T + CH - 1) / CH);
-    return (size_t)B * nck * (size_t)H * BLOB_BYTES;
+    const int nck = (int)((T + CH - 1) / CH);
+    return batched_head_bytes(B, nck, H) + (size_t)B * nck * (size_t)H * BLOB_BYTES;
 }
 
 cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, const float *log_alpha,
@@ -970,11 +1287,38 @@ cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, const
     int32_t *chunk_off = nullptr;
     unsigned char *blobs = ws;
     int64_t slots = (int64_t)B * nck;
+    int dev = 0, n_sm = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess)
+        cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
     if (packed) {
         chunk_off = reinterpret_cast<int32_t *>(ws);
         blobs = ws + (((size_t)(n_seqs + 1) * 4 + 255) / 256) * 256;
         slots = T / CH + n_seqs;
         chunk_offsets_kernel<<<1, 1024, 0, stream>>>(cu_seqlens, n_seqs, chunk_off);
+    } else {
+        blobs = ws + batched_head_bytes(B, nck, H);
+        const FusedPlan plan = n_tok > 0 ? fused_plan(B, H, nck, n_sm) : FusedPlan{0, 0};
+        if (plan.n) {
+            int32_t *ready = reinterpret_cast<int32_t *>(ws);
+            FusedQueue *queue = reinterpret_cast<FusedQueue *>(ready + (size_t)B * nck * H);
+            cudaError_t err = cudaMemsetAsync(ws, 0, (size_t)B * nck * H * 4 + sizeof(FusedQueue), stream);
+            if (err != cudaSuccess) return err;
+            CUtensorMap mq, mk, mla, mv;
+            if (!make_map(&mq, q, true, n_tok, H) || !make_map(&mk, k, true, n_tok, H) ||
+                !make_map(&mla, log_alpha, false, n_tok, H) || !make_map(&mv, v, true, n_tok, H))
+                return cudaErrorInvalidValue;
+            const __nv_bfloat16 *qb = (const __nv_bfloat16 *)q, *kb = (const __nv_bfloat16 *)k;
+            __nv_bfloat16 *ob = (__nv_bfloat16 *)o;
+            int n_chain = B * H * (D / plan.n), n_first = plan.n_first;
+            void *args[] = {&mq, &mk, &mla, &mv, &qb, &kb, (void *)&log_alpha, (void *)&beta, &blobs,
+                            &ready, &queue, (void *)&S0, &ob, &S_T, &T, &H, &B, (void *)&nck,
+                            &n_first, &n_chain};
+            if (plan.n == 64)
+                return cudaLaunchCooperativeKernel((const void *)kda_fused_kernel<64>, dim3((unsigned)n_sm),
+                                                   dim3(FUSED_NT), args, fused_smem<64>(), stream);
+            return cudaLaunchCooperativeKernel((const void *)kda_fused_kernel<128>, dim3((unsigned)n_sm),
+                                               dim3(FUSED_NT), args, fused_smem<128>(), stream);
+        }
     }
     cudaError_t err;
     if (n_tok > 0 && slots > 0) {
@@ -998,9 +1342,6 @@ cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, const
     if (n_tok > 0 && !make_map(&mv, v, true, n_tok, H)) return cudaErrorInvalidValue;
     // 128-column slices (one CTA per sequence-head) when there are enough pairs to fill
     // the GPU; otherwise 64-column slices for twice the parallelism.
-    int dev = 0, n_sm = 148;
-    if (cudaGetDevice(&dev) == cudaSuccess)
-        cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
     if ((int64_t)nseq * H >= n_sm) return launch_chain<128>(mv, blobs, chunk_off, S0, o, S_T, cu_seqlens, T, H, nck, nseq, stream);
     return launch_chain<64>(mv, blobs, chunk_off, S0, o, S_T, cu_seqlens, T, H, nck, nseq, stream);
 }

@@ -19,6 +19,10 @@ __device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count)
                  : "memory");
 }
+// Ends an mbarrier's life; required before its memory is used for anything else.
+__device__ __forceinline__ void mbar_inval(uint64_t *bar) {
+    asm volatile("mbarrier.inval.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
 __device__ __forceinline__ void fence_mbar_init() {
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
 }
@@ -58,6 +62,81 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, bool &
     const uint64_t t0 = global_ns();
     for (uint32_t i = 1;; ++i) {
         if (mbar_try_wait(bar, parity)) return true;
+        if ((i & 255u) == 0) {
+            if (*reinterpret_cast<volatile int *>(status) != 0 || global_ns() - t0 > WAIT_LIMIT_NS)
+                break;
+        }
+    }
+    dead = true;
+    atomicExch(status, 1);
+    return false;
+}
+
+// ------------------------------------------------------------------ cross-CTA flags
+// Between CTAs of one cooperative grid (all resident at once): a producer publishes
+// data it wrote to global memory with bulk copies by waiting for the copies to
+// complete, then flag_publish; a consumer that sees the flag set (flag_wait) may then
+// read that data, also with bulk copies. The producer must never wait on its consumer.
+__device__ __forceinline__ void fence_proxy_async_global() {
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+__device__ __forceinline__ void flag_publish(int32_t *flag) {
+    fence_proxy_async_global();
+    asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(flag), "r"(1) : "memory");
+}
+__device__ __forceinline__ int32_t ld_acquire_gpu(const int32_t *p) {
+    int32_t v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+// Waits until *flag != 0, with the same limit and failure reporting as mbar_wait.
+__device__ __forceinline__ bool flag_wait(const int32_t *flag, bool &dead, int *status) {
+    if (dead) return false;
+    if (ld_acquire_gpu(flag) != 0) {
+        fence_proxy_async_global();
+        return true;
+    }
+    const uint64_t t0 = global_ns();
+    for (uint32_t i = 1;; ++i) {
+        __nanosleep(100);
+        if (ld_acquire_gpu(flag) != 0) {
+            fence_proxy_async_global();
+            return true;
+        }
+        if ((i & 63u) == 0) {
+            if (*reinterpret_cast<volatile int *>(status) != 0 || global_ns() - t0 > WAIT_LIMIT_NS)
+                break;
+        }
+    }
+    dead = true;
+    atomicExch(status, 1);
+    return false;
+}
+
+// Counter in shared memory raised by one thread and read by others in the CTA.
+__device__ __forceinline__ int32_t ld_acquire_cta(const int32_t *p) {
+    int32_t v;
+    asm volatile("ld.acquire.cta.shared::cta.b32 %0, [%1];" : "=r"(v) : "r"(smem_u32(p)) : "memory");
+    return v;
+}
+__device__ __forceinline__ void st_release_cta(int32_t *p, int32_t v) {
+    asm volatile("st.release.cta.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(p)), "r"(v) : "memory");
+}
+// Waits until the shared counter *p exceeds v, with the limit and failure reporting of
+// mbar_wait; the counter's writer has seen global data the caller will then read with
+// bulk copies.
+__device__ __forceinline__ bool counter_wait_gt(const int32_t *p, int32_t v, bool &dead, int *status) {
+    if (dead) return false;
+    if (ld_acquire_cta(p) > v) {
+        fence_proxy_async_global();
+        return true;
+    }
+    const uint64_t t0 = global_ns();
+    for (uint32_t i = 1;; ++i) {
+        if (ld_acquire_cta(p) > v) {
+            fence_proxy_async_global();
+            return true;
+        }
         if ((i & 255u) == 0) {
             if (*reinterpret_cast<volatile int *>(status) != 0 || global_ns() - t0 > WAIT_LIMIT_NS)
                 break;
@@ -142,6 +221,19 @@ __device__ __forceinline__ void tma_prefetch_l2_2d(const CUtensorMap *map, int x
                      reinterpret_cast<uint64_t>(map)),
                  "r"(x), "r"(y)
                  : "memory");
+}
+
+// ------------------------------------------------------------------ register budget
+// Moves registers between the warpgroups of a CTA (all four warps of a warpgroup
+// execute it). The counts must be multiples of 8 in [24, 256], and the increases of
+// all warpgroups together must not exceed what the decreases and the launch leave.
+template <int R>
+__device__ __forceinline__ void setmaxnreg_inc() {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(R));
+}
+template <int R>
+__device__ __forceinline__ void setmaxnreg_dec() {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(R));
 }
 
 // ------------------------------------------------------------------ tcgen05
