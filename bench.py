@@ -34,6 +34,8 @@ sys.path.insert(0, ROOT)
 METRIC = "KDA prefill tokens/s + decode tokens/s on 1 B200; % of tensor/HBM roofline"
 PREFILL = dict(B=4, T=4096, H=16, s0_std=0.1, la_range=(0.001, 0.1), seed=20261)
 DECODE = dict(N=256, H=32, steps=1024, s0_std=0.1, la_range=(0.001, 0.1), seed=20263)
+VARLEN = dict(n_seqs=64, len_range=(512, 16384), H=32, la_range=(0.001, 0.1), seed=20262)
+LONG = dict(T_call=65536, calls=16, H=32, la_range=(0.0001, 0.05), seed=20264)
 L2_FLUSH_BYTES = 256 << 20  # larger than the 126 MB L2
 D = 128
 # algorithmic bytes (single pass) per token-head: q,k,v,o bf16 + log_alpha fp32 + beta fp32
@@ -218,7 +220,8 @@ def prefill_config(world: int) -> dict:
     return {"workload": f"KDA prefill B={B} T={T} H={H} d=128 C=64, bf16 q/k/v, fp32 log_alpha/beta/"
                         "state, S0~N(0,0.1^2)",
             "global_batch": B * world, "seq_len": T, "parallelism": f"dp{world}",
-            "l2": "flushed before every step (256 MiB write); inputs 412 MB > L2"}
+            "l2": f"flushed before every step (256 MiB write); the step moves "
+                  f"{(PREFILL_BYTES_PER_TOKEN_HEAD * B * T * H + 2 * STATE_BYTES * B * H) / 1e6:.0f} MB"}
 
 
 # ------------------------------------------------------------------ arms
@@ -262,6 +265,79 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
+def other_prefill_workloads(kda, dev, stream, flush, pk, world, rank):
+    """The packed variable-length batch and the long-context sequence, each timed on
+    the device (CUDA events on the launching stream, L2 flushed before the packed call;
+    the long-context calls stream 3.2 GB of inputs each, far more than L2)."""
+    from gated_delta_rule_101_b200.inputs import cu_from_lengths, prefill_inputs, varlen_lengths
+
+    out = {}
+    barrier(world)
+    # packed: 64 sequences, lengths ~ U[512, 16384], H = 32, S0 = 0
+    lengths = varlen_lengths(VARLEN["n_seqs"], *VARLEN["len_range"], seed=VARLEN["seed"] + 1000 * rank)
+    cu = cu_from_lengths(lengths)
+    T, H = int(cu[-1]), VARLEN["H"]
+    inp = prefill_inputs(T=T, H=H, cu_seqlens=cu, dtype=torch.bfloat16, la_range=VARLEN["la_range"],
+                         seed=VARLEN["seed"] + 1000 * rank, device=dev)
+    o = torch.empty_like(inp.v)
+    S_T = torch.empty(len(lengths), H, 128, 128, device=dev)
+    ws = torch.empty(kda.workspace_size(1, T, H, len(lengths)), dtype=torch.uint8, device=dev)
+    n_l = kda.chunk_fwd_launches(1, T, H, len(lengths))
+
+    def call():
+        kda.chunk_fwd(inp.q, inp.k, inp.v, inp.log_alpha, inp.beta, None, cu_seqlens=inp.cu_seqlens,
+                      out=o, state_out=S_T, workspace=ws, stream=stream)
+
+    times = time_steps(call, 3, 3, stream, flush)
+    ms = max_over_ranks(sum(times), world, dev) / len(times)
+    alg = PREFILL_BYTES_PER_TOKEN_HEAD * T * H + 2 * STATE_BYTES * len(lengths) * H
+    out["varlen"] = {"value": T * world / (ms * 1e-3), "unit": "tokens/s", "ms_per_call": ms,
+                     "config": {"workload": f"KDA packed prefill, {len(lengths)} sequences "
+                                            f"(lengths U[{VARLEN['len_range'][0]}, "
+                                            f"{VARLEN['len_range'][1]}], {T} tokens), H={H}, bf16",
+                                "l2": "flushed before every call; inputs far above L2"},
+                     "roofline": {"bound": "hbm", "achieved": alg / (ms * 1e-3) / 1e9,
+                                  "peak": pk["hbm_gbs"], "unit": "GB/s",
+                                  "frac": alg / (ms * 1e-3) / 1e9 / pk["hbm_gbs"],
+                                  "alg_bytes_per_launch": alg},
+                     "gpu_launches": n_l * len(times)}
+    del inp, o, S_T, ws
+    torch.cuda.empty_cache()
+    # long context: 2^20 tokens as 16 calls of 65,536 with the state carried in place
+    Tc, H, calls = LONG["T_call"], LONG["H"], LONG["calls"]
+    inps = [prefill_inputs(B=1, T=Tc, H=H, dtype=torch.bfloat16, la_range=LONG["la_range"],
+                           seed=LONG["seed"] * 100 + c + 1000 * rank, device=dev) for c in range(2)]
+    S = torch.zeros(1, H, 128, 128, device=dev)
+    o = torch.empty_like(inps[0].v)
+    ws = torch.empty(kda.workspace_size(1, Tc, H), dtype=torch.uint8, device=dev)
+    n_l = kda.chunk_fwd_launches(1, Tc, H)
+
+    def sequence():
+        S.zero_()
+        for c in range(calls):  # two input sets alternate: the data differs, the work does not
+            x = inps[c % 2]
+            kda.chunk_fwd(x.q, x.k, x.v, x.log_alpha, x.beta, S, out=o, state_out=S, workspace=ws,
+                          stream=stream)
+
+    times = time_steps(sequence, 2, 3, stream)
+    ms = max_over_ranks(sum(times), world, dev) / len(times)
+    alg = (PREFILL_BYTES_PER_TOKEN_HEAD * Tc * H + 2 * STATE_BYTES * H) * calls
+    out["long_context"] = {"value": Tc * calls * world / (ms * 1e-3), "unit": "tokens/s",
+                           "ms_per_sequence": ms, "ms_per_call": ms / calls,
+                           "config": {"workload": f"KDA long-context prefill, one sequence of "
+                                                  f"{Tc * calls} tokens as {calls} calls of {Tc} "
+                                                  f"with S_T carried as the next S0, H={H}, bf16",
+                                      "l2": "not flushed; each call streams 3.2 GB of inputs"},
+                           "roofline": {"bound": "hbm", "achieved": alg / (ms * 1e-3) / 1e9,
+                                        "peak": pk["hbm_gbs"], "unit": "GB/s",
+                                        "frac": alg / (ms * 1e-3) / 1e9 / pk["hbm_gbs"],
+                                        "alg_bytes_per_launch": alg / calls},
+                           "gpu_launches": n_l * calls * len(times)}
+    del inps, S, o, ws
+    torch.cuda.empty_cache()
+    return out
+
+
 def run_kda(args, rank, world, local_rank):
     import gated_delta_rule_101_b200 as kda
     from gated_delta_rule_101_b200.inputs import decode_inputs, prefill_inputs
@@ -301,7 +377,7 @@ def run_kda(args, rank, world, local_rank):
     ms_per_step = total_ms / args.steps
     tokens_per_step = B * T * world
     value = tokens_per_step / (ms_per_step * 1e-3)
-    launches_per_call = 1
+    launches_per_call = kda.chunk_fwd_launches(B, T, H)
     avg_kernel_s = sum(times) / len(times) * 1e-3
     alg_bytes = PREFILL_BYTES_PER_TOKEN_HEAD * B * T * H + 2 * STATE_BYTES * B * H
     achieved = alg_bytes / avg_kernel_s / 1e9
@@ -310,7 +386,9 @@ def run_kda(args, rank, world, local_rank):
     roofline = {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
                 "frac": achieved / pk["hbm_gbs"], "traffic": traffic("prefill", args.traffic),
                 "peak_source": pk_kind,
-                "kernel": "kda_chunk_fwd: kda_prep_kernel + kda_chain_kernel (one call, timed together)",
+                "kernel": "kda_chunk_fwd (one call, timed as a whole): "
+                          + ("kda_prep_kernel + kda_chain_kernel" if launches_per_call == 2
+                             else "kda_fused_kernel"),
                 "alg_bytes_per_launch": alg_bytes,
                 "tensor_pages_flops": {"achieved_tflops": tflops, "peak": pk["bf16_tflops"],
                                        "frac": tflops / pk["bf16_tflops"],
@@ -382,6 +460,9 @@ def run_kda(args, rank, world, local_rank):
                   "gpu_launches": nsteps * len(d_times), "clocks": dclk}
         del graph, dinp, S, od
 
+    # ---------------- the other prefill workloads (reported beside the step, not the step)
+    extra = {} if args.no_extra else other_prefill_workloads(kda, dev, stream, flush, pk, world, rank)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_oracle_sample(inp)
@@ -393,7 +474,8 @@ def run_kda(args, rank, world, local_rank):
                 "data": "synthetic",
                 "config": prefill_config(world),
                 "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
-                "gpu_launches": launches_per_call * args.steps, "clocks": clk, "decode": decode}
+                "gpu_launches": launches_per_call * args.steps, "clocks": clk, "decode": decode,
+                **extra}
         print(json.dumps(line), flush=True)
 
 
@@ -405,6 +487,10 @@ def main():
     ap.add_argument("--impl", choices=["kda", "reference"], default="kda")
     ap.add_argument("--decode-steps", type=int, default=DECODE["steps"])
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="skip the packed and long-context prefill workloads")
+    ap.add_argument("--shape", default=None,
+                    help="B,T,H of the prefill step instead of 4,4096,16 (for profiling captures)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true",
                     help="skip the host-buffer end-to-end leg (for short profiling runs)")
@@ -415,6 +501,12 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.shape:
+        try:
+            B, T, H = (int(x) for x in args.shape.split(","))
+        except ValueError:
+            ap.error("--shape takes B,T,H")
+        PREFILL.update(B=B, T=T, H=H)
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

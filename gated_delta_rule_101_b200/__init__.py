@@ -50,6 +50,8 @@ def _bind(lib: ctypes.CDLL) -> ctypes.CDLL:
     lib.kda_chunk_fwd_workspace_size.restype = i32
     lib.kda_chunk_fwd_workspace_size.argtypes = [i32, i64, i32, i32, i32, i32,
                                                  ctypes.POINTER(ctypes.c_size_t)]
+    lib.kda_chunk_fwd_launches.restype = i32
+    lib.kda_chunk_fwd_launches.argtypes = [i32, i64, i32, i32, i32, i32, ctypes.POINTER(ctypes.c_int)]
     lib.kda_chunk_fwd.restype = i32
     lib.kda_chunk_fwd.argtypes = [vp, vp, vp, fp, fp, fp, vp, fp, i32, i64, i32, i32, vp, i32,
                                   vp, i32, vp, ctypes.c_size_t, vp]
@@ -120,6 +122,18 @@ def workspace_size(B: int, T: int, H: int, n_seqs: int = 0, dtype=torch.bfloat16
                                             ctypes.byref(out))
     if st != KDA_OK:
         raise KDAError(st, "kda_chunk_fwd_workspace_size")
+    return int(out.value)
+
+
+def chunk_fwd_launches(B: int, T: int, H: int, n_seqs: int = 0, dtype=torch.bfloat16,
+                       C: int = CHUNK) -> int:
+    """Number of libkda kernels one chunk_fwd call with these sizes launches."""
+    out = ctypes.c_int(0)
+    code = KDA_BF16 if dtype == torch.bfloat16 else KDA_F32
+    st = lib().kda_chunk_fwd_launches(int(B), int(T), int(H), int(C), int(n_seqs), code,
+                                      ctypes.byref(out))
+    if st != KDA_OK:
+        raise KDAError(st, "kda_chunk_fwd_launches")
     return int(out.value)
 
 

@@ -54,6 +54,14 @@ int kda_chunk_fwd_workspace_size(int B, int64_t T, int H, int C, int n_seqs, int
     return KDA_OK;
 }
 
+int kda_chunk_fwd_launches(int B, int64_t T, int H, int C, int n_seqs, int dtype, int *n_kernels) {
+    if (!n_kernels) return KDA_ERR_INVALID_ARG;
+    const int st = check_prefill_shape(B, T, H, C, n_seqs, dtype);
+    if (st != KDA_OK) return st;
+    *n_kernels = dtype == KDA_BF16 ? kda::prefill_tc_launches(B, T, H, n_seqs) : 1;
+    return KDA_OK;
+}
+
 int kda_chunk_fwd(const void *q, const void *k, const void *v, const float *log_alpha,
                   const float *beta, const float *S0, void *o, float *S_T, int B, int64_t T,
                   int H, int C, const int32_t *cu_seqlens, int n_seqs,

@@ -50,6 +50,7 @@ cudaError_t launch_prefill_simt(const void *q, const void *k, const void *v,
 
 // Tensor-core prefill (bf16 q/k/v): workspace bytes and launcher.
 size_t prefill_tc_workspace(int B, int64_t T, int H, int n_seqs);
+int prefill_tc_launches(int B, int64_t T, int H, int n_seqs);
 cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, const float *log_alpha,
                               const float *beta, const float *S0, void *o, float *S_T, int B,
                               int64_t T, int H, const int32_t *cu_seqlens, int n_seqs,

@@ -1275,6 +1275,23 @@ size_t prefill_tc_workspace(int B, int64_t T, int H, int n_seqs) {
     return batched_head_bytes(B, nck, H) + (size_t)B * nck * (size_t)H * BLOB_BYTES;
 }
 
+int sm_count() {
+    int dev = 0, n_sm = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess)
+        cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
+    return n_sm;
+}
+
+// Kernels launch_prefill_tc launches for these arguments (its decisions, restated).
+int prefill_tc_launches(int B, int64_t T, int H, int n_seqs) {
+    const bool packed = n_seqs > 0;
+    const int64_t n_tok = packed ? T : (int64_t)B * T;
+    const int nck = (int)((T + CH - 1) / CH);
+    if (!packed && n_tok > 0 && fused_plan(B, H, nck, sm_count()).n) return 1;
+    const int64_t slots = packed ? T / CH + n_seqs : (int64_t)B * nck;
+    return (packed ? 1 : 0) + (n_tok > 0 && slots > 0 ? 1 : 0) + 1;
+}
+
 cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, const float *log_alpha,
                               const float *beta, const float *S0, void *o, float *S_T, int B,
                               int64_t T, int H, const int32_t *cu_seqlens, int n_seqs,
@@ -1287,9 +1304,7 @@ cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, const
     int32_t *chunk_off = nullptr;
     unsigned char *blobs = ws;
     int64_t slots = (int64_t)B * nck;
-    int dev = 0, n_sm = 148;
-    if (cudaGetDevice(&dev) == cudaSuccess)
-        cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
+    const int n_sm = sm_count();
     if (packed) {
         chunk_off = reinterpret_cast<int32_t *>(ws);
         blobs = ws + (((size_t)(n_seqs + 1) * 4 + 255) / 256) * 256;

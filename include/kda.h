@@ -86,6 +86,17 @@ KDA_API int kda_chunk_fwd_workspace_size(int B, int64_t T, int H, int C, int n_s
                                  size_t *bytes);
 
 /*
+ * Number of libkda kernels that one kda_chunk_fwd call with these arguments
+ * launches on the current device (*n_kernels), for launch accounting. The
+ * bf16 path launches its prep and chain kernels (plus a chunk-offset scan for
+ * packed sequences), or one fused cooperative kernel for batched inputs with
+ * few sequence-heads; the fp32 path launches one kernel. Returns KDA_OK, or
+ * KDA_ERR_INVALID_ARG / KDA_ERR_UNSUPPORTED as kda_chunk_fwd would.
+ */
+KDA_API int kda_chunk_fwd_launches(int B, int64_t T, int H, int C, int n_seqs, int dtype,
+                                   int *n_kernels);
+
+/*
  * Chunk-parallel KDA prefill (blog.gzher.com section 4; chunked form of the
  * mokono.cn explainer section 2.1: S_r = P_r S_0 + H_r within a chunk).
  *
@@ -148,8 +159,8 @@ KDA_API int kda_decode_step(const void *q, const void *k, const void *v, const f
  * kda_noalloc_scratch_bytes() bytes (64 MiB) that lives in the library's
  * device image: every GPU that loads the library holds it until the process
  * exits. A problem whose kda_chunk_fwd_workspace_size exceeds it is rejected
- * with KDA_ERR_SCRATCH_LIMIT before anything is launched (roughly 900
- * chunk-head pairs for bf16, i.e. B * ceil(T/64) * H <= 903 for unpacked
+ * with KDA_ERR_SCRATCH_LIMIT before anything is launched (about a thousand
+ * chunk-head pairs for bf16, i.e. B * ceil(T/64) * H <= 1015 for unpacked
  * input; fp32 input needs no scratch). All calls on a GPU share the buffer and
  * it keeps the previous call's contents; nothing in it has to start at zero.
  * Calls that may overlap on the GPU (different streams, no ordering between
