@@ -225,6 +225,51 @@ def test_many_sequence_heads_take_full_width_chain():
     check(st, rs, "bf16", "128-column chain S_T")
 
 
+# ---------------------------------------------------------------- each bf16 path
+# A batched bf16 call runs either one fused cooperative grid (few sequence-heads, many
+# chunks) or the prep kernel and then the chain kernel; kda_chunk_fwd_launches tells
+# which. Both get ragged tails, strongly decayed channels, alpha = 0 / 1 tokens and a
+# carried state. (B, T, H) are chosen far from the boundary between the two.
+PATHS = {"fused_grid": (1, 1000, 32, 1), "prep_then_chain": (1, 300, 72, 2)}
+
+
+def _stress_gates(inp):
+    inp.log_alpha[..., 5] = -3.0             # one channel decays fast everywhere
+    inp.log_alpha[0, 100:140, 3, 77] = -40.0  # a burst beyond the factorised range
+    inp.log_alpha[0, 10, 3, 100] = -1e4       # alpha = 0 for one channel of one token
+    inp.log_alpha[0, 20:30, 0] = 0.0          # alpha = 1 tokens
+    return inp
+
+
+@pytest.mark.parametrize("path", list(PATHS))
+def test_each_bf16_path_against_the_oracle(path):
+    B, T, H, launches = PATHS[path]
+    assert kda.chunk_fwd_launches(B, T, H) == launches
+    inp = _stress_gates(prefill_inputs(B=B, T=T, H=H, dtype=torch.bfloat16, s0_std=0.1, seed=31,
+                                       device=DEV))
+    o, st = run(inp)
+    assert torch.isfinite(o.float()).all() and torch.isfinite(st).all()
+    _check_sampled(inp, o, st, [0, 0, 0], [0, 3, H - 1], list(range(128)), "bf16", path)
+
+
+def test_fused_grid_carries_state_across_calls():
+    """Two fused calls of 500 tokens with the state carried in place equal the oracle
+    run over all 1000 tokens."""
+    H = 32
+    assert kda.chunk_fwd_launches(1, 500, H) == 1
+    inp = _stress_gates(prefill_inputs(B=1, T=1000, H=H, dtype=torch.bfloat16, s0_std=0.1,
+                                       seed=32, device=DEV))
+    S = inp.S0.clone()
+    o = torch.empty_like(inp.v)
+    for a in (0, 500):
+        sl = lambda x: x[:, a:a + 500].contiguous()
+        oc, _ = kda.chunk_fwd(sl(inp.q), sl(inp.k), sl(inp.v), sl(inp.log_alpha), sl(inp.beta), S,
+                              state_out=S)
+        o[:, a:a + 500] = oc
+    torch.cuda.synchronize()
+    _check_sampled(inp, o, S, [0, 0], [3, 17], list(range(128)), "bf16", "fused, two calls")
+
+
 def test_no_bounded_wait_timed_out():
     """Every tensor-core kernel run so far finished without a wait giving up."""
     import ctypes
