@@ -92,7 +92,7 @@ constexpr uint32_t P_BADL = 66816;    // 128 int
 constexpr uint32_t P_BAR = 67328;     // 2 mbarriers
 constexpr uint32_t P_TMEM = 67344;
 constexpr uint32_t P_NBAD = 67348;    // number of listed bad channels
-constexpr uint32_t P_CLAIM = 67352;   // item index handed to the worker's threads
+constexpr uint32_t P_CLAIM = 67352;   // [2] item indices handed to the worker's threads
 constexpr uint32_t PREP_SMEM = 67360 + 1024;
 constexpr uint32_t PREP_TMEM_COLS = 128;  // Gram 64, then W 128
 constexpr uint32_t PREP_TMA_BYTES = 32768;  // q, k
@@ -231,7 +231,7 @@ struct PrepWorker {
     bool dead;
     // Thread 0: ready-flag index of the worker's last blob, not yet published (or -1).
     // It is published once that blob's stores have completed, which the worker checks
-    // after issuing its next item's loads, so that the wait overlaps them.
+    // while it waits for its next item's loads, so that the two waits overlap.
     int pending;
     __device__ __forceinline__ static int g() { return SINGLE ? 0 : (int)(threadIdx.x / PREP_NT); }
     __device__ __forceinline__ static int tid() { return SINGLE ? (int)threadIdx.x : (int)(threadIdx.x % PREP_NT); }
@@ -297,11 +297,17 @@ struct PrepWorker {
 // Prep of one (chunk, head): the chunk's gates, Grams, inverse and W, written to the
 // chunk's workspace blob. pf(x, y) is called by thread 0 after it has issued the
 // item's loads; it returns false or the coordinates of a later item's tiles, which are
-// then warmed in L2. ready != null: publish the blob's ready flag.
-template <class Worker, class Prefetch>
+// then warmed in L2. ready != null: publish the blob's ready flag. Thread 0 calls
+// hook.before_wait() and hook.after_wait() around its wait for the item's loads (work
+// whose latency that wait can hide).
+struct NoHook {
+    __device__ __forceinline__ void before_wait() {}
+    __device__ __forceinline__ void after_wait() {}
+};
+template <class Worker, class Prefetch, class Hook = NoHook>
 __device__ __forceinline__ void prep_item(Worker &w, const PrepArgs &a, int slot, int h,
                                           SeqSpan span, int n, Prefetch pf,
-                                          int32_t *__restrict__ ready) {
+                                          int32_t *__restrict__ ready, Hook hook = Hook()) {
     unsigned char *sm = Worker::sm();
     const int tid = Worker::tid(), warp = tid >> 5, lane = tid & 31;
     const int H = a.H;
@@ -330,7 +336,6 @@ __device__ __forceinline__ void prep_item(Worker &w, const PrepArgs &a, int slot
             tma_prefetch_l2_2d(a.tm_k, pf_x + 64, pf_y);
             tma_prefetch_l2_2d(a.tm_la, pf_x, pf_y);
         }
-        w.publish_pending(ready);  // the previous item's stores are the only ones in flight
     }
     if (tid < CH) sbeta[tid] = tid < L ? a.beta[(tok0 + tid) * H + h] : 0.f;
 
@@ -387,7 +392,14 @@ __device__ __forceinline__ void prep_item(Worker &w, const PrepArgs &a, int slot
     tc_fence_after();
     const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(sm + P_TMEM);
     const uint32_t sm_base = smem_u32(sm);
+    if (tid == 0) {
+        hook.before_wait();
+        // The previous item's stores are the only bulk stores in flight; waiting for
+        // them here overlaps this item's loads and keeps warp 0 free until now.
+        w.publish_pending(ready);
+    }
     w.wait(bar_tma, w.tma_phase);
+    if (tid == 0) hook.after_wait();
     w.tma_phase ^= 1u;
 
     // ---- gates and operand images, row by row. BAD selects the exact handling of key
@@ -1097,15 +1109,26 @@ kda_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         using Worker = PrepWorker<false>;
         Worker w;
         w.init(false);
+        // Thread 0 claims each item one item ahead: the claim's atomics are issued while
+        // the current item's loads are in flight. The two slots alternate, so a slot is
+        // rewritten only after every thread has passed the item that read it.
         volatile int32_t *claim = reinterpret_cast<volatile int32_t *>(Worker::sm() + P_CLAIM);
-        for (;;) {
-            if (Worker::tid() == 0) {
-                int it = atomicAdd(&queue->next_shared, 1);
-                if (it >= n_shared) it = chain_cta ? -1 : n_shared + atomicAdd(&queue->next_rest, 1);
-                *claim = it < n_total ? it : -1;
-            }
+        auto claim_next = [&]() {
+            int it = atomicAdd(&queue->next_shared, 1);
+            if (it >= n_shared) it = chain_cta ? -1 : n_shared + atomicAdd(&queue->next_rest, 1);
+            return it < n_total ? it : -1;
+        };
+        struct ClaimAhead {
+            decltype(claim_next) &next;
+            volatile int32_t *slot;
+            int value;
+            __device__ __forceinline__ void before_wait() { value = next(); }
+            __device__ __forceinline__ void after_wait() { *slot = value; }
+        };
+        if (Worker::tid() == 0) claim[0] = claim_next();
+        for (int j = 0;; ++j) {
             Worker::sync();
-            const int it = *claim;  // read before the item's first barrier; rewritten after it
+            const int it = claim[j & 1];
             if (it < 0 || w.dead) break;
             const int n = it / P, p = it % P, seq = p / H, h = p % H;
             // warm L2 for the item about one round of all workers later
@@ -1117,7 +1140,8 @@ kda_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 y = (int)((int64_t)(pp / H) * T + (int64_t)(pit / P) * CH);
                 return true;
             };
-            prep_item(w, pa, seq * nck + n, h, SeqSpan{(int64_t)seq * T, T}, n, pf, ready);
+            prep_item(w, pa, seq * nck + n, h, SeqSpan{(int64_t)seq * T, T}, n, pf, ready,
+                      ClaimAhead{claim_next, claim + ((j + 1) & 1), -1});
         }
         w.release(ready);
     }
