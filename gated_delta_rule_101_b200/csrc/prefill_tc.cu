@@ -198,12 +198,6 @@ __device__ __forceinline__ void st_chunk(unsigned char *p, const float (&v)[8]) 
     *reinterpret_cast<uint4 *>(p) = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]),
                                                pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
 }
-__device__ __forceinline__ void ld_chunk(const unsigned char *p, float (&v)[8]) {
-    const uint4 u = *reinterpret_cast<const uint4 *>(p);
-    const __nv_bfloat16 *b = reinterpret_cast<const __nv_bfloat16 *>(&u);
-#pragma unroll
-    for (int e = 0; e < 8; ++e) v[e] = __bfloat162float(b[e]);
-}
 
 // Shared-memory stride between the prep workers of one CTA.
 constexpr uint32_t PREP_PART = ((PREP_SMEM - 1024 + 1023) / 1024) * 1024;
@@ -1100,7 +1094,7 @@ kda_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                  int nck, int n_first, int n_chain) {
     extern __shared__ unsigned char smem_raw[];
     unsigned char *sm = aligned_smem(smem_raw);
-    const int tid = threadIdx.x, g = tid / PREP_NT;
+    const int tid = threadIdx.x;
     const int P = B * H;
     const int n_shared = n_first * P, n_total = nck * P;
     const bool chain_cta = (int)blockIdx.x < n_chain;
