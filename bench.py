@@ -133,9 +133,9 @@ class ClockSampler:
 # from; otherwise the roofline's traffic is null.
 TRAFFIC_SOURCES = {"prefill": ("prefill_tc.cu", "tc_ptx.cuh", "kda_internal.cuh"),
                    "decode": ("decode.cu", "kda_internal.cuh")}
-TRAFFIC = {"prefill": {"source_hash": "ad83ac7aec4312e9",  # prep + chain
-                       "bytes": 270749696 + 215545856 + 341876992 + 56629504},
-           "decode": {"source_hash": "bfbc16685498d103", "bytes": 547402496 + 480379392}}
+TRAFFIC = {"prefill": {"source_hash": "fc45713cebf7a436",  # prep + chain
+                       "bytes": 270942720 + 217313792 + 341919488 + 56497152},
+           "decode": {"source_hash": "1e7a03f630c48f57", "bytes": 547436544 + 479846400}}
 
 
 def source_hash(kind: str) -> str:
