@@ -772,6 +772,25 @@ struct ChainArgs {
     const int32_t *ready;  // non-null: wait for each blob's ready flag before reading it
 };
 
+// The part of one (sequence, head, slice) recurrence a chain task runs: chunks [c0, c1)
+// of the sequence (c1 < 0: to its end), starting from s0 (the (sequence, head) 128 x 128
+// state block; null: zeros; s0_identity: the identity) and writing the end state to st
+// (a block, or null) and, if write_o, the outputs. u_zero drops U (V_new = -W S): the
+// recurrence then applies the chunks' transition matrix Prod (Diag(gamma_L) - K~^T W)
+// to s0, which with s0 = I yields that matrix itself.
+struct ChainWindow {
+    int c0, c1;
+    const float *s0;
+    bool s0_identity;
+    float *st;
+    bool write_o;
+    bool u_zero;
+};
+__device__ __forceinline__ ChainWindow full_window(const ChainArgs &a, int seq, int h) {
+    const int64_t off = ((int64_t)seq * a.H + h) * (int64_t)(D * D);
+    return {0, -1, a.S0 ? a.S0 + off : nullptr, false, a.S_T ? a.S_T + off : nullptr, true, false};
+}
+
 // The state recurrence of one (sequence, head, N-column value slice), run by threads
 // 0 .. CHAIN_NT-1 of the CTA (tid) on shared memory `sm` (1024-aligned,
 // ChainLayout<N>::BYTES - 1024 bytes). ROLE 0: the calling thread's warp decides its
@@ -782,7 +801,8 @@ struct ChainArgs {
 // that issue the loads only poll shared memory.
 template <int N, int ROLE = 0>
 __device__ __forceinline__ void chain_task(unsigned char *sm, const int tid, const ChainArgs &a,
-                                           const int seq, const int h, const int j0) {
+                                           const int seq, const int h, const int j0,
+                                           const ChainWindow &win) {
     static_assert(N == 64 || N == 128, "value slices of 64 or 128 columns");
     constexpr int NH = N / 2;  // columns per epilogue thread
     using Lay = ChainLayout<N>;
@@ -794,15 +814,15 @@ __device__ __forceinline__ void chain_task(unsigned char *sm, const int tid, con
     const CUtensorMap &tm_v = *a.tm_v;
     const unsigned char *ws_blobs = a.ws_blobs;
     const int32_t *chunk_off = a.chunk_off;
-    const float *S0 = a.S0;
     __nv_bfloat16 *o = a.o;
-    float *S_T = a.S_T;
     const int64_t T = a.T;
     const int H = a.H, nck = a.nck;
     const SeqSpan span = seq_span(a.cu, T, seq);
-    const int nchunks = (int)((span.len + CH - 1) / CH);
-    const int64_t slot0 = chunk_off ? (int64_t)chunk_off[seq] : (int64_t)seq * nck;
-    const int64_t state_off = ((int64_t)seq * H + h) * (int64_t)(D * D);
+    const int c0 = win.c0;  // chunk indices below are relative to the window's first chunk
+    const int seq_chunks = (int)((span.len + CH - 1) / CH);
+    const int c_end = win.c1 < 0 || win.c1 > seq_chunks ? seq_chunks : win.c1;
+    const int nchunks = c_end > c0 ? c_end - c0 : 0;
+    const int64_t slot0 = (chunk_off ? (int64_t)chunk_off[seq] : (int64_t)seq * nck) + c0;
 
     uint64_t *bar_ld1 = reinterpret_cast<uint64_t *>(sm + Lay::BAR);  // [2] load part 1, per stage
     uint64_t *bar_ld2 = bar_ld1 + 2;  // [2] load part 2, per stage
@@ -826,7 +846,7 @@ __device__ __forceinline__ void chain_task(unsigned char *sm, const int tid, con
 #pragma unroll
         for (int b = 0; b < N / 64; ++b)
             tma_load_2d(st + Lay::V + b * 8192, &tm_v, h * D + j0 + 64 * b,
-                        (int)(span.start + (int64_t)chunk * CH), &bar_ld1[stage]);
+                        (int)(span.start + (int64_t)(c0 + chunk) * CH), &bar_ld1[stage]);
     };
     auto issue_load2 = [&](int chunk, int stage) {
         const unsigned char *blob = blob_of(chunk);
@@ -852,8 +872,12 @@ __device__ __forceinline__ void chain_task(unsigned char *sm, const int tid, con
     if (epi) {
 #pragma unroll
         for (int j = 0; j < NH; j += 4) {
-            float4 v4 = S0 ? *reinterpret_cast<const float4 *>(S0 + state_off + (int64_t)c * D + j0 + jh + j)
-                           : make_float4(0.f, 0.f, 0.f, 0.f);
+            float4 v4 = win.s0 ? *reinterpret_cast<const float4 *>(win.s0 + (int64_t)c * D + j0 + jh + j)
+                               : make_float4(0.f, 0.f, 0.f, 0.f);
+            if (win.s0_identity) {
+                const int col = j0 + jh + j;
+                v4 = make_float4(c == col, c == col + 1, c == col + 2, c == col + 3);
+            }
             s_reg[j] = v4.x; s_reg[j + 1] = v4.y; s_reg[j + 2] = v4.z; s_reg[j + 3] = v4.w;
         }
 #pragma unroll
@@ -936,8 +960,9 @@ __device__ __forceinline__ void chain_task(unsigned char *sm, const int tid, con
             mbar_wait(&bar_c[m & 1], (uint32_t)(m >> 1) & 1u, dead, &g_kda_device_status);
             tc_fence_after();
             const int r = c;
-            const bool live = r < chunk_rows(span.len, (int64_t)m * CH);
-            __nv_bfloat16 *dst = o + ((span.start + (int64_t)m * CH + r) * H + h) * (int64_t)D + j0;
+            const int64_t m0 = (int64_t)(c0 + m) * CH;  // first token of the chunk
+            const bool live = r < chunk_rows(span.len, m0);
+            __nv_bfloat16 *dst = o + ((span.start + m0 + r) * H + h) * (int64_t)D + j0;
 #pragma unroll
             for (int b = 0; b < N / 32; ++b) {
                 float ov[32];
@@ -972,7 +997,7 @@ __device__ __forceinline__ void chain_task(unsigned char *sm, const int tid, con
                     for (int jc = 0; jc < 4; ++jc) {
                         float v[8];
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) v[e] = us[jc * 8 + e] - ws[jc * 8 + e];
+                        for (int e = 0; e < 8; ++e) v[e] = (win.u_zero ? 0.f : us[jc * 8 + e]) - ws[jc * 8 + e];
                         st_chunk(sm + Lay::VIMG + sw128_chunk_off(r, ((jh + 32 * p) >> 3) + jc, 64), v);
                     }
                 }
@@ -980,7 +1005,7 @@ __device__ __forceinline__ void chain_task(unsigned char *sm, const int tid, con
                 tc_fence_before();
                 named_bar_arrive(BAR_VNEW, BAR_VNEW_COUNT);
             } else if (hf == 1) {
-                if (n > 0) store_output(n - 1);
+                if (win.write_o && n > 0) store_output(n - 1);
             } else if (warp == 1) {
                 // Part 1 of the stage is free once the first MMAs have completed: refill it
                 // with chunk n + 2 while this chunk is still being processed.
@@ -1025,11 +1050,11 @@ __device__ __forceinline__ void chain_task(unsigned char *sm, const int tid, con
                 if (!dead) issue_load2(n + 2, stage);
             }
         }
-        if (nchunks > 0 && !dead && q4 < 2 && hf == 1) store_output(nchunks - 1);
-        if (S_T) {
+        if (win.write_o && nchunks > 0 && !dead && q4 < 2 && hf == 1) store_output(nchunks - 1);
+        if (win.st) {
 #pragma unroll
             for (int j = 0; j < NH; j += 4)
-                *reinterpret_cast<float4 *>(S_T + state_off + (int64_t)c * D + j0 + jh + j) =
+                *reinterpret_cast<float4 *>(win.st + (int64_t)c * D + j0 + jh + j) =
                     make_float4(s_reg[j], s_reg[j + 1], s_reg[j + 2], s_reg[j + 3]);
         }
     }
@@ -1047,7 +1072,100 @@ kda_chain_kernel(const __grid_constant__ CUtensorMap tm_v,
                  int nck) {
     extern __shared__ unsigned char smem_raw[];
     const ChainArgs a{&tm_v, ws_blobs, chunk_off, S0, o, S_T, cu, T, H, nck, nullptr};
-    chain_task<N>(aligned_smem(smem_raw), threadIdx.x, a, blockIdx.x, blockIdx.y, blockIdx.z * N);
+    chain_task<N>(aligned_smem(smem_raw), threadIdx.x, a, blockIdx.x, blockIdx.y, blockIdx.z * N,
+                  full_window(a, blockIdx.x, blockIdx.y));
+}
+
+// =====================================================================================
+// segment scan: long sequences with few sequence-heads (batched inputs)
+// =====================================================================================
+// The chunks of every sequence are cut into n_seg segments of seg_len chunks (the last
+// one takes the rest). Within a segment the state obeys S_end = P_k S_start + H_k, with
+// P_k the product of the chunks' transitions Diag(gamma_L) - K~^T W and H_k the end
+// state reached from zero (mokono.cn "Kimi Linear：高效注意力机制在长序列处理中的创新应用"
+// section 2.1: S_r = P_r S_0 + H_r, applied per segment instead of per chunk).
+//  * pass 1, all in parallel: segment 0 runs its true chain (outputs; its end state is
+//    the start of segment 1); each middle segment k = 1 .. n_seg-2 runs its chain from
+//    zero (giving H_k) and, with U dropped, from the identity (giving P_k).
+//  * combine: S_start[k+1] = P_k S_start[k] + H_k for k = 1 .. n_seg-2, in fp32.
+//  * pass 2, in parallel: segments 1 .. n_seg-1 replay their chains from their true start
+//    states (outputs; the last one writes S_T).
+// The chain work is about three segments' worth per slice instead of n_seg, spread over
+// up to 2 (2 n_seg - 3) CTAs per sequence-head.
+struct SegScan {
+    float *p, *hh, *start;  // per (sequence-head, segment) 128 x 128 fp32 blocks
+    int n_seg, seg_len;
+    __host__ __device__ float *blk(float *base, int pair, int k) const {
+        return base + ((size_t)pair * n_seg + k) * (size_t)(D * D);
+    }
+};
+
+template <int N>
+__global__ void __launch_bounds__(CHAIN_NT, 1)
+kda_seg_pass_kernel(const __grid_constant__ CUtensorMap tm_v,
+                    const unsigned char *__restrict__ ws_blobs, const float *__restrict__ S0,
+                    __nv_bfloat16 *__restrict__ o, float *__restrict__ S_T, int64_t T, int H,
+                    int nck, SegScan sg, int pass) {
+    extern __shared__ unsigned char smem_raw[];
+    constexpr int SLICES = D / N;
+    const int pair = blockIdx.x / SLICES, j0 = (blockIdx.x % SLICES) * N;
+    const int seq = pair / H, h = pair % H;
+    const int64_t off = (int64_t)pair * (D * D);
+    const ChainArgs a{&tm_v, ws_blobs, nullptr, S0, o, S_T, nullptr, T, H, nck, nullptr};
+    const int L = sg.seg_len;
+    ChainWindow win;
+    if (pass == 1) {
+        const int t = blockIdx.y;  // 0: segment 0; 2k - 1: H_k; 2k: P_k
+        const int k = (t + 1) / 2;
+        if (t == 0)
+            win = {0, L, S0 ? S0 + off : nullptr, false, sg.blk(sg.start, pair, 1), true, false};
+        else if (t & 1)
+            win = {k * L, (k + 1) * L, nullptr, false, sg.blk(sg.hh, pair, k), false, false};
+        else
+            win = {k * L, (k + 1) * L, nullptr, true, sg.blk(sg.p, pair, k), false, true};
+    } else {
+        const int k = blockIdx.y + 1;
+        const bool last = k == sg.n_seg - 1;
+        win = {k * L, last ? -1 : (k + 1) * L, sg.blk(sg.start, pair, k), false,
+               last ? (S_T ? S_T + off : nullptr) : nullptr, true, false};
+    }
+    chain_task<N>(aligned_smem(smem_raw), threadIdx.x, a, seq, h, j0, win);
+}
+
+// S_start[k+1][:, slice] = P_k S_start[k][:, slice] + H_k[:, slice] for k = 1 .. n_seg-2.
+// One CTA per (sequence-head, 64-column slice); thread t owns row t/2, 32 columns.
+constexpr int SEG_COMBINE_NT = 256;
+__global__ void __launch_bounds__(SEG_COMBINE_NT)
+kda_seg_combine_kernel(SegScan sg) {
+    __shared__ __align__(16) float s[D][64];
+    const int pair = blockIdx.x >> 1, j0 = (blockIdx.x & 1) * 64;
+    const int tid = threadIdx.x, r = tid >> 1, jb = (tid & 1) * 32;
+    const float *s1 = sg.blk(sg.start, pair, 1);
+    for (int e = tid; e < D * 64; e += SEG_COMBINE_NT) s[e >> 6][e & 63] = s1[(e >> 6) * D + j0 + (e & 63)];
+    __syncthreads();
+    for (int k = 1; k + 1 < sg.n_seg; ++k) {
+        const float *pk = sg.blk(sg.p, pair, k) + (size_t)r * D;
+        const float *hk = sg.blk(sg.hh, pair, k) + (size_t)r * D + j0 + jb;
+        float acc[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) acc[j] = hk[j];
+        for (int c = 0; c < D; ++c) {
+            const float pv = pk[c];
+#pragma unroll
+            for (int j = 0; j < 32; j += 4) {
+                const float4 sv = *reinterpret_cast<const float4 *>(&s[c][jb + j]);
+                acc[j] += pv * sv.x; acc[j + 1] += pv * sv.y; acc[j + 2] += pv * sv.z; acc[j + 3] += pv * sv.w;
+            }
+        }
+        __syncthreads();  // every thread has read the old state
+        float *out = sg.blk(sg.start, pair, k + 1) + (size_t)r * D + j0 + jb;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+            s[r][jb + j] = acc[j];
+            out[j] = acc[j];
+        }
+        __syncthreads();
+    }
 }
 
 // =====================================================================================
@@ -1146,13 +1264,14 @@ kda_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     constexpr int SLICES = D / N;
     const int task = blockIdx.x, pair = task / SLICES, seq = pair / H, h = pair % H;
     const int j0 = (task % SLICES) * N;
+    const ChainWindow win = full_window(ca, seq, h);
     if (wg < 2) {
         setmaxnreg_inc<fused_reg_epi<N>()>();
-        chain_task<N, 1>(sm, tid, ca, seq, h, j0);
+        chain_task<N, 1>(sm, tid, ca, seq, h, j0, win);
     } else if (wg == 2) {
         setmaxnreg_dec<FUSED_REG_MMA>();
-        if (tid < CHAIN_NT) chain_task<N, 2>(sm, tid, ca, seq, h, j0);
-        else if (tid < CHAIN_NT + 32) chain_task<N, 3>(sm, tid, ca, seq, h, j0);
+        if (tid < CHAIN_NT) chain_task<N, 2>(sm, tid, ca, seq, h, j0, win);
+        else if (tid < CHAIN_NT + 32) chain_task<N, 3>(sm, tid, ca, seq, h, j0, win);
     } else {
         setmaxnreg_dec<FUSED_REG_IDLE>();
     }
@@ -1224,60 +1343,85 @@ size_t batched_head_bytes(int B, int nck, int H) {
     return (((size_t)B * nck * H * 4 + sizeof(FusedQueue) + 255) / 256) * 256;
 }
 
-// Plan of the fused kernel for batched inputs. The model (B200 measurements): a prep
-// worker finishes an item about every PREP_US, three per SM; a chain takes about
-// CHAIN_US[N] per chunk. With n_chain chain CTAs, the other SMs produce the items of
-// the last chunks while the chains run; the split puts the end of that production at
-// about the end of the chains. The two-kernel path (prep on every SM, then the
-// chains) is kept when the model gives the fused kernel no clear gain.
-struct FusedPlan {
-    int n;        // value columns per chain CTA (64 or 128); 0: do not fuse
-    int n_first;  // chunks whose items every CTA shares
+// Plan for batched inputs: prep then chains (two kernels), the fused grid, or the
+// segment scan. Model (B200 measurements): the standalone prep kernel finishes a
+// chunk-head about every PREP_US_TWO per CTA slot, the fused grid's workers about
+// every PREP_US_FUSED, three per SM; a 64-column chain takes about CHAIN_US_64 per
+// chunk (CHAIN_US_128 for 128 columns). Each alternative is costed and the cheapest
+// taken; the fused grid only with a clear margin.
+//  * fused grid: n_chain chain CTAs run while the other SMs produce the items of the
+//    last chunks; n_first puts the end of that production at about the end of the chains.
+//  * segment scan: n_seg segments of seg_len chunks; two passes of about seg_len chunks
+//    each after the prep, plus the sequential combine.
+struct BatchedPlan {
+    int kind;     // 0: prep then chains; 1: fused grid; 2: segment scan
+    int n_first;  // fused grid: chunks whose items every CTA shares
+    int n_seg, seg_len;
 };
 bool fused_supported() {
     static int ok = -1;  // device capabilities, queried once
     if (ok < 0) {
-        int dev = 0, coop = 0, per64 = 0, per128 = 0;
+        int dev = 0, coop = 0, per64 = 0;
         ok = cudaGetDevice(&dev) == cudaSuccess &&
              cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev) == cudaSuccess && coop &&
              cudaFuncSetAttribute(kda_fused_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   (int)fused_smem<64>()) == cudaSuccess &&
-             cudaFuncSetAttribute(kda_fused_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  (int)fused_smem<128>()) == cudaSuccess &&
              cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per64, kda_fused_kernel<64>, FUSED_NT,
                                                            fused_smem<64>()) == cudaSuccess &&
-             cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per128, kda_fused_kernel<128>, FUSED_NT,
-                                                           fused_smem<128>()) == cudaSuccess &&
-             per64 >= 1 && per128 >= 1;
+             per64 >= 1;
     }
     return ok == 1;
 }
-FusedPlan fused_plan(int B, int H, int nck, int n_sm) {
-    constexpr double PREP_US = 16.5, CHAIN_US_64 = 1.45, CHAIN_US_128 = 2.3;
+// Segments the workspace has room for (it is sized without knowing the device: at most
+// 16 segments of at least 8 chunks, and only where 3 segments fit 256 SMs).
+int seg_capacity(int B, int H, int nck) {
+    const int P = B * H;
+    if (2 * P * 3 > 256) return 0;
+    const int c = nck / 8;
+    return c < 16 ? c : 16;
+}
+size_t seg_bytes(int B, int H, int nck) {
+    const int cap = seg_capacity(B, H, nck);
+    return cap >= 3 ? (size_t)3 * B * H * cap * (size_t)(D * D) * sizeof(float) : 0;
+}
+BatchedPlan batched_plan(int B, int H, int nck, int n_sm) {
+    constexpr double PREP_US_TWO = 14.4, PREP_US_FUSED = 16.5, CHAIN_US_64 = 1.45,
+                     CHAIN_US_128 = 2.3, COMBINE_US = 6.0, LAUNCH_US = 4.0;
     constexpr int MIN_PREP_CTAS = 8;
     const int P = B * H;
-    const double r = 3.0 / PREP_US;  // items per microsecond per SM
-    if ((int64_t)nck * P >= (1ll << 30) || !fused_supported()) return {0, 0};
-    // the two-kernel path: prep on every SM, then the chains in waves
+    const double r2 = 3.0 / PREP_US_TWO, rf = 3.0 / PREP_US_FUSED;  // items per us per SM
+    const double t_prep = nck * (double)P / (n_sm * r2);
+    // prep on every SM, then the chains in waves
     const int n2 = P >= n_sm ? 128 : 64;
     const double waves = (double)((P * (D / n2) + n_sm - 1) / n_sm);
-    const double t_two = nck * (double)P / (n_sm * r) + waves * nck * (n2 == 64 ? CHAIN_US_64 : CHAIN_US_128);
-    FusedPlan best{0, 0};
-    double t_best = 0.95 * t_two;
-    for (int n : {64}) {  // 128-column chains run about 2.3 us per chunk here: no gain
-        const int n_chain = P * (D / n);
-        if (n_chain + MIN_PREP_CTAS > n_sm) continue;
-        const double tau = n == 64 ? CHAIN_US_64 : CHAIN_US_128;
+    BatchedPlan best{0, 0, 0, 0};
+    double t_best = t_prep + waves * nck * (n2 == 64 ? CHAIN_US_64 : CHAIN_US_128);
+    // segment scan
+    int n_seg = (n_sm / (2 * P) + 3) / 2;  // pass 1: 2 P (2 n_seg - 3) CTAs in one wave
+    const int cap = seg_capacity(B, H, nck);
+    n_seg = n_seg < cap ? n_seg : cap;
+    if (n_seg >= 3) {
+        const int seg_len = (nck + n_seg - 1) / n_seg;
+        n_seg = (nck + seg_len - 1) / seg_len;
+        const double t = t_prep + 2.0 * seg_len * CHAIN_US_64 + (n_seg - 2) * COMBINE_US + 2 * LAUNCH_US;
+        if (n_seg >= 3 && t < t_best) {
+            t_best = t;
+            best = {2, 0, n_seg, seg_len};
+        }
+    }
+    // fused grid (64-column chains; 128-column chains run about 2.3 us per chunk: no gain)
+    const int n_chain = 2 * P;
+    if (n_chain + MIN_PREP_CTAS <= n_sm && (int64_t)nck * P < (1ll << 30) && fused_supported()) {
         const int n_prep = n_sm - n_chain;
-        int n_first = nck - (int)((double)nck * tau * n_prep * r / P);
+        int n_first = nck - (int)((double)nck * CHAIN_US_64 * n_prep * rf / P);
         const int lo = nck < 2 ? nck : 2;
         n_first = n_first < lo ? lo : (n_first > nck ? nck : n_first);
-        const double t_a = (double)n_first * P / (n_sm * r);
-        const double t_b = (double)(nck - n_first) * P / (n_prep * r);
-        const double t = t_a + (nck * tau > t_b ? nck * tau : t_b);
-        if (t < t_best) {
+        const double t_a = (double)n_first * P / (n_sm * rf);
+        const double t_b = (double)(nck - n_first) * P / (n_prep * rf);
+        const double t = t_a + (nck * CHAIN_US_64 > t_b ? nck * CHAIN_US_64 : t_b);
+        if (t < 0.95 * t_best) {
             t_best = t;
-            best = {n, n_first};
+            best = {1, n_first, 0, 0};
         }
     }
     return best;
@@ -1290,7 +1434,8 @@ size_t prefill_tc_workspace(int B, int64_t T, int H, int n_seqs) {
         return head + slots * (size_t)H * BLOB_BYTES;
     }
     const int nck = (int)((T + CH - 1) / CH);
-    return batched_head_bytes(B, nck, H) + (size_t)B * nck * (size_t)H * BLOB_BYTES;
+    return batched_head_bytes(B, nck, H) + (size_t)B * nck * (size_t)H * BLOB_BYTES +
+           seg_bytes(B, H, nck);
 }
 
 int sm_count() {
@@ -1305,7 +1450,11 @@ int prefill_tc_launches(int B, int64_t T, int H, int n_seqs) {
     const bool packed = n_seqs > 0;
     const int64_t n_tok = packed ? T : (int64_t)B * T;
     const int nck = (int)((T + CH - 1) / CH);
-    if (!packed && n_tok > 0 && fused_plan(B, H, nck, sm_count()).n) return 1;
+    if (!packed && n_tok > 0) {
+        const BatchedPlan plan = batched_plan(B, H, nck, sm_count());
+        if (plan.kind == 1) return 1;  // the fused grid
+        if (plan.kind == 2) return 4;  // prep, pass 1, combine, pass 2
+    }
     const int64_t slots = packed ? T / CH + n_seqs : (int64_t)B * nck;
     return (packed ? 1 : 0) + (n_tok > 0 && slots > 0 ? 1 : 0) + 1;
 }
@@ -1323,6 +1472,7 @@ cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, const
     unsigned char *blobs = ws;
     int64_t slots = (int64_t)B * nck;
     const int n_sm = sm_count();
+    BatchedPlan plan{0, 0, 0, 0};
     if (packed) {
         chunk_off = reinterpret_cast<int32_t *>(ws);
         blobs = ws + (((size_t)(n_seqs + 1) * 4 + 255) / 256) * 256;
@@ -1330,8 +1480,8 @@ cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, const
         chunk_offsets_kernel<<<1, 1024, 0, stream>>>(cu_seqlens, n_seqs, chunk_off);
     } else {
         blobs = ws + batched_head_bytes(B, nck, H);
-        const FusedPlan plan = n_tok > 0 ? fused_plan(B, H, nck, n_sm) : FusedPlan{0, 0};
-        if (plan.n) {
+        plan = n_tok > 0 ? batched_plan(B, H, nck, n_sm) : BatchedPlan{0, 0, 0, 0};
+        if (plan.kind == 1) {
             int32_t *ready = reinterpret_cast<int32_t *>(ws);
             FusedQueue *queue = reinterpret_cast<FusedQueue *>(ready + (size_t)B * nck * H);
             cudaError_t err = cudaMemsetAsync(ws, 0, (size_t)B * nck * H * 4 + sizeof(FusedQueue), stream);
@@ -1342,15 +1492,12 @@ cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, const
                 return cudaErrorInvalidValue;
             const __nv_bfloat16 *qb = (const __nv_bfloat16 *)q, *kb = (const __nv_bfloat16 *)k;
             __nv_bfloat16 *ob = (__nv_bfloat16 *)o;
-            int n_chain = B * H * (D / plan.n), n_first = plan.n_first;
+            int n_chain = 2 * B * H, n_first = plan.n_first;
             void *args[] = {&mq, &mk, &mla, &mv, &qb, &kb, (void *)&log_alpha, (void *)&beta, &blobs,
                             &ready, &queue, (void *)&S0, &ob, &S_T, &T, &H, &B, (void *)&nck,
                             &n_first, &n_chain};
-            if (plan.n == 64)
-                return cudaLaunchCooperativeKernel((const void *)kda_fused_kernel<64>, dim3((unsigned)n_sm),
-                                                   dim3(FUSED_NT), args, fused_smem<64>(), stream);
-            return cudaLaunchCooperativeKernel((const void *)kda_fused_kernel<128>, dim3((unsigned)n_sm),
-                                               dim3(FUSED_NT), args, fused_smem<128>(), stream);
+            return cudaLaunchCooperativeKernel((const void *)kda_fused_kernel<64>, dim3((unsigned)n_sm),
+                                               dim3(FUSED_NT), args, fused_smem<64>(), stream);
         }
     }
     cudaError_t err;
@@ -1373,6 +1520,23 @@ cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, const
     }
     CUtensorMap mv;
     if (n_tok > 0 && !make_map(&mv, v, true, n_tok, H)) return cudaErrorInvalidValue;
+    if (plan.kind == 2) {  // segment scan: pass 1, combine, pass 2
+        const int P = B * H, cap = seg_capacity(B, H, nck);
+        float *base = reinterpret_cast<float *>(blobs + (size_t)B * nck * H * BLOB_BYTES);
+        const size_t per = (size_t)P * cap * (D * D);
+        const SegScan sg{base, base + per, base + 2 * per, plan.n_seg, plan.seg_len};
+        using Lay = ChainLayout<64>;
+        err = cudaFuncSetAttribute(kda_seg_pass_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   (int)Lay::BYTES);
+        if (err != cudaSuccess) return err;
+        __nv_bfloat16 *ob = (__nv_bfloat16 *)o;
+        kda_seg_pass_kernel<64><<<dim3((unsigned)(2 * P), (unsigned)(2 * plan.n_seg - 3)), CHAIN_NT,
+                                  Lay::BYTES, stream>>>(mv, blobs, S0, ob, S_T, T, H, nck, sg, 1);
+        kda_seg_combine_kernel<<<2 * P, SEG_COMBINE_NT, 0, stream>>>(sg);
+        kda_seg_pass_kernel<64><<<dim3((unsigned)(2 * P), (unsigned)(plan.n_seg - 1)), CHAIN_NT,
+                                  Lay::BYTES, stream>>>(mv, blobs, S0, ob, S_T, T, H, nck, sg, 2);
+        return cudaGetLastError();
+    }
     // 128-column slices (one CTA per sequence-head) when there are enough pairs to fill
     // the GPU; otherwise 64-column slices for twice the parallelism.
     if ((int64_t)nseq * H >= n_sm) return launch_chain<128>(mv, blobs, chunk_off, S0, o, S_T, cu_seqlens, T, H, nck, nseq, stream);

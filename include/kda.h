@@ -89,8 +89,10 @@ KDA_API int kda_chunk_fwd_workspace_size(int B, int64_t T, int H, int C, int n_s
  * Number of libkda kernels that one kda_chunk_fwd call with these arguments
  * launches on the current device (*n_kernels), for launch accounting. The
  * bf16 path launches its prep and chain kernels (plus a chunk-offset scan for
- * packed sequences), or one fused cooperative kernel for batched inputs with
- * few sequence-heads; the fp32 path launches one kernel. Returns KDA_OK, or
+ * packed sequences: 2 or 3), one fused cooperative kernel for batched inputs
+ * with few sequence-heads and many chunks (1), or, for long batched sequences
+ * with very few sequence-heads, the segment scan: prep, two chain passes and
+ * a combine (4). The fp32 path launches one kernel. Returns KDA_OK, or
  * KDA_ERR_INVALID_ARG / KDA_ERR_UNSUPPORTED as kda_chunk_fwd would.
  */
 KDA_API int kda_chunk_fwd_launches(int B, int64_t T, int H, int C, int n_seqs, int dtype,

@@ -226,18 +226,22 @@ def test_many_sequence_heads_take_full_width_chain():
 
 
 # ---------------------------------------------------------------- each bf16 path
-# A batched bf16 call runs either one fused cooperative grid (few sequence-heads, many
-# chunks) or the prep kernel and then the chain kernel; kda_chunk_fwd_launches tells
-# which. Both get ragged tails, strongly decayed channels, alpha = 0 / 1 tokens and a
-# carried state. (B, T, H) are chosen far from the boundary between the two.
-PATHS = {"fused_grid": (1, 1000, 32, 1), "prep_then_chain": (1, 300, 72, 2)}
+# A batched bf16 call runs one of three plans; kda_chunk_fwd_launches tells which:
+# prep then chains (2 launches), the fused cooperative grid (1), or the segment scan
+# for long sequences with few sequence-heads (4: prep, pass 1, combine, pass 2). Each
+# gets ragged tails, strongly decayed channels, alpha = 0 / 1 tokens and a carried
+# state. (B, T, H) are chosen far from the boundaries between the plans.
+PATHS = {"fused_grid": (1, 1000, 32, 1), "prep_then_chain": (1, 300, 72, 2),
+         "segment_scan": (1, 3000, 2, 4), "segment_scan_batched": (2, 8000, 2, 4)}
 
 
 def _stress_gates(inp):
-    inp.log_alpha[..., 5] = -3.0             # one channel decays fast everywhere
-    inp.log_alpha[0, 100:140, 3, 77] = -40.0  # a burst beyond the factorised range
-    inp.log_alpha[0, 10, 3, 100] = -1e4       # alpha = 0 for one channel of one token
-    inp.log_alpha[0, 20:30, 0] = 0.0          # alpha = 1 tokens
+    H = inp.q.shape[2]
+    hh = min(3, H - 1)
+    inp.log_alpha[..., 5] = -3.0               # one channel decays fast everywhere
+    inp.log_alpha[0, 100:140, hh, 77] = -40.0  # a burst beyond the factorised range
+    inp.log_alpha[0, 10, hh, 100] = -1e4       # alpha = 0 for one channel of one token
+    inp.log_alpha[0, 20:30, 0] = 0.0           # alpha = 1 tokens
     return inp
 
 
@@ -249,7 +253,9 @@ def test_each_bf16_path_against_the_oracle(path):
                                        device=DEV))
     o, st = run(inp)
     assert torch.isfinite(o.float()).all() and torch.isfinite(st).all()
-    _check_sampled(inp, o, st, [0, 0, 0], [0, 3, H - 1], list(range(128)), "bf16", path)
+    seqs = [0, 0, B - 1]
+    heads = [0, min(3, H - 1), H - 1]
+    _check_sampled(inp, o, st, seqs, heads, list(range(128)), "bf16", path)
 
 
 def test_fused_grid_carries_state_across_calls():
