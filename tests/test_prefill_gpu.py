@@ -276,6 +276,24 @@ def test_fused_grid_carries_state_across_calls():
     _check_sampled(inp, o, S, [0, 0], [3, 17], list(range(128)), "bf16", "fused, two calls")
 
 
+def test_segment_scan_carries_state_across_calls():
+    """Two segment-scan calls of 3,000 tokens with the state carried in place equal the
+    oracle run over all 6,000 tokens."""
+    H, Tc = 2, 3000
+    assert kda.chunk_fwd_launches(1, Tc, H) == 4
+    inp = _stress_gates(prefill_inputs(B=1, T=2 * Tc, H=H, dtype=torch.bfloat16, s0_std=0.1,
+                                       seed=33, device=DEV))
+    S = inp.S0.clone()
+    o = torch.empty_like(inp.v)
+    for a in (0, Tc):
+        sl = lambda x: x[:, a:a + Tc].contiguous()
+        oc, _ = kda.chunk_fwd(sl(inp.q), sl(inp.k), sl(inp.v), sl(inp.log_alpha), sl(inp.beta), S,
+                              state_out=S)
+        o[:, a:a + Tc] = oc
+    torch.cuda.synchronize()
+    _check_sampled(inp, o, S, [0, 0], [0, 1], list(range(128)), "bf16", "segment scan, two calls")
+
+
 def test_no_bounded_wait_timed_out():
     """Every tensor-core kernel run so far finished without a wait giving up."""
     import ctypes
