@@ -387,8 +387,9 @@ def run_kda(args, rank, world, local_rank):
                 "frac": achieved / pk["hbm_gbs"], "traffic": traffic("prefill", args.traffic),
                 "peak_source": pk_kind,
                 "kernel": "kda_chunk_fwd (one call, timed as a whole): "
-                          + ("kda_prep_kernel + kda_chain_kernel" if launches_per_call == 2
-                             else "kda_fused_kernel"),
+                          + {1: "kda_fused_kernel", 2: "kda_prep_kernel + kda_chain_kernel",
+                             4: "kda_prep_kernel + kda_seg_pass_kernel x2 + kda_seg_combine_kernel"}
+                          .get(launches_per_call, f"{launches_per_call} kernels"),
                 "alg_bytes_per_launch": alg_bytes,
                 "tensor_pages_flops": {"achieved_tflops": tflops, "peak": pk["bf16_tflops"],
                                        "frac": tflops / pk["bf16_tflops"],

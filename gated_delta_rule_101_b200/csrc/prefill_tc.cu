@@ -1133,38 +1133,58 @@ kda_seg_pass_kernel(const __grid_constant__ CUtensorMap tm_v,
 }
 
 // S_start[k+1][:, slice] = P_k S_start[k][:, slice] + H_k[:, slice] for k = 1 .. n_seg-2.
-// One CTA per (sequence-head, 64-column slice); thread t owns row t/2, 32 columns.
+// One CTA per (sequence-head, 64-column slice); thread t owns row t/2, 32 columns. Each
+// step stages P_k in shared memory (rows padded to 129 floats, so that the 16 rows a
+// warp reads at one column fall in distinct banks).
 constexpr int SEG_COMBINE_NT = 256;
+constexpr int SEG_PLD = D + 1;
+constexpr uint32_t SEG_COMBINE_SMEM = (D * 64 + D * SEG_PLD) * sizeof(float);
 __global__ void __launch_bounds__(SEG_COMBINE_NT)
 kda_seg_combine_kernel(SegScan sg) {
-    __shared__ __align__(16) float s[D][64];
+    extern __shared__ __align__(16) float seg_smem[];
+    float (*s)[64] = reinterpret_cast<float (*)[64]>(seg_smem);  // [128][64] current state slice
+    float *pm = seg_smem + D * 64;                                  // [128][SEG_PLD] P_k
     const int pair = blockIdx.x >> 1, j0 = (blockIdx.x & 1) * 64;
     const int tid = threadIdx.x, r = tid >> 1, jb = (tid & 1) * 32;
     const float *s1 = sg.blk(sg.start, pair, 1);
-    for (int e = tid; e < D * 64; e += SEG_COMBINE_NT) s[e >> 6][e & 63] = s1[(e >> 6) * D + j0 + (e & 63)];
-    __syncthreads();
+    for (int e = tid; e < D * 16; e += SEG_COMBINE_NT) {  // 16 float4 per row
+        const int row = e >> 4, c4 = (e & 15) * 4;
+        *reinterpret_cast<float4 *>(&s[row][c4]) = *reinterpret_cast<const float4 *>(s1 + row * D + j0 + c4);
+    }
     for (int k = 1; k + 1 < sg.n_seg; ++k) {
-        const float *pk = sg.blk(sg.p, pair, k) + (size_t)r * D;
+        const float *pk = sg.blk(sg.p, pair, k);
+        for (int e = tid; e < D * 32; e += SEG_COMBINE_NT) {  // 32 float4 per row of P_k
+            const int row = e >> 5, c4 = (e & 31) * 4;
+            const float4 v = *reinterpret_cast<const float4 *>(pk + row * D + c4);
+            float *dst = pm + row * SEG_PLD + c4;
+            dst[0] = v.x; dst[1] = v.y; dst[2] = v.z; dst[3] = v.w;
+        }
+        __syncthreads();  // P_k and the state are in shared memory
         const float *hk = sg.blk(sg.hh, pair, k) + (size_t)r * D + j0 + jb;
         float acc[32];
 #pragma unroll
-        for (int j = 0; j < 32; ++j) acc[j] = hk[j];
+        for (int j = 0; j < 32; j += 4) {
+            const float4 hv = *reinterpret_cast<const float4 *>(hk + j);
+            acc[j] = hv.x; acc[j + 1] = hv.y; acc[j + 2] = hv.z; acc[j + 3] = hv.w;
+        }
+        const float *prow = pm + r * SEG_PLD;
+#pragma unroll 4
         for (int c = 0; c < D; ++c) {
-            const float pv = pk[c];
+            const float pv = prow[c];
 #pragma unroll
             for (int j = 0; j < 32; j += 4) {
                 const float4 sv = *reinterpret_cast<const float4 *>(&s[c][jb + j]);
                 acc[j] += pv * sv.x; acc[j + 1] += pv * sv.y; acc[j + 2] += pv * sv.z; acc[j + 3] += pv * sv.w;
             }
         }
-        __syncthreads();  // every thread has read the old state
+        __syncthreads();  // every thread has read the old state and P_k
         float *out = sg.blk(sg.start, pair, k + 1) + (size_t)r * D + j0 + jb;
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-            s[r][jb + j] = acc[j];
-            out[j] = acc[j];
+        for (int j = 0; j < 32; j += 4) {
+            const float4 v = make_float4(acc[j], acc[j + 1], acc[j + 2], acc[j + 3]);
+            *reinterpret_cast<float4 *>(&s[r][jb + j]) = v;
+            *reinterpret_cast<float4 *>(out + j) = v;
         }
-        __syncthreads();
     }
 }
 
@@ -1532,7 +1552,10 @@ cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, const
         __nv_bfloat16 *ob = (__nv_bfloat16 *)o;
         kda_seg_pass_kernel<64><<<dim3((unsigned)(2 * P), (unsigned)(2 * plan.n_seg - 3)), CHAIN_NT,
                                   Lay::BYTES, stream>>>(mv, blobs, S0, ob, S_T, T, H, nck, sg, 1);
-        kda_seg_combine_kernel<<<2 * P, SEG_COMBINE_NT, 0, stream>>>(sg);
+        err = cudaFuncSetAttribute(kda_seg_combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   (int)SEG_COMBINE_SMEM);
+        if (err != cudaSuccess) return err;
+        kda_seg_combine_kernel<<<2 * P, SEG_COMBINE_NT, SEG_COMBINE_SMEM, stream>>>(sg);
         kda_seg_pass_kernel<64><<<dim3((unsigned)(2 * P), (unsigned)(plan.n_seg - 1)), CHAIN_NT,
                                   Lay::BYTES, stream>>>(mv, blobs, S0, ob, S_T, T, H, nck, sg, 2);
         return cudaGetLastError();
