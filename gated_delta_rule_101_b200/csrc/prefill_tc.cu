@@ -1147,17 +1147,27 @@ kda_seg_combine_kernel(SegScan sg) {
     const int pair = blockIdx.x >> 1, j0 = (blockIdx.x & 1) * 64;
     const int tid = threadIdx.x, r = tid >> 1, jb = (tid & 1) * 32;
     const float *s1 = sg.blk(sg.start, pair, 1);
-    for (int e = tid; e < D * 16; e += SEG_COMBINE_NT) {  // 16 float4 per row
-        const int row = e >> 4, c4 = (e & 15) * 4;
+#pragma unroll
+    for (int i = 0; i < D * 16 / SEG_COMBINE_NT; ++i) {  // 16 float4 per row of the slice
+        const int e = tid + i * SEG_COMBINE_NT, row = e >> 4, c4 = (e & 15) * 4;
         *reinterpret_cast<float4 *>(&s[row][c4]) = *reinterpret_cast<const float4 *>(s1 + row * D + j0 + c4);
     }
     for (int k = 1; k + 1 < sg.n_seg; ++k) {
         const float *pk = sg.blk(sg.p, pair, k);
-        for (int e = tid; e < D * 32; e += SEG_COMBINE_NT) {  // 32 float4 per row of P_k
-            const int row = e >> 5, c4 = (e & 31) * 4;
-            const float4 v = *reinterpret_cast<const float4 *>(pk + row * D + c4);
-            float *dst = pm + row * SEG_PLD + c4;
-            dst[0] = v.x; dst[1] = v.y; dst[2] = v.z; dst[3] = v.w;
+        {  // all of this thread's loads first, so that they are in flight together
+            constexpr int PER = D * 32 / SEG_COMBINE_NT;  // float4 of P_k per thread
+            float4 v[PER];
+#pragma unroll
+            for (int i = 0; i < PER; ++i) {
+                const int e = tid + i * SEG_COMBINE_NT;
+                v[i] = *reinterpret_cast<const float4 *>(pk + (e >> 5) * D + (e & 31) * 4);
+            }
+#pragma unroll
+            for (int i = 0; i < PER; ++i) {
+                const int e = tid + i * SEG_COMBINE_NT;
+                float *dst = pm + (e >> 5) * SEG_PLD + (e & 31) * 4;
+                dst[0] = v[i].x; dst[1] = v[i].y; dst[2] = v[i].z; dst[3] = v[i].w;
+            }
         }
         __syncthreads();  // P_k and the state are in shared memory
         const float *hk = sg.blk(sg.hh, pair, k) + (size_t)r * D + j0 + jb;
