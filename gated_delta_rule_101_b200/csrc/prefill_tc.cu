@@ -1133,9 +1133,11 @@ kda_seg_pass_kernel(const __grid_constant__ CUtensorMap tm_v,
 }
 
 // S_start[k+1][:, slice] = P_k S_start[k][:, slice] + H_k[:, slice] for k = 1 .. n_seg-2.
-// One CTA per (sequence-head, 64-column slice); thread t owns row t/2, 32 columns. Each
-// step stages P_k in shared memory (rows padded to 129 floats, so that the 16 rows a
-// warp reads at one column fall in distinct banks).
+// One CTA per (sequence-head, 64-column slice). Thread t owns rows t/4 and t/4 + 64 and
+// the 16 columns 4 (t % 4) + 16 m + {0..3}, m = 0..3: per column index the four threads
+// of a row read four different banks of the state, and two row values of P_k serve 32
+// products. Each step stages P_k in shared memory (rows padded to 129 floats, so that
+// the rows a warp reads at one column fall in distinct banks).
 constexpr int SEG_COMBINE_NT = 256;
 constexpr int SEG_PLD = D + 1;
 constexpr uint32_t SEG_COMBINE_SMEM = (D * 64 + D * SEG_PLD) * sizeof(float);
@@ -1145,7 +1147,7 @@ kda_seg_combine_kernel(SegScan sg) {
     float (*s)[64] = reinterpret_cast<float (*)[64]>(seg_smem);  // [128][64] current state slice
     float *pm = seg_smem + D * 64;                                  // [128][SEG_PLD] P_k
     const int pair = blockIdx.x >> 1, j0 = (blockIdx.x & 1) * 64;
-    const int tid = threadIdx.x, r = tid >> 1, jb = (tid & 1) * 32;
+    const int tid = threadIdx.x, r0 = tid >> 2, jq = (tid & 3) * 4;
     const float *s1 = sg.blk(sg.start, pair, 1);
 #pragma unroll
     for (int i = 0; i < D * 16 / SEG_COMBINE_NT; ++i) {  // 16 float4 per row of the slice
@@ -1170,30 +1172,40 @@ kda_seg_combine_kernel(SegScan sg) {
             }
         }
         __syncthreads();  // P_k and the state are in shared memory
-        const float *hk = sg.blk(sg.hh, pair, k) + (size_t)r * D + j0 + jb;
-        float acc[32];
+        float acc[2][16];
 #pragma unroll
-        for (int j = 0; j < 32; j += 4) {
-            const float4 hv = *reinterpret_cast<const float4 *>(hk + j);
-            acc[j] = hv.x; acc[j + 1] = hv.y; acc[j + 2] = hv.z; acc[j + 3] = hv.w;
+        for (int h2 = 0; h2 < 2; ++h2) {
+            const float *hk = sg.blk(sg.hh, pair, k) + (size_t)(r0 + 64 * h2) * D + j0 + jq;
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {
+                const float4 hv = *reinterpret_cast<const float4 *>(hk + 16 * m);
+                acc[h2][4 * m] = hv.x; acc[h2][4 * m + 1] = hv.y; acc[h2][4 * m + 2] = hv.z; acc[h2][4 * m + 3] = hv.w;
+            }
         }
-        const float *prow = pm + r * SEG_PLD;
+        const float *p0 = pm + r0 * SEG_PLD, *p1 = pm + (r0 + 64) * SEG_PLD;
 #pragma unroll 4
         for (int c = 0; c < D; ++c) {
-            const float pv = prow[c];
+            const float a0 = p0[c], a1 = p1[c];
 #pragma unroll
-            for (int j = 0; j < 32; j += 4) {
-                const float4 sv = *reinterpret_cast<const float4 *>(&s[c][jb + j]);
-                acc[j] += pv * sv.x; acc[j + 1] += pv * sv.y; acc[j + 2] += pv * sv.z; acc[j + 3] += pv * sv.w;
+            for (int m = 0; m < 4; ++m) {
+                const float4 sv = *reinterpret_cast<const float4 *>(&s[c][jq + 16 * m]);
+                acc[0][4 * m] += a0 * sv.x; acc[0][4 * m + 1] += a0 * sv.y;
+                acc[0][4 * m + 2] += a0 * sv.z; acc[0][4 * m + 3] += a0 * sv.w;
+                acc[1][4 * m] += a1 * sv.x; acc[1][4 * m + 1] += a1 * sv.y;
+                acc[1][4 * m + 2] += a1 * sv.z; acc[1][4 * m + 3] += a1 * sv.w;
             }
         }
         __syncthreads();  // every thread has read the old state and P_k
-        float *out = sg.blk(sg.start, pair, k + 1) + (size_t)r * D + j0 + jb;
 #pragma unroll
-        for (int j = 0; j < 32; j += 4) {
-            const float4 v = make_float4(acc[j], acc[j + 1], acc[j + 2], acc[j + 3]);
-            *reinterpret_cast<float4 *>(&s[r][jb + j]) = v;
-            *reinterpret_cast<float4 *>(out + j) = v;
+        for (int h2 = 0; h2 < 2; ++h2) {
+            const int r = r0 + 64 * h2;
+            float *out = sg.blk(sg.start, pair, k + 1) + (size_t)r * D + j0 + jq;
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {
+                const float4 v = make_float4(acc[h2][4 * m], acc[h2][4 * m + 1], acc[h2][4 * m + 2], acc[h2][4 * m + 3]);
+                *reinterpret_cast<float4 *>(&s[r][jq + 16 * m]) = v;
+                *reinterpret_cast<float4 *>(out + 16 * m) = v;
+            }
         }
     }
 }
