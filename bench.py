@@ -133,8 +133,8 @@ class ClockSampler:
 # from; otherwise the roofline's traffic is null.
 TRAFFIC_SOURCES = {"prefill": ("prefill_tc.cu", "tc_ptx.cuh", "kda_internal.cuh"),
                    "decode": ("decode.cu", "kda_internal.cuh")}
-TRAFFIC = {"prefill": {"source_hash": "fc45713cebf7a436",  # prep + chain
-                       "bytes": 270942720 + 217313792 + 341919488 + 56497152},
+TRAFFIC = {"prefill": {"source_hash": "226299f94bcc1aae",  # prep + chain
+                       "bytes": 270968832 + 216843264 + 341876992 + 55703296},
            "decode": {"source_hash": "1e7a03f630c48f57", "bytes": 547436544 + 479846400}}
 
 
