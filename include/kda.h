@@ -162,8 +162,8 @@ KDA_API int kda_decode_step(const void *q, const void *k, const void *v, const f
  * device image: every GPU that loads the library holds it until the process
  * exits. A problem whose kda_chunk_fwd_workspace_size exceeds it is rejected
  * with KDA_ERR_SCRATCH_LIMIT before anything is launched (about a thousand
- * chunk-head pairs for bf16, i.e. B * ceil(T/64) * H <= 1015 for unpacked
- * input; fp32 input needs no scratch). All calls on a GPU share the buffer and
+ * chunk-head pairs for bf16: B * ceil(T/64) * H <= 1015 for unpacked input
+ * without segment-scan room; fp32 input needs no scratch). All calls on a GPU share the buffer and
  * it keeps the previous call's contents; nothing in it has to start at zero.
  * Calls that may overlap on the GPU (different streams, no ordering between
  * them) race on the buffer: issue them on one stream. The first call on each
