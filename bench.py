@@ -133,7 +133,7 @@ class ClockSampler:
 # from; otherwise the roofline's traffic is null.
 TRAFFIC_SOURCES = {"prefill": ("prefill_tc.cu", "tc_ptx.cuh", "kda_internal.cuh"),
                    "decode": ("decode.cu", "kda_internal.cuh")}
-TRAFFIC = {"prefill": {"source_hash": "226299f94bcc1aae",  # prep + chain
+TRAFFIC = {"prefill": {"source_hash": "4bcc50ac00615650",  # prep + chain
                        "bytes": 270968832 + 216843264 + 341876992 + 55703296},
            "decode": {"source_hash": "1e7a03f630c48f57", "bytes": 547436544 + 479846400}}
 

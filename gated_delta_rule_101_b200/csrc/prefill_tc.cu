@@ -1400,19 +1400,26 @@ struct BatchedPlan {
     int n_first;  // fused grid: chunks whose items every CTA shares
     int n_seg, seg_len;
 };
+// Whether the current device can run the fused grid (cooperative launch, one CTA per
+// SM). The kernel's shared-memory attribute is set here, once per device, as the check
+// needs it; the answer is cached per device.
 bool fused_supported() {
-    static int ok = -1;  // device capabilities, queried once
-    if (ok < 0) {
-        int dev = 0, coop = 0, per64 = 0;
-        ok = cudaGetDevice(&dev) == cudaSuccess &&
-             cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev) == cudaSuccess && coop &&
-             cudaFuncSetAttribute(kda_fused_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  (int)fused_smem<64>()) == cudaSuccess &&
-             cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per64, kda_fused_kernel<64>, FUSED_NT,
-                                                           fused_smem<64>()) == cudaSuccess &&
-             per64 >= 1;
+    constexpr int MAX_DEVICES = 128;
+    static int ok[MAX_DEVICES];  // 0: not checked, 1: yes, 2: no
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= MAX_DEVICES) return false;
+    if (ok[dev] == 0) {
+        int coop = 0, per64 = 0;
+        const bool yes =
+            cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev) == cudaSuccess && coop &&
+            cudaFuncSetAttribute(kda_fused_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)fused_smem<64>()) == cudaSuccess &&
+            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per64, kda_fused_kernel<64>, FUSED_NT,
+                                                          fused_smem<64>()) == cudaSuccess &&
+            per64 >= 1;
+        ok[dev] = yes ? 1 : 2;
     }
-    return ok == 1;
+    return ok[dev] == 1;
 }
 // Segments the workspace has room for (it is sized without knowing the device: at most
 // 16 segments of at least 8 chunks, and only where 3 segments fit 256 SMs).
