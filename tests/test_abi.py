@@ -6,6 +6,7 @@ device pointers are safe: nothing dereferences them.
 import ctypes
 
 import pytest
+import torch
 
 import gated_delta_rule_101_b200 as kda
 from gated_delta_rule_101_b200 import build as kbuild
@@ -80,6 +81,21 @@ def test_chunk_fwd_rejects_short_workspace(lib):
         pytest.skip("this build needs no workspace for bf16 prefill")
     assert _chunk(lib, B=4, T=4096, H=16, ws=FAKE, ws_bytes=need.value - 1) == WORKSPACE
     assert _chunk(lib, B=4, T=4096, H=16, ws=None, ws_bytes=need.value) == WORKSPACE
+
+
+def test_launch_count_query_follows_the_plan():
+    """kda_chunk_fwd_launches reports the plan a call takes. Without a GPU the fused grid
+    is unavailable (it needs a cooperative-launch check), but the rest of the planning
+    is host logic: a long sequence with very few heads takes the segment scan (prep,
+    two chain passes, combine), many heads take prep then chains, packed sequences add
+    the offset scan, and fp32 input runs one kernel."""
+    assert kda.chunk_fwd_launches(1, 3000, 2) == 4
+    assert kda.chunk_fwd_launches(1, 300, 72) == 2
+    assert kda.chunk_fwd_launches(4, 4096, 16) == 2
+    assert kda.chunk_fwd_launches(1, 1000, 2, n_seqs=3) == 3
+    assert kda.chunk_fwd_launches(1, 256, 2, dtype=torch.float32) == 1
+    with pytest.raises(kda.KDAError):
+        kda.chunk_fwd_launches(1, 256, 2, C=32)
 
 
 def test_decode_rejects_bad_arguments(lib):
