@@ -43,6 +43,11 @@ PREFILL_BYTES_PER_TOKEN_HEAD = 3 * D * 2 + D * 4 + 4 + D * 2  # 1540
 STATE_BYTES = D * D * 4
 PAGES_FLOPS_PER_TOKEN_HEAD = 6 * D * D + 3 * 64 * D + 64 * 64  # 6Td^2 + 3TCd + TC^2 per token
 DECODE_BYTES_PER_HEAD_STEP = 2 * STATE_BYTES + PREFILL_BYTES_PER_TOKEN_HEAD  # 132612
+# gate bytes per token-head in each layout of the forget gate (the rest is 1028 B)
+GATE_BYTES = {"channel": D * 4, "channel_bf16": D * 2, "head": 4, "none": 0}
+GATE_MODELS = {"channel_bf16": "KDA with a bf16 per-channel gate",
+               "head": "Gated DeltaNet (one forget rate per head)",
+               "none": "DeltaNet (no forget gate)"}
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -133,9 +138,9 @@ class ClockSampler:
 # from; otherwise the roofline's traffic is null.
 TRAFFIC_SOURCES = {"prefill": ("prefill_tc.cu", "tc_ptx.cuh", "kda_internal.cuh"),
                    "decode": ("decode.cu", "kda_internal.cuh")}
-TRAFFIC = {"prefill": {"source_hash": "4bcc50ac00615650",  # prep + chain
-                       "bytes": 270968832 + 216843264 + 341876992 + 55703296},
-           "decode": {"source_hash": "1e7a03f630c48f57", "bytes": 547436544 + 479846400}}
+TRAFFIC = {"prefill": {"source_hash": "427a56f8d9b960cc",  # prep + chain
+                       "bytes": 270915328 + 215513088 + 341882624 + 53068544},
+           "decode": {"source_hash": "5e83d1dd83fc2ca5", "bytes": 547408640 + 479616512}}
 
 
 def source_hash(kind: str) -> str:
@@ -193,26 +198,23 @@ def time_steps(fn, steps, warmup, stream, flush=None):
     return times
 
 
-def cpu_oracle_sample(inp, n_heads=None):
-    """Times the fp64 oracle on sequence 0 of the prefill batch (all heads)."""
+def cpu_oracle_sample(inp, min_s: float = 10.0, max_reps: int = 40):
+    """Times the fp64 oracle on the whole prefill batch (every sequence and head),
+    repeated until at least ``min_s`` seconds of CPU time (at most ``max_reps`` passes)."""
     import oracle
 
-    H = inp.q.shape[2] if n_heads is None else n_heads
-    sl = lambda x: x[0:1, :, :H]
-    q, k, v, la = sl(inp.q), sl(inp.k), sl(inp.v), sl(inp.log_alpha)
-    b = inp.beta[0:1, :, :H]
-    S0 = None if inp.S0 is None else inp.S0[0:1, :H]
-    args = [oracle._f64(t) for t in (q, k, v, la, b, S0)]
+    args = [oracle._f64(t) for t in (inp.q, inp.k, inp.v, inp.log_alpha, inp.beta, inp.S0)]
     threads = oracle.default_threads()
-    t0 = time.perf_counter()
-    oracle.kda_fwd(*args, threads=threads)
-    dt = time.perf_counter() - t0
-    T = inp.q.shape[1]
-    full_H = inp.q.shape[2]
-    tokens = T * H / full_H  # token positions (all heads) equivalent
-    return {"value": tokens / dt, "unit": "tokens/s", "cores": threads, "kind": "oracle",
-            "sample": f"1 of {inp.q.shape[0]} sequences ({T} tokens x {H} heads) of the prefill "
-                      f"batch, fp64 recurrence, {dt:.2f} s"}
+    B, T, H = inp.q.shape[:3]
+    reps, total = 0, 0.0
+    while total < min_s and reps < max_reps:
+        t0 = time.perf_counter()
+        oracle.kda_fwd(*args, threads=threads)
+        total += time.perf_counter() - t0
+        reps += 1
+    return {"value": B * T * reps / total, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "sample": f"the whole prefill batch ({B} sequences x {T} tokens x {H} heads, bf16 "
+                      f"inputs widened to fp64) {reps} times, {total:.1f} s on {threads} threads"}
 
 
 def prefill_config(world: int) -> dict:
@@ -226,12 +228,12 @@ def prefill_config(world: int) -> dict:
 
 # ------------------------------------------------------------------ arms
 def run_reference(args, rank, world):
-    """The fp64 CPU oracle timed on host cores, a bounded sample per step."""
+    """The fp64 CPU oracle timed on host cores, the whole prefill workload per step."""
     if rank != 0:
         return
     from gated_delta_rule_101_b200.inputs import prefill_inputs
 
-    inp = prefill_inputs(B=1, T=PREFILL["T"], H=PREFILL["H"], dtype=torch.bfloat16,
+    inp = prefill_inputs(B=PREFILL["B"], T=PREFILL["T"], H=PREFILL["H"], dtype=torch.bfloat16,
                          s0_std=PREFILL["s0_std"], la_range=PREFILL["la_range"],
                          seed=PREFILL["seed"], device="cpu")
     import oracle
@@ -247,11 +249,10 @@ def run_reference(args, rank, world):
         oracle.kda_fwd(*args_np, threads=threads)
         times.append(time.perf_counter() - t0)
     total = sum(times)
-    tokens = PREFILL["T"] * args.steps
+    tokens = PREFILL["B"] * PREFILL["T"] * args.steps
     value = tokens / total
-    sample = (f"one of the {PREFILL['B']} sequences of the prefill workload per step "
-              f"({PREFILL['T']} tokens x {H} heads, bf16 inputs widened to fp64), {threads} threads; "
-              f"value = tokens of that sequence / CPU time")
+    sample = (f"the whole prefill workload per step ({PREFILL['B']} sequences x {PREFILL['T']} "
+              f"tokens x {H} heads, bf16 inputs widened to fp64), {threads} threads")
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True, "scaling": "weak",
@@ -336,6 +337,45 @@ def other_prefill_workloads(kda, dev, stream, flush, pk, world, rank):
     del inps, S, o, ws
     torch.cuda.empty_cache()
     return out
+
+
+def gate_layout_workloads(kda, dev, stream, flush, pk, world, rank):
+    """The step's workload with the forget gate in the other layouts (bf16 per channel,
+    one rate per head, none), each call timed on the device with L2 flushed before it."""
+    from gated_delta_rule_101_b200.inputs import prefill_inputs
+
+    B, T, H = PREFILL["B"], PREFILL["T"], PREFILL["H"]
+    ws = torch.empty(kda.workspace_size(B, T, H), dtype=torch.uint8, device=dev)
+    n_l = kda.chunk_fwd_launches(B, T, H)
+    out = {}
+    for gate, model in GATE_MODELS.items():
+        inp = prefill_inputs(B=B, T=T, H=H, dtype=torch.bfloat16, s0_std=PREFILL["s0_std"],
+                             la_range=PREFILL["la_range"], seed=PREFILL["seed"] + 1000 * rank,
+                             gate=gate, device=dev)
+        o = torch.empty_like(inp.v)
+        S_T = torch.empty_like(inp.S0)
+
+        def call():
+            kda.chunk_fwd(inp.q, inp.k, inp.v, inp.log_alpha, inp.beta, inp.S0, out=o, state_out=S_T,
+                          workspace=ws, stream=stream)
+
+        barrier(world)
+        times = time_steps(call, 10, 3, stream, flush)
+        ms = max_over_ranks(sum(times), world, dev) / len(times)
+        alg = (PREFILL_BYTES_PER_TOKEN_HEAD - GATE_BYTES["channel"] + GATE_BYTES[gate]) * B * T * H \
+            + 2 * STATE_BYTES * B * H
+        out[gate] = {"value": B * T * world / (ms * 1e-3), "unit": "tokens/s", "ms_per_call": ms,
+                     "config": {"workload": f"{model}: prefill B={B} T={T} H={H} d=128, bf16",
+                                "l2": "flushed before every call"},
+                     "roofline": {"bound": "hbm", "achieved": alg / (ms * 1e-3) / 1e9,
+                                  "peak": pk["hbm_gbs"], "unit": "GB/s",
+                                  "frac": alg / (ms * 1e-3) / 1e9 / pk["hbm_gbs"],
+                                  "alg_bytes_per_launch": alg},
+                     "gpu_launches": n_l * len(times)}
+        del inp, o, S_T
+    del ws
+    torch.cuda.empty_cache()
+    return {"gate_layouts": out}
 
 
 def run_kda(args, rank, world, local_rank):
@@ -462,7 +502,9 @@ def run_kda(args, rank, world, local_rank):
         del graph, dinp, S, od
 
     # ---------------- the other prefill workloads (reported beside the step, not the step)
-    extra = {} if args.no_extra else other_prefill_workloads(kda, dev, stream, flush, pk, world, rank)
+    extra = {} if args.no_extra else {
+        **other_prefill_workloads(kda, dev, stream, flush, pk, world, rank),
+        **gate_layout_workloads(kda, dev, stream, flush, pk, world, rank)}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -489,7 +531,7 @@ def main():
     ap.add_argument("--decode-steps", type=int, default=DECODE["steps"])
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-extra", action="store_true",
-                    help="skip the packed and long-context prefill workloads")
+                    help="skip the packed, long-context and gate-layout prefill workloads")
     ap.add_argument("--shape", default=None,
                     help="B,T,H of the prefill step instead of 4,4096,16 (for profiling captures)")
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -6,6 +6,13 @@ libkda (``libkda.so`` next to this file, built by ``build.py`` from
 * ``chunk_fwd``   -> ``kda_chunk_fwd``: chunk-parallel prefill, C = 64;
 * ``decode_step`` -> ``kda_decode_step``: one recurrent decode token.
 
+Both take the forget gate as ``log_alpha`` in any of the library's gate
+layouts (``kda_gate``), told apart by shape and dtype: ``[..., H, 128]``
+fp32 (KDA, one rate per key channel; ``kda_chunk_fwd``), the same in bf16,
+``[..., H]`` fp32 (one rate per head: Gated DeltaNet), or ``None`` (no gate:
+DeltaNet); the last three go through ``kda_chunk_fwd_gated`` /
+``kda_decode_step_gated``.
+
 This module only marshals arguments: it checks dtypes, shapes and devices,
 allocates outputs with PyTorch (device memory is PyTorch's job here), and
 passes raw device pointers and the current CUDA stream to the C ABI. Every
@@ -25,6 +32,9 @@ LIB_PATH = os.path.join(_PKG, "libkda.so")
 HEADER = os.path.join(os.path.dirname(_PKG), "include", "kda.h")
 
 KDA_BF16, KDA_F32 = 0, 1
+KDA_GATE_CHANNEL, KDA_GATE_CHANNEL_BF16, KDA_GATE_HEAD, KDA_GATE_NONE = 0, 1, 2, 3
+GATE_NAMES = {KDA_GATE_CHANNEL: "channel", KDA_GATE_CHANNEL_BF16: "channel_bf16",
+              KDA_GATE_HEAD: "head", KDA_GATE_NONE: "none"}
 KDA_OK = 0
 STATUS = {0: "KDA_OK", -1: "KDA_ERR_INVALID_ARG", -2: "KDA_ERR_UNSUPPORTED",
           -3: "KDA_ERR_WORKSPACE", -4: "KDA_ERR_CUDA", -5: "KDA_ERR_TIMEOUT",
@@ -64,6 +74,11 @@ def _bind(lib: ctypes.CDLL) -> ctypes.CDLL:
     lib.kda_get_device_status.argtypes = [ctypes.POINTER(ctypes.c_int)]
     lib.kda_decode_step.restype = i32
     lib.kda_decode_step.argtypes = [vp, vp, vp, fp, fp, fp, vp, i32, i32, i32, vp]
+    lib.kda_chunk_fwd_gated.restype = i32
+    lib.kda_chunk_fwd_gated.argtypes = [vp, vp, vp, vp, i32, fp, fp, vp, fp, i32, i64, i32, i32,
+                                        vp, i32, vp, i32, vp, ctypes.c_size_t, vp]
+    lib.kda_decode_step_gated.restype = i32
+    lib.kda_decode_step_gated.argtypes = [vp, vp, vp, vp, i32, fp, fp, vp, i32, i32, i32, vp]
     return lib
 
 
@@ -109,6 +124,25 @@ def _need(t: torch.Tensor, name: str, dtype, device) -> None:
         raise ValueError(f"{name} must be contiguous")
 
 
+def gate_kind(log_alpha: torch.Tensor | None, q: torch.Tensor) -> int:
+    """The kda_gate layout of ``log_alpha`` for inputs shaped like ``q``."""
+    if log_alpha is None:
+        return KDA_GATE_NONE
+    if log_alpha.shape == q.shape and log_alpha.dtype == torch.float32:
+        return KDA_GATE_CHANNEL
+    if log_alpha.shape == q.shape and log_alpha.dtype == torch.bfloat16:
+        return KDA_GATE_CHANNEL_BF16
+    if log_alpha.shape == q.shape[:-1] and log_alpha.dtype == torch.float32:
+        return KDA_GATE_HEAD
+    raise ValueError(f"log_alpha must be None, fp32/bf16 {tuple(q.shape)} or fp32 "
+                     f"{tuple(q.shape[:-1])}; got {log_alpha.dtype} {tuple(log_alpha.shape)}")
+
+
+def _need_gate(log_alpha, gate: int, device) -> None:
+    if gate != KDA_GATE_NONE:
+        _need(log_alpha, "log_alpha", log_alpha.dtype, device)
+
+
 def _stream_handle(stream: torch.cuda.Stream | None, device) -> ctypes.c_void_p:
     s = stream if stream is not None else torch.cuda.current_stream(device)
     return ctypes.c_void_p(s.cuda_stream)
@@ -141,9 +175,10 @@ def chunk_fwd(q, k, v, log_alpha, beta, S0=None, *, cu_seqlens=None, cu_seqlens_
               out=None, final_state=True, state_out=None, workspace=None, stream=None, C=CHUNK):
     """KDA prefill through ``kda_chunk_fwd``; returns ``(o, S_T)`` (S_T None if not requested).
 
-    ``q, k, v, log_alpha``: ``[B, T, H, 128]`` (or packed ``[T, H, 128]`` with
+    ``q, k, v``: ``[B, T, H, 128]`` (or packed ``[T, H, 128]`` with
     ``cu_seqlens``, an int32 device tensor of ``n_seqs + 1`` offsets).
-    ``beta``: ``[B, T, H]``. ``S0``: fp32 ``[n_seqs, H, 128, 128]`` or None.
+    ``log_alpha``: like ``q`` (fp32 or bf16), ``[B, T, H]`` fp32, or None (see
+    ``gate_kind``). ``beta``: ``[B, T, H]``. ``S0``: fp32 ``[n_seqs, H, 128, 128]`` or None.
     ``state_out`` may be ``S0`` itself for in-place carry.
     """
     dev = q.device
@@ -163,10 +198,11 @@ def chunk_fwd(q, k, v, log_alpha, beta, S0=None, *, cu_seqlens=None, cu_seqlens_
         _need(t, name, q.dtype, dev)
         if t.shape != q.shape:
             raise ValueError(f"{name} shape {tuple(t.shape)} != q shape {tuple(q.shape)}")
-    _need(log_alpha, "log_alpha", torch.float32, dev)
+    gate = gate_kind(log_alpha, q)
+    _need_gate(log_alpha, gate, dev)
     _need(beta, "beta", torch.float32, dev)
-    if log_alpha.shape != q.shape or beta.shape != q.shape[:-1]:
-        raise ValueError("log_alpha must match q; beta must be q.shape[:-1]")
+    if beta.shape != q.shape[:-1]:
+        raise ValueError("beta must be q.shape[:-1]")
     nseq = n_seqs if packed else B
     sshape = (nseq, H, HEAD_DIM, HEAD_DIM)
     if S0 is not None:
@@ -189,20 +225,23 @@ def chunk_fwd(q, k, v, log_alpha, beta, S0=None, *, cu_seqlens=None, cu_seqlens_
     if need and workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=dev)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    st = lib().kda_chunk_fwd(
-        _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(S0), _ptr(out), _ptr(S_T),
-        B, T, H, C, _ptr(cu_seqlens), n_seqs, _ptr(host_cu), code, _ptr(workspace), ws_bytes,
-        _stream_handle(stream, dev))
+    tail = (_ptr(beta), _ptr(S0), _ptr(out), _ptr(S_T), B, T, H, C, _ptr(cu_seqlens), n_seqs,
+            _ptr(host_cu), code, _ptr(workspace), ws_bytes, _stream_handle(stream, dev))
+    if gate == KDA_GATE_CHANNEL:
+        st, where = lib().kda_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), *tail), "kda_chunk_fwd"
+    else:
+        st = lib().kda_chunk_fwd_gated(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), gate, *tail)
+        where = "kda_chunk_fwd_gated"
     if st != KDA_OK:
-        raise KDAError(st, "kda_chunk_fwd")
+        raise KDAError(st, where)
     return out, S_T
 
 
 def decode_step(q, k, v, log_alpha, beta, S, *, out=None, stream=None):
     """One decode token through ``kda_decode_step``; updates ``S`` in place, returns ``o``.
 
-    ``q, k, v, log_alpha``: ``[N, H, 128]``; ``beta``: ``[N, H]``;
-    ``S``: fp32 ``[N, H, 128, 128]``.
+    ``q, k, v``: ``[N, H, 128]``; ``log_alpha``: like ``q`` (fp32 or bf16), ``[N, H]``
+    fp32, or None (see ``gate_kind``); ``beta``: ``[N, H]``; ``S``: fp32 ``[N, H, 128, 128]``.
     """
     dev = q.device
     code = _dtype_code(q)
@@ -211,17 +250,22 @@ def decode_step(q, k, v, log_alpha, beta, S, *, out=None, stream=None):
         raise ValueError(f"head dim must be {HEAD_DIM}, got {dk}")
     for name, t in (("q", q), ("k", k), ("v", v)):
         _need(t, name, q.dtype, dev)
-    _need(log_alpha, "log_alpha", torch.float32, dev)
+    gate = gate_kind(log_alpha, q)
+    _need_gate(log_alpha, gate, dev)
     _need(beta, "beta", torch.float32, dev)
     _need(S, "S", torch.float32, dev)
     if tuple(S.shape) != (N, H, HEAD_DIM, HEAD_DIM):
         raise ValueError("S must be [N, H, 128, 128]")
     if out is None:
         out = torch.empty_like(v)
-    st = lib().kda_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(S),
-                               _ptr(out), N, H, code, _stream_handle(stream, dev))
+    tail = (_ptr(beta), _ptr(S), _ptr(out), N, H, code, _stream_handle(stream, dev))
+    if gate == KDA_GATE_CHANNEL:
+        st, where = lib().kda_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), *tail), "kda_decode_step"
+    else:
+        st = lib().kda_decode_step_gated(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), gate, *tail)
+        where = "kda_decode_step_gated"
     if st != KDA_OK:
-        raise KDAError(st, "kda_decode_step")
+        raise KDAError(st, where)
     return out
 
 

@@ -10,6 +10,16 @@ namespace {
 constexpr int KDA_VERSION = 100;  // 0.1.0
 
 bool valid_dtype(int dtype) { return dtype == KDA_BF16 || dtype == KDA_F32; }
+bool valid_gate(int gate) { return gate >= KDA_GATE_CHANNEL && gate <= KDA_GATE_NONE; }
+
+// The gate tensor is required unless there is no gate; the tensor-core path reads
+// per-channel gates through TMA (16-byte base) and head gates as fp32 scalars.
+int check_gate_ptr(const void *log_alpha, int gate, bool tma) {
+    if (gate == KDA_GATE_NONE) return KDA_OK;
+    if (!log_alpha) return KDA_ERR_INVALID_ARG;
+    const uintptr_t align = gate == KDA_GATE_HEAD ? 4u : (tma ? 16u : (gate == KDA_GATE_CHANNEL ? 4u : 2u));
+    return ((uintptr_t)log_alpha & (align - 1)) == 0 ? KDA_OK : KDA_ERR_INVALID_ARG;
+}
 
 // Validates the shape arguments shared by the size query and the call.
 int check_prefill_shape(int B, int64_t T, int H, int C, int n_seqs, int dtype) {
@@ -32,7 +42,7 @@ const char *kda_strerror(int status) {
     switch (status) {
     case KDA_OK: return "KDA_OK";
     case KDA_ERR_INVALID_ARG: return "KDA_ERR_INVALID_ARG: invalid argument";
-    case KDA_ERR_UNSUPPORTED: return "KDA_ERR_UNSUPPORTED: unsupported chunk size or dtype";
+    case KDA_ERR_UNSUPPORTED: return "KDA_ERR_UNSUPPORTED: unsupported chunk size, dtype or gate layout";
     case KDA_ERR_WORKSPACE: return "KDA_ERR_WORKSPACE: workspace missing or too small";
     case KDA_ERR_CUDA: return "KDA_ERR_CUDA: kernel launch failed";
     case KDA_ERR_TIMEOUT: return "KDA_ERR_TIMEOUT: bounded device wait expired";
@@ -67,11 +77,24 @@ int kda_chunk_fwd(const void *q, const void *k, const void *v, const float *log_
                   int H, int C, const int32_t *cu_seqlens, int n_seqs,
                   const int32_t *cu_seqlens_host, int dtype, void *workspace,
                   size_t workspace_bytes, void *stream) {
+    return kda_chunk_fwd_gated(q, k, v, log_alpha, KDA_GATE_CHANNEL, beta, S0, o, S_T, B, T, H, C,
+                               cu_seqlens, n_seqs, cu_seqlens_host, dtype, workspace,
+                               workspace_bytes, stream);
+}
+
+int kda_chunk_fwd_gated(const void *q, const void *k, const void *v, const void *log_alpha,
+                        int gate, const float *beta, const float *S0, void *o, float *S_T, int B,
+                        int64_t T, int H, int C, const int32_t *cu_seqlens, int n_seqs,
+                        const int32_t *cu_seqlens_host, int dtype, void *workspace,
+                        size_t workspace_bytes, void *stream) {
     int st = check_prefill_shape(B, T, H, C, n_seqs, dtype);
     if (st != KDA_OK) return st;
+    if (!valid_gate(gate)) return KDA_ERR_UNSUPPORTED;
     const bool packed = n_seqs > 0;
     if (packed != (cu_seqlens != nullptr)) return KDA_ERR_INVALID_ARG;
-    if (T > 0 && (!q || !k || !v || !log_alpha || !beta || !o)) return KDA_ERR_INVALID_ARG;
+    if (T > 0 && (!q || !k || !v || !beta || !o)) return KDA_ERR_INVALID_ARG;
+    if (T > 0 && check_gate_ptr(log_alpha, gate, dtype == KDA_BF16) != KDA_OK)
+        return KDA_ERR_INVALID_ARG;
     if (cu_seqlens_host) {
         if (!packed || cu_seqlens_host[0] != 0 || cu_seqlens_host[n_seqs] != T)
             return KDA_ERR_INVALID_ARG;
@@ -89,14 +112,14 @@ int kda_chunk_fwd(const void *q, const void *k, const void *v, const float *log_
     cudaError_t err;
     if (dtype == KDA_BF16) {
         // TMA requires 16-byte aligned tensor bases
-        if (T > 0 && ((((uintptr_t)q | (uintptr_t)k | (uintptr_t)v | (uintptr_t)log_alpha) & 15u) != 0))
+        if (T > 0 && ((((uintptr_t)q | (uintptr_t)k | (uintptr_t)v) & 15u) != 0))
             return KDA_ERR_INVALID_ARG;
         if ((S0 && ((uintptr_t)S0 & 15u)) || (S_T && ((uintptr_t)S_T & 15u)) || ((uintptr_t)o & 15u))
             return KDA_ERR_INVALID_ARG;
-        err = kda::launch_prefill_tc(q, k, v, log_alpha, beta, S0, o, S_T, B, T, H, cu_seqlens,
-                                     n_seqs, workspace, s);
+        err = kda::launch_prefill_tc(q, k, v, log_alpha, gate, beta, S0, o, S_T, B, T, H,
+                                     cu_seqlens, n_seqs, workspace, s);
     } else {
-        err = kda::launch_prefill_simt(q, k, v, log_alpha, beta, S0, o, S_T, nseq, T, H,
+        err = kda::launch_prefill_simt(q, k, v, log_alpha, gate, beta, S0, o, S_T, nseq, T, H,
                                        cu_seqlens, dtype, s);
     }
     if (err == cudaErrorInvalidValue) return KDA_ERR_INVALID_ARG;
@@ -111,13 +134,21 @@ int kda_get_device_status(int *status) {
 int kda_decode_step(const void *q, const void *k, const void *v, const float *log_alpha,
                     const float *beta, float *S, void *o, int N, int H, int dtype,
                     void *stream) {
-    if (!valid_dtype(dtype)) return KDA_ERR_UNSUPPORTED;
+    return kda_decode_step_gated(q, k, v, log_alpha, KDA_GATE_CHANNEL, beta, S, o, N, H, dtype,
+                                 stream);
+}
+
+int kda_decode_step_gated(const void *q, const void *k, const void *v, const void *log_alpha,
+                          int gate, const float *beta, float *S, void *o, int N, int H,
+                          int dtype, void *stream) {
+    if (!valid_dtype(dtype) || !valid_gate(gate)) return KDA_ERR_UNSUPPORTED;
     if (N <= 0 || H <= 0) return KDA_ERR_INVALID_ARG;
     if ((int64_t)N * H > (int64_t)INT32_MAX) return KDA_ERR_INVALID_ARG;
-    if (!q || !k || !v || !log_alpha || !beta || !S || !o) return KDA_ERR_INVALID_ARG;
+    if (!q || !k || !v || !beta || !S || !o) return KDA_ERR_INVALID_ARG;
+    if (check_gate_ptr(log_alpha, gate, false) != KDA_OK) return KDA_ERR_INVALID_ARG;
     if (((uintptr_t)S & 15u) != 0) return KDA_ERR_INVALID_ARG;  // 128-bit state accesses
-    const cudaError_t err =
-        kda::launch_decode(q, k, v, log_alpha, beta, S, o, N, H, dtype, (cudaStream_t)stream);
+    const cudaError_t err = kda::launch_decode(q, k, v, log_alpha, gate, beta, S, o, N, H, dtype,
+                                               (cudaStream_t)stream);
     return err == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 

@@ -23,10 +23,10 @@ constexpr int DEC_THREADS = 256;
 constexpr int DEC_WARPS = DEC_THREADS / 32;
 constexpr int ROWS_PER_WARP = D / DEC_WARPS;  // 16
 
-template <typename TIn>
+template <typename TIn, int GATE>
 __global__ void __launch_bounds__(DEC_THREADS)
 decode_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const TIn *__restrict__ v,
-              const float *__restrict__ log_alpha, const float *__restrict__ beta,
+              const void *__restrict__ log_alpha, const float *__restrict__ beta,
               float *__restrict__ S, TIn *__restrict__ o) {
     const int64_t nh = blockIdx.x;  // sequence * H + head
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -45,7 +45,7 @@ decode_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const TIn *_
     if (tid < D) {
         const float kk = to_f32(k[nh * D + tid]);
         const float qq = to_f32(q[nh * D + tid]);
-        const float a = expf(log_alpha[nh * D + tid]);
+        const float a = GATE == KDA_GATE_NONE ? 1.f : expf(gate_log<GATE>(log_alpha, nh, tid));
         s_k[tid] = kk;
         s_a[tid] = a;
         s_ka[tid] = kk * a;
@@ -102,18 +102,23 @@ decode_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const TIn *_
 
 }  // namespace
 
-cudaError_t launch_decode(const void *q, const void *k, const void *v, const float *log_alpha,
-                          const float *beta, float *S, void *o, int N, int H, int dtype,
-                          cudaStream_t stream) {
+cudaError_t launch_decode(const void *q, const void *k, const void *v, const void *log_alpha,
+                          int gate, const float *beta, float *S, void *o, int N, int H,
+                          int dtype, cudaStream_t stream) {
     const unsigned grid = (unsigned)((int64_t)N * H);
-    if (dtype == KDA_BF16) {
-        decode_kernel<__nv_bfloat16><<<grid, DEC_THREADS, 0, stream>>>(
-            (const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k, (const __nv_bfloat16 *)v,
-            log_alpha, beta, S, (__nv_bfloat16 *)o);
-    } else {
-        decode_kernel<float><<<grid, DEC_THREADS, 0, stream>>>(
-            (const float *)q, (const float *)k, (const float *)v, log_alpha, beta, S, (float *)o);
-    }
+    with_gate(gate, [&](auto g) {
+        constexpr int G = decltype(g)::value;
+        if (dtype == KDA_BF16) {
+            decode_kernel<__nv_bfloat16, G><<<grid, DEC_THREADS, 0, stream>>>(
+                (const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k, (const __nv_bfloat16 *)v,
+                log_alpha, beta, S, (__nv_bfloat16 *)o);
+        } else {
+            decode_kernel<float, G><<<grid, DEC_THREADS, 0, stream>>>(
+                (const float *)q, (const float *)k, (const float *)v, log_alpha, beta, S,
+                (float *)o);
+        }
+        return 0;
+    });
     return cudaGetLastError();
 }
 

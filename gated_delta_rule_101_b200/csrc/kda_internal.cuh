@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <type_traits>
+
 #include "kda.h"
 
 namespace kda {
@@ -19,6 +21,34 @@ template <typename T> __device__ __forceinline__ T from_f32(float x);
 template <> __device__ __forceinline__ float from_f32<float>(float x) { return x; }
 template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
     return __float2bfloat16_rn(x);
+}
+
+// Log forget rate of key channel c for token-head row `row` (= token * H + head), in
+// each kda_gate layout: per channel (fp32 or bf16, rows of 128), one per row (a
+// head-wide scalar gate), or none (rate 1, log 0).
+template <int GATE>
+__device__ __forceinline__ float gate_log(const void *la, int64_t row, int c) {
+    if constexpr (GATE == KDA_GATE_CHANNEL) {
+        return static_cast<const float *>(la)[row * D + c];
+    } else if constexpr (GATE == KDA_GATE_CHANNEL_BF16) {
+        return __bfloat162float(static_cast<const __nv_bfloat16 *>(la)[row * D + c]);
+    } else if constexpr (GATE == KDA_GATE_HEAD) {
+        return static_cast<const float *>(la)[row];
+    } else {
+        return 0.f;
+    }
+}
+
+// Calls f(std::integral_constant<int, GATE>) for a runtime gate layout (validated by
+// the caller).
+template <class F>
+auto with_gate(int gate, F &&f) {
+    switch (gate) {
+    case KDA_GATE_CHANNEL_BF16: return f(std::integral_constant<int, KDA_GATE_CHANNEL_BF16>{});
+    case KDA_GATE_HEAD: return f(std::integral_constant<int, KDA_GATE_HEAD>{});
+    case KDA_GATE_NONE: return f(std::integral_constant<int, KDA_GATE_NONE>{});
+    default: return f(std::integral_constant<int, KDA_GATE_CHANNEL>{});
+    }
 }
 
 // Where a sequence's tokens live: [start, start + len) in token rows.
@@ -39,20 +69,20 @@ __device__ __forceinline__ SeqSpan seq_span(const int32_t *cu, int64_t T, int s)
 }
 
 // ---- launchers (host side); each returns cudaGetLastError() of its launch ----
-cudaError_t launch_decode(const void *q, const void *k, const void *v, const float *log_alpha,
-                          const float *beta, float *S, void *o, int N, int H, int dtype,
-                          cudaStream_t stream);
+cudaError_t launch_decode(const void *q, const void *k, const void *v, const void *log_alpha,
+                          int gate, const float *beta, float *S, void *o, int N, int H,
+                          int dtype, cudaStream_t stream);
 
 cudaError_t launch_prefill_simt(const void *q, const void *k, const void *v,
-                                const float *log_alpha, const float *beta, const float *S0,
+                                const void *log_alpha, int gate, const float *beta, const float *S0,
                                 void *o, float *S_T, int n_seqs, int64_t T, int H,
                                 const int32_t *cu_seqlens, int dtype, cudaStream_t stream);
 
 // Tensor-core prefill (bf16 q/k/v): workspace bytes and launcher.
 size_t prefill_tc_workspace(int B, int64_t T, int H, int n_seqs);
 int prefill_tc_launches(int B, int64_t T, int H, int n_seqs);
-cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, const float *log_alpha,
-                              const float *beta, const float *S0, void *o, float *S_T, int B,
+cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, const void *log_alpha,
+                              int gate, const float *beta, const float *S0, void *o, float *S_T, int B,
                               int64_t T, int H, const int32_t *cu_seqlens, int n_seqs,
                               void *workspace, cudaStream_t stream);
 

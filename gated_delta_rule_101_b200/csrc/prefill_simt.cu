@@ -59,10 +59,10 @@ __device__ __forceinline__ void load_row8(const TIn *src, float *dst) {
     for (int e = 0; e < 8; ++e) dst[e] = to_f32(src[e]);
 }
 
-template <typename TIn>
+template <typename TIn, int GATE>
 __global__ void __launch_bounds__(NT, 1)
 prefill_simt_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k,
-                    const TIn *__restrict__ v, const float *__restrict__ log_alpha,
+                    const TIn *__restrict__ v, const void *__restrict__ log_alpha,
                     const float *__restrict__ beta, const float *__restrict__ S0,
                     TIn *__restrict__ o, float *__restrict__ S_T, int64_t T, int H,
                     const int32_t *__restrict__ cu_seqlens) {
@@ -93,7 +93,7 @@ prefill_simt_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k,
                 load_row8(q + off, dq);
                 load_row8(k + off, dk);
 #pragma unroll
-                for (int x = 0; x < 8; ++x) dg[x] = log_alpha[off + x];
+                for (int x = 0; x < 8; ++x) dg[x] = gate_log<GATE>(log_alpha, (tok0 + r) * H + h, c8 + x);
             } else {
 #pragma unroll
                 for (int x = 0; x < 8; ++x) dq[x] = dk[x] = dg[x] = 0.f;
@@ -254,16 +254,16 @@ prefill_simt_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k,
         }
 }
 
-template <typename TIn>
-cudaError_t launch_t(const void *q, const void *k, const void *v, const float *la,
+template <typename TIn, int GATE>
+cudaError_t launch_t(const void *q, const void *k, const void *v, const void *la,
                      const float *beta, const float *S0, void *o, float *S_T, int n_seqs,
                      int64_t T, int H, const int32_t *cu, cudaStream_t stream) {
     const size_t smem = sizeof(SimtSmem);
-    cudaError_t err = cudaFuncSetAttribute(prefill_simt_kernel<TIn>,
+    cudaError_t err = cudaFuncSetAttribute(prefill_simt_kernel<TIn, GATE>,
                                            cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (err != cudaSuccess) return err;
     dim3 grid((unsigned)n_seqs, (unsigned)H, D / DVS);
-    prefill_simt_kernel<TIn><<<grid, NT, smem, stream>>>(
+    prefill_simt_kernel<TIn, GATE><<<grid, NT, smem, stream>>>(
         (const TIn *)q, (const TIn *)k, (const TIn *)v, la, beta, S0, (TIn *)o, S_T, T, H, cu);
     return cudaGetLastError();
 }
@@ -271,14 +271,18 @@ cudaError_t launch_t(const void *q, const void *k, const void *v, const float *l
 }  // namespace
 
 cudaError_t launch_prefill_simt(const void *q, const void *k, const void *v,
-                                const float *log_alpha, const float *beta, const float *S0,
-                                void *o, float *S_T, int n_seqs, int64_t T, int H,
-                                const int32_t *cu_seqlens, int dtype, cudaStream_t stream) {
-    if (dtype == KDA_BF16)
-        return launch_t<__nv_bfloat16>(q, k, v, log_alpha, beta, S0, o, S_T, n_seqs, T, H,
-                                       cu_seqlens, stream);
-    return launch_t<float>(q, k, v, log_alpha, beta, S0, o, S_T, n_seqs, T, H, cu_seqlens,
-                           stream);
+                                const void *log_alpha, int gate, const float *beta,
+                                const float *S0, void *o, float *S_T, int n_seqs, int64_t T,
+                                int H, const int32_t *cu_seqlens, int dtype,
+                                cudaStream_t stream) {
+    return with_gate(gate, [&](auto g) {
+        constexpr int G = decltype(g)::value;
+        if (dtype == KDA_BF16)
+            return launch_t<__nv_bfloat16, G>(q, k, v, log_alpha, beta, S0, o, S_T, n_seqs, T, H,
+                                              cu_seqlens, stream);
+        return launch_t<float, G>(q, k, v, log_alpha, beta, S0, o, S_T, n_seqs, T, H,
+                                  cu_seqlens, stream);
+    });
 }
 
 }  // namespace kda

@@ -204,9 +204,10 @@ constexpr uint32_t PREP_PART = ((PREP_SMEM - 1024 + 1023) / 1024) * 1024;
 
 // Arguments of the prep work that are fixed for a launch.
 struct PrepArgs {
-    const CUtensorMap *tm_q, *tm_k, *tm_la;
+    const CUtensorMap *tm_q, *tm_k, *tm_la;  // tm_la: per-channel gate layouts only
     const __nv_bfloat16 *q, *k;
-    const float *log_alpha, *beta;
+    const void *log_alpha;  // in the kernel's kda_gate layout
+    const float *beta;
     unsigned char *ws_blobs;
     int64_t T;
     int H;
@@ -294,11 +295,30 @@ struct PrepWorker {
 // then warmed in L2. ready != null: publish the blob's ready flag. Thread 0 calls
 // hook.before_wait() and hook.after_wait() around its wait for the item's loads (work
 // whose latency that wait can hide).
+// Log gate of channels c .. c+3 of token-head row `row` (read once: streamed past L1).
+template <int GATE>
+__device__ __forceinline__ float4 load_gate4(const void *la, int64_t row, int c) {
+    if constexpr (GATE == KDA_GATE_CHANNEL) {
+        return __ldcs(reinterpret_cast<const float4 *>(static_cast<const float *>(la) + row * D + c));
+    } else if constexpr (GATE == KDA_GATE_CHANNEL_BF16) {
+        const uint2 raw = __ldcs(reinterpret_cast<const uint2 *>(
+            static_cast<const __nv_bfloat16 *>(la) + row * D + c));
+        const float2 lo = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&raw.x));
+        const float2 hi = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&raw.y));
+        return make_float4(lo.x, lo.y, hi.x, hi.y);
+    } else if constexpr (GATE == KDA_GATE_HEAD) {
+        const float x = __ldcs(static_cast<const float *>(la) + row);
+        return make_float4(x, x, x, x);
+    } else {
+        return make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+}
+
 struct NoHook {
     __device__ __forceinline__ void before_wait() {}
     __device__ __forceinline__ void after_wait() {}
 };
-template <class Worker, class Prefetch, class Hook = NoHook>
+template <int GATE, class Worker, class Prefetch, class Hook = NoHook>
 __device__ __forceinline__ void prep_item(Worker &w, const PrepArgs &a, int slot, int h,
                                           SeqSpan span, int n, Prefetch pf,
                                           int32_t *__restrict__ ready, Hook hook = Hook()) {
@@ -328,7 +348,12 @@ __device__ __forceinline__ void prep_item(Worker &w, const PrepArgs &a, int slot
             tma_prefetch_l2_2d(a.tm_q, pf_x + 64, pf_y);
             tma_prefetch_l2_2d(a.tm_k, pf_x, pf_y);
             tma_prefetch_l2_2d(a.tm_k, pf_x + 64, pf_y);
-            tma_prefetch_l2_2d(a.tm_la, pf_x, pf_y);
+            if constexpr (GATE == KDA_GATE_CHANNEL) {  // fp32 boxes of 128 channels
+                tma_prefetch_l2_2d(a.tm_la, pf_x, pf_y);
+            } else if constexpr (GATE == KDA_GATE_CHANNEL_BF16) {  // bf16 boxes of 64
+                tma_prefetch_l2_2d(a.tm_la, pf_x, pf_y);
+                tma_prefetch_l2_2d(a.tm_la, pf_x + 64, pf_y);
+            }
         }
     }
     if (tid < CH) sbeta[tid] = tid < L ? a.beta[(tok0 + tid) * H + h] : 0.f;
@@ -340,12 +365,21 @@ __device__ __forceinline__ void prep_item(Worker &w, const PrepArgs &a, int slot
     const int f = lane, fblk = f >> 4, fchunk = (f & 15) >> 1, fhalf = (f & 1) * 8;
     float4 g4[8];
     float gls[4], gams[4];
-    {
-        const float *la = a.log_alpha + (tok0 * H + h) * (int64_t)D + 4 * f;
+    if constexpr (GATE == KDA_GATE_NONE) {  // no decay: g = 0, exp(g_L) = 1
+#pragma unroll
+        for (int v = 0; v < 8; ++v) g4[v] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) { gls[e] = 0.f; gams[e] = 1.f; }
+        if (warp == 0) {
+            *reinterpret_cast<float4 *>(sgl + 4 * f) = make_float4(0.f, 0.f, 0.f, 0.f);
+            *reinterpret_cast<float4 *>(sgam + 4 * f) = make_float4(1.f, 1.f, 1.f, 1.f);
+        }
+    } else {
+        const int64_t row0 = tok0 * H + h;  // token-head row of the chunk's first token
 #pragma unroll
         for (int v = 0; v < 8; ++v) {
             const int r = 8 * warp + v;
-            g4[v] = r < L ? __ldcs(reinterpret_cast<const float4 *>(la + (int64_t)r * H * D))
+            g4[v] = r < L ? load_gate4<GATE>(a.log_alpha, row0 + (int64_t)r * H, 4 * f)
                           : make_float4(0.f, 0.f, 0.f, 0.f);
         }
 #pragma unroll
@@ -411,15 +445,20 @@ __device__ __forceinline__ void prep_item(Worker &w, const PrepArgs &a, int slot
             const __nv_bfloat16 *qb = reinterpret_cast<const __nv_bfloat16 *>(&qraw);
             const __nv_bfloat16 *kb = reinterpret_cast<const __nv_bfloat16 *>(&kraw);
             const float gs[4] = {g4[v].x, g4[v].y, g4[v].z, g4[v].w};
+            // a head-wide gate has one g per row: its two exponentials serve all channels
+            const float eg_row = GATE == KDA_GATE_NONE ? 1.f : __expf(gs[0]);
+            const float ein_row = GATE == KDA_GATE_NONE ? 1.f : __expf(-gs[0]);
+            constexpr bool ROW_GATE = GATE == KDA_GATE_HEAD || GATE == KDA_GATE_NONE;
             float qe[4], ke[4], kin[4], kt[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
                 const float x = live ? __bfloat162float(qb[e]) : 0.f;
                 const float kk = live ? __bfloat162float(kb[e]) : 0.f;
-                const float eg = __expf(gs[e]);
+                const float eg = ROW_GATE ? eg_row : __expf(gs[e]);
                 qe[e] = x * eg;
                 ke[e] = kk * eg;
-                const float kin_ = kk * __expf(-gs[e]);  // exp(-g) <= exp(80) for good channels
+                // exp(-g) <= exp(80) for good channels
+                const float kin_ = kk * (ROW_GATE ? ein_row : __expf(-gs[e]));
                 if constexpr (BAD) {
                     kin[e] = badc[e] ? 0.f : kin_;
                     kt[e] = badc[e] ? kk * __expf(gls[e] - gs[e]) : kin_ * gams[e];
@@ -438,7 +477,7 @@ __device__ __forceinline__ void prep_item(Worker &w, const PrepArgs &a, int slot
                 make_uint2(pack_bf16x2(kin[0], kin[1]), pack_bf16x2(kin[2], kin[3]));
         }
     };
-    if (n_bad) gate_rows(std::true_type{});
+    if (GATE != KDA_GATE_NONE && n_bad) gate_rows(std::true_type{});
     else gate_rows(std::false_type{});
     fence_async_smem();
     tc_fence_before();
@@ -492,10 +531,11 @@ __device__ __forceinline__ void prep_item(Worker &w, const PrepArgs &a, int slot
                     const int bi = e >> 6, r = e & 63;
                     float qx = 0.f, kx = 0.f, gx = 0.f;
                     if (b0 + bi < nb_total) {
-                        const int64_t ccol = (int64_t)h * D + badl[b0 + bi];
+                        const int cc = badl[b0 + bi];
+                        const int64_t ccol = (int64_t)h * D + cc;
                         float gsum = 0.f;
                         for (int j = 0; j <= r; ++j)
-                            gsum += j < L ? a.log_alpha[(tok0 + j) * H * D + ccol] : 0.f;
+                            gsum += j < L ? gate_log<GATE>(a.log_alpha, (tok0 + j) * H + h, cc) : 0.f;
                         gx = gsum;
                         if (r < L) {
                             qx = __bfloat162float(a.q[(tok0 + r) * H * D + ccol]);
@@ -555,7 +595,7 @@ __device__ __forceinline__ void prep_item(Worker &w, const PrepArgs &a, int slot
             }
         }
     };
-    if (n_bad) gram_readout(std::true_type{});
+    if (GATE != KDA_GATE_NONE && n_bad) gram_readout(std::true_type{});
     else gram_readout(std::false_type{});
     fence_async_smem();
     tc_fence_before();
@@ -703,11 +743,12 @@ __device__ __forceinline__ void prep_item(Worker &w, const PrepArgs &a, int slot
 }
 
 
+template <int GATE>
 __global__ void __launch_bounds__(PREP_NT, 3)
 kda_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_la, int pf_dist,
                 const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
-                const float *__restrict__ log_alpha, const float *__restrict__ beta,
+                const void *__restrict__ log_alpha, const float *__restrict__ beta,
                 unsigned char *__restrict__ ws_blobs, const int32_t *__restrict__ chunk_off,
                 const int32_t *__restrict__ cu, int64_t T, int H, int n_seqs, int nck) {
     extern __shared__ unsigned char smem_raw[];
@@ -730,7 +771,7 @@ kda_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const PrepArgs a{&tm_q, &tm_k, &tm_la, q, k, log_alpha, beta, ws_blobs, T, H};
     PrepWorker<true> w;
     w.init(true);
-    prep_item(w, a, slot, h, seq_span(cu, T, seq), n, pf, nullptr);
+    prep_item<GATE>(w, a, slot, h, seq_span(cu, T, seq), n, pf, nullptr);
     w.release(nullptr);
 }
 
@@ -1242,12 +1283,12 @@ struct FusedQueue {
     int32_t next_rest;    // the other items, claimed by prep-only CTAs
 };
 
-template <int N>
+template <int N, int GATE>
 __global__ void __launch_bounds__(FUSED_NT, 1)
 kda_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                  const __grid_constant__ CUtensorMap tm_la, const __grid_constant__ CUtensorMap tm_v,
                  const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
-                 const float *__restrict__ log_alpha, const float *__restrict__ beta,
+                 const void *__restrict__ log_alpha, const float *__restrict__ beta,
                  unsigned char *__restrict__ ws_blobs, int32_t *__restrict__ ready,
                  FusedQueue *__restrict__ queue, const float *__restrict__ S0,
                  __nv_bfloat16 *__restrict__ o, float *__restrict__ S_T, int64_t T, int H, int B,
@@ -1294,7 +1335,7 @@ kda_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 y = (int)((int64_t)(pp / H) * T + (int64_t)(pit / P) * CH);
                 return true;
             };
-            prep_item(w, pa, seq * nck + n, h, SeqSpan{(int64_t)seq * T, T}, n, pf, ready,
+            prep_item<GATE>(w, pa, seq * nck + n, h, SeqSpan{(int64_t)seq * T, T}, n, pf, ready,
                       ClaimAhead{claim_next, claim + ((j + 1) & 1), -1});
         }
         w.release(ready);
@@ -1371,7 +1412,8 @@ int prep_residency() {
     int dev = 0, n_sm = 0, per_sm = 0;
     if (cudaGetDevice(&dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kda_prep_kernel, PREP_NT, PREP_SMEM) !=
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kda_prep_kernel<KDA_GATE_CHANNEL>,
+                                                      PREP_NT, PREP_SMEM) !=
             cudaSuccess)
         return 0;
     return n_sm * per_sm;
@@ -1403,6 +1445,11 @@ struct BatchedPlan {
 // Whether the current device can run the fused grid (cooperative launch, one CTA per
 // SM). The kernel's shared-memory attribute is set here, once per device, as the check
 // needs it; the answer is cached per device.
+template <int GATE>
+bool fused_smem_attr() {
+    return cudaFuncSetAttribute(kda_fused_kernel<64, GATE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)fused_smem<64>()) == cudaSuccess;
+}
 bool fused_supported() {
     constexpr int MAX_DEVICES = 128;
     static int ok[MAX_DEVICES];  // 0: not checked, 1: yes, 2: no
@@ -1412,10 +1459,10 @@ bool fused_supported() {
         int coop = 0, per64 = 0;
         const bool yes =
             cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev) == cudaSuccess && coop &&
-            cudaFuncSetAttribute(kda_fused_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)fused_smem<64>()) == cudaSuccess &&
-            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per64, kda_fused_kernel<64>, FUSED_NT,
-                                                          fused_smem<64>()) == cudaSuccess &&
+            fused_smem_attr<KDA_GATE_CHANNEL>() && fused_smem_attr<KDA_GATE_CHANNEL_BF16>() &&
+            fused_smem_attr<KDA_GATE_HEAD>() && fused_smem_attr<KDA_GATE_NONE>() &&
+            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per64, kda_fused_kernel<64, KDA_GATE_CHANNEL>,
+                                                          FUSED_NT, fused_smem<64>()) == cudaSuccess &&
             per64 >= 1;
         ok[dev] = yes ? 1 : 2;
     }
@@ -1508,8 +1555,18 @@ int prefill_tc_launches(int B, int64_t T, int H, int n_seqs) {
     return (packed ? 1 : 0) + (n_tok > 0 && slots > 0 ? 1 : 0) + 1;
 }
 
-cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, const float *log_alpha,
-                              const float *beta, const float *S0, void *o, float *S_T, int B,
+// Tensor map of a per-channel gate (fp32 boxes of 128 channels, bf16 boxes of 64), used
+// only for L2 prefetch; the other layouts get a copy of `fallback`, which no kernel reads.
+bool make_gate_map(CUtensorMap *m, const void *la, int gate, int64_t n_tok, int H,
+                   const CUtensorMap &fallback) {
+    if (gate == KDA_GATE_CHANNEL) return make_map(m, la, false, n_tok, H);
+    if (gate == KDA_GATE_CHANNEL_BF16) return make_map(m, la, true, n_tok, H);
+    *m = fallback;
+    return true;
+}
+
+cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, const void *log_alpha,
+                              int gate, const float *beta, const float *S0, void *o, float *S_T, int B,
                               int64_t T, int H, const int32_t *cu_seqlens, int n_seqs,
                               void *workspace, cudaStream_t stream) {
     const bool packed = n_seqs > 0;
@@ -1537,7 +1594,7 @@ cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, const
             if (err != cudaSuccess) return err;
             CUtensorMap mq, mk, mla, mv;
             if (!make_map(&mq, q, true, n_tok, H) || !make_map(&mk, k, true, n_tok, H) ||
-                !make_map(&mla, log_alpha, false, n_tok, H) || !make_map(&mv, v, true, n_tok, H))
+                !make_gate_map(&mla, log_alpha, gate, n_tok, H, mq) || !make_map(&mv, v, true, n_tok, H))
                 return cudaErrorInvalidValue;
             const __nv_bfloat16 *qb = (const __nv_bfloat16 *)q, *kb = (const __nv_bfloat16 *)k;
             __nv_bfloat16 *ob = (__nv_bfloat16 *)o;
@@ -1545,26 +1602,33 @@ cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, const
             void *args[] = {&mq, &mk, &mla, &mv, &qb, &kb, (void *)&log_alpha, (void *)&beta, &blobs,
                             &ready, &queue, (void *)&S0, &ob, &S_T, &T, &H, &B, (void *)&nck,
                             &n_first, &n_chain};
-            return cudaLaunchCooperativeKernel((const void *)kda_fused_kernel<64>, dim3((unsigned)n_sm),
-                                               dim3(FUSED_NT), args, fused_smem<64>(), stream);
+            return with_gate(gate, [&](auto g) {
+                return cudaLaunchCooperativeKernel((const void *)kda_fused_kernel<64, decltype(g)::value>,
+                                                   dim3((unsigned)n_sm), dim3(FUSED_NT), args,
+                                                   fused_smem<64>(), stream);
+            });
         }
     }
     cudaError_t err;
     if (n_tok > 0 && slots > 0) {
         CUtensorMap mq, mk, mla;
         if (!make_map(&mq, q, true, n_tok, H) || !make_map(&mk, k, true, n_tok, H) ||
-            !make_map(&mla, log_alpha, false, n_tok, H))
+            !make_gate_map(&mla, log_alpha, gate, n_tok, H, mq))
             return cudaErrorInvalidValue;
-        err = cudaFuncSetAttribute(kda_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                   (int)PREP_SMEM);
-        if (err == cudaSuccess)  // three CTAs per SM need the largest shared-memory carveout
-            err = cudaFuncSetAttribute(kda_prep_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
-                                       (int)cudaSharedmemCarveoutMaxShared);
-        if (err != cudaSuccess) return err;
-        kda_prep_kernel<<<dim3((unsigned)slots, (unsigned)H), PREP_NT, PREP_SMEM, stream>>>(
-            mq, mk, mla, prep_residency(), (const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k, log_alpha, beta,
-            blobs, chunk_off, cu_seqlens, T, H, n_seqs, nck);
-        err = cudaGetLastError();
+        const int pf_dist = prep_residency();
+        err = with_gate(gate, [&](auto g) {
+            constexpr int G = decltype(g)::value;
+            cudaError_t e = cudaFuncSetAttribute(kda_prep_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 (int)PREP_SMEM);
+            if (e == cudaSuccess)  // three CTAs per SM need the largest shared-memory carveout
+                e = cudaFuncSetAttribute(kda_prep_kernel<G>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                         (int)cudaSharedmemCarveoutMaxShared);
+            if (e != cudaSuccess) return e;
+            kda_prep_kernel<G><<<dim3((unsigned)slots, (unsigned)H), PREP_NT, PREP_SMEM, stream>>>(
+                mq, mk, mla, pf_dist, (const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k, log_alpha,
+                beta, blobs, chunk_off, cu_seqlens, T, H, n_seqs, nck);
+            return cudaGetLastError();
+        });
         if (err != cudaSuccess) return err;
     }
     CUtensorMap mv;

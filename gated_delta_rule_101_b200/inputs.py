@@ -30,10 +30,11 @@ class PrefillInputs:
     q: torch.Tensor
     k: torch.Tensor
     v: torch.Tensor
-    log_alpha: torch.Tensor
+    log_alpha: torch.Tensor | None  # in the layout of `gate` (GATES)
     beta: torch.Tensor
     S0: torch.Tensor | None
     cu_seqlens: torch.Tensor | None  # int32 [n_seqs + 1] on the inputs' device, or None
+    gate: str = "channel"
 
     @property
     def n_seqs(self) -> int:
@@ -52,6 +53,20 @@ def _unit_normal_rows(shape, gen, device, dtype) -> torch.Tensor:
     return x.to(dtype)
 
 
+# Forget-gate layouts (the library's kda_gate): per key channel in fp32 or bf16, one per
+# (token, head) in fp32, or none. Values are drawn as -U(lo, hi) in fp32.
+GATES = ("channel", "channel_bf16", "head", "none")
+
+
+def _draw_gate(gate: str, lead, H: int, dk: int, la_range, gen, device):
+    lo, hi = la_range
+    if gate == "none":
+        return None
+    shape = lead + ((H,) if gate == "head" else (H, dk))
+    la = -(lo + (hi - lo) * torch.rand(shape, generator=gen, device=device, dtype=torch.float32))
+    return la.to(torch.bfloat16) if gate == "channel_bf16" else la
+
+
 def varlen_lengths(n_seqs: int, lo: int, hi: int, seed: int) -> list[int]:
     """Sequence lengths drawn uniformly from the integers [lo, hi] (CPU generator)."""
     g = _gen(seed, "cpu")
@@ -67,12 +82,13 @@ def cu_from_lengths(lengths, device="cpu") -> torch.Tensor:
 
 def prefill_inputs(*, T: int, H: int, B: int = 1, cu_seqlens=None, dtype=torch.bfloat16,
                    la_range=(0.001, 0.1), s0_std: float = 0.0, seed: int = 0,
-                   device="cpu", dk: int = DK, dv: int = DV) -> PrefillInputs:
+                   device="cpu", dk: int = DK, dv: int = DV, gate: str = "channel") -> PrefillInputs:
     """Inputs for one ``kda_chunk_fwd`` call.
 
     Without ``cu_seqlens`` the tensors are ``[B, T, H, .]``; with it (a list or
     tensor of ``n_seqs + 1`` offsets ending at ``T``) they are packed
-    ``[T, H, .]`` and ``B`` must be 1.
+    ``[T, H, .]`` and ``B`` must be 1. ``gate`` picks the layout of
+    ``log_alpha`` (one of GATES).
     """
     gen = _gen(seed, device)
     if cu_seqlens is None:
@@ -88,13 +104,12 @@ def prefill_inputs(*, T: int, H: int, B: int = 1, cu_seqlens=None, dtype=torch.b
     q = _unit_normal_rows(lead + (H, dk), gen, device, dtype)
     k = _unit_normal_rows(lead + (H, dk), gen, device, dtype)
     v = torch.randn(lead + (H, dv), generator=gen, device=device, dtype=torch.float32).to(dtype)
-    lo, hi = la_range
-    la = -(lo + (hi - lo) * torch.rand(lead + (H, dk), generator=gen, device=device, dtype=torch.float32))
+    la = _draw_gate(gate, lead, H, dk, la_range, gen, device)
     beta = torch.sigmoid(torch.randn(lead + (H,), generator=gen, device=device, dtype=torch.float32))
     S0 = None
     if s0_std > 0:
         S0 = s0_std * torch.randn((n_seqs, H, dk, dv), generator=gen, device=device, dtype=torch.float32)
-    return PrefillInputs(q, k, v, la, beta, S0, cu)
+    return PrefillInputs(q, k, v, la, beta, S0, cu, gate)
 
 
 @dataclass
@@ -102,22 +117,22 @@ class DecodeInputs:
     q: torch.Tensor          # [steps, N, H, dk]
     k: torch.Tensor          # [steps, N, H, dk]
     v: torch.Tensor          # [steps, N, H, dv]
-    log_alpha: torch.Tensor  # [steps, N, H, dk] fp32
+    log_alpha: torch.Tensor | None  # [steps, N, H, dk] fp32 (layout of `gate`)
     beta: torch.Tensor       # [steps, N, H] fp32
     S: torch.Tensor          # [N, H, dk, dv] fp32 initial state
+    gate: str = "channel"
 
 
 def decode_inputs(*, steps: int, N: int, H: int, dtype=torch.bfloat16, la_range=(0.001, 0.1),
                   s0_std: float = 0.1, seed: int = 0, device="cpu", dk: int = DK,
-                  dv: int = DV) -> DecodeInputs:
+                  dv: int = DV, gate: str = "channel") -> DecodeInputs:
     """Per-step token inputs for ``steps`` consecutive ``kda_decode_step`` calls."""
     gen = _gen(seed, device)
     lead = (steps, N)
     q = _unit_normal_rows(lead + (H, dk), gen, device, dtype)
     k = _unit_normal_rows(lead + (H, dk), gen, device, dtype)
     v = torch.randn(lead + (H, dv), generator=gen, device=device, dtype=torch.float32).to(dtype)
-    lo, hi = la_range
-    la = -(lo + (hi - lo) * torch.rand(lead + (H, dk), generator=gen, device=device, dtype=torch.float32))
+    la = _draw_gate(gate, lead, H, dk, la_range, gen, device)
     beta = torch.sigmoid(torch.randn(lead + (H,), generator=gen, device=device, dtype=torch.float32))
     S = s0_std * torch.randn((N, H, dk, dv), generator=gen, device=device, dtype=torch.float32)
-    return DecodeInputs(q, k, v, la, beta, S)
+    return DecodeInputs(q, k, v, la, beta, S, gate)

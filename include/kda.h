@@ -22,8 +22,9 @@
  *     (a cudaStream_t, NULL = the legacy default stream).
  *   - All tensors are contiguous, row-major, in the layouts given below.
  *     Token-major tensors index [token][head][channel].
- *   - q, k, v and o share one element type, `dtype` (kda_dtype). log_alpha,
- *     beta and the state are always fp32.
+ *   - q, k, v and o share one element type, `dtype` (kda_dtype). beta and
+ *     the state are always fp32; log_alpha is fp32 except in the bf16 gate
+ *     layout of the *_gated calls (kda_gate).
  *   - Preconditions that are not checked element by element: q and k rows
  *     L2-normalised per head (the layer's L2Norm, section 3), log_alpha
  *     finite and <= 0 (use a large finite negative number, not -inf, for
@@ -57,10 +58,28 @@ typedef enum kda_dtype {
     KDA_F32 = 1   /* q, k, v, o are float32 */
 } kda_dtype;
 
+/*
+ * How the forget gate alpha_t is given. KDA gives every key channel its own
+ * rate (blog.gzher.com "Kimi K3论文：Kimi Linear", section 3). The two models
+ * that section 2 of the same page builds it from are special cases of it:
+ * Gated DeltaNet has one scalar rate per head, and alpha_t times
+ * (I - beta_t k_t k_t^T) S equals (I - beta_t k_t k_t^T) Diag(alpha_t 1) S
+ * because a scalar commutes with the matrix. DeltaNet has no forget gate
+ * (alpha_t = 1).
+ * The gate is always passed as log_alpha (natural log), in one of these
+ * layouts:
+ */
+typedef enum kda_gate {
+    KDA_GATE_CHANNEL = 0,      /* fp32 [token][head][128]: one rate per key channel (KDA) */
+    KDA_GATE_CHANNEL_BF16 = 1, /* the same, bfloat16 */
+    KDA_GATE_HEAD = 2,         /* fp32 [token][head]: one rate per head (Gated DeltaNet) */
+    KDA_GATE_NONE = 3          /* no gate, alpha = 1 (DeltaNet); log_alpha is not read */
+} kda_gate;
+
 typedef enum kda_status {
     KDA_OK = 0,
     KDA_ERR_INVALID_ARG = -1, /* null pointer, bad size, bad offsets */
-    KDA_ERR_UNSUPPORTED = -2, /* C != 64 or unknown dtype */
+    KDA_ERR_UNSUPPORTED = -2, /* C != 64, unknown dtype or unknown gate layout */
     KDA_ERR_WORKSPACE = -3,   /* workspace missing or smaller than required */
     KDA_ERR_CUDA = -4,        /* a kernel launch failed */
     KDA_ERR_TIMEOUT = -5,     /* a bounded device-side wait expired */
@@ -133,6 +152,22 @@ KDA_API int kda_chunk_fwd(const void *q, const void *k, const void *v, const flo
                   size_t workspace_bytes, void *stream);
 
 /*
+ * kda_chunk_fwd with the forget gate in any kda_gate layout. All other
+ * arguments are those of kda_chunk_fwd. log_alpha points to a tensor of
+ * `gate`'s layout ([B, T, H, 128] fp32 or bf16, or [B, T, H] fp32; packed
+ * inputs drop B), finite and <= 0. For KDA_GATE_NONE it is not read and may
+ * be NULL. kda_chunk_fwd(...) is kda_chunk_fwd_gated(..., KDA_GATE_CHANNEL, ...).
+ * The gate layout changes neither the workspace size nor the kernels
+ * launched. An unknown `gate` returns KDA_ERR_UNSUPPORTED.
+ */
+KDA_API int kda_chunk_fwd_gated(const void *q, const void *k, const void *v,
+                                const void *log_alpha, int gate, const float *beta,
+                                const float *S0, void *o, float *S_T, int B, int64_t T, int H,
+                                int C, const int32_t *cu_seqlens, int n_seqs,
+                                const int32_t *cu_seqlens_host, int dtype, void *workspace,
+                                size_t workspace_bytes, void *stream);
+
+/*
  * One recurrent decode step for N sequences (eq. (1) applied to one token;
  * blog.gzher.com section 4: decode uses the recurrent kernel).
  *
@@ -144,6 +179,15 @@ KDA_API int kda_chunk_fwd(const void *q, const void *k, const void *v, const flo
  */
 KDA_API int kda_decode_step(const void *q, const void *k, const void *v, const float *log_alpha,
                     const float *beta, float *S, void *o, int N, int H, int dtype, void *stream);
+
+/*
+ * kda_decode_step with the forget gate in any kda_gate layout: log_alpha is
+ * [N, H, 128] fp32 or bf16, [N, H] fp32, or not read (KDA_GATE_NONE, may be
+ * NULL). Everything else is as for kda_decode_step.
+ */
+KDA_API int kda_decode_step_gated(const void *q, const void *k, const void *v,
+                                  const void *log_alpha, int gate, const float *beta, float *S,
+                                  void *o, int N, int H, int dtype, void *stream);
 
 /*
  * kda_chunk_fwd for callers that cannot allocate device memory. The pages

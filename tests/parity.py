@@ -36,3 +36,16 @@ def check(x, ref, kind, what):
         assert mabs <= tol["max_abs_frac"] * mx, \
             f"{what}: max-abs {mabs:.3e} > {tol['max_abs_frac']:.0e} x {mx:.3e}"
     return rel, mabs
+
+
+def per_channel_gate(log_alpha, gate, like):
+    """The forget gate in the form the oracle takes: fp32 log rates, one per key channel,
+    shaped like ``like`` (q). A head-wide rate (Gated DeltaNet) is the same rate on every
+    channel, a bf16 gate is widened exactly, and no gate (DeltaNet) is log 1 = 0."""
+    import torch
+
+    if gate == "none":
+        return torch.zeros(like.shape, dtype=torch.float32, device=like.device)
+    if gate == "head":
+        return log_alpha[..., None].expand(like.shape).float()
+    return log_alpha.float()

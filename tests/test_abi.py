@@ -113,6 +113,44 @@ def test_decode_rejects_bad_arguments(lib):
     assert call(S=ctypes.c_void_p((1 << 20) + 4)) == INVALID  # state must be 16-byte aligned
 
 
+def test_gated_entry_points_validate_the_gate(lib):
+    G = kda
+
+    def chunk(gate, la=FAKE, dtype=BF16):
+        return lib.kda_chunk_fwd_gated(FAKE, FAKE, FAKE, la, gate, FAKE, None, FAKE, None, 1, 128, 2,
+                                       64, None, 0, None, dtype, None, 0, None)
+
+    def decode(gate, la=FAKE):
+        return lib.kda_decode_step_gated(FAKE, FAKE, FAKE, la, gate, FAKE, FAKE, FAKE, 4, 2, BF16,
+                                         None)
+
+    for bad in (-1, 4, 99):
+        assert chunk(bad) == UNSUPPORTED and decode(bad) == UNSUPPORTED
+    for gate in (G.KDA_GATE_CHANNEL, G.KDA_GATE_CHANNEL_BF16, G.KDA_GATE_HEAD):
+        assert chunk(gate, la=None) == INVALID and decode(gate, la=None) == INVALID
+    # no gate: log_alpha is not needed (validation goes on to the missing workspace)
+    assert chunk(G.KDA_GATE_NONE, la=None) == WORKSPACE
+    # per-channel gates are read by TMA on the bf16 path (16-byte base); head gates are fp32
+    off8, off2 = ctypes.c_void_p((1 << 20) + 8), ctypes.c_void_p((1 << 20) + 2)
+    assert chunk(G.KDA_GATE_CHANNEL, la=off8) == INVALID
+    assert chunk(G.KDA_GATE_CHANNEL_BF16, la=off8) == INVALID
+    assert chunk(G.KDA_GATE_HEAD, la=off8) == WORKSPACE
+    assert chunk(G.KDA_GATE_HEAD, la=off2) == INVALID
+    assert decode(G.KDA_GATE_HEAD, la=off2) == INVALID
+
+
+def test_binding_infers_the_gate_layout():
+    q = torch.zeros(2, 64, 3, 128, dtype=torch.bfloat16)
+    assert kda.gate_kind(torch.zeros(2, 64, 3, 128), q) == kda.KDA_GATE_CHANNEL
+    assert kda.gate_kind(torch.zeros(2, 64, 3, 128, dtype=torch.bfloat16), q) == kda.KDA_GATE_CHANNEL_BF16
+    assert kda.gate_kind(torch.zeros(2, 64, 3), q) == kda.KDA_GATE_HEAD
+    assert kda.gate_kind(None, q) == kda.KDA_GATE_NONE
+    for bad in (torch.zeros(2, 64, 3, 1), torch.zeros(2, 64, 3, dtype=torch.bfloat16),
+                torch.zeros(2, 64, 3, 128, dtype=torch.float16)):
+        with pytest.raises(ValueError):
+            kda.gate_kind(bad, q)
+
+
 def test_binding_refuses_wrong_dtypes_before_calling():
     import torch
 

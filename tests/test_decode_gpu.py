@@ -5,7 +5,7 @@ import torch
 import gated_delta_rule_101_b200 as kda
 import oracle
 from gated_delta_rule_101_b200.inputs import decode_inputs
-from parity import check
+from parity import check, per_channel_gate
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda:0"
@@ -14,15 +14,20 @@ DEV = "cuda:0"
 def _oracle_for(inp, n_idx, h_idx):
     """Oracle over the token sequence of each sampled (sequence, head) pair."""
     outs = []
+    la_full = per_channel_gate(inp.log_alpha, inp.gate, inp.q)
     for n, h in zip(n_idx, h_idx):
         q = inp.q[:, n, h][None, :, None]  # [1, steps, 1, dk]
         k = inp.k[:, n, h][None, :, None]
         v = inp.v[:, n, h][None, :, None]
-        la = inp.log_alpha[:, n, h][None, :, None]
+        la = la_full[:, n, h][None, :, None]
         b = inp.beta[:, n, h][None, :, None]
         S0 = inp.S[n, h][None, None]
         outs.append(oracle.kda_fwd(q, k, v, la, b, S0))
     return outs
+
+
+def _gate_at(inp, t):
+    return None if inp.log_alpha is None else inp.log_alpha[t]
 
 
 def _run_decode(inp, graph: bool):
@@ -31,18 +36,18 @@ def _run_decode(inp, graph: bool):
     o = torch.empty_like(inp.v)
     if not graph:
         for t in range(steps):
-            kda.decode_step(inp.q[t], inp.k[t], inp.v[t], inp.log_alpha[t], inp.beta[t], S, out=o[t])
+            kda.decode_step(inp.q[t], inp.k[t], inp.v[t], _gate_at(inp, t), inp.beta[t], S, out=o[t])
     else:
         s = torch.cuda.Stream()
         s.wait_stream(torch.cuda.current_stream())
         with torch.cuda.stream(s):  # first call outside capture
-            kda.decode_step(inp.q[0], inp.k[0], inp.v[0], inp.log_alpha[0], inp.beta[0], S.clone(),
+            kda.decode_step(inp.q[0], inp.k[0], inp.v[0], _gate_at(inp, 0), inp.beta[0], S.clone(),
                             out=o[0])
         torch.cuda.current_stream().wait_stream(s)
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g):
             for t in range(steps):
-                kda.decode_step(inp.q[t], inp.k[t], inp.v[t], inp.log_alpha[t], inp.beta[t], S,
+                kda.decode_step(inp.q[t], inp.k[t], inp.v[t], _gate_at(inp, t), inp.beta[t], S,
                                 out=o[t])
         g.replay()
     torch.cuda.synchronize()
@@ -90,3 +95,16 @@ def test_decode_deterministic():
     o1, S1 = _run_decode(inp, graph=False)
     o2, S2 = _run_decode(inp, graph=False)
     assert torch.equal(o1, o2) and torch.equal(S1, S2)
+
+
+@pytest.mark.parametrize("gate", ["channel_bf16", "head", "none"])
+@pytest.mark.parametrize("dtype,kind", [(torch.bfloat16, "bf16"), (torch.float32, "f32")])
+def test_decode_gate_layouts(gate, dtype, kind):
+    """Gated DeltaNet (one rate per head), DeltaNet (no gate) and a bf16 gate."""
+    inp = decode_inputs(steps=24, N=2, H=3, dtype=dtype, seed=46, gate=gate, device=DEV)
+    o, S = _run_decode(inp, graph=gate == "head")
+    for n in range(2):
+        for h in range(3):
+            (ro, rs), = _oracle_for(inp, [n], [h])
+            check(o[:, n, h], ro[0, :, 0], kind, f"decode {gate} o (n={n}, h={h})")
+            check(S[n, h], rs[0, 0], kind, f"decode {gate} S (n={n}, h={h})")

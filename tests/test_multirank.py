@@ -48,7 +48,7 @@ def _worker(rank, world, port, out):
 
 def test_two_rank_max_reduce_and_distinct_batches():
     world, port = 2, _free_port()
-    with mp.Manager() as mgr:
+    with mp.get_context("spawn").Manager() as mgr:
         out = mgr.dict()
         mp.spawn(_worker, args=(world, port, out), nprocs=world, join=True)
         res = dict(out)

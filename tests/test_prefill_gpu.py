@@ -6,7 +6,7 @@ import torch
 import gated_delta_rule_101_b200 as kda
 import oracle
 from gated_delta_rule_101_b200.inputs import cu_from_lengths, prefill_inputs, varlen_lengths
-from parity import check
+from parity import check, per_channel_gate
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda:0"
@@ -21,7 +21,8 @@ def run(inp, **kw):
 
 
 def ref(inp):
-    return oracle.kda_fwd(inp.q, inp.k, inp.v, inp.log_alpha, inp.beta, inp.S0,
+    la = per_channel_gate(inp.log_alpha, inp.gate, inp.q)
+    return oracle.kda_fwd(inp.q, inp.k, inp.v, la, inp.beta, inp.S0,
                           cu_seqlens=None if inp.cu_seqlens is None else inp.cu_seqlens.cpu())
 
 
@@ -152,6 +153,7 @@ def _sample_ref(inp, seqs, heads, cols):
     """Oracle on sampled (sequence, head) pairs and value columns, whole sequences."""
     out = []
     cu = None if inp.cu_seqlens is None else inp.cu_seqlens.cpu().tolist()
+    la_full = per_channel_gate(inp.log_alpha, inp.gate, inp.q)
     for s, h in zip(seqs, heads):
         if cu is None:
             sl = (slice(s, s + 1), slice(None))
@@ -159,7 +161,7 @@ def _sample_ref(inp, seqs, heads, cols):
         else:
             a, z = cu[s], cu[s + 1]
             pick = lambda x: x[a:z, h:h + 1][None]
-        q, k, la = pick(inp.q), pick(inp.k), pick(inp.log_alpha)
+        q, k, la = pick(inp.q), pick(inp.k), pick(la_full)
         v = pick(inp.v)[..., cols]
         b = pick(inp.beta[..., None])[..., 0]
         S0 = None if inp.S0 is None else inp.S0[s, h][:, cols][None, None]
@@ -292,6 +294,67 @@ def test_segment_scan_carries_state_across_calls():
         o[:, a:a + Tc] = oc
     torch.cuda.synchronize()
     _check_sampled(inp, o, S, [0, 0], [0, 1], list(range(128)), "bf16", "segment scan, two calls")
+
+
+# ---- gate layouts: Gated DeltaNet (one rate per head), DeltaNet (no gate), bf16 gate
+LAYOUTS = ["channel_bf16", "head", "none"]
+
+
+@pytest.mark.parametrize("gate", LAYOUTS)
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_gate_layouts_against_the_oracle(gate, dtype):
+    inp = prefill_inputs(B=2, T=300, H=3, dtype=dtype, s0_std=0.1, seed=41, gate=gate, device=DEV)
+    o, st = run(inp)
+    ro, rs = ref(inp)
+    check(o, ro, KIND[dtype], f"{gate} o")
+    check(st, rs, KIND[dtype], f"{gate} S_T")
+
+
+@pytest.mark.parametrize("gate", ["channel_bf16", "head"])
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_gate_layouts_strong_decay(gate, dtype):
+    """Chunk log-decay beyond the factorised range in every channel (head gate) or in
+    many (bf16 gate): the exact pairwise path reads the gate in its own layout."""
+    inp = prefill_inputs(B=1, T=200, H=2, dtype=dtype, la_range=(0.5, 3.0), s0_std=0.1,
+                         seed=42, gate=gate, device=DEV)
+    o, st = run(inp)
+    ro, rs = ref(inp)
+    check(o, ro, KIND[dtype], f"{gate} strong decay o")
+    check(st, rs, KIND[dtype], f"{gate} strong decay S_T")
+
+
+@pytest.mark.parametrize("gate", LAYOUTS)
+@pytest.mark.parametrize("path", ["fused_grid", "segment_scan"])
+def test_gate_layouts_on_each_bf16_plan(gate, path):
+    B, T, H, launches = PATHS[path]
+    assert kda.chunk_fwd_launches(B, T, H) == launches
+    inp = prefill_inputs(B=B, T=T, H=H, dtype=torch.bfloat16, s0_std=0.1, seed=43, gate=gate,
+                         device=DEV)
+    o, st = run(inp)
+    assert torch.isfinite(o.float()).all() and torch.isfinite(st).all()
+    _check_sampled(inp, o, st, [0, B - 1], [0, H - 1], list(range(128)), "bf16", f"{path} {gate}")
+
+
+@pytest.mark.parametrize("gate", ["channel_bf16", "head"])
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_gate_layout_equals_the_widened_channel_gate(gate, dtype):
+    """A head-wide or bf16 gate gives bit-for-bit the result of the same gate widened to
+    fp32 per channel: the layouts differ only in how the rates are read."""
+    inp = prefill_inputs(B=2, T=200, H=3, dtype=dtype, s0_std=0.1, seed=44, gate=gate, device=DEV)
+    o1, s1 = run(inp)
+    wide = per_channel_gate(inp.log_alpha, gate, inp.q).contiguous()
+    o2, s2 = kda.chunk_fwd(inp.q, inp.k, inp.v, wide, inp.beta, inp.S0)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(s1, s2)
+
+
+def test_gate_layout_none_needs_no_tensor_and_is_checked():
+    """No gate: log_alpha may be None; a gate tensor of another shape is refused."""
+    inp = prefill_inputs(B=1, T=70, H=2, dtype=torch.bfloat16, seed=45, gate="head", device=DEV)
+    with pytest.raises(ValueError):
+        kda.chunk_fwd(inp.q, inp.k, inp.v, inp.log_alpha[..., :1], inp.beta)
+    assert kda.gate_kind(None, inp.q) == kda.KDA_GATE_NONE
+    assert kda.gate_kind(inp.log_alpha, inp.q) == kda.KDA_GATE_HEAD
 
 
 def test_no_bounded_wait_timed_out():
