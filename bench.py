@@ -502,9 +502,10 @@ def run_kda(args, rank, world, local_rank):
         del graph, dinp, S, od
 
     # ---------------- the other prefill workloads (reported beside the step, not the step)
-    extra = {} if args.no_extra else {
-        **other_prefill_workloads(kda, dev, stream, flush, pk, world, rank),
-        **gate_layout_workloads(kda, dev, stream, flush, pk, world, rank)}
+    extra = {}
+    if not args.no_extra:  # the gate layouts first, next to the step they vary
+        extra.update(gate_layout_workloads(kda, dev, stream, flush, pk, world, rank))
+        extra.update(other_prefill_workloads(kda, dev, stream, flush, pk, world, rank))
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

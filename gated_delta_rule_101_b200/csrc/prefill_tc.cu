@@ -40,6 +40,8 @@
 
 #include <type_traits>
 
+#include <utility>
+
 #include "kda_internal.cuh"
 #include "tc_ptx.cuh"
 
@@ -752,6 +754,9 @@ kda_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 unsigned char *__restrict__ ws_blobs, const int32_t *__restrict__ chunk_off,
                 const int32_t *__restrict__ cu, int64_t T, int H, int n_seqs, int nck) {
     extern __shared__ unsigned char smem_raw[];
+    // The chain kernel after this one may start its CTAs (they wait for this grid to
+    // complete before reading a blob): they then take SMs as this grid's last CTAs leave.
+    griddep_launch_dependents();
     const int slot = blockIdx.x, h = blockIdx.y;
     int seq, n;
     if (!resolve_slot(slot, chunk_off, n_seqs, nck, seq, n)) return;
@@ -811,6 +816,9 @@ struct ChainArgs {
     int H;
     int nck;
     const int32_t *ready;  // non-null: wait for each blob's ready flag before reading it
+    // Launched as a dependent of the prep kernel (which may still run): everything up
+    // to the first blob load only touches the call's inputs, then griddep_wait.
+    bool wait_prior = false;
 };
 
 // The part of one (sequence, head, slice) recurrence a chain task runs: chunks [c0, c1)
@@ -934,6 +942,10 @@ __device__ __forceinline__ void chain_task(unsigned char *sm, const int tid, con
     named_bar_sync(BAR_CHAIN, bar_chain_count);
     tc_fence_after();
     const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(tmem_slot);
+    if (a.wait_prior) {  // the blobs exist once the prep grid has completed
+        griddep_wait();
+        fence_proxy_async_global();
+    }
     const uint32_t d3 = tmem + 2 * N;  // D1 buffers at columns 0 and N
     const uint32_t du = tmem + 3 * N;  // U = T Diag(beta) V (rows 64..127)
     const uint32_t sm_base = smem_u32(sm);
@@ -1110,9 +1122,9 @@ kda_chain_kernel(const __grid_constant__ CUtensorMap tm_v,
                  const unsigned char *__restrict__ ws_blobs, const int32_t *__restrict__ chunk_off,
                  const float *__restrict__ S0, __nv_bfloat16 *__restrict__ o,
                  float *__restrict__ S_T, const int32_t *__restrict__ cu, int64_t T, int H,
-                 int nck) {
+                 int nck, int wait_prior) {
     extern __shared__ unsigned char smem_raw[];
-    const ChainArgs a{&tm_v, ws_blobs, chunk_off, S0, o, S_T, cu, T, H, nck, nullptr};
+    const ChainArgs a{&tm_v, ws_blobs, chunk_off, S0, o, S_T, cu, T, H, nck, nullptr, wait_prior != 0};
     chain_task<N>(aligned_smem(smem_raw), threadIdx.x, a, blockIdx.x, blockIdx.y, blockIdx.z * N,
                   full_window(a, blockIdx.x, blockIdx.y));
 }
@@ -1152,7 +1164,8 @@ kda_seg_pass_kernel(const __grid_constant__ CUtensorMap tm_v,
     const int pair = blockIdx.x / SLICES, j0 = (blockIdx.x % SLICES) * N;
     const int seq = pair / H, h = pair % H;
     const int64_t off = (int64_t)pair * (D * D);
-    const ChainArgs a{&tm_v, ws_blobs, nullptr, S0, o, S_T, nullptr, T, H, nck, nullptr};
+    // pass 1 follows the prep kernel as its dependent; pass 2 follows the combine
+    const ChainArgs a{&tm_v, ws_blobs, nullptr, S0, o, S_T, nullptr, T, H, nck, nullptr, pass == 1};
     const int L = sg.seg_len;
     ChainWindow win;
     if (pass == 1) {
@@ -1393,17 +1406,36 @@ bool make_map(CUtensorMap *m, const void *ptr, bool bf16, int64_t n_tok, int H) 
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Launches `kernel`; with `after_prep` as a programmatic dependent of the prep kernel just
+// launched on the stream, so that its CTAs may start while that kernel's last CTAs run.
+template <class... KArgs, class... Args>
+cudaError_t launch_maybe_dependent(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                                   cudaStream_t stream, bool after_prep, Args &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = after_prep ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 template <int N>
 cudaError_t launch_chain(const CUtensorMap &mv, const unsigned char *blobs, const int32_t *chunk_off,
                          const float *S0, void *o, float *S_T, const int32_t *cu, int64_t T, int H,
-                         int nck, int nseq, cudaStream_t stream) {
+                         int nck, int nseq, bool after_prep, cudaStream_t stream) {
     using Lay = ChainLayout<N>;
     cudaError_t err = cudaFuncSetAttribute(kda_chain_kernel<N>,
                                            cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Lay::BYTES);
     if (err != cudaSuccess) return err;
-    kda_chain_kernel<N><<<dim3((unsigned)nseq, (unsigned)H, D / N), CHAIN_NT, Lay::BYTES, stream>>>(
-        mv, blobs, chunk_off, S0, (__nv_bfloat16 *)o, S_T, cu, T, H, nck);
-    return cudaGetLastError();
+    err = launch_maybe_dependent(kda_chain_kernel<N>, dim3((unsigned)nseq, (unsigned)H, D / N),
+                                 dim3(CHAIN_NT), Lay::BYTES, stream, after_prep, mv, blobs, chunk_off,
+                                 S0, (__nv_bfloat16 *)o, S_T, cu, T, H, nck, after_prep ? 1 : 0);
+    return err != cudaSuccess ? err : cudaGetLastError();
 }
 
 // CTAs of the prep kernel resident on the whole GPU at once (its L2 prefetch
@@ -1610,7 +1642,8 @@ cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, const
         }
     }
     cudaError_t err;
-    if (n_tok > 0 && slots > 0) {
+    const bool prep_launched = n_tok > 0 && slots > 0;
+    if (prep_launched) {
         CUtensorMap mq, mk, mla;
         if (!make_map(&mq, q, true, n_tok, H) || !make_map(&mk, k, true, n_tok, H) ||
             !make_gate_map(&mla, log_alpha, gate, n_tok, H, mq))
@@ -1643,8 +1676,10 @@ cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, const
                                    (int)Lay::BYTES);
         if (err != cudaSuccess) return err;
         __nv_bfloat16 *ob = (__nv_bfloat16 *)o;
-        kda_seg_pass_kernel<64><<<dim3((unsigned)(2 * P), (unsigned)(2 * plan.n_seg - 3)), CHAIN_NT,
-                                  Lay::BYTES, stream>>>(mv, blobs, S0, ob, S_T, T, H, nck, sg, 1);
+        err = launch_maybe_dependent(kda_seg_pass_kernel<64>, dim3((unsigned)(2 * P), (unsigned)(2 * plan.n_seg - 3)),
+                                     dim3(CHAIN_NT), Lay::BYTES, stream, prep_launched, mv, blobs, S0, ob,
+                                     S_T, T, H, nck, sg, 1);
+        if (err != cudaSuccess) return err;
         err = cudaFuncSetAttribute(kda_seg_combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                    (int)SEG_COMBINE_SMEM);
         if (err != cudaSuccess) return err;
@@ -1655,8 +1690,11 @@ cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, const
     }
     // 128-column slices (one CTA per sequence-head) when there are enough pairs to fill
     // the GPU; otherwise 64-column slices for twice the parallelism.
-    if ((int64_t)nseq * H >= n_sm) return launch_chain<128>(mv, blobs, chunk_off, S0, o, S_T, cu_seqlens, T, H, nck, nseq, stream);
-    return launch_chain<64>(mv, blobs, chunk_off, S0, o, S_T, cu_seqlens, T, H, nck, nseq, stream);
+    if ((int64_t)nseq * H >= n_sm)
+        return launch_chain<128>(mv, blobs, chunk_off, S0, o, S_T, cu_seqlens, T, H, nck, nseq,
+                                 prep_launched, stream);
+    return launch_chain<64>(mv, blobs, chunk_off, S0, o, S_T, cu_seqlens, T, H, nck, nseq,
+                            prep_launched, stream);
 }
 
 int read_device_status(int *status) {

@@ -72,6 +72,17 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, bool &
     return false;
 }
 
+// ------------------------------------------------------------------ dependent launch
+// A kernel launched with programmatic stream serialization may start while the kernel
+// before it on the stream still runs, once every CTA of that one has called
+// griddep_launch_dependents (or exited). It must call griddep_wait, which returns when
+// the earlier kernel has completed and its writes are visible, before reading them.
+// Both are no-ops for kernels launched the ordinary way.
+__device__ __forceinline__ void griddep_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // ------------------------------------------------------------------ cross-CTA flags
 // Between CTAs of one cooperative grid (all resident at once): a producer publishes
 // data it wrote to global memory with bulk copies by waiting for the copies to

@@ -296,6 +296,34 @@ def test_segment_scan_carries_state_across_calls():
     _check_sampled(inp, o, S, [0, 0], [0, 1], list(range(128)), "bf16", "segment scan, two calls")
 
 
+@pytest.mark.parametrize("path", ["prep_then_chain", "segment_scan"])
+def test_prefill_captured_in_a_cuda_graph(path):
+    """A call captured in a CUDA graph replays to the eager result bit for bit; the
+    chain (or the segment scan's first pass) is launched as a dependent of the prep."""
+    B, T, H, launches = PATHS[path]
+    assert kda.chunk_fwd_launches(B, T, H) == launches
+    inp = prefill_inputs(B=B, T=T, H=H, dtype=torch.bfloat16, s0_std=0.1, seed=47, device=DEV)
+    o_eager, s_eager = run(inp)
+    ws = torch.empty(kda.workspace_size(B, T, H), dtype=torch.uint8, device=DEV)
+    o, st = torch.empty_like(inp.v), torch.empty_like(inp.S0)
+    call = lambda: kda.chunk_fwd(inp.q, inp.k, inp.v, inp.log_alpha, inp.beta, inp.S0, out=o,
+                                 state_out=st, workspace=ws)
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        call()
+    torch.cuda.current_stream().wait_stream(side)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        call()
+    o.zero_()
+    st.zero_()
+    graph.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(o, o_eager) and torch.equal(st, s_eager)
+    del graph
+
+
 # ---- gate layouts: Gated DeltaNet (one rate per head), DeltaNet (no gate), bf16 gate
 LAYOUTS = ["channel_bf16", "head", "none"]
 
