@@ -296,6 +296,31 @@ def test_segment_scan_carries_state_across_calls():
     _check_sampled(inp, o, S, [0, 0], [0, 1], list(range(128)), "bf16", "segment scan, two calls")
 
 
+def test_wide_chain_all_outputs():
+    """Enough sequence-heads to fill the GPU: one 128-column chain CTA per sequence-head.
+    Ragged last chunk, carried state, every output."""
+    assert kda.chunk_fwd_launches(2, 200, 80) == 2
+    inp = prefill_inputs(B=2, T=200, H=80, dtype=torch.bfloat16, s0_std=0.1, seed=48, device=DEV)
+    o, st = run(inp)
+    ro, rs = ref(inp)
+    check(o, ro, "bf16", "wide chain o")
+    check(st, rs, "bf16", "wide chain S_T")
+
+
+def test_wide_chain_packed_with_empty_sequences():
+    lengths = [0, 130, 64, 1, 257, 0, 65, 190]
+    cu = cu_from_lengths(lengths)
+    inp = prefill_inputs(T=int(cu[-1]), H=40, cu_seqlens=cu, dtype=torch.bfloat16, s0_std=0.1,
+                         seed=49, gate="head", device=DEV)
+    o, st = run(inp, cu_seqlens_host=cu)
+    ro, rs = ref(inp)
+    check(o, ro, "bf16", "wide chain packed o")
+    check(st, rs, "bf16", "wide chain packed S_T")
+    for i, n in enumerate(lengths):
+        if n == 0:
+            assert torch.equal(st[i], inp.S0[i])
+
+
 @pytest.mark.parametrize("path", ["prep_then_chain", "segment_scan"])
 def test_prefill_captured_in_a_cuda_graph(path):
     """A call captured in a CUDA graph replays to the eager result bit for bit; the
