@@ -138,8 +138,8 @@ class ClockSampler:
 # from; otherwise the roofline's traffic is null.
 TRAFFIC_SOURCES = {"prefill": ("prefill_tc.cu", "tc_ptx.cuh", "kda_internal.cuh"),
                    "decode": ("decode.cu", "kda_internal.cuh")}
-TRAFFIC = {"prefill": {"source_hash": "427a56f8d9b960cc",  # prep + chain
-                       "bytes": 270915328 + 215513088 + 341882624 + 53068544},
+TRAFFIC = {"prefill": {"source_hash": "74907cbf3b761b00",  # prep + chain
+                       "bytes": 270917888 + 215580928 + 341895168 + 52601856},
            "decode": {"source_hash": "5e83d1dd83fc2ca5", "bytes": 547408640 + 479616512}}
 
 
