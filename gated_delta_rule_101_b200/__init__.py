@@ -171,24 +171,22 @@ def chunk_fwd_launches(B: int, T: int, H: int, n_seqs: int = 0, dtype=torch.bflo
     return int(out.value)
 
 
-def chunk_fwd(q, k, v, log_alpha, beta, S0=None, *, cu_seqlens=None, cu_seqlens_host=None,
-              out=None, final_state=True, state_out=None, workspace=None, stream=None, C=CHUNK):
-    """KDA prefill through ``kda_chunk_fwd``; returns ``(o, S_T)`` (S_T None if not requested).
-
-    ``q, k, v``: ``[B, T, H, 128]`` (or packed ``[T, H, 128]`` with
-    ``cu_seqlens``, an int32 device tensor of ``n_seqs + 1`` offsets).
-    ``log_alpha``: like ``q`` (fp32 or bf16), ``[B, T, H]`` fp32, or None (see
-    ``gate_kind``). ``beta``: ``[B, T, H]``. ``S0``: fp32 ``[n_seqs, H, 128, 128]`` or None.
-    ``state_out`` may be ``S0`` itself for in-place carry.
-    """
+def _prefill_args(q, k, v, log_alpha, beta, S0, cu_seqlens, out, state_out):
+    """Checks the prefill tensors (dtypes, devices, contiguity, shapes) before any pointer
+    reaches the library, which trusts the sizes it is given. Returns
+    ``(B, T, H, n_seqs, gate, state_shape)``."""
     dev = q.device
-    code = _dtype_code(q)
+    _dtype_code(q)
     packed = cu_seqlens is not None
+    if q.dim() != (3 if packed else 4):
+        raise ValueError(f"q must be {'[T, H, 128]' if packed else '[B, T, H, 128]'}, got {tuple(q.shape)}")
     if packed:
         T, H, dk = q.shape
         B = 1
         n_seqs = cu_seqlens.numel() - 1
         _need(cu_seqlens, "cu_seqlens", torch.int32, dev)
+        if cu_seqlens.dim() != 1 or n_seqs < 1:
+            raise ValueError("cu_seqlens must be 1-D with n_seqs + 1 >= 2 offsets")
     else:
         B, T, H, dk = q.shape
         n_seqs = 0
@@ -203,20 +201,37 @@ def chunk_fwd(q, k, v, log_alpha, beta, S0=None, *, cu_seqlens=None, cu_seqlens_
     _need(beta, "beta", torch.float32, dev)
     if beta.shape != q.shape[:-1]:
         raise ValueError("beta must be q.shape[:-1]")
-    nseq = n_seqs if packed else B
-    sshape = (nseq, H, HEAD_DIM, HEAD_DIM)
-    if S0 is not None:
-        _need(S0, "S0", torch.float32, dev)
-        if tuple(S0.shape) != sshape:
-            raise ValueError(f"S0 must be {sshape}")
+    sshape = (n_seqs if packed else B, H, HEAD_DIM, HEAD_DIM)
+    for name, t in (("S0", S0), ("state_out", state_out)):
+        if t is not None:
+            _need(t, name, torch.float32, dev)
+            if tuple(t.shape) != sshape:
+                raise ValueError(f"{name} must be {sshape}, got {tuple(t.shape)}")
+    if out is not None:
+        _need(out, "out", q.dtype, dev)
+        if out.shape != q.shape:
+            raise ValueError(f"out shape {tuple(out.shape)} != q shape {tuple(q.shape)}")
+    return B, T, H, n_seqs, gate, sshape
+
+
+def chunk_fwd(q, k, v, log_alpha, beta, S0=None, *, cu_seqlens=None, cu_seqlens_host=None,
+              out=None, final_state=True, state_out=None, workspace=None, stream=None, C=CHUNK):
+    """KDA prefill through ``kda_chunk_fwd``; returns ``(o, S_T)`` (S_T None if not requested).
+
+    ``q, k, v``: ``[B, T, H, 128]`` (or packed ``[T, H, 128]`` with
+    ``cu_seqlens``, an int32 device tensor of ``n_seqs + 1`` offsets).
+    ``log_alpha``: like ``q`` (fp32 or bf16), ``[B, T, H]`` fp32, or None (see
+    ``gate_kind``). ``beta``: ``[B, T, H]``. ``S0``: fp32 ``[n_seqs, H, 128, 128]`` or None.
+    ``state_out`` may be ``S0`` itself for in-place carry.
+    """
+    dev = q.device
+    code = _dtype_code(q)
+    B, T, H, n_seqs, gate, sshape = _prefill_args(q, k, v, log_alpha, beta, S0, cu_seqlens, out,
+                                                  state_out)
     if out is None:
         out = torch.empty_like(v)
-    _need(out, "out", q.dtype, dev)
-    S_T = None
-    if state_out is not None:
-        _need(state_out, "state_out", torch.float32, dev)
-        S_T = state_out
-    elif final_state:
+    S_T = state_out
+    if S_T is None and final_state:
         S_T = torch.empty(sshape, dtype=torch.float32, device=dev)
     host_cu = None
     if cu_seqlens_host is not None:
@@ -245,19 +260,28 @@ def decode_step(q, k, v, log_alpha, beta, S, *, out=None, stream=None):
     """
     dev = q.device
     code = _dtype_code(q)
+    if q.dim() != 3:
+        raise ValueError(f"q must be [N, H, 128], got {tuple(q.shape)}")
     N, H, dk = q.shape
     if dk != HEAD_DIM:
         raise ValueError(f"head dim must be {HEAD_DIM}, got {dk}")
     for name, t in (("q", q), ("k", k), ("v", v)):
         _need(t, name, q.dtype, dev)
+        if t.shape != q.shape:
+            raise ValueError(f"{name} shape {tuple(t.shape)} != q shape {tuple(q.shape)}")
     gate = gate_kind(log_alpha, q)
     _need_gate(log_alpha, gate, dev)
     _need(beta, "beta", torch.float32, dev)
+    if beta.shape != q.shape[:-1]:
+        raise ValueError("beta must be [N, H]")
     _need(S, "S", torch.float32, dev)
     if tuple(S.shape) != (N, H, HEAD_DIM, HEAD_DIM):
         raise ValueError("S must be [N, H, 128, 128]")
     if out is None:
         out = torch.empty_like(v)
+    _need(out, "out", q.dtype, dev)
+    if out.shape != q.shape:
+        raise ValueError(f"out shape {tuple(out.shape)} != q shape {tuple(q.shape)}")
     tail = (_ptr(beta), _ptr(S), _ptr(out), N, H, code, _stream_handle(stream, dev))
     if gate == KDA_GATE_CHANNEL:
         st, where = lib().kda_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), *tail), "kda_decode_step"
@@ -281,13 +305,11 @@ def chunk_fwd_noalloc(q, k, v, log_alpha, beta, S0=None, *, out, state_out=None,
     """
     dev = q.device
     code = _dtype_code(q)
-    packed = cu_seqlens is not None
-    if packed:
-        T, H, _ = q.shape
-        B, n_seqs = 1, cu_seqlens.numel() - 1
-    else:
-        B, T, H, _ = q.shape
-        n_seqs = 0
+    if out is None:
+        raise ValueError("chunk_fwd_noalloc writes into the caller's `out`")
+    B, T, H, n_seqs, gate, _ = _prefill_args(q, k, v, log_alpha, beta, S0, cu_seqlens, out, state_out)
+    if gate != KDA_GATE_CHANNEL:
+        raise ValueError("kda_chunk_fwd_noalloc takes the per-channel fp32 gate only")
     host_cu = None
     if cu_seqlens_host is not None:
         host_cu = torch.as_tensor(cu_seqlens_host, dtype=torch.int32).contiguous().cpu()
