@@ -539,9 +539,9 @@ def main():
     ap.add_argument("--no-e2e", action="store_true",
                     help="skip the host-buffer end-to-end leg (for short profiling runs)")
     ap.add_argument("--traffic", type=float, default=None,
-                    help="ncu dram bytes per prefill launch, if captured for this build")
+                    help="ncu dram bytes per prefill launch, if captured for the current sources")
     ap.add_argument("--decode-traffic", type=float, default=None,
-                    help="ncu dram bytes per decode launch, if captured for this build")
+                    help="ncu dram bytes per decode launch, if captured for the current sources")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

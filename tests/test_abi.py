@@ -78,7 +78,7 @@ def test_chunk_fwd_rejects_short_workspace(lib):
     need = ctypes.c_size_t(0)
     assert lib.kda_chunk_fwd_workspace_size(4, 4096, 16, 64, 0, BF16, ctypes.byref(need)) == 0
     if need.value == 0:
-        pytest.skip("this build needs no workspace for bf16 prefill")
+        pytest.skip("the library needs no workspace for bf16 prefill")
     assert _chunk(lib, B=4, T=4096, H=16, ws=FAKE, ws_bytes=need.value - 1) == WORKSPACE
     assert _chunk(lib, B=4, T=4096, H=16, ws=None, ws_bytes=need.value) == WORKSPACE
 
