@@ -19,7 +19,11 @@
  * Conventions shared by every call
  *   - Every pointer is DEVICE memory owned by the caller. The library never
  *     allocates, frees or synchronises; calls are asynchronous on `stream`
- *     (a cudaStream_t, NULL = the legacy default stream).
+ *     (a cudaStream_t, NULL = the legacy default stream) and may be captured
+ *     in a CUDA graph (except the first kda_chunk_fwd_noalloc call on a GPU).
+ *     Within a prefill call, later kernels may start while earlier ones finish
+ *     (programmatic dependent launch); they wait for the earlier results on
+ *     the device, so callers see ordinary stream order.
  *   - All tensors are contiguous, row-major, in the layouts given below.
  *     Token-major tensors index [token][head][channel].
  *   - q, k, v and o share one element type, `dtype` (kda_dtype). beta and
