@@ -14,7 +14,8 @@ runs its own batch; the only collectives are the barrier and the max-reduce
 of the timings).
 
 ``--impl reference`` times the fp64 CPU oracle (the slow, obviously correct
-definition of the recurrence) on a bounded sample of the same workload.
+definition of the recurrence) on the host cores, the whole prefill workload per
+step (rank 0 only under torchrun).
 """
 from __future__ import annotations
 
@@ -150,9 +151,10 @@ def clock_rejected(clk: dict) -> bool:
 # from; otherwise the roofline's traffic is null.
 TRAFFIC_SOURCES = {"prefill": ("prefill_tc.cu", "tc_ptx.cuh", "kda_internal.cuh"),
                    "decode": ("decode.cu", "kda_internal.cuh")}
-TRAFFIC = {"prefill": {"source_hash": "74907cbf3b761b00",  # prep + chain
+TRAFFIC = {"prefill": {"source_hash": "74907cbf3b761b00", "shape": (4, 4096, 16),  # prep + chain
                        "bytes": 270917888 + 215580928 + 341895168 + 52601856},
-           "decode": {"source_hash": "5e83d1dd83fc2ca5", "bytes": 547408640 + 479616512}}
+           "decode": {"source_hash": "5e83d1dd83fc2ca5", "shape": (256, 32),
+                      "bytes": 547408640 + 479616512}}
 
 
 def source_hash(kind: str) -> str:
@@ -167,11 +169,13 @@ def source_hash(kind: str) -> str:
     return h.hexdigest()[:16]
 
 
-def traffic(kind: str, override):
+def traffic(kind: str, override, shape):
+    """DRAM bytes per launch: the override, else the committed capture if it was taken
+    from the current sources at this shape, else None."""
     if override is not None:
         return override
     t = TRAFFIC[kind]
-    return t["bytes"] if t["source_hash"] == source_hash(kind) else None
+    return t["bytes"] if t["source_hash"] == source_hash(kind) and tuple(shape) == t["shape"] else None
 
 
 # ------------------------------------------------------------------ helpers
@@ -444,7 +448,7 @@ def run_kda(args, rank, world, local_rank):
     pages_flops = PAGES_FLOPS_PER_TOKEN_HEAD * B * T * H
     tflops = pages_flops / avg_kernel_s / 1e12
     roofline = {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
-                "frac": achieved / pk["hbm_gbs"], "traffic": traffic("prefill", args.traffic),
+                "frac": achieved / pk["hbm_gbs"], "traffic": traffic("prefill", args.traffic, (B, T, H)),
                 "peak_source": pk_kind,
                 "kernel": "kda_chunk_fwd (one call, timed as a whole): "
                           + {1: "kda_fused_kernel", 2: "kda_prep_kernel + kda_chain_kernel",
@@ -516,7 +520,7 @@ def run_kda(args, rank, world, local_rank):
                                          "steps in one CUDA graph", "l2": "state 512 MiB > L2"},
                   "roofline": {"bound": "hbm", "achieved": d_ach, "peak": pk["hbm_gbs"],
                                "unit": "GB/s", "frac": d_ach / pk["hbm_gbs"],
-                               "traffic": traffic("decode", args.decode_traffic), "peak_source": pk_kind,
+                               "traffic": traffic("decode", args.decode_traffic, (N, Hd)), "peak_source": pk_kind,
                                "kernel": "kda_decode_step", "alg_bytes_per_launch": d_bytes},
                   "gpu_launches": nsteps * len(d_times), "clocks": dclk}
         del graph, dinp, S, od

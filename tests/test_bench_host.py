@@ -16,8 +16,11 @@ def test_clock_record_rejection():
                                      "reasons": ["clock sampling unavailable"]})
 
 
-def test_traffic_is_reported_only_for_the_captured_sources():
+def test_traffic_is_reported_only_for_the_captured_sources_and_shape():
     for kind in ("prefill", "decode"):
         t = bench.TRAFFIC[kind]
-        assert bench.traffic(kind, None) == (t["bytes"] if t["source_hash"] == bench.source_hash(kind) else None)
-    assert bench.traffic("prefill", 123) == 123  # an explicit capture overrides
+        same = t["source_hash"] == bench.source_hash(kind)
+        assert bench.traffic(kind, None, t["shape"]) == (t["bytes"] if same else None)
+        other = tuple(x + 1 for x in t["shape"])
+        assert bench.traffic(kind, None, other) is None
+    assert bench.traffic("prefill", 123, (1, 1, 1)) == 123  # an explicit capture overrides
