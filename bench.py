@@ -192,16 +192,19 @@ def max_over_ranks(x: float, world: int, device) -> float:
     return float(t.item())
 
 
-def time_steps(fn, steps, warmup, stream, flush=None):
+def time_steps(fn, steps, warmup, stream, flush=None, name="kda"):
     """Runs fn warmup times, then times each of `steps` calls with CUDA events
-    on `stream` (L2 flushed before each call, outside the events). Returns ms list."""
-    for _ in range(warmup):
-        fn()
-    torch.cuda.synchronize()
+    on `stream` (L2 flushed before each call, outside the events). Returns ms list.
+    The warm-up and the timed calls sit in NVTX ranges `name`/warmup and `name`/timed
+    (for `ncu --nvtx --nvtx-include`)."""
+    with torch.cuda.nvtx.range(f"{name}/warmup"):
+        for _ in range(warmup):
+            fn()
+        torch.cuda.synchronize()
     times = []
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
            for _ in range(steps)]
-    with torch.cuda.stream(stream):
+    with torch.cuda.nvtx.range(f"{name}/timed"), torch.cuda.stream(stream):
         for a, b in evs:
             if flush is not None:
                 flush()
@@ -305,7 +308,7 @@ def other_prefill_workloads(kda, dev, stream, flush, pk, world, rank):
         kda.chunk_fwd(inp.q, inp.k, inp.v, inp.log_alpha, inp.beta, None, cu_seqlens=inp.cu_seqlens,
                       out=o, state_out=S_T, workspace=ws, stream=stream)
 
-    times = time_steps(call, 3, 3, stream, flush)
+    times = time_steps(call, 3, 3, stream, flush, name="kda.varlen")
     ms = max_over_ranks(sum(times), world, dev) / len(times)
     alg = PREFILL_BYTES_PER_TOKEN_HEAD * T * H + 2 * STATE_BYTES * len(lengths) * H
     out["varlen"] = {"value": T * world / (ms * 1e-3), "unit": "tokens/s", "ms_per_call": ms,
@@ -336,7 +339,7 @@ def other_prefill_workloads(kda, dev, stream, flush, pk, world, rank):
             kda.chunk_fwd(x.q, x.k, x.v, x.log_alpha, x.beta, S, out=o, state_out=S, workspace=ws,
                           stream=stream)
 
-    times = time_steps(sequence, 2, 3, stream)
+    times = time_steps(sequence, 2, 3, stream, name="kda.long_context")
     ms = max_over_ranks(sum(times), world, dev) / len(times)
     alg = (PREFILL_BYTES_PER_TOKEN_HEAD * Tc * H + 2 * STATE_BYTES * H) * calls
     out["long_context"] = {"value": Tc * calls * world / (ms * 1e-3), "unit": "tokens/s",
@@ -376,7 +379,7 @@ def gate_layout_workloads(kda, dev, stream, flush, pk, world, rank):
                           workspace=ws, stream=stream)
 
         barrier(world)
-        times = time_steps(call, 10, 3, stream, flush)
+        times = time_steps(call, 10, 3, stream, flush, name=f"kda.gate.{gate}")
         ms = max_over_ranks(sum(times), world, dev) / len(times)
         alg = (PREFILL_BYTES_PER_TOKEN_HEAD - GATE_BYTES["channel"] + GATE_BYTES[gate]) * B * T * H \
             + 2 * STATE_BYTES * B * H
@@ -425,7 +428,7 @@ def run_kda(args, rank, world, local_rank):
         barrier(world)
         torch.cuda.synchronize()
         clocks = ClockSampler(dev.index)
-        t = time_steps(step, args.steps, args.warmup, stream, flush)
+        t = time_steps(step, args.steps, args.warmup, stream, flush, name="kda.prefill")
         torch.cuda.synchronize()
         barrier(world)
         torch.cuda.synchronize()
@@ -480,7 +483,7 @@ def run_kda(args, rank, world, local_rank):
     if not args.no_e2e:
         e2e_steps = max(3, min(args.steps, 10))
         barrier(world)
-        e_times = time_steps(e2e_step, e2e_steps, max(3, args.warmup // 2), stream)
+        e_times = time_steps(e2e_step, e2e_steps, max(3, args.warmup // 2), stream, name="kda.e2e")
         barrier(world)
         e_ms = max_over_ranks(sum(e_times), world, dev) / e2e_steps
         e2e = {"value": tokens_per_step / (e_ms * 1e-3), "unit": "tokens/s",
@@ -507,7 +510,7 @@ def run_kda(args, rank, world, local_rank):
                                 out=od[t], stream=stream)
         barrier(world)
         dclk = ClockSampler(dev.index)
-        d_times = time_steps(graph.replay, 2, 1, stream, flush)
+        d_times = time_steps(graph.replay, 2, 1, stream, flush, name="kda.decode")
         dclk = dclk.stop()
         barrier(world)
         d_ms = max_over_ranks(sum(d_times), world, dev) / len(d_times)
