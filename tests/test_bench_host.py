@@ -24,3 +24,124 @@ def test_traffic_is_reported_only_for_the_captured_sources_and_shape():
         other = tuple(x + 1 for x in t["shape"])
         assert bench.traffic(kind, None, other) is None
     assert bench.traffic("prefill", 123, (1, 1, 1)) == 123  # an explicit capture overrides
+
+
+def _fake_cuda(monkeypatch):
+    """Runs bench.py's GPU arm on the CPU: CUDA streams, events and graphs become
+    no-ops, the device becomes the CPU and libkda a stand-in that records its calls."""
+    import contextlib
+    import types
+
+    import torch
+
+    import gated_delta_rule_101_b200 as kda
+
+    class Recorder:
+        def __init__(self):
+            self.calls = []
+
+        def __getattr__(self, name):
+            def call(*args):
+                self.calls.append(name)
+                return 0
+
+            return call
+
+    class Event:
+        def __init__(self, **kw):
+            pass
+
+        def record(self, stream=None):
+            pass
+
+        def elapsed_time(self, other):
+            return 0.25
+
+    class Stream:
+        cuda_stream = 0
+
+        def __init__(self, *a, **kw):
+            pass
+
+        def wait_stream(self, other):
+            pass
+
+    class Graph:
+        def replay(self):
+            pass
+
+    class Props:
+        uuid = "00000000-0000-0000-0000-000000000000"
+
+    cuda = types.SimpleNamespace(
+        synchronize=lambda *a, **kw: None, Event=Event, Stream=Stream,
+        stream=lambda s: contextlib.nullcontext(), current_stream=lambda *a, **kw: Stream(),
+        set_device=lambda *a: None, get_device_properties=lambda i: Props(), CUDAGraph=Graph,
+        graph=lambda g, **kw: contextlib.nullcontext(), empty_cache=lambda: None, nvtx=torch.cuda.nvtx)
+    shim = types.ModuleType("torch_on_cpu")
+    for k in dir(torch):
+        if not k.startswith("__"):
+            setattr(shim, k, getattr(torch, k))
+    shim.device = lambda *a, **kw: torch.device("cpu")
+    shim.cuda = cuda
+    rec = Recorder()
+    monkeypatch.setattr(bench, "torch", shim)
+    monkeypatch.setattr(kda, "_lib", rec)
+    monkeypatch.setattr(torch.Tensor, "pin_memory", lambda self: self)
+    for d, kw in ((bench.PREFILL, dict(B=2, T=130, H=2)), (bench.DECODE, dict(N=2, H=2, steps=3)),
+                  (bench.VARLEN, dict(n_seqs=3, len_range=(5, 70), H=2)),
+                  (bench.LONG, dict(T_call=128, calls=3, H=2))):
+        for key, val in kw.items():
+            monkeypatch.setitem(d, key, val)
+    monkeypatch.setattr(bench, "L2_FLUSH_BYTES", 1 << 10)
+    return rec
+
+
+def _run_kda_line(**flags):
+    import contextlib
+    import io
+    import json
+    import types
+
+    args = types.SimpleNamespace(steps=3, warmup=3, no_extra=False, no_cpu_baseline=True, no_e2e=False,
+                                 no_decode=False, decode_steps=3, traffic=None, decode_traffic=None)
+    for k, v in flags.items():
+        setattr(args, k, v)
+    out = io.StringIO()
+    with contextlib.redirect_stdout(out):
+        bench.run_kda(args, 0, 1, 0)
+    return json.loads(out.getvalue().strip().splitlines()[-1])
+
+
+def test_gpu_arm_runs_end_to_end_on_fakes(monkeypatch):
+    rec = _fake_cuda(monkeypatch)
+    line = _run_kda_line()
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+                "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config", "roofline",
+                "e2e", "gpu_launches", "clocks", "decode", "varlen", "long_context", "gate_layouts"):
+        assert key in line, key
+    assert set(line["gate_layouts"]) == {"channel_bf16", "head", "none"}
+    for r in (line["roofline"], line["decode"]["roofline"]):
+        assert {"bound", "achieved", "peak", "unit", "frac", "traffic"} <= set(r)
+    assert line["roofline"]["traffic"] is None  # captured at another shape
+    assert {"kda_chunk_fwd", "kda_chunk_fwd_gated", "kda_decode_step"} <= set(rec.calls)
+
+
+def test_gpu_arm_remeasures_a_throttled_step(monkeypatch):
+    _fake_cuda(monkeypatch)
+
+    class Clocks:
+        n = 0
+
+        def __init__(self, index):
+            pass
+
+        def stop(self):
+            Clocks.n += 1
+            return {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0,
+                    "reasons": ["hw_thermal_slowdown"] if Clocks.n == 1 else []}
+
+    monkeypatch.setattr(bench, "ClockSampler", Clocks)
+    line = _run_kda_line(no_extra=True, no_decode=True, no_e2e=True)
+    assert line["clocks"]["reasons"] == []
+    assert line["clocks"]["remeasured_after"]["reasons"] == ["hw_thermal_slowdown"]
