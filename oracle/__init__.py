@@ -6,7 +6,8 @@ CPU-baseline leg of ``bench.py`` may import this package. The CUDA library
 no code: the only thing both sides use is the seeded input generator, which
 holds none of the method's arithmetic.
 
-What is computed is Kimi Delta Attention's recurrence, eq. (1) of the
+``kda_fwd`` runs the recurrence; ``backward.kda_bwd`` gives its gradients (the
+reverse pass, plain numpy). What is computed is Kimi Delta Attention's recurrence, eq. (1) of the
 blog.gzher.com review "Kimi K3论文：Kimi Linear" (section 3):
 
     S_t = (I - beta_t k_t k_t^T) Diag(alpha_t) S_{t-1} + beta_t k_t v_t^T,
