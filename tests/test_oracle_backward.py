@@ -142,3 +142,17 @@ def test_each_planted_mistake_fails_the_autograd_pin(old, new):
     got = mod.kda_bwd(*c, cu_seqlens=cu)
     with pytest.raises(AssertionError):
         _assert_close(got, want, 1e-10, "mutant")
+
+
+@pytest.mark.parametrize("C", [1, 16, 64])
+@pytest.mark.parametrize("la_range", [(0.05, 0.5), (2.0, 6.0)])
+def test_chunked_backward_equals_the_reverse_pass_oracle(C, la_range):
+    """The chunk algebra's reverse pass (tests/chunked_backward.py, the blueprint of a
+    chunked backward) reproduces the token-by-token gradients, ragged last chunk and
+    strong decay included."""
+    from chunked_backward import kda_chunked_bwd_fp64
+
+    c = _case(7, (2, 37), dk=8, dv=5, la_range=la_range)
+    want = kda_bwd(*c)
+    got = kda_chunked_bwd_fp64(*c, C=C)
+    _assert_close(got, want, 1e-10, f"chunked C={C}")
