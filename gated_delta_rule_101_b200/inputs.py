@@ -11,7 +11,9 @@ Recipe (every draw from one ``torch.Generator`` seeded with ``seed``, in the
 order listed, on ``device``):
   q, k       ~ N(0, 1), L2-normalised over the key dimension, cast to ``dtype``
   v          ~ N(0, 1), cast to ``dtype``
-  log_alpha  = -U(lo, hi), fp32, independent per (token, head, key channel)
+  log_alpha  = -U(lo, hi), fp32, independent per (token, head, key channel); with
+               gate="head" one per (token, head), with gate="channel_bf16" the
+               same draw cast to bf16, with gate="none" no draw (None)
   beta       = sigmoid(N(0, 1)), fp32, one per (token, head)
   S0         ~ N(0, s0_std^2) fp32 per (sequence, head, dk, dv); zeros if s0_std == 0
 """
