@@ -79,6 +79,10 @@ def _bind(lib: ctypes.CDLL) -> ctypes.CDLL:
                                         vp, i32, vp, i32, vp, ctypes.c_size_t, vp]
     lib.kda_decode_step_gated.restype = i32
     lib.kda_decode_step_gated.argtypes = [vp, vp, vp, vp, i32, fp, fp, vp, i32, i32, i32, vp]
+    lib.kda_set_wait_limit_ns.restype = i32
+    lib.kda_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
+    lib.kda_selftest_wait_timeout.restype = i32
+    lib.kda_selftest_wait_timeout.argtypes = [vp, vp, vp]
     return lib
 
 
@@ -320,3 +324,29 @@ def chunk_fwd_noalloc(q, k, v, log_alpha, beta, S0=None, *, out, state_out=None,
     if st != KDA_OK:
         raise KDAError(st, "kda_chunk_fwd_noalloc")
     return out, state_out
+
+
+def device_status() -> int:
+    """Reads and clears libkda's device status: 0, or 1 if a bounded wait gave up."""
+    st = ctypes.c_int(0)
+    rc = lib().kda_get_device_status(ctypes.byref(st))
+    if rc != KDA_OK:
+        raise KDAError(rc, "kda_get_device_status")
+    return st.value
+
+
+def set_wait_limit_ns(ns: int) -> None:
+    """Sets the bounded waits' time limit (0 restores the default of one second)."""
+    rc = lib().kda_set_wait_limit_ns(int(ns))
+    if rc != KDA_OK:
+        raise KDAError(rc, "kda_set_wait_limit_ns")
+
+
+def selftest_wait_timeout(flag: torch.Tensor, result: torch.Tensor, stream=None) -> None:
+    """Launches ``kda_selftest_wait_timeout`` on device int32 tensors ``flag`` (kept at
+    0 by the caller) and ``result`` (receives the bitmask of waits that gave up)."""
+    for t, name in ((flag, "flag"), (result, "result")):
+        _need(t, name, torch.int32, flag.device)
+    rc = lib().kda_selftest_wait_timeout(_ptr(flag), _ptr(result), _stream_handle(stream, flag.device))
+    if rc != KDA_OK:
+        raise KDAError(rc, "kda_selftest_wait_timeout")

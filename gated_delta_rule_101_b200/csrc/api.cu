@@ -131,6 +131,17 @@ int kda_get_device_status(int *status) {
     return kda::read_device_status(status) == 0 ? KDA_OK : KDA_ERR_CUDA;
 }
 
+int kda_set_wait_limit_ns(uint64_t ns) {
+    return kda::set_wait_limit_ns((unsigned long long)ns) == 0 ? KDA_OK : KDA_ERR_CUDA;
+}
+
+int kda_selftest_wait_timeout(const int32_t *flag, int32_t *result, void *stream) {
+    if (!flag || !result) return KDA_ERR_INVALID_ARG;
+    if (((uintptr_t)flag & 3u) != 0 || ((uintptr_t)result & 3u) != 0) return KDA_ERR_INVALID_ARG;
+    return kda::launch_wait_selftest(flag, result, (cudaStream_t)stream) == cudaSuccess ? KDA_OK
+                                                                                        : KDA_ERR_CUDA;
+}
+
 int kda_decode_step(const void *q, const void *k, const void *v, const float *log_alpha,
                     const float *beta, float *S, void *o, int N, int H, int dtype,
                     void *stream) {

@@ -86,7 +86,11 @@ cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, const
                               int64_t T, int H, const int32_t *cu_seqlens, int n_seqs,
                               void *workspace, cudaStream_t stream);
 
-// Reads and clears the device status word set by bounded waits (0 = no timeout).
+// Reads and clears the count of bounded waits that gave up (*status: 0 none, 1 some).
 int read_device_status(int *status);
+// Sets the bounded waits' time limit (0: the default of one second).
+int set_wait_limit_ns(unsigned long long ns);
+// Runs the bounded-wait self-test kernel (see kda_selftest_wait_timeout).
+cudaError_t launch_wait_selftest(const int32_t *flag, int32_t *result, cudaStream_t stream);
 
 }  // namespace kda

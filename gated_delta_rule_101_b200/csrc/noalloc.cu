@@ -12,8 +12,11 @@
 //
 // Properties a caller must know:
 //   - The scratch is KDA_NOALLOC_SCRATCH_BYTES (64 MiB) per GPU. It is part of
-//     the library's device image, so every GPU that loads the library holds
-//     it until the process exits, whether or not this entry point is used.
+//     the library's device image: it is reserved on each GPU where that image
+//     is loaded (when the CUDA context loads the library's module: at context
+//     creation with CUDA_MODULE_LOADING=EAGER, otherwise on the first use of
+//     one of its kernels or symbols) and held until the process exits, whether
+//     or not this entry point is used.
 //   - Problems whose workspace would exceed it are rejected with
 //     KDA_ERR_SCRATCH_LIMIT before anything is launched.
 //   - All calls on a GPU share the one buffer, and it keeps whatever the last
@@ -24,6 +27,9 @@
 //   - The first call on each GPU looks up the buffer's device address
 //     (cudaGetSymbolAddress, with that GPU current). Make that first call
 //     before any stream capture begins.
+//   - The address is kept for the life of the process. A device reset
+//     (cudaDeviceReset) unloads the module and invalidates it, so this entry
+//     point must not be used after one.
 //   - Nothing here calls cudaMalloc, cudaFree or any allocating routine.
 #include <mutex>
 

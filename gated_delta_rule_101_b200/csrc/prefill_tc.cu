@@ -47,9 +47,9 @@
 
 namespace kda {
 
-// Status word of the tensor-core kernels: 1 after a bounded wait gave up.
-// Read and cleared by kda_get_device_status().
-__device__ int g_kda_device_status = 0;
+// Status of the tensor-core kernels: the count of bounded waits that gave up (read and
+// cleared by kda_get_device_status()) and the waits' time limit.
+__device__ ptx::DeviceStatus g_kda_status = {0, 0, ptx::WAIT_LIMIT_NS};
 
 namespace {
 
@@ -249,7 +249,7 @@ struct PrepWorker {
     // Worker-wide wait: thread 0 polls, the others sleep at the worker's barrier.
     __device__ __forceinline__ void wait(uint64_t *bar, uint32_t parity) {
         bool ok = true;
-        if (tid() == 0) ok = mbar_wait(bar, parity, dead, &g_kda_device_status);
+        if (tid() == 0) ok = mbar_wait(bar, parity, dead, &g_kda_status);
         dead = sync_or(!ok || dead);
     }
     // Barriers and TMEM; every thread of the worker calls this once, before any item.
@@ -883,7 +883,7 @@ __device__ __forceinline__ void chain_task(unsigned char *sm, const int tid, con
     bool dead = false;
 
     auto blob_of = [&](int chunk) {
-        if (a.ready) counter_wait_gt(ready_upto, chunk, dead, &g_kda_device_status);
+        if (a.ready) counter_wait_gt(ready_upto, chunk, dead, &g_kda_status);
         return ws_blobs + ((size_t)(slot0 + chunk) * H + h) * BLOB_BYTES;
     };
     auto issue_load1 = [&](int chunk, int stage) {
@@ -955,7 +955,7 @@ __device__ __forceinline__ void chain_task(unsigned char *sm, const int tid, con
         // ------------------------------------------------------------ flag watcher
         if (lane == 0) {
             for (int m = 0; m < nchunks; ++m) {
-                if (!flag_wait(a.ready + (size_t)(slot0 + m) * H + h, dead, &g_kda_device_status)) break;
+                if (!flag_wait(a.ready + (size_t)(slot0 + m) * H + h, dead, &g_kda_status)) break;
                 st_release_cta(ready_upto, m + 1);
             }
         }
@@ -975,7 +975,7 @@ __device__ __forceinline__ void chain_task(unsigned char *sm, const int tid, con
             const uint32_t d1 = tmem + (uint32_t)((n & 1) * N);
             const uint32_t lph = (uint32_t)(n >> 1) & 1u;
             if (lane == 0) {
-                mbar_wait(&bar_ld1[stage], lph, dead, &g_kda_device_status);
+                mbar_wait(&bar_ld1[stage], lph, dead, &g_kda_status);
                 if (!dead) {  // D1 = [Q~; W] S, DU = [.; T Diag(beta)] V
                     tc_fence_after();
                     mma_run<D>(d1, kmajor(st_base + Lay::A1, 128), mnmajor(sm_base + Lay::SIMG, 16384),
@@ -987,7 +987,7 @@ __device__ __forceinline__ void chain_task(unsigned char *sm, const int tid, con
             }
             __syncwarp();
             named_bar_sync(BAR_VNEW, BAR_VNEW_COUNT);  // V_new image of chunk n written
-            if (lane == 0) mbar_wait(&bar_ld2[stage], lph, dead, &g_kda_device_status);
+            if (lane == 0) mbar_wait(&bar_ld2[stage], lph, dead, &g_kda_status);
             if (lane == 0 && !dead) {
                 // D3 = K~^T V_new (the state path first), then D1 += [A_qk; 0] V_new
                 tc_fence_after();
@@ -1010,7 +1010,7 @@ __device__ __forceinline__ void chain_task(unsigned char *sm, const int tid, con
         // 4 and 5 (lane quarters 0 and 1) once the output MMA of chunk m has completed,
         // while the next chunk's first MMAs run.
         auto store_output = [&](int m) {
-            mbar_wait(&bar_c[m & 1], (uint32_t)(m >> 1) & 1u, dead, &g_kda_device_status);
+            mbar_wait(&bar_c[m & 1], (uint32_t)(m >> 1) & 1u, dead, &g_kda_status);
             tc_fence_after();
             const int r = c;
             const int64_t m0 = (int64_t)(c0 + m) * CH;  // first token of the chunk
@@ -1038,7 +1038,7 @@ __device__ __forceinline__ void chain_task(unsigned char *sm, const int tid, con
             const uint32_t d1 = tmem + (uint32_t)((n & 1) * N);
             const uint32_t lph = (uint32_t)(n >> 1) & 1u;
             if (q4 >= 2) {  // rows 64..127 hold (W S)[r] in D1 and U[r] in DU; V_new = U - W S
-                mbar_wait(bar_a, ph, dead, &g_kda_device_status);
+                mbar_wait(bar_a, ph, dead, &g_kda_status);
                 tc_fence_after();
                 const int r = c - 64;
 #pragma unroll
@@ -1063,14 +1063,14 @@ __device__ __forceinline__ void chain_task(unsigned char *sm, const int tid, con
                 // Part 1 of the stage is free once the first MMAs have completed: refill it
                 // with chunk n + 2 while this chunk is still being processed.
                 if (lane == 0 && n + 2 < nchunks) {
-                    mbar_wait(bar_a, ph, dead, &g_kda_device_status);
+                    mbar_wait(bar_a, ph, dead, &g_kda_status);
                     if (!dead) issue_load1(n + 2, stage);
                 }
                 __syncwarp();
             }
             {  // S <- Diag(exp(g_L)) S + K~^T V_new
-                mbar_wait(&bar_ld2[stage], lph, dead, &g_kda_device_status);  // GAM
-                mbar_wait(bar_b, ph, dead, &g_kda_device_status);
+                mbar_wait(&bar_ld2[stage], lph, dead, &g_kda_status);  // GAM
+                mbar_wait(bar_b, ph, dead, &g_kda_status);
                 tc_fence_after();
                 const float gam = reinterpret_cast<const float *>(st + Lay::GAM)[c];
 #pragma unroll
@@ -1099,7 +1099,7 @@ __device__ __forceinline__ void chain_task(unsigned char *sm, const int tid, con
             // Part 2 is free once the output MMA (the last reader of A2 and KTT) has
             // completed and the state update (the reader of GAM) has passed BAR_END.
             if (tid == 32 && n + 2 < nchunks) {
-                mbar_wait(&bar_c[stage], lph, dead, &g_kda_device_status);
+                mbar_wait(&bar_c[stage], lph, dead, &g_kda_status);
                 if (!dead) issue_load2(n + 2, stage);
             }
         }
@@ -1698,12 +1698,53 @@ cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, const
 }
 
 int read_device_status(int *status) {
-    int v = 0;
-    if (cudaMemcpyFromSymbol(&v, g_kda_device_status, sizeof(int)) != cudaSuccess) return -1;
+    ptx::DeviceStatus v{};
+    if (cudaMemcpyFromSymbol(&v, g_kda_status, sizeof(int)) != cudaSuccess) return -1;
     const int zero = 0;
-    if (cudaMemcpyToSymbol(g_kda_device_status, &zero, sizeof(int)) != cudaSuccess) return -1;
-    *status = v;
+    if (cudaMemcpyToSymbol(g_kda_status, &zero, sizeof(int)) != cudaSuccess) return -1;
+    *status = v.timeouts != 0 ? 1 : 0;
     return 0;
+}
+
+int set_wait_limit_ns(unsigned long long ns) {
+    const unsigned long long limit = ns ? ns : ptx::WAIT_LIMIT_NS;
+    return cudaMemcpyToSymbol(g_kda_status, &limit, sizeof(limit),
+                              offsetof(ptx::DeviceStatus, wait_limit_ns)) == cudaSuccess
+               ? 0
+               : -1;
+}
+
+namespace {
+// Self-test of the failure path: one warp runs the three kinds of bounded wait the
+// kernels use on conditions that never come true (an mbarrier nobody arrives on, a
+// global flag nobody sets, a shared counter nobody raises), each with its own `dead`
+// flag so that every one of them runs its slow path. No copy or MMA is in flight, so
+// the kernel leaves nothing behind when it returns. Bit b of *result is set when wait
+// b gave up.
+__global__ void __launch_bounds__(32) kda_wait_selftest_kernel(const int32_t *flag, int32_t *result) {
+    __shared__ uint64_t bar;
+    __shared__ int32_t counter;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        counter = 0;
+        fence_mbar_init();
+    }
+    __syncwarp();
+    if (threadIdx.x == 0) {
+        int32_t bits = 0;
+        bool dead0 = false, dead1 = false, dead2 = false;
+        if (!mbar_wait(&bar, 0, dead0, &g_kda_status)) bits |= 1;
+        if (!flag_wait(flag, dead1, &g_kda_status)) bits |= 2;
+        if (!counter_wait_gt(&counter, 0, dead2, &g_kda_status)) bits |= 4;
+        *result = bits;
+        mbar_inval(&bar);
+    }
+}
+}  // namespace
+
+cudaError_t launch_wait_selftest(const int32_t *flag, int32_t *result, cudaStream_t stream) {
+    kda_wait_selftest_kernel<<<1, 32, 0, stream>>>(flag, result);
+    return cudaGetLastError();
 }
 
 }  // namespace kda

@@ -49,26 +49,53 @@ __device__ __forceinline__ uint64_t global_ns() {
     return t;
 }
 
-constexpr uint64_t WAIT_LIMIT_NS = 1000000000ull;  // give up a wait after one second
+// Device status shared by the tensor-core kernels of the library.
+//   timeouts:      number of bounded waits that have given up since the host last
+//                  read and cleared it (kda_get_device_status).
+//   wait_limit_ns: how long a wait may take before it gives up (one second; tests of
+//                  the failure path shorten it through kda_set_wait_limit_ns).
+struct DeviceStatus {
+    int timeouts;
+    int reserved;
+    unsigned long long wait_limit_ns;
+};
+constexpr unsigned long long WAIT_LIMIT_NS = 1000000000ull;  // the default limit: one second
 
-// Waits for `parity` on `bar`. Gives up after WAIT_LIMIT_NS, or as soon as any
-// CTA has recorded a timeout in *status (so one failure does not make every
-// other CTA wait its full limit in turn). On giving up it sets *status to 1
-// and `dead`; once `dead` is set every later wait returns at once, so the
-// kernel unwinds instead of hanging.
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, bool &dead, int *status) {
+// Bookkeeping of one wait's slow path. It starts when the wait is first found not
+// complete: it notes the time, the limit in force and the timeout count at that moment.
+// The wait gives up when its limit has passed, or as soon as the count has moved, that
+// is when any CTA has given up on a wait since this one began (so one failure does not
+// make every other CTA wait its full limit in turn). A count left over from an earlier
+// launch does not count: only changes seen while waiting do, so a timeout that nobody
+// has read yet cannot make a later call give up early.
+struct WaitClock {
+    uint64_t t0, limit;
+    int base;
+    __device__ __forceinline__ explicit WaitClock(const DeviceStatus *st)
+        : t0(global_ns()),
+          limit(*reinterpret_cast<const volatile unsigned long long *>(&st->wait_limit_ns)),
+          base(*reinterpret_cast<const volatile int *>(&st->timeouts)) {}
+    __device__ __forceinline__ bool expired(const DeviceStatus *st) const {
+        return *reinterpret_cast<const volatile int *>(&st->timeouts) != base || global_ns() - t0 > limit;
+    }
+};
+__device__ __forceinline__ void record_timeout(DeviceStatus *st, bool &dead) {
+    dead = true;
+    atomicAdd(&st->timeouts, 1);
+}
+
+// Waits for `parity` on `bar`, bounded as WaitClock describes. On giving up it
+// counts a timeout in *st and sets `dead`; once `dead` is set every later wait
+// returns at once, so the kernel unwinds instead of hanging.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, bool &dead, DeviceStatus *st) {
     if (dead) return false;
     if (mbar_try_wait(bar, parity)) return true;
-    const uint64_t t0 = global_ns();
+    const WaitClock clk(st);
     for (uint32_t i = 1;; ++i) {
         if (mbar_try_wait(bar, parity)) return true;
-        if ((i & 255u) == 0) {
-            if (*reinterpret_cast<volatile int *>(status) != 0 || global_ns() - t0 > WAIT_LIMIT_NS)
-                break;
-        }
+        if ((i & 255u) == 0 && clk.expired(st)) break;
     }
-    dead = true;
-    atomicExch(status, 1);
+    record_timeout(st, dead);
     return false;
 }
 
@@ -101,26 +128,22 @@ __device__ __forceinline__ int32_t ld_acquire_gpu(const int32_t *p) {
     return v;
 }
 // Waits until *flag != 0, with the same limit and failure reporting as mbar_wait.
-__device__ __forceinline__ bool flag_wait(const int32_t *flag, bool &dead, int *status) {
+__device__ __forceinline__ bool flag_wait(const int32_t *flag, bool &dead, DeviceStatus *st) {
     if (dead) return false;
     if (ld_acquire_gpu(flag) != 0) {
         fence_proxy_async_global();
         return true;
     }
-    const uint64_t t0 = global_ns();
+    const WaitClock clk(st);
     for (uint32_t i = 1;; ++i) {
         __nanosleep(100);
         if (ld_acquire_gpu(flag) != 0) {
             fence_proxy_async_global();
             return true;
         }
-        if ((i & 63u) == 0) {
-            if (*reinterpret_cast<volatile int *>(status) != 0 || global_ns() - t0 > WAIT_LIMIT_NS)
-                break;
-        }
+        if ((i & 63u) == 0 && clk.expired(st)) break;
     }
-    dead = true;
-    atomicExch(status, 1);
+    record_timeout(st, dead);
     return false;
 }
 
@@ -136,32 +159,28 @@ __device__ __forceinline__ void st_release_cta(int32_t *p, int32_t v) {
 // Waits until the shared counter *p exceeds v, with the limit and failure reporting of
 // mbar_wait; the counter's writer has seen global data the caller will then read with
 // bulk copies.
-__device__ __forceinline__ bool counter_wait_gt(const int32_t *p, int32_t v, bool &dead, int *status) {
+__device__ __forceinline__ bool counter_wait_gt(const int32_t *p, int32_t v, bool &dead, DeviceStatus *st) {
     if (dead) return false;
     if (ld_acquire_cta(p) > v) {
         fence_proxy_async_global();
         return true;
     }
-    const uint64_t t0 = global_ns();
+    const WaitClock clk(st);
     for (uint32_t i = 1;; ++i) {
         if (ld_acquire_cta(p) > v) {
             fence_proxy_async_global();
             return true;
         }
-        if ((i & 255u) == 0) {
-            if (*reinterpret_cast<volatile int *>(status) != 0 || global_ns() - t0 > WAIT_LIMIT_NS)
-                break;
-        }
+        if ((i & 255u) == 0 && clk.expired(st)) break;
     }
-    dead = true;
-    atomicExch(status, 1);
+    record_timeout(st, dead);
     return false;
 }
 
 // CTA-wide wait: thread 0 polls the barrier while every other thread sleeps at
 // the CTA barrier (polling threads would take issue slots from co-resident
 // CTAs). All threads leave with the same `dead` value.
-__device__ __forceinline__ void cta_wait(uint64_t *bar, uint32_t parity, bool &dead, int *status) {
+__device__ __forceinline__ void cta_wait(uint64_t *bar, uint32_t parity, bool &dead, DeviceStatus *status) {
     bool ok = true;
     if (threadIdx.x == 0) ok = mbar_wait(bar, parity, dead, status);
     dead = __syncthreads_or(!ok || dead) != 0;

@@ -207,7 +207,9 @@ KDA_API int kda_decode_step_gated(const void *q, const void *k, const void *v,
  *
  * Instead of a workspace the call uses one fixed scratch buffer of
  * kda_noalloc_scratch_bytes() bytes (64 MiB) that lives in the library's
- * device image: every GPU that loads the library holds it until the process
+ * device image: it is reserved on each GPU where that image is loaded (at
+ * context creation with CUDA_MODULE_LOADING=EAGER, otherwise on the first use
+ * of the library's device code on that GPU) and held until the process
  * exits. A problem whose kda_chunk_fwd_workspace_size exceeds it is rejected
  * with KDA_ERR_SCRATCH_LIMIT before anything is launched (about a thousand
  * chunk-head pairs for bf16: B * ceil(T/64) * H <= 1015 for unpacked input
@@ -216,7 +218,9 @@ KDA_API int kda_decode_step_gated(const void *q, const void *k, const void *v,
  * Calls that may overlap on the GPU (different streams, no ordering between
  * them) race on the buffer: issue them on one stream. The first call on each
  * GPU looks up the buffer's device address with that GPU current; make it
- * before any stream capture begins. The function itself allocates nothing.
+ * before any stream capture begins. The address is kept for the life of the
+ * process: do not use this entry point after a device reset
+ * (cudaDeviceReset). The function itself allocates nothing.
  */
 KDA_API int kda_chunk_fwd_noalloc(const void *q, const void *k, const void *v,
                                   const float *log_alpha, const float *beta, const float *S0,
@@ -228,13 +232,39 @@ KDA_API int kda_chunk_fwd_noalloc(const void *q, const void *k, const void *v,
 KDA_API size_t kda_noalloc_scratch_bytes(void);
 
 /*
- * Reads and clears the library's device status word. *status is 0 when no
- * kernel has given up on a bounded wait since the last read, 1 otherwise
- * (the affected call's outputs are then invalid; KDA_ERR_TIMEOUT describes
- * it). Synchronises with the device (a blocking symbol copy on the legacy
+ * Reads and clears the library's device status. *status is 0 when no kernel
+ * has given up on a bounded wait since the last read, 1 otherwise (the
+ * outputs of the call that timed out are then invalid; KDA_ERR_TIMEOUT
+ * describes it). A timeout that has not been read yet does not affect later
+ * calls: a wait gives up early only when another wait gives up while it is
+ * waiting, so calls made after the failed one compute normally.
+ * Synchronises with the device (a blocking symbol copy on the legacy
  * stream); do not call it inside stream capture.
  */
 KDA_API int kda_get_device_status(int *status);
+
+/*
+ * Failure-detection support (no counterpart on the pages; library plumbing).
+ *
+ * Every wait of the tensor-core kernels on an mbarrier, a ready flag or a
+ * shared counter gives up after a time limit (default one second), counts a
+ * timeout in the device status and lets its kernel unwind and return.
+ * kda_set_wait_limit_ns sets that limit for later launches on the current
+ * GPU (ns = 0 restores the default). It is meant for tests of the failure
+ * path; a limit shorter than a kernel's ordinary waits makes correct calls
+ * time out. Synchronises with the device like kda_get_device_status.
+ *
+ * kda_selftest_wait_timeout runs, on `stream`, one small kernel that makes
+ * each of the three kinds of bounded wait run out: an mbarrier that nothing
+ * arrives on, the device int32 *flag (which the caller keeps at 0) and a
+ * shared counter that nothing raises. It writes to the device int32 *result
+ * a bitmask of the waits that gave up (bit 0 mbarrier, bit 1 flag, bit 2
+ * counter; 7 when all three did) and counts three timeouts in the device
+ * status. It takes about three wait limits. Both pointers must be 4-byte
+ * aligned device memory.
+ */
+KDA_API int kda_set_wait_limit_ns(uint64_t ns);
+KDA_API int kda_selftest_wait_timeout(const int32_t *flag, int32_t *result, void *stream);
 
 #ifdef __cplusplus
 }

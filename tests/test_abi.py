@@ -157,3 +157,11 @@ def test_binding_refuses_wrong_dtypes_before_calling():
     q = torch.zeros(1, 64, 1, 128, dtype=torch.float16)
     with pytest.raises(TypeError):
         kda.chunk_fwd(q, q, q, q.float(), q[..., 0].float())
+
+
+def test_wait_selftest_rejects_bad_pointers(lib):
+    """The failure-path self-test checks its pointers before launching anything."""
+    assert lib.kda_selftest_wait_timeout(None, FAKE, None) == INVALID
+    assert lib.kda_selftest_wait_timeout(FAKE, None, None) == INVALID
+    assert lib.kda_selftest_wait_timeout(ctypes.c_void_p((1 << 20) + 2), FAKE, None) == INVALID
+    assert lib.kda_selftest_wait_timeout(FAKE, ctypes.c_void_p((1 << 20) + 1), None) == INVALID
