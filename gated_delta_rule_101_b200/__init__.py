@@ -28,7 +28,10 @@ import re
 import torch
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "libkda.so")
+# KDA_DEBUG=1 in the environment selects the KDA_DEBUG build (device-side checks of
+# packed-sequence offsets; see include/kda.h).
+DEBUG_BUILD = os.environ.get("KDA_DEBUG", "0") not in ("", "0")
+LIB_PATH = os.path.join(_PKG, "libkda_debug.so" if DEBUG_BUILD else "libkda.so")
 HEADER = os.path.join(os.path.dirname(_PKG), "include", "kda.h")
 
 KDA_BF16, KDA_F32 = 0, 1
@@ -326,8 +329,13 @@ def chunk_fwd_noalloc(q, k, v, log_alpha, beta, S0=None, *, out, state_out=None,
     return out, state_out
 
 
+STATUS_TIMEOUT, STATUS_BAD_INPUT = 1, 2
+
+
 def device_status() -> int:
-    """Reads and clears libkda's device status: 0, or 1 if a bounded wait gave up."""
+    """Reads and clears libkda's device status: 0, or a mask of STATUS_TIMEOUT (a
+    bounded wait gave up) and STATUS_BAD_INPUT (a KDA_DEBUG build refused device
+    offsets)."""
     st = ctypes.c_int(0)
     rc = lib().kda_get_device_status(ctypes.byref(st))
     if rc != KDA_OK:

@@ -17,6 +17,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libkda.so")
+DEBUG_LIB = os.path.join(PKG, "libkda_debug.so")  # the same sources with KDA_DEBUG defined
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 
@@ -31,21 +32,25 @@ def sources() -> list[str]:
     return sorted(glob.glob(os.path.join(CSRC, "*.cu")))
 
 
-def _stale() -> bool:
-    if not os.path.exists(LIB):
+def _stale(lib: str) -> bool:
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     deps = sources() + glob.glob(os.path.join(CSRC, "*.cuh")) + glob.glob(os.path.join(INCLUDE, "*.h"))
     return any(os.path.getmtime(p) > t for p in deps)
 
 
-def build(force: bool = False, verbose: bool = False, extra: list[str] | None = None) -> str:
-    """Compile every csrc/*.cu into libkda.so; returns the library path."""
-    if not force and not _stale():
-        return LIB
+def build(force: bool = False, verbose: bool = False, extra: list[str] | None = None,
+          debug: bool = False) -> str:
+    """Compile every csrc/*.cu into libkda.so (with ``debug``: libkda_debug.so, built with
+    KDA_DEBUG defined); returns the library path."""
+    lib = DEBUG_LIB if debug else LIB
+    if not force and not _stale(lib):
+        return lib
     cmd = [nvcc(), *ARCH, "-O3", "-lineinfo", "-std=c++17", "-shared", "-Xcompiler", "-fPIC",
            "-Xcompiler", "-fvisibility=hidden", "--expt-relaxed-constexpr",
-           f"-I{INCLUDE}", f"-I{CSRC}", *(extra or []), "-o", LIB + ".tmp", *sources()]
+           *(["-DKDA_DEBUG"] if debug else []),
+           f"-I{INCLUDE}", f"-I{CSRC}", *(extra or []), "-o", lib + ".tmp", *sources()]
     if verbose:
         print(" ".join(cmd), file=sys.stderr)
     res = subprocess.run(cmd, capture_output=True, text=True)
@@ -53,10 +58,21 @@ def build(force: bool = False, verbose: bool = False, extra: list[str] | None = 
         raise RuntimeError(f"nvcc failed ({res.returncode}):\n{res.stderr}")
     if verbose and res.stderr:
         print(res.stderr, file=sys.stderr)
-    os.replace(LIB + ".tmp", LIB)
-    return LIB
+    os.replace(lib + ".tmp", lib)
+    return lib
+
+
+def build_all(force: bool = False, verbose: bool = False) -> list[str]:
+    """Both libraries: libkda.so and its KDA_DEBUG variant, compiled in parallel."""
+    from concurrent.futures import ThreadPoolExecutor
+
+    with ThreadPoolExecutor(2) as ex:
+        jobs = [ex.submit(build, force, verbose, None, d) for d in (False, True)]
+        return [j.result() for j in jobs]
 
 
 if __name__ == "__main__":
-    print(build(force="--force" in sys.argv, verbose=True,
-                extra=["-Xptxas", "-v"] if "--ptxas-v" in sys.argv else None))
+    if "--ptxas-v" in sys.argv:
+        print(build(force=True, verbose=True, extra=["-Xptxas", "-v"], debug="--debug" in sys.argv))
+    else:
+        print(build_all(force="--force" in sys.argv, verbose=True))

@@ -86,8 +86,11 @@ cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, const
                               int64_t T, int H, const int32_t *cu_seqlens, int n_seqs,
                               void *workspace, cudaStream_t stream);
 
-// Reads and clears the count of bounded waits that gave up (*status: 0 none, 1 some).
+// Reads and clears the device status: *status is a mask of KDA_STATUS_TIMEOUT (a bounded
+// wait gave up) and KDA_STATUS_BAD_INPUT (a KDA_DEBUG build refused device offsets).
 int read_device_status(int *status);
+// Reads and clears the fp32 path's count of refused device offsets (KDA_DEBUG builds).
+int read_simt_bad_input(int *count);
 // Sets the bounded waits' time limit (0: the default of one second).
 int set_wait_limit_ns(unsigned long long ns);
 // Runs the bounded-wait self-test kernel (see kda_selftest_wait_timeout).

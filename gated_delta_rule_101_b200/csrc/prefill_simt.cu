@@ -53,6 +53,10 @@ struct SimtSmem {
     float beta[CH];
 };
 
+// Calls of a KDA_DEBUG build whose device offsets failed the checks (always 0 in the
+// ordinary build); read and cleared with the rest of the device status.
+__device__ int g_simt_bad_input = 0;
+
 template <typename TIn>
 __device__ __forceinline__ void load_row8(const TIn *src, float *dst) {
 #pragma unroll
@@ -71,6 +75,22 @@ prefill_simt_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k,
 
     const int seq = blockIdx.x, h = blockIdx.y, j0 = blockIdx.z * DVS;
     const int tid = threadIdx.x;
+#ifdef KDA_DEBUG
+    // Device offsets of packed sequences are checked by every CTA before any is used
+    // (cu[0] = 0, non-decreasing, cu[n_seqs] = T, with n_seqs = gridDim.x); on failure
+    // the CTA returns without touching the caller's tensors and the first CTA counts
+    // the call in the debug status.
+    if (cu_seqlens) {
+        const int n_seqs = (int)gridDim.x;
+        bool bad = tid == 0 && (cu_seqlens[0] != 0 || (int64_t)cu_seqlens[n_seqs] != T);
+        for (int s2 = tid; s2 < n_seqs; s2 += NT) bad |= cu_seqlens[s2 + 1] < cu_seqlens[s2];
+        if (__syncthreads_or(bad)) {
+            if (tid == 0 && blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0)
+                atomicAdd(&g_simt_bad_input, 1);
+            return;
+        }
+    }
+#endif
     const SeqSpan span = seq_span(cu_seqlens, T, seq);
     const int64_t state_off = ((int64_t)seq * H + h) * (int64_t)(D * D);
 
@@ -283,6 +303,15 @@ cudaError_t launch_prefill_simt(const void *q, const void *k, const void *v,
         return launch_t<float, G>(q, k, v, log_alpha, beta, S0, o, S_T, n_seqs, T, H,
                                   cu_seqlens, stream);
     });
+}
+
+int read_simt_bad_input(int *count) {
+    int v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_simt_bad_input, sizeof(int)) != cudaSuccess) return -1;
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(g_simt_bad_input, &zero, sizeof(int)) != cudaSuccess) return -1;
+    *count = v;
+    return 0;
 }
 
 }  // namespace kda

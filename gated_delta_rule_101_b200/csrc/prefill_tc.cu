@@ -169,12 +169,39 @@ __device__ __forceinline__ bool resolve_slot(int slot, const int32_t *chunk_off,
 // =====================================================================================
 // chunk offsets of packed sequences: chunk_off[s] = sum_{t<s} ceil(len_t / 64)
 // =====================================================================================
+// The workspace of packed inputs starts with n_seqs + 2 int32: the n_seqs + 1 chunk
+// offsets and a validity word, 1 when the offsets may be used. The ordinary build sets
+// it to 1 unconditionally (the device offsets are trusted, or were checked on the host
+// from their host copy). A KDA_DEBUG build checks them here (cu[0] = 0, non-decreasing,
+// cu[n_seqs] = T); if they fail it counts the call in the device status, writes zero
+// chunk offsets and a validity word of 0, and every later kernel of the call returns
+// at entry without reading cu_seqlens, so nothing outside the caller's tensors is
+// touched and no output is written.
+__host__ __device__ constexpr size_t packed_head_bytes(int n_seqs) {
+    return (((size_t)(n_seqs + 2) * 4 + 255) / 256) * 256;
+}
+__device__ __forceinline__ bool packed_offsets_ok(const int32_t *chunk_off, int n_seqs) {
+    return chunk_off[n_seqs + 1] != 0;
+}
+
 __global__ void __launch_bounds__(1024)
-chunk_offsets_kernel(const int32_t *__restrict__ cu, int n_seqs, int32_t *__restrict__ out) {
+chunk_offsets_kernel(const int32_t *__restrict__ cu, int n_seqs, int64_t T, int32_t *__restrict__ out) {
     __shared__ int32_t part[1024];
     const int tid = threadIdx.x;
     const int per = (n_seqs + 1023) / 1024;
     const int s0 = min(tid * per, n_seqs), s1 = min(s0 + per, n_seqs);
+#ifdef KDA_DEBUG
+    bool bad = tid == 0 && (cu[0] != 0 || (int64_t)cu[n_seqs] != T);
+    for (int s = s0; s < s1; ++s) bad |= cu[s + 1] < cu[s];
+    if (__syncthreads_or(bad)) {
+        for (int s = tid; s <= n_seqs; s += 1024) out[s] = 0;
+        if (tid == 0) {
+            out[n_seqs + 1] = 0;
+            atomicAdd(&g_kda_status.bad_input, 1);
+        }
+        return;
+    }
+#endif
     int32_t local = 0;
     for (int s = s0; s < s1; ++s) local += (cu[s + 1] - cu[s] + CH - 1) / CH;
     part[tid] = local;
@@ -190,7 +217,10 @@ chunk_offsets_kernel(const int32_t *__restrict__ cu, int n_seqs, int32_t *__rest
         out[s] = run;
         run += (cu[s + 1] - cu[s] + CH - 1) / CH;
     }
-    if (tid == 1023) out[n_seqs] = part[1023];
+    if (tid == 1023) {
+        out[n_seqs] = part[1023];
+        out[n_seqs + 1] = 1;
+    }
 }
 
 // =====================================================================================
@@ -757,6 +787,7 @@ kda_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     // The chain kernel after this one may start its CTAs (they wait for this grid to
     // complete before reading a blob): they then take SMs as this grid's last CTAs leave.
     griddep_launch_dependents();
+    if (chunk_off && !packed_offsets_ok(chunk_off, n_seqs)) return;
     const int slot = blockIdx.x, h = blockIdx.y;
     int seq, n;
     if (!resolve_slot(slot, chunk_off, n_seqs, nck, seq, n)) return;
@@ -1124,6 +1155,7 @@ kda_chain_kernel(const __grid_constant__ CUtensorMap tm_v,
                  float *__restrict__ S_T, const int32_t *__restrict__ cu, int64_t T, int H,
                  int nck, int wait_prior) {
     extern __shared__ unsigned char smem_raw[];
+    if (chunk_off && !packed_offsets_ok(chunk_off, (int)gridDim.x)) return;
     const ChainArgs a{&tm_v, ws_blobs, chunk_off, S0, o, S_T, cu, T, H, nck, nullptr, wait_prior != 0};
     chain_task<N>(aligned_smem(smem_raw), threadIdx.x, a, blockIdx.x, blockIdx.y, blockIdx.z * N,
                   full_window(a, blockIdx.x, blockIdx.y));
@@ -1557,7 +1589,7 @@ BatchedPlan batched_plan(int B, int H, int nck, int n_sm) {
 
 size_t prefill_tc_workspace(int B, int64_t T, int H, int n_seqs) {
     if (n_seqs > 0) {
-        const size_t head = (((size_t)(n_seqs + 1) * 4 + 255) / 256) * 256;
+        const size_t head = packed_head_bytes(n_seqs);
         const size_t slots = (size_t)(T / CH) + (size_t)n_seqs;
         return head + slots * (size_t)H * BLOB_BYTES;
     }
@@ -1613,9 +1645,9 @@ cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, const
     BatchedPlan plan{0, 0, 0, 0};
     if (packed) {
         chunk_off = reinterpret_cast<int32_t *>(ws);
-        blobs = ws + (((size_t)(n_seqs + 1) * 4 + 255) / 256) * 256;
+        blobs = ws + packed_head_bytes(n_seqs);
         slots = T / CH + n_seqs;
-        chunk_offsets_kernel<<<1, 1024, 0, stream>>>(cu_seqlens, n_seqs, chunk_off);
+        chunk_offsets_kernel<<<1, 1024, 0, stream>>>(cu_seqlens, n_seqs, T, chunk_off);
     } else {
         blobs = ws + batched_head_bytes(B, nck, H);
         plan = n_tok > 0 ? batched_plan(B, H, nck, n_sm) : BatchedPlan{0, 0, 0, 0};
@@ -1698,11 +1730,13 @@ cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, const
 }
 
 int read_device_status(int *status) {
-    ptx::DeviceStatus v{};
-    if (cudaMemcpyFromSymbol(&v, g_kda_status, sizeof(int)) != cudaSuccess) return -1;
-    const int zero = 0;
-    if (cudaMemcpyToSymbol(g_kda_status, &zero, sizeof(int)) != cudaSuccess) return -1;
-    *status = v.timeouts != 0 ? 1 : 0;
+    int v[2] = {0, 0};  // timeouts, bad_input
+    if (cudaMemcpyFromSymbol(v, g_kda_status, sizeof(v)) != cudaSuccess) return -1;
+    const int zero[2] = {0, 0};
+    if (cudaMemcpyToSymbol(g_kda_status, zero, sizeof(zero)) != cudaSuccess) return -1;
+    int simt_bad = 0;
+    if (read_simt_bad_input(&simt_bad) != 0) return -1;
+    *status = (v[0] != 0 ? KDA_STATUS_TIMEOUT : 0) | (v[1] + simt_bad != 0 ? KDA_STATUS_BAD_INPUT : 0);
     return 0;
 }
 

@@ -52,11 +52,13 @@ __device__ __forceinline__ uint64_t global_ns() {
 // Device status shared by the tensor-core kernels of the library.
 //   timeouts:      number of bounded waits that have given up since the host last
 //                  read and cleared it (kda_get_device_status).
+//   bad_input:     number of calls whose device-side sequence offsets failed the
+//                  checks of a KDA_DEBUG build (always 0 in the ordinary build).
 //   wait_limit_ns: how long a wait may take before it gives up (one second; tests of
 //                  the failure path shorten it through kda_set_wait_limit_ns).
 struct DeviceStatus {
     int timeouts;
-    int reserved;
+    int bad_input;
     unsigned long long wait_limit_ns;
 };
 constexpr unsigned long long WAIT_LIMIT_NS = 1000000000ull;  // the default limit: one second

@@ -232,15 +232,31 @@ KDA_API int kda_chunk_fwd_noalloc(const void *q, const void *k, const void *v,
 KDA_API size_t kda_noalloc_scratch_bytes(void);
 
 /*
- * Reads and clears the library's device status. *status is 0 when no kernel
- * has given up on a bounded wait since the last read, 1 otherwise (the
- * outputs of the call that timed out are then invalid; KDA_ERR_TIMEOUT
- * describes it). A timeout that has not been read yet does not affect later
- * calls: a wait gives up early only when another wait gives up while it is
- * waiting, so calls made after the failed one compute normally.
+ * Reads and clears the library's device status. *status is 0 when nothing
+ * has been recorded since the last read, otherwise a mask of:
+ *   KDA_STATUS_TIMEOUT    a kernel gave up on a bounded wait (the outputs of
+ *                         the call that timed out are invalid; KDA_ERR_TIMEOUT
+ *                         describes it);
+ *   KDA_STATUS_BAD_INPUT  a KDA_DEBUG build found device cu_seqlens that
+ *                         break the documented contract (cu_seqlens[0] = 0,
+ *                         non-decreasing, cu_seqlens[n_seqs] = T) and left
+ *                         that call's outputs unwritten.
+ * A timeout that has not been read yet does not affect later calls: a wait
+ * gives up early only when another wait gives up while it is waiting, so
+ * calls made after the failed one compute normally.
  * Synchronises with the device (a blocking symbol copy on the legacy
  * stream); do not call it inside stream capture.
+ *
+ * KDA_DEBUG builds. libkda_debug.so is the same library compiled with
+ * KDA_DEBUG defined. Device offsets passed without a host copy are then
+ * checked on the device before any kernel of the call reads a sequence span:
+ * on failure the call is counted as KDA_STATUS_BAD_INPUT and its kernels
+ * return at entry, so nothing outside the caller's tensors is read or
+ * written. Nothing traps or faults on purpose. The ordinary build trusts
+ * device offsets that come without a host copy.
  */
+#define KDA_STATUS_TIMEOUT 1
+#define KDA_STATUS_BAD_INPUT 2
 KDA_API int kda_get_device_status(int *status);
 
 /*

@@ -72,7 +72,8 @@ def test_noalloc_matches_workspace_entry_point_on_two_calls():
     assert _noalloc_call(junk, jo, js) == kda.KDA_OK
     packed = cu_from_lengths([70, 0, 129, 5])
     cases = [  # (inputs, kernels a workspace call launches: the plan it takes)
-        (prefill_inputs(B=2, T=300, H=3, dtype=torch.bfloat16, s0_std=0.1, seed=101, device=DEV), 2),
+        (prefill_inputs(B=1, T=300, H=72, dtype=torch.bfloat16, s0_std=0.1, seed=101, device=DEV), 2),
+        (prefill_inputs(B=2, T=300, H=3, dtype=torch.bfloat16, s0_std=0.1, seed=105, device=DEV), 1),
         (prefill_inputs(T=int(packed[-1]), H=2, cu_seqlens=packed, dtype=torch.bfloat16,
                         s0_std=0.1, seed=102, device=DEV), 3),
         (prefill_inputs(B=1, T=1000, H=32, dtype=torch.bfloat16, s0_std=0.1, seed=103, device=DEV), 1),
