@@ -397,6 +397,92 @@ def gate_layout_workloads(kda, dev, stream, flush, pk, world, rank):
     return {"gate_layouts": out}
 
 
+def fused_io_workload(kda, dev, stream, flush, pk, world, rank):
+    """The step's shape through kda_chunk_fwd_io with every fused step of the layer:
+    the gate's pre-activation z as bf16 logits (alpha = sigmoid(z)), q and k
+    L2-normalised in the kernel, beta as logits, and the output RMSNorm and sigmoid
+    output gate. Inputs: q, k, v, output gate ~ N(0, 1) bf16 (q, k not normalised),
+    z ~ U(2, 7) bf16, beta logits ~ N(0, 1), RMSNorm weights ~ U(0.5, 1.5),
+    S0 ~ N(0, 0.1^2). Timed like the step (L2 flushed before each call)."""
+    B, T, H = PREFILL["B"], PREFILL["T"], PREFILL["H"]
+    g = torch.Generator(device=dev).manual_seed(PREFILL["seed"] + 77 + 1000 * rank)
+    shape = (B, T, H, 128)
+    bf = lambda: torch.randn(shape, generator=g, device=dev).to(torch.bfloat16)
+    q, k, v, og = bf(), bf(), bf(), bf()
+    z = (torch.rand(shape, generator=g, device=dev) * 5 + 2).to(torch.bfloat16)
+    b = torch.randn((B, T, H), generator=g, device=dev)
+    w = torch.rand(128, generator=g, device=dev) + 0.5
+    S0 = 0.1 * torch.randn((B, H, 128, 128), generator=g, device=dev)
+    ws = torch.empty(kda.workspace_size(B, T, H), dtype=torch.uint8, device=dev)
+    o, S_T = torch.empty_like(v), torch.empty_like(S0)
+
+    def call():
+        kda.chunk_fwd(q, k, v, z, b, S0, out=o, state_out=S_T, workspace=ws, stream=stream,
+                      gate_logits=True, qk_l2norm=True, beta_logits=True, out_gate=og,
+                      out_norm_weight=w)
+
+    barrier(world)
+    times = time_steps(call, 10, 3, stream, flush, name="kda.fused_io")
+    ms = max_over_ranks(sum(times), world, dev) / len(times)
+    # q, k, v, o, output gate and z in bf16, beta fp32; plus S0 and S_T
+    per_tok = 4 * 256 + 256 + 256 + 4
+    alg = per_tok * B * T * H + 2 * STATE_BYTES * B * H
+    # the same layer steps as separate passes: normalise q and k (read + write), log
+    # sigmoid of z (bf16 in, fp32 log_alpha out), sigmoid of beta, the KDA call with an
+    # fp32 gate, then RMSNorm and the output gate (read o and the gate, write o)
+    unfused = (2 * 512 + (256 + 512) + 8 + PREFILL_BYTES_PER_TOKEN_HEAD + 3 * 256) * B * T * H
+    n_l = kda.chunk_fwd_launches(B, T, H, out_epilogue=True)
+    del q, k, v, og, z, b, S0, ws, o, S_T
+    torch.cuda.empty_cache()
+    return {"fused_io": {
+        "value": B * T * world / (ms * 1e-3), "unit": "tokens/s", "ms_per_call": ms,
+        "config": {"workload": f"KDA prefill B={B} T={T} H={H} d=128, bf16, with the layer's gate "
+                               "pre-activation, q/k L2Norm, beta sigmoid, output RMSNorm and sigmoid "
+                               "gate fused", "l2": "flushed before every call"},
+        "roofline": {"bound": "hbm", "achieved": alg / (ms * 1e-3) / 1e9, "peak": pk["hbm_gbs"],
+                     "unit": "GB/s", "frac": alg / (ms * 1e-3) / 1e9 / pk["hbm_gbs"],
+                     "alg_bytes_per_launch": alg},
+        "bytes_per_token_head": per_tok, "unfused_bytes_per_token_head": unfused // (B * T * H),
+        "gpu_launches": n_l * len(times)}}
+
+
+def backward_workload(kda, dev, stream, flush, pk, world, rank):
+    """kda_chunk_bwd on the step's shape (B=4, T=4096, H=16, bf16 inputs, fp32 per-channel
+    gate): the gradients of sum(o * dout) + sum(S_T * dS_T), dout ~ N(0, 1) bf16, dS_T ~
+    N(0, 1). Timed like the step (L2 flushed before each call)."""
+    from gated_delta_rule_101_b200.inputs import prefill_inputs
+
+    B, T, H = PREFILL["B"], PREFILL["T"], PREFILL["H"]
+    inp = prefill_inputs(B=B, T=T, H=H, dtype=torch.bfloat16, s0_std=PREFILL["s0_std"],
+                         la_range=PREFILL["la_range"], seed=PREFILL["seed"] + 2000 + 1000 * rank, device=dev)
+    g = torch.Generator(device=dev).manual_seed(PREFILL["seed"] + 3000 + 1000 * rank)
+    dout = torch.randn(inp.v.shape, generator=g, device=dev).to(torch.bfloat16)
+    dS_T = torch.randn(inp.S0.shape, generator=g, device=dev)
+    ws = torch.empty(kda.bwd_workspace_size(B, T, H), dtype=torch.uint8, device=dev)
+
+    def call():
+        kda.chunk_bwd(inp.q, inp.k, inp.v, inp.log_alpha, inp.beta, inp.S0, dout, dS_T, workspace=ws,
+                      stream=stream)
+
+    barrier(world)
+    times = time_steps(call, 3, 1, stream, flush, name="kda.backward")
+    ms = max_over_ranks(sum(times), world, dev) / len(times)
+    # inputs q, k, v, dout bf16, log_alpha fp32, beta; outputs dq, dk, dv, dlog_alpha fp32,
+    # dbeta; plus S0, dS_T in and dS0 out
+    per_tok = 4 * 256 + 512 + 4 + 4 * 512 + 4
+    alg = per_tok * B * T * H + 3 * STATE_BYTES * B * H
+    del inp, dout, dS_T, ws
+    torch.cuda.empty_cache()
+    return {"backward": {
+        "value": B * T * world / (ms * 1e-3), "unit": "tokens/s", "ms_per_call": ms,
+        "config": {"workload": f"KDA backward (kda_chunk_bwd) B={B} T={T} H={H} d=128, bf16 inputs, "
+                               "fp32 gradients", "l2": "flushed before every call"},
+        "roofline": {"bound": "hbm", "achieved": alg / (ms * 1e-3) / 1e9, "peak": pk["hbm_gbs"],
+                     "unit": "GB/s", "frac": alg / (ms * 1e-3) / 1e9 / pk["hbm_gbs"],
+                     "alg_bytes_per_launch": alg, "kernel": "kda_bwd_slice_kernel + kda_bwd_reduce_kernel"},
+        "gpu_launches": 2 * len(times)}}
+
+
 def run_kda(args, rank, world, local_rank):
     import gated_delta_rule_101_b200 as kda
     from gated_delta_rule_101_b200.inputs import decode_inputs, prefill_inputs
@@ -532,6 +618,8 @@ def run_kda(args, rank, world, local_rank):
     extra = {}
     if not args.no_extra:  # the gate layouts first, next to the step they vary
         extra.update(gate_layout_workloads(kda, dev, stream, flush, pk, world, rank))
+        extra.update(fused_io_workload(kda, dev, stream, flush, pk, world, rank))
+        extra.update(backward_workload(kda, dev, stream, flush, pk, world, rank))
         extra.update(other_prefill_workloads(kda, dev, stream, flush, pk, world, rank))
 
     cpu = None

@@ -10,14 +10,15 @@ namespace {
 constexpr int KDA_VERSION = 100;  // 0.1.0
 
 bool valid_dtype(int dtype) { return dtype == KDA_BF16 || dtype == KDA_F32; }
-bool valid_gate(int gate) { return gate >= KDA_GATE_CHANNEL && gate <= KDA_GATE_NONE; }
+bool valid_gate(int gate) { return gate >= KDA_GATE_CHANNEL && gate <= KDA_GATE_CHANNEL_LOGIT_BF16; }
 
 // The gate tensor is required unless there is no gate; the tensor-core path reads
 // per-channel gates through TMA (16-byte base) and head gates as fp32 scalars.
 int check_gate_ptr(const void *log_alpha, int gate, bool tma) {
     if (gate == KDA_GATE_NONE) return KDA_OK;
     if (!log_alpha) return KDA_ERR_INVALID_ARG;
-    const uintptr_t align = gate == KDA_GATE_HEAD ? 4u : (tma ? 16u : (gate == KDA_GATE_CHANNEL ? 4u : 2u));
+    const bool fp32 = gate == KDA_GATE_CHANNEL || gate == KDA_GATE_CHANNEL_LOGIT;
+    const uintptr_t align = gate == KDA_GATE_HEAD ? 4u : (tma ? 16u : (fp32 ? 4u : 2u));
     return ((uintptr_t)log_alpha & (align - 1)) == 0 ? KDA_OK : KDA_ERR_INVALID_ARG;
 }
 
@@ -31,6 +32,28 @@ int check_prefill_shape(int B, int64_t T, int H, int C, int n_seqs, int dtype) {
     // grid limits: y = H (<= 65535); x = sequences
     if (H > 65535) return KDA_ERR_INVALID_ARG;
     if (T > (int64_t)INT32_MAX) return KDA_ERR_INVALID_ARG;  // offsets are int32
+    return KDA_OK;
+}
+
+// Checks a kda_io and turns it into the kernels' options. `out_ok`: the call supports an
+// output gate; `esize`: bytes per element of the output gate (it has q's dtype).
+int make_io(const kda_io *io, bool out_ok, int esize, kda::IoOpts *opts) {
+    *opts = kda::IoOpts{};
+    if (!io) return KDA_OK;
+    if (!(io->qk_l2norm_eps >= 0.f) || !(io->out_norm_eps >= 0.f)) return KDA_ERR_INVALID_ARG;  // also NaN
+    if (io->qk_l2norm_eps > 1e30f || io->out_norm_eps > 1e30f) return KDA_ERR_INVALID_ARG;
+    opts->flags = (io->qk_l2norm ? kda::IO_QK_L2NORM : 0) | (io->beta_logits ? kda::IO_BETA_LOGITS : 0);
+    opts->l2_eps = io->qk_l2norm_eps;
+    if (io->out_gate) {
+        if (!out_ok) return KDA_ERR_UNSUPPORTED;
+        // the prefill epilogue reads four gate values (8 bytes) per lane, the weights as float4
+        const uintptr_t align = esize == 2 ? 8u : (uintptr_t)esize;
+        if (((uintptr_t)io->out_gate & (align - 1)) != 0) return KDA_ERR_INVALID_ARG;
+        if (io->out_norm_weight && ((uintptr_t)io->out_norm_weight & 15u) != 0) return KDA_ERR_INVALID_ARG;
+        opts->out_gate = io->out_gate;
+        opts->out_w = io->out_norm_weight;
+        opts->out_eps = io->out_norm_eps;
+    }
     return KDA_OK;
 }
 
@@ -65,10 +88,17 @@ int kda_chunk_fwd_workspace_size(int B, int64_t T, int H, int C, int n_seqs, int
 }
 
 int kda_chunk_fwd_launches(int B, int64_t T, int H, int C, int n_seqs, int dtype, int *n_kernels) {
+    return kda_chunk_fwd_io_launches(B, T, H, C, n_seqs, dtype, nullptr, n_kernels);
+}
+
+int kda_chunk_fwd_io_launches(int B, int64_t T, int H, int C, int n_seqs, int dtype, const kda_io *io,
+                              int *n_kernels) {
     if (!n_kernels) return KDA_ERR_INVALID_ARG;
     const int st = check_prefill_shape(B, T, H, C, n_seqs, dtype);
     if (st != KDA_OK) return st;
-    *n_kernels = dtype == KDA_BF16 ? kda::prefill_tc_launches(B, T, H, n_seqs) : 1;
+    const bool out_epi = io && io->out_gate;
+    if (out_epi && dtype != KDA_BF16) return KDA_ERR_UNSUPPORTED;
+    *n_kernels = dtype == KDA_BF16 ? kda::prefill_tc_launches(B, T, H, n_seqs, out_epi) : 1;
     return KDA_OK;
 }
 
@@ -87,9 +117,21 @@ int kda_chunk_fwd_gated(const void *q, const void *k, const void *v, const void 
                         int64_t T, int H, int C, const int32_t *cu_seqlens, int n_seqs,
                         const int32_t *cu_seqlens_host, int dtype, void *workspace,
                         size_t workspace_bytes, void *stream) {
+    return kda_chunk_fwd_io(q, k, v, log_alpha, gate, beta, S0, o, S_T, B, T, H, C, cu_seqlens, n_seqs,
+                            cu_seqlens_host, dtype, workspace, workspace_bytes, nullptr, stream);
+}
+
+int kda_chunk_fwd_io(const void *q, const void *k, const void *v, const void *log_alpha, int gate,
+                     const float *beta, const float *S0, void *o, float *S_T, int B, int64_t T, int H,
+                     int C, const int32_t *cu_seqlens, int n_seqs, const int32_t *cu_seqlens_host,
+                     int dtype, void *workspace, size_t workspace_bytes, const kda_io *io,
+                     void *stream) {
     int st = check_prefill_shape(B, T, H, C, n_seqs, dtype);
     if (st != KDA_OK) return st;
     if (!valid_gate(gate)) return KDA_ERR_UNSUPPORTED;
+    kda::IoOpts opts;
+    st = make_io(io, dtype == KDA_BF16, dtype == KDA_BF16 ? 2 : 4, &opts);
+    if (st != KDA_OK) return st;
     const bool packed = n_seqs > 0;
     if (packed != (cu_seqlens != nullptr)) return KDA_ERR_INVALID_ARG;
     if (T > 0 && (!q || !k || !v || !beta || !o)) return KDA_ERR_INVALID_ARG;
@@ -117,12 +159,61 @@ int kda_chunk_fwd_gated(const void *q, const void *k, const void *v, const void 
         if ((S0 && ((uintptr_t)S0 & 15u)) || (S_T && ((uintptr_t)S_T & 15u)) || ((uintptr_t)o & 15u))
             return KDA_ERR_INVALID_ARG;
         err = kda::launch_prefill_tc(q, k, v, log_alpha, gate, beta, S0, o, S_T, B, T, H,
-                                     cu_seqlens, n_seqs, workspace, s);
+                                     cu_seqlens, n_seqs, workspace, opts, s);
     } else {
         err = kda::launch_prefill_simt(q, k, v, log_alpha, gate, beta, S0, o, S_T, nseq, T, H,
-                                       cu_seqlens, dtype, s);
+                                       cu_seqlens, dtype, opts, s);
     }
     if (err == cudaErrorInvalidValue) return KDA_ERR_INVALID_ARG;
+    return err == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+int kda_chunk_bwd_workspace_size(int B, int64_t T, int H, int n_seqs, size_t *bytes) {
+    if (!bytes) return KDA_ERR_INVALID_ARG;
+    const int st = check_prefill_shape(B, T, H, KDA_CHUNK, n_seqs, KDA_F32);
+    if (st != KDA_OK) return st;
+    const bool packed = n_seqs > 0;
+    const int64_t n_tok = packed ? T : (int64_t)B * T;
+    const int64_t slots = packed ? T / KDA_CHUNK + n_seqs : (int64_t)B * ((T + KDA_CHUNK - 1) / KDA_CHUNK);
+    *bytes = kda::bwd_workspace(n_tok, H, slots);
+    return KDA_OK;
+}
+
+int kda_chunk_bwd(const void *q, const void *k, const void *v, const void *log_alpha, int gate,
+                  const float *beta, const float *S0, const void *dout, const float *dS_T, float *dq,
+                  float *dk, float *dv, float *dgate, float *dbeta, float *dS0, int B, int64_t T, int H,
+                  const int32_t *cu_seqlens, int n_seqs, const int32_t *cu_seqlens_host, int dtype,
+                  const kda_io *io, void *workspace, size_t workspace_bytes, void *stream) {
+    int st = check_prefill_shape(B, T, H, KDA_CHUNK, n_seqs, dtype);
+    if (st != KDA_OK) return st;
+    if (!valid_gate(gate)) return KDA_ERR_UNSUPPORTED;
+    kda::IoOpts opts;
+    st = make_io(io, false, dtype == KDA_BF16 ? 2 : 4, &opts);  // no output epilogue
+    if (st != KDA_OK) return st;
+    const bool packed = n_seqs > 0;
+    if (packed != (cu_seqlens != nullptr)) return KDA_ERR_INVALID_ARG;
+    if (T > 0 && (!q || !k || !v || !beta || !dout || !dq || !dk || !dv || !dbeta))
+        return KDA_ERR_INVALID_ARG;
+    if (T > 0 && gate != KDA_GATE_NONE && !dgate) return KDA_ERR_INVALID_ARG;
+    if (T > 0 && check_gate_ptr(log_alpha, gate, false) != KDA_OK) return KDA_ERR_INVALID_ARG;
+    if (cu_seqlens_host) {
+        if (!packed || cu_seqlens_host[0] != 0 || cu_seqlens_host[n_seqs] != T) return KDA_ERR_INVALID_ARG;
+        for (int s2 = 0; s2 < n_seqs; ++s2)
+            if (cu_seqlens_host[s2 + 1] < cu_seqlens_host[s2]) return KDA_ERR_INVALID_ARG;
+    }
+    size_t need = 0;
+    st = kda_chunk_bwd_workspace_size(B, T, H, n_seqs, &need);
+    if (st != KDA_OK) return st;
+    if (!workspace || workspace_bytes < need || ((uintptr_t)workspace & 15u) != 0) return KDA_ERR_WORKSPACE;
+    kda::BwdArgs a{};
+    a.q = q; a.k = k; a.v = v; a.log_alpha = log_alpha; a.beta = beta; a.S0 = S0; a.dout = dout;
+    a.dS_T = dS_T; a.dq = dq; a.dk = dk; a.dv = dv; a.dgate = dgate; a.dbeta = dbeta; a.dS0 = dS0;
+    a.B = B; a.T = T; a.H = H; a.cu = cu_seqlens; a.n_seqs = n_seqs;
+    a.n_tok = packed ? T : (int64_t)B * T;
+    a.chunk_slots = packed ? T / KDA_CHUNK + n_seqs : (int64_t)B * ((T + KDA_CHUNK - 1) / KDA_CHUNK);
+    a.workspace = workspace;
+    a.io = opts;
+    const cudaError_t err = kda::launch_bwd(a, gate, dtype, (cudaStream_t)stream);
     return err == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 
@@ -152,13 +243,22 @@ int kda_decode_step(const void *q, const void *k, const void *v, const float *lo
 int kda_decode_step_gated(const void *q, const void *k, const void *v, const void *log_alpha,
                           int gate, const float *beta, float *S, void *o, int N, int H,
                           int dtype, void *stream) {
+    return kda_decode_step_io(q, k, v, log_alpha, gate, beta, S, o, N, H, dtype, nullptr, stream);
+}
+
+int kda_decode_step_io(const void *q, const void *k, const void *v, const void *log_alpha, int gate,
+                       const float *beta, float *S, void *o, int N, int H, int dtype, const kda_io *io,
+                       void *stream) {
     if (!valid_dtype(dtype) || !valid_gate(gate)) return KDA_ERR_UNSUPPORTED;
+    kda::IoOpts opts;
+    const int io_st = make_io(io, true, dtype == KDA_BF16 ? 2 : 4, &opts);
+    if (io_st != KDA_OK) return io_st;
     if (N <= 0 || H <= 0) return KDA_ERR_INVALID_ARG;
     if ((int64_t)N * H > (int64_t)INT32_MAX) return KDA_ERR_INVALID_ARG;
     if (!q || !k || !v || !beta || !S || !o) return KDA_ERR_INVALID_ARG;
     if (check_gate_ptr(log_alpha, gate, false) != KDA_OK) return KDA_ERR_INVALID_ARG;
     if (((uintptr_t)S & 15u) != 0) return KDA_ERR_INVALID_ARG;  // 128-bit state accesses
-    const cudaError_t err = kda::launch_decode(q, k, v, log_alpha, gate, beta, S, o, N, H, dtype,
+    const cudaError_t err = kda::launch_decode(q, k, v, log_alpha, gate, beta, S, o, N, H, dtype, opts,
                                                (cudaStream_t)stream);
     return err == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }

@@ -10,6 +10,9 @@
 // so the 64 KiB fp32 state of a head is read once and written once, and the
 // step is bound by HBM bandwidth (0.86 FLOP per byte).
 //
+// Optional fused transformations (IoOpts): q and k L2-normalised, beta given as logits,
+// and the output passed through the head-wise RMSNorm and sigmoid output gate.
+//
 // Layout: one CTA of 256 threads per (sequence, head). Warp w owns state rows
 // 16w .. 16w+15; lane l owns columns 4l .. 4l+3, so every warp access to a row
 // is one contiguous 512-byte segment (float4 per lane). All 16 row loads are
@@ -23,11 +26,23 @@ constexpr int DEC_THREADS = 256;
 constexpr int DEC_WARPS = DEC_THREADS / 32;
 constexpr int ROWS_PER_WARP = D / DEC_WARPS;  // 16
 
+// Sum over the first four warps (the D = 128 threads that hold one channel each) of a
+// value per thread; every one of those threads gets the total. `slot`: 4 floats of
+// shared memory. Called by all threads of the CTA (it contains a barrier).
+__device__ __forceinline__ float sum_channels(float x, float *slot) {
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
+    if (tid < D && lane == 0) slot[warp] = x;
+    __syncthreads();
+    return slot[0] + slot[1] + slot[2] + slot[3];
+}
+
 template <typename TIn, int GATE>
 __global__ void __launch_bounds__(DEC_THREADS)
 decode_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const TIn *__restrict__ v,
               const void *__restrict__ log_alpha, const float *__restrict__ beta,
-              float *__restrict__ S, TIn *__restrict__ o) {
+              float *__restrict__ S, TIn *__restrict__ o, IoOpts io) {
     const int64_t nh = blockIdx.x;  // sequence * H + head
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
@@ -35,6 +50,7 @@ decode_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const TIn *_
     __shared__ float4 s_red[2][DEC_WARPS][D / 4];
     __shared__ float s_delta[D];
     __shared__ float s_qk[4];
+    __shared__ float s_sum[3][4];
 
     float4 *Sp = reinterpret_cast<float4 *>(S + nh * (int64_t)(D * D));
     float4 st[ROWS_PER_WARP];
@@ -42,9 +58,15 @@ decode_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const TIn *_
     for (int rr = 0; rr < ROWS_PER_WARP; ++rr)
         st[rr] = __ldcs(Sp + (warp * ROWS_PER_WARP + rr) * (D / 4) + lane);
 
+    float kk = tid < D ? to_f32(k[nh * D + tid]) : 0.f;
+    float qq = tid < D ? to_f32(q[nh * D + tid]) : 0.f;
+    if (io.flags & IO_QK_L2NORM) {  // uniform over the CTA
+        const float sk = sum_channels(kk * kk, s_sum[0]);
+        const float sq = sum_channels(qq * qq, s_sum[1]);
+        kk *= sk + io.l2_eps > 0.f ? rsqrtf(sk + io.l2_eps) : 0.f;
+        qq *= sq + io.l2_eps > 0.f ? rsqrtf(sq + io.l2_eps) : 0.f;
+    }
     if (tid < D) {
-        const float kk = to_f32(k[nh * D + tid]);
-        const float qq = to_f32(q[nh * D + tid]);
         const float a = GATE == KDA_GATE_NONE ? 1.f : expf(gate_log<GATE>(log_alpha, nh, tid));
         s_k[tid] = kk;
         s_a[tid] = a;
@@ -69,6 +91,7 @@ decode_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const TIn *_
     s_red[1][warp][lane] = p;
     __syncthreads();
 
+    float oj = 0.f;
     if (tid < D) {
         const float *ru = reinterpret_cast<const float *>(&s_red[0][0][0]);
         const float *rp = reinterpret_cast<const float *>(&s_red[1][0][0]);
@@ -78,12 +101,22 @@ decode_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const TIn *_
             uj += ru[w * D + tid];
             pj += rp[w * D + tid];
         }
-        const float b = beta[nh];
+        float b = beta[nh];
+        if (io.flags & IO_BETA_LOGITS) b = sigmoid(b);
         const float d = b * (to_f32(v[nh * D + tid]) - uj);
         s_delta[tid] = d;
         const float qk = s_qk[0] + s_qk[1] + s_qk[2] + s_qk[3];
-        o[nh * D + tid] = from_f32<TIn>(pj + qk * d);
+        oj = pj + qk * d;
     }
+    if (io.out_gate) {  // o <- RMSNorm(o) * w * sigmoid(gate), over the head's 128 channels
+        const float ms = sum_channels(oj * oj, s_sum[2]) * (1.f / D);
+        if (tid < D) {
+            const float w = io.out_w ? io.out_w[tid] : 1.f;
+            const float g = to_f32(static_cast<const TIn *>(io.out_gate)[nh * D + tid]);
+            oj *= rsqrtf(ms + io.out_eps) * w * sigmoid(g);
+        }
+    }
+    if (tid < D) o[nh * D + tid] = from_f32<TIn>(oj);
     __syncthreads();
 
     const float4 d4 = reinterpret_cast<const float4 *>(s_delta)[lane];
@@ -104,18 +137,18 @@ decode_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const TIn *_
 
 cudaError_t launch_decode(const void *q, const void *k, const void *v, const void *log_alpha,
                           int gate, const float *beta, float *S, void *o, int N, int H,
-                          int dtype, cudaStream_t stream) {
+                          int dtype, const IoOpts &io, cudaStream_t stream) {
     const unsigned grid = (unsigned)((int64_t)N * H);
     with_gate(gate, [&](auto g) {
         constexpr int G = decltype(g)::value;
         if (dtype == KDA_BF16) {
             decode_kernel<__nv_bfloat16, G><<<grid, DEC_THREADS, 0, stream>>>(
                 (const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k, (const __nv_bfloat16 *)v,
-                log_alpha, beta, S, (__nv_bfloat16 *)o);
+                log_alpha, beta, S, (__nv_bfloat16 *)o, io);
         } else {
             decode_kernel<float, G><<<grid, DEC_THREADS, 0, stream>>>(
                 (const float *)q, (const float *)k, (const float *)v, log_alpha, beta, S,
-                (float *)o);
+                (float *)o, io);
         }
         return 0;
     });

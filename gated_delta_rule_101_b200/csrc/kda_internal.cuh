@@ -26,6 +26,45 @@ template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(flo
 // Log forget rate of key channel c for token-head row `row` (= token * H + head), in
 // each kda_gate layout: per channel (fp32 or bf16, rows of 128), one per row (a
 // head-wide scalar gate), or none (rate 1, log 0).
+// log sigmoid(z) = min(z, 0) - log(1 + exp(-|z|)), so that nothing overflows; for small
+// x = exp(-|z|) the logarithm is its Taylor series x - x^2 / 2 (relative error below
+// x^2 / 3 < 4e-7), which keeps full relative precision where 1 + x would round to 1.
+__device__ __forceinline__ float log_sigmoid(float z) {
+    const float x = __expf(-fabsf(z));
+    const float l = x < 1e-3f ? x * (1.f - 0.5f * x) : __logf(1.f + x);
+    return fminf(z, 0.f) - l;
+}
+__device__ __forceinline__ float sigmoid(float z) { return 1.f / (1.f + __expf(-z)); }
+
+// Fused input and output transformations of the layer around the operator
+// (blog.gzher.com "Kimi K3论文：Kimi Linear", section 3: q, k = L2Norm(...),
+// beta = Sigmoid(W_beta x), and a head-wise RMSNorm with a sigmoid output gate before
+// the output projection). Flags of IoOpts::flags:
+constexpr int IO_QK_L2NORM = 1;    // q and k rows are L2-normalised in the kernel
+constexpr int IO_BETA_LOGITS = 2;  // beta holds logits: the kernel uses sigmoid(beta)
+struct IoOpts {
+    int flags = 0;
+    float l2_eps = 0.f;             // added to the sum of squares of a q / k row
+    const void *out_gate = nullptr;  // [tokens][H][128] dtype, or null: no output gate and norm
+    const float *out_w = nullptr;    // [128] RMSNorm weight, or null for ones
+    float out_eps = 0.f;             // added to the mean square of an output row
+};
+
+// Per-channel gate layouts (one value per key channel, fp32 or bf16): log rates or logits.
+template <int GATE>
+constexpr bool per_channel_gate() {
+    return GATE == KDA_GATE_CHANNEL || GATE == KDA_GATE_CHANNEL_BF16 || GATE == KDA_GATE_CHANNEL_LOGIT ||
+           GATE == KDA_GATE_CHANNEL_LOGIT_BF16;
+}
+template <int GATE>
+constexpr bool bf16_gate() {
+    return GATE == KDA_GATE_CHANNEL_BF16 || GATE == KDA_GATE_CHANNEL_LOGIT_BF16;
+}
+template <int GATE>
+constexpr bool logit_gate() {
+    return GATE == KDA_GATE_CHANNEL_LOGIT || GATE == KDA_GATE_CHANNEL_LOGIT_BF16;
+}
+
 template <int GATE>
 __device__ __forceinline__ float gate_log(const void *la, int64_t row, int c) {
     if constexpr (GATE == KDA_GATE_CHANNEL) {
@@ -34,6 +73,10 @@ __device__ __forceinline__ float gate_log(const void *la, int64_t row, int c) {
         return __bfloat162float(static_cast<const __nv_bfloat16 *>(la)[row * D + c]);
     } else if constexpr (GATE == KDA_GATE_HEAD) {
         return static_cast<const float *>(la)[row];
+    } else if constexpr (GATE == KDA_GATE_CHANNEL_LOGIT) {
+        return log_sigmoid(static_cast<const float *>(la)[row * D + c]);
+    } else if constexpr (GATE == KDA_GATE_CHANNEL_LOGIT_BF16) {
+        return log_sigmoid(__bfloat162float(static_cast<const __nv_bfloat16 *>(la)[row * D + c]));
     } else {
         return 0.f;
     }
@@ -47,6 +90,8 @@ auto with_gate(int gate, F &&f) {
     case KDA_GATE_CHANNEL_BF16: return f(std::integral_constant<int, KDA_GATE_CHANNEL_BF16>{});
     case KDA_GATE_HEAD: return f(std::integral_constant<int, KDA_GATE_HEAD>{});
     case KDA_GATE_NONE: return f(std::integral_constant<int, KDA_GATE_NONE>{});
+    case KDA_GATE_CHANNEL_LOGIT: return f(std::integral_constant<int, KDA_GATE_CHANNEL_LOGIT>{});
+    case KDA_GATE_CHANNEL_LOGIT_BF16: return f(std::integral_constant<int, KDA_GATE_CHANNEL_LOGIT_BF16>{});
     default: return f(std::integral_constant<int, KDA_GATE_CHANNEL>{});
     }
 }
@@ -71,20 +116,42 @@ __device__ __forceinline__ SeqSpan seq_span(const int32_t *cu, int64_t T, int s)
 // ---- launchers (host side); each returns cudaGetLastError() of its launch ----
 cudaError_t launch_decode(const void *q, const void *k, const void *v, const void *log_alpha,
                           int gate, const float *beta, float *S, void *o, int N, int H,
-                          int dtype, cudaStream_t stream);
+                          int dtype, const IoOpts &io, cudaStream_t stream);
 
 cudaError_t launch_prefill_simt(const void *q, const void *k, const void *v,
                                 const void *log_alpha, int gate, const float *beta, const float *S0,
                                 void *o, float *S_T, int n_seqs, int64_t T, int H,
-                                const int32_t *cu_seqlens, int dtype, cudaStream_t stream);
+                                const int32_t *cu_seqlens, int dtype, const IoOpts &io,
+                                cudaStream_t stream);
 
 // Tensor-core prefill (bf16 q/k/v): workspace bytes and launcher.
 size_t prefill_tc_workspace(int B, int64_t T, int H, int n_seqs);
-int prefill_tc_launches(int B, int64_t T, int H, int n_seqs);
+// out_epilogue: the call applies an output gate and norm (runs prep and the full-head chain).
+int prefill_tc_launches(int B, int64_t T, int H, int n_seqs, bool out_epilogue = false);
 cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, const void *log_alpha,
                               int gate, const float *beta, const float *S0, void *o, float *S_T, int B,
                               int64_t T, int H, const int32_t *cu_seqlens, int n_seqs,
-                              void *workspace, cudaStream_t stream);
+                              void *workspace, const IoOpts &io, cudaStream_t stream);
+
+// Backward pass (kda_chunk_bwd): arguments of one call.
+struct BwdArgs {
+    const void *q, *k, *v, *log_alpha;
+    const float *beta, *S0;
+    const void *dout;
+    const float *dS_T;
+    float *dq, *dk, *dv, *dgate, *dbeta, *dS0;
+    int B;
+    int64_t T;
+    int H;
+    const int32_t *cu;
+    int n_seqs;
+    int64_t n_tok;        // tokens in all (B * T, or T packed)
+    int64_t chunk_slots;  // chunks in all (B * ceil(T / 64), or T / 64 + n_seqs packed)
+    void *workspace;
+    IoOpts io;
+};
+size_t bwd_workspace(int64_t n_tok, int H, int64_t chunk_slots);
+cudaError_t launch_bwd(const BwdArgs &a, int gate, int dtype, cudaStream_t stream);
 
 // Reads and clears the device status: *status is a mask of KDA_STATUS_TIMEOUT (a bounded
 // wait gave up) and KDA_STATUS_BAD_INPUT (a KDA_DEBUG build refused device offsets).

@@ -69,7 +69,7 @@ prefill_simt_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k,
                     const TIn *__restrict__ v, const void *__restrict__ log_alpha,
                     const float *__restrict__ beta, const float *__restrict__ S0,
                     TIn *__restrict__ o, float *__restrict__ S_T, int64_t T, int H,
-                    const int32_t *__restrict__ cu_seqlens) {
+                    const int32_t *__restrict__ cu_seqlens, int io_flags, float l2_eps) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     SimtSmem &sm = *reinterpret_cast<SimtSmem *>(smem_raw);
 
@@ -123,8 +123,34 @@ prefill_simt_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k,
             const int r = e / DVS, j = e % DVS;
             sm.vu[e] = r < L ? to_f32(v[((tok0 + r) * H + h) * (int64_t)D + j0 + j]) : 0.f;
         }
-        if (tid < CH) sm.beta[tid] = tid < L ? beta[(tok0 + tid) * H + h] : 0.f;
+        if (tid < CH) {
+            float b = tid < L ? beta[(tok0 + tid) * H + h] : 0.f;
+            if ((io_flags & IO_BETA_LOGITS) && tid < L) b = sigmoid(b);
+            sm.beta[tid] = b;
+        }
         __syncthreads();
+        if (io_flags & IO_QK_L2NORM) {  // q and k rows to unit length (rows >= L stay zero)
+            const int warp = tid >> 5, lane = tid & 31;
+            for (int r = warp; r < CH; r += NT / 32) {
+                float sq = 0.f, sk = 0.f;
+                for (int c = lane; c < D; c += 32) {
+                    sq += sm.q[r * LD + c] * sm.q[r * LD + c];
+                    sk += sm.k[r * LD + c] * sm.k[r * LD + c];
+                }
+#pragma unroll
+                for (int off = 16; off > 0; off >>= 1) {
+                    sq += __shfl_xor_sync(0xffffffffu, sq, off);
+                    sk += __shfl_xor_sync(0xffffffffu, sk, off);
+                }
+                const float nq = sq + l2_eps > 0.f ? rsqrtf(sq + l2_eps) : 0.f;
+                const float nk = sk + l2_eps > 0.f ? rsqrtf(sk + l2_eps) : 0.f;
+                for (int c = lane; c < D; c += 32) {
+                    sm.q[r * LD + c] *= nq;
+                    sm.k[r * LD + c] *= nk;
+                }
+            }
+            __syncthreads();
+        }
 
         // ---- g = chunk-local inclusive cumulative sum of log_alpha, per channel
         bool unsafe = false;
@@ -277,14 +303,15 @@ prefill_simt_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k,
 template <typename TIn, int GATE>
 cudaError_t launch_t(const void *q, const void *k, const void *v, const void *la,
                      const float *beta, const float *S0, void *o, float *S_T, int n_seqs,
-                     int64_t T, int H, const int32_t *cu, cudaStream_t stream) {
+                     int64_t T, int H, const int32_t *cu, const IoOpts &io, cudaStream_t stream) {
     const size_t smem = sizeof(SimtSmem);
     cudaError_t err = cudaFuncSetAttribute(prefill_simt_kernel<TIn, GATE>,
                                            cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (err != cudaSuccess) return err;
     dim3 grid((unsigned)n_seqs, (unsigned)H, D / DVS);
     prefill_simt_kernel<TIn, GATE><<<grid, NT, smem, stream>>>(
-        (const TIn *)q, (const TIn *)k, (const TIn *)v, la, beta, S0, (TIn *)o, S_T, T, H, cu);
+        (const TIn *)q, (const TIn *)k, (const TIn *)v, la, beta, S0, (TIn *)o, S_T, T, H, cu, io.flags,
+        io.l2_eps);
     return cudaGetLastError();
 }
 
@@ -293,15 +320,15 @@ cudaError_t launch_t(const void *q, const void *k, const void *v, const void *la
 cudaError_t launch_prefill_simt(const void *q, const void *k, const void *v,
                                 const void *log_alpha, int gate, const float *beta,
                                 const float *S0, void *o, float *S_T, int n_seqs, int64_t T,
-                                int H, const int32_t *cu_seqlens, int dtype,
+                                int H, const int32_t *cu_seqlens, int dtype, const IoOpts &io,
                                 cudaStream_t stream) {
     return with_gate(gate, [&](auto g) {
         constexpr int G = decltype(g)::value;
         if (dtype == KDA_BF16)
             return launch_t<__nv_bfloat16, G>(q, k, v, log_alpha, beta, S0, o, S_T, n_seqs, T, H,
-                                              cu_seqlens, stream);
+                                              cu_seqlens, io, stream);
         return launch_t<float, G>(q, k, v, log_alpha, beta, S0, o, S_T, n_seqs, T, H,
-                                  cu_seqlens, stream);
+                                  cu_seqlens, io, stream);
     });
 }
 

@@ -77,7 +77,13 @@ typedef enum kda_gate {
     KDA_GATE_CHANNEL = 0,      /* fp32 [token][head][128]: one rate per key channel (KDA) */
     KDA_GATE_CHANNEL_BF16 = 1, /* the same, bfloat16 */
     KDA_GATE_HEAD = 2,         /* fp32 [token][head]: one rate per head (Gated DeltaNet) */
-    KDA_GATE_NONE = 3          /* no gate, alpha = 1 (DeltaNet); log_alpha is not read */
+    KDA_GATE_NONE = 3,         /* no gate, alpha = 1 (DeltaNet); log_alpha is not read */
+    /* The gate's pre-activation z (the output of the gate's low-rank projection,
+     * section 3: alpha_t = f(W_up W_down x_t)), with f = sigmoid: alpha = sigmoid(z),
+     * so the kernels use log alpha = log sigmoid(z) = -log(1 + exp(-z)). The page
+     * leaves f open; sigmoid is the plainest map onto [0, 1]. z is any finite value. */
+    KDA_GATE_CHANNEL_LOGIT = 4,     /* fp32 [token][head][128] */
+    KDA_GATE_CHANNEL_LOGIT_BF16 = 5 /* the same, bfloat16 */
 } kda_gate;
 
 typedef enum kda_status {
@@ -172,6 +178,90 @@ KDA_API int kda_chunk_fwd_gated(const void *q, const void *k, const void *v,
                                 size_t workspace_bytes, void *stream);
 
 /*
+ * Fused input and output transformations (blog.gzher.com "Kimi K3论文：Kimi
+ * Linear", section 3, the neural parameterisation around the operator):
+ *   q_t, k_t = L2Norm(...),  beta_t = Sigmoid(W_beta x_t),
+ * and before the output projection a head-wise RMSNorm and a data-dependent
+ * sigmoid output gate. The section does not write the epilogue as a formula;
+ * the reading taken is, per (token, head) row o of 128 values,
+ *   o <- o / sqrt(mean(o^2) + out_norm_eps) * w * sigmoid(out_gate),
+ * with w the norm's weight. A zero field leaves that step out:
+ *   qk_l2norm        nonzero: q and k rows (128 channels) are divided by
+ *                    sqrt(sum of squares + qk_l2norm_eps) inside the kernels
+ *                    (a row whose sum plus eps is 0 becomes 0); the inputs then
+ *                    need not be normalised
+ *   beta_logits      nonzero: beta holds logits, the kernels use sigmoid(beta)
+ *   out_gate         NULL, or the gate's input, shaped like o ([B, T, H, 128] or
+ *                    [N, H, 128], q's dtype; 8-byte aligned for bf16): applies
+ *                    the output epilogue above to o
+ *   out_norm_weight  [128] fp32, 16-byte aligned, or NULL for ones
+ * eps values must be finite and >= 0. The gate's own pre-activation is a gate
+ * layout (KDA_GATE_CHANNEL_LOGIT*), not a field here.
+ */
+typedef struct kda_io {
+    int qk_l2norm;
+    float qk_l2norm_eps;
+    int beta_logits;
+    const void *out_gate;
+    const float *out_norm_weight;
+    float out_norm_eps;
+} kda_io;
+
+/*
+ * kda_chunk_fwd_gated with the fused transformations of `io` (NULL: none, which
+ * is kda_chunk_fwd_gated itself). The output epilogue is available for bf16
+ * inputs (the fp32 path returns KDA_ERR_UNSUPPORTED for out_gate != NULL); it
+ * runs the prep kernel and a chain kernel that holds whole output rows (one
+ * CTA per sequence-head), whatever plan the call would otherwise take, in the
+ * same workspace. The other fields work on every path.
+ */
+KDA_API int kda_chunk_fwd_io(const void *q, const void *k, const void *v, const void *log_alpha,
+                             int gate, const float *beta, const float *S0, void *o, float *S_T,
+                             int B, int64_t T, int H, int C, const int32_t *cu_seqlens, int n_seqs,
+                             const int32_t *cu_seqlens_host, int dtype, void *workspace,
+                             size_t workspace_bytes, const kda_io *io, void *stream);
+
+/* kda_chunk_fwd_launches for a kda_chunk_fwd_io call with these options. */
+KDA_API int kda_chunk_fwd_io_launches(int B, int64_t T, int H, int C, int n_seqs, int dtype,
+                                      const kda_io *io, int *n_kernels);
+
+/*
+ * Backward pass of kda_chunk_fwd (training): the gradients of
+ *   L = sum(o * dout) + sum(S_T * dS_T)
+ * with respect to every input, for given dout (and dS_T). The recurrence of eq. (1)
+ * (section 3) is differentiated token by token in reverse (section 4 of the same
+ * page counts the training cost of the chunked form; these are the same
+ * gradients). All arithmetic is fp32 on CUDA cores, for both dtypes.
+ *
+ *   q, k, v, log_alpha, gate, beta, S0, B, T, H, cu_seqlens, n_seqs,
+ *   cu_seqlens_host, dtype, io: as for kda_chunk_fwd_io (io->out_gate must be
+ *              NULL: the output epilogue has no backward here)
+ *   dout       like o (dtype): dL/do
+ *   dS_T       [Nseq, H, 128, 128] fp32: dL/dS_T, or NULL for zeros
+ *   dq, dk, dv [.., H, 128] fp32 (written): dL/dq, dL/dk, dL/dv (with io->qk_l2norm,
+ *              the gradients of the un-normalised q and k)
+ *   dgate      the gate's gradient (written), fp32, in its layout's shape:
+ *              [.., H, 128] for per-channel layouts (dL/dlog_alpha, or dL/dz for
+ *              the logit layouts), [.., H] for KDA_GATE_HEAD; not written (may be
+ *              NULL) for KDA_GATE_NONE
+ *   dbeta      [.., H] fp32 (written): dL/dbeta (dL/d logit with io->beta_logits)
+ *   dS0        [Nseq, H, 128, 128] fp32 (written), or NULL: dL/dS0
+ *   workspace  device buffer of kda_chunk_bwd_workspace_size bytes, 16-byte
+ *              aligned. It holds each token's per-slice gradient shares (6.2 KB
+ *              per token-head), the state at every chunk start (64 KB per
+ *              chunk-head) and a replay scratch of 256 x 1 MiB.
+ * The call launches two kernels; the result is bitwise reproducible.
+ * Concurrent calls must not share a workspace.
+ */
+KDA_API int kda_chunk_bwd_workspace_size(int B, int64_t T, int H, int n_seqs, size_t *bytes);
+KDA_API int kda_chunk_bwd(const void *q, const void *k, const void *v, const void *log_alpha, int gate,
+                          const float *beta, const float *S0, const void *dout, const float *dS_T,
+                          float *dq, float *dk, float *dv, float *dgate, float *dbeta, float *dS0,
+                          int B, int64_t T, int H, const int32_t *cu_seqlens, int n_seqs,
+                          const int32_t *cu_seqlens_host, int dtype, const kda_io *io,
+                          void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * One recurrent decode step for N sequences (eq. (1) applied to one token;
  * blog.gzher.com section 4: decode uses the recurrent kernel).
  *
@@ -192,6 +282,11 @@ KDA_API int kda_decode_step(const void *q, const void *k, const void *v, const f
 KDA_API int kda_decode_step_gated(const void *q, const void *k, const void *v,
                                   const void *log_alpha, int gate, const float *beta, float *S,
                                   void *o, int N, int H, int dtype, void *stream);
+
+/* kda_decode_step_gated with the fused transformations of `io` (NULL: none). */
+KDA_API int kda_decode_step_io(const void *q, const void *k, const void *v, const void *log_alpha,
+                               int gate, const float *beta, float *S, void *o, int N, int H,
+                               int dtype, const kda_io *io, void *stream);
 
 /*
  * kda_chunk_fwd for callers that cannot allocate device memory. The pages

@@ -124,9 +124,10 @@ def test_gated_entry_points_validate_the_gate(lib):
         return lib.kda_decode_step_gated(FAKE, FAKE, FAKE, la, gate, FAKE, FAKE, FAKE, 4, 2, BF16,
                                          None)
 
-    for bad in (-1, 4, 99):
+    for bad in (-1, 6, 99):
         assert chunk(bad) == UNSUPPORTED and decode(bad) == UNSUPPORTED
-    for gate in (G.KDA_GATE_CHANNEL, G.KDA_GATE_CHANNEL_BF16, G.KDA_GATE_HEAD):
+    for gate in (G.KDA_GATE_CHANNEL, G.KDA_GATE_CHANNEL_BF16, G.KDA_GATE_HEAD,
+                 G.KDA_GATE_CHANNEL_LOGIT, G.KDA_GATE_CHANNEL_LOGIT_BF16):
         assert chunk(gate, la=None) == INVALID and decode(gate, la=None) == INVALID
     # no gate: log_alpha is not needed (validation goes on to the missing workspace)
     assert chunk(G.KDA_GATE_NONE, la=None) == WORKSPACE
@@ -134,6 +135,8 @@ def test_gated_entry_points_validate_the_gate(lib):
     off8, off2 = ctypes.c_void_p((1 << 20) + 8), ctypes.c_void_p((1 << 20) + 2)
     assert chunk(G.KDA_GATE_CHANNEL, la=off8) == INVALID
     assert chunk(G.KDA_GATE_CHANNEL_BF16, la=off8) == INVALID
+    assert chunk(G.KDA_GATE_CHANNEL_LOGIT, la=off8) == INVALID
+    assert chunk(G.KDA_GATE_CHANNEL_LOGIT_BF16, la=off8) == INVALID
     assert chunk(G.KDA_GATE_HEAD, la=off8) == WORKSPACE
     assert chunk(G.KDA_GATE_HEAD, la=off2) == INVALID
     assert decode(G.KDA_GATE_HEAD, la=off2) == INVALID
@@ -165,3 +168,57 @@ def test_wait_selftest_rejects_bad_pointers(lib):
     assert lib.kda_selftest_wait_timeout(FAKE, None, None) == INVALID
     assert lib.kda_selftest_wait_timeout(ctypes.c_void_p((1 << 20) + 2), FAKE, None) == INVALID
     assert lib.kda_selftest_wait_timeout(FAKE, ctypes.c_void_p((1 << 20) + 1), None) == INVALID
+
+
+def test_io_entry_points_validate_their_options(lib):
+    """kda_chunk_fwd_io / kda_decode_step_io check the fused options before launching."""
+    Io = kda.KdaIo
+
+    def chunk(io, dtype=BF16, gate=kda.KDA_GATE_CHANNEL):
+        return lib.kda_chunk_fwd_io(FAKE, FAKE, FAKE, FAKE, gate, FAKE, None, FAKE, None, 1, 128, 2, 64,
+                                    None, 0, None, dtype, None, 0, ctypes.byref(io), None)
+
+    def decode(io):
+        return lib.kda_decode_step_io(FAKE, FAKE, FAKE, FAKE, kda.KDA_GATE_CHANNEL, FAKE, FAKE, FAKE, 4, 2,
+                                      BF16, ctypes.byref(io), None)
+
+    gate16 = (1 << 20)
+    assert chunk(Io(1, -1.0, 0, None, None, 0.0)) == INVALID            # negative eps
+    assert chunk(Io(1, float("nan"), 0, None, None, 0.0)) == INVALID   # NaN eps
+    assert chunk(Io(0, 0.0, 0, gate16, None, -1.0)) == INVALID          # negative output eps
+    assert chunk(Io(0, 0.0, 0, gate16, None, 1e-6), dtype=F32) == UNSUPPORTED  # fp32: no epilogue
+    assert chunk(Io(0, 0.0, 0, gate16 + 2, None, 1e-6)) == INVALID     # bf16 gate: 8-byte aligned
+    assert chunk(Io(0, 0.0, 0, gate16, gate16 + 4, 1e-6)) == INVALID    # weights: 16-byte aligned
+    assert decode(Io(1, -1.0, 0, None, None, 0.0)) == INVALID
+    assert decode(Io(0, 0.0, 0, gate16 + 2, None, 1e-6)) == INVALID
+    # valid options go on to the next check (the missing workspace)
+    assert chunk(Io(1, 1e-6, 1, gate16, gate16, 1e-6)) == WORKSPACE
+    n = ctypes.c_int(0)
+    assert lib.kda_chunk_fwd_io_launches(1, 128, 2, 64, 0, F32, ctypes.byref(Io(0, 0.0, 0, gate16, None, 0.0)),
+                                         ctypes.byref(n)) == UNSUPPORTED
+
+
+def test_backward_validates_before_launching(lib):
+    def bwd(**kw):
+        a = dict(q=FAKE, k=FAKE, v=FAKE, la=FAKE, gate=kda.KDA_GATE_CHANNEL, beta=FAKE, S0=None, do=FAKE,
+                 dST=None, dq=FAKE, dk=FAKE, dv=FAKE, dg=FAKE, db=FAKE, dS0=None, B=1, T=128, H=2,
+                 cu=None, n=0, cuh=None, dtype=BF16, io=None, ws=None, wsb=0)
+        a.update(kw)
+        return lib.kda_chunk_bwd(a["q"], a["k"], a["v"], a["la"], a["gate"], a["beta"], a["S0"], a["do"],
+                                 a["dST"], a["dq"], a["dk"], a["dv"], a["dg"], a["db"], a["dS0"], a["B"],
+                                 a["T"], a["H"], a["cu"], a["n"], a["cuh"], a["dtype"], a["io"], a["ws"],
+                                 a["wsb"], None)
+
+    for field in ("q", "k", "v", "beta", "do", "dq", "dk", "dv", "db", "dg"):
+        assert bwd(**{field: None}) == INVALID, field
+    assert bwd(gate=kda.KDA_GATE_NONE, dg=None) == WORKSPACE  # no gate: no gate gradient needed
+    assert bwd(gate=9) == UNSUPPORTED
+    assert bwd(dtype=5) == UNSUPPORTED
+    assert bwd(B=0) == INVALID
+    io = kda.KdaIo(0, 0.0, 0, 1 << 20, None, 1e-6)  # the output epilogue has no backward
+    assert bwd(io=ctypes.byref(io)) == UNSUPPORTED
+    assert bwd() == WORKSPACE
+    n = ctypes.c_size_t(0)
+    assert lib.kda_chunk_bwd_workspace_size(4, 4096, 16, 0, ctypes.byref(n)) == 0
+    # slot words, shares 6.2 KB per token-head, 64 KB per chunk-head, 256 MiB replay scratch
+    assert n.value == (256 + 4 * 4096 * 16 * 4 * 385 + 4 * 64 * 16 * 4 * 4096 + 256 * 64 * 4096) * 4
