@@ -46,8 +46,8 @@ int make_io(const kda_io *io, bool out_ok, int esize, kda::IoOpts *opts) {
     opts->l2_eps = io->qk_l2norm_eps;
     if (io->out_gate) {
         if (!out_ok) return KDA_ERR_UNSUPPORTED;
-        // the prefill epilogue reads four gate values (8 bytes) per lane, the weights as float4
-        const uintptr_t align = esize == 2 ? 8u : (uintptr_t)esize;
+        // the prefill epilogue reads eight gate values (16 bytes) per lane, the weights as float4
+        const uintptr_t align = esize == 2 ? 16u : (uintptr_t)esize;
         if (((uintptr_t)io->out_gate & (align - 1)) != 0) return KDA_ERR_INVALID_ARG;
         if (io->out_norm_weight && ((uintptr_t)io->out_norm_weight & 15u) != 0) return KDA_ERR_INVALID_ARG;
         opts->out_gate = io->out_gate;
@@ -98,7 +98,7 @@ int kda_chunk_fwd_io_launches(int B, int64_t T, int H, int C, int n_seqs, int dt
     if (st != KDA_OK) return st;
     const bool out_epi = io && io->out_gate;
     if (out_epi && dtype != KDA_BF16) return KDA_ERR_UNSUPPORTED;
-    *n_kernels = dtype == KDA_BF16 ? kda::prefill_tc_launches(B, T, H, n_seqs, out_epi) : 1;
+    *n_kernels = dtype == KDA_BF16 ? kda::prefill_tc_launches(B, T, H, n_seqs, out_epi, io && io->qk_l2norm) : 1;
     return KDA_OK;
 }
 

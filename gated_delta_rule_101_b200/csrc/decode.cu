@@ -38,7 +38,9 @@ __device__ __forceinline__ float sum_channels(float x, float *slot) {
     return slot[0] + slot[1] + slot[2] + slot[3];
 }
 
-template <typename TIn, int GATE>
+// IO: the call has fused transformations (io); a template parameter, so that the plain
+// step carries none of their code.
+template <typename TIn, int GATE, bool IO>
 __global__ void __launch_bounds__(DEC_THREADS)
 decode_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const TIn *__restrict__ v,
               const void *__restrict__ log_alpha, const float *__restrict__ beta,
@@ -58,15 +60,22 @@ decode_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const TIn *_
     for (int rr = 0; rr < ROWS_PER_WARP; ++rr)
         st[rr] = __ldcs(Sp + (warp * ROWS_PER_WARP + rr) * (D / 4) + lane);
 
-    float kk = tid < D ? to_f32(k[nh * D + tid]) : 0.f;
-    float qq = tid < D ? to_f32(q[nh * D + tid]) : 0.f;
-    if (io.flags & IO_QK_L2NORM) {  // uniform over the CTA
-        const float sk = sum_channels(kk * kk, s_sum[0]);
-        const float sq = sum_channels(qq * qq, s_sum[1]);
-        kk *= sk + io.l2_eps > 0.f ? rsqrtf(sk + io.l2_eps) : 0.f;
-        qq *= sq + io.l2_eps > 0.f ? rsqrtf(sq + io.l2_eps) : 0.f;
+    float kk = 0.f, qq = 0.f;
+    if constexpr (IO) {
+        kk = tid < D ? to_f32(k[nh * D + tid]) : 0.f;
+        qq = tid < D ? to_f32(q[nh * D + tid]) : 0.f;
+        if (io.flags & IO_QK_L2NORM) {  // uniform over the CTA
+            const float sk = sum_channels(kk * kk, s_sum[0]);
+            const float sq = sum_channels(qq * qq, s_sum[1]);
+            kk *= sk + io.l2_eps > 0.f ? rsqrtf(sk + io.l2_eps) : 0.f;
+            qq *= sq + io.l2_eps > 0.f ? rsqrtf(sq + io.l2_eps) : 0.f;
+        }
     }
     if (tid < D) {
+        if constexpr (!IO) {
+            kk = to_f32(k[nh * D + tid]);
+            qq = to_f32(q[nh * D + tid]);
+        }
         const float a = GATE == KDA_GATE_NONE ? 1.f : expf(gate_log<GATE>(log_alpha, nh, tid));
         s_k[tid] = kk;
         s_a[tid] = a;
@@ -102,13 +111,13 @@ decode_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const TIn *_
             pj += rp[w * D + tid];
         }
         float b = beta[nh];
-        if (io.flags & IO_BETA_LOGITS) b = sigmoid(b);
+        if (IO && (io.flags & IO_BETA_LOGITS)) b = sigmoid(b);
         const float d = b * (to_f32(v[nh * D + tid]) - uj);
         s_delta[tid] = d;
         const float qk = s_qk[0] + s_qk[1] + s_qk[2] + s_qk[3];
         oj = pj + qk * d;
     }
-    if (io.out_gate) {  // o <- RMSNorm(o) * w * sigmoid(gate), over the head's 128 channels
+    if (IO && io.out_gate) {  // o <- RMSNorm(o) * w * sigmoid(gate), over the head's 128 channels
         const float ms = sum_channels(oj * oj, s_sum[2]) * (1.f / D);
         if (tid < D) {
             const float w = io.out_w ? io.out_w[tid] : 1.f;
@@ -139,16 +148,20 @@ cudaError_t launch_decode(const void *q, const void *k, const void *v, const voi
                           int gate, const float *beta, float *S, void *o, int N, int H,
                           int dtype, const IoOpts &io, cudaStream_t stream) {
     const unsigned grid = (unsigned)((int64_t)N * H);
+    const bool has_io = io.flags != 0 || io.out_gate != nullptr;
     with_gate(gate, [&](auto g) {
         constexpr int G = decltype(g)::value;
+        auto run = [&](auto kernel, auto tin) {
+            using TIn = decltype(tin);
+            kernel<<<grid, DEC_THREADS, 0, stream>>>((const TIn *)q, (const TIn *)k, (const TIn *)v, log_alpha,
+                                                     beta, S, (TIn *)o, io);
+        };
         if (dtype == KDA_BF16) {
-            decode_kernel<__nv_bfloat16, G><<<grid, DEC_THREADS, 0, stream>>>(
-                (const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k, (const __nv_bfloat16 *)v,
-                log_alpha, beta, S, (__nv_bfloat16 *)o, io);
+            if (has_io) run(decode_kernel<__nv_bfloat16, G, true>, __nv_bfloat16{});
+            else run(decode_kernel<__nv_bfloat16, G, false>, __nv_bfloat16{});
         } else {
-            decode_kernel<float, G><<<grid, DEC_THREADS, 0, stream>>>(
-                (const float *)q, (const float *)k, (const float *)v, log_alpha, beta, S,
-                (float *)o, io);
+            if (has_io) run(decode_kernel<float, G, true>, float{});
+            else run(decode_kernel<float, G, false>, float{});
         }
         return 0;
     });

@@ -126,8 +126,9 @@ cudaError_t launch_prefill_simt(const void *q, const void *k, const void *v,
 
 // Tensor-core prefill (bf16 q/k/v): workspace bytes and launcher.
 size_t prefill_tc_workspace(int B, int64_t T, int H, int n_seqs);
-// out_epilogue: the call applies an output gate and norm (runs prep and the full-head chain).
-int prefill_tc_launches(int B, int64_t T, int H, int n_seqs, bool out_epilogue = false);
+// out_epilogue: the call applies an output gate and norm (runs prep and the full-head chain);
+// l2norm: q and k are normalised in the kernel (no fused grid).
+int prefill_tc_launches(int B, int64_t T, int H, int n_seqs, bool out_epilogue = false, bool l2norm = false);
 cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, const void *log_alpha,
                               int gate, const float *beta, const float *S0, void *o, float *S_T, int B,
                               int64_t T, int H, const int32_t *cu_seqlens, int n_seqs,

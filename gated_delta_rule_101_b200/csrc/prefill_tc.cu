@@ -358,7 +358,9 @@ struct NoHook {
     __device__ __forceinline__ void before_wait() {}
     __device__ __forceinline__ void after_wait() {}
 };
-template <int GATE, class Worker, class Prefetch, class Hook = NoHook>
+// L2: q and k rows are L2-normalised here (IO_QK_L2NORM); a template parameter, so that
+// kernels without it carry none of its code.
+template <int GATE, bool L2, class Worker, class Prefetch, class Hook = NoHook>
 __device__ __forceinline__ void prep_item(Worker &w, const PrepArgs &a, int slot, int h,
                                           SeqSpan span, int n, Prefetch pf,
                                           int32_t *__restrict__ ready, Hook hook = Hook()) {
@@ -477,7 +479,7 @@ __device__ __forceinline__ void prep_item(Worker &w, const PrepArgs &a, int slot
     // ---- gates and operand images, row by row. BAD selects the exact handling of key
     //      channels whose chunk log-decay exceeds SAFE_SPAN (kept out of the unrolled
     //      common path so that it stays branch-free).
-    const bool l2 = (a.io_flags & IO_QK_L2NORM) != 0;
+    constexpr bool l2 = L2;
     float *sqn = reinterpret_cast<float *>(sm + P_QN);
     float *skn = reinterpret_cast<float *>(sm + P_KN);
     auto gate_rows = [&](auto bad_tag) {
@@ -497,7 +499,7 @@ __device__ __forceinline__ void prep_item(Worker &w, const PrepArgs &a, int slot
                 xq[e] = live ? __bfloat162float(qb[e]) : 0.f;
                 xk[e] = live ? __bfloat162float(kb[e]) : 0.f;
             }
-            if (l2) {  // the warp holds the whole row (lane f: channels 4f .. 4f+3)
+            if constexpr (L2) {  // the warp holds the whole row (lane f: channels 4f .. 4f+3)
                 float sq = xq[0] * xq[0] + xq[1] * xq[1] + xq[2] * xq[2] + xq[3] * xq[3];
                 float sk = xk[0] * xk[0] + xk[1] * xk[1] + xk[2] * xk[2] + xk[3] * xk[3];
 #pragma unroll
@@ -613,7 +615,7 @@ __device__ __forceinline__ void prep_item(Worker &w, const PrepArgs &a, int slot
                         if (r < L) {
                             qx = __bfloat162float(a.q[(tok0 + r) * H * D + ccol]);
                             kx = __bfloat162float(a.k[(tok0 + r) * H * D + ccol]);
-                            if (l2) {  // the row norms gate_rows found
+                            if constexpr (L2) {  // the row norms gate_rows found
                                 qx *= sqn[r];
                                 kx *= skn[r];
                             }
@@ -820,7 +822,7 @@ __device__ __forceinline__ void prep_item(Worker &w, const PrepArgs &a, int slot
 }
 
 
-template <int GATE>
+template <int GATE, bool L2>
 __global__ void __launch_bounds__(PREP_NT, 3)
 kda_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_la, int pf_dist,
@@ -853,7 +855,7 @@ kda_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const PrepArgs a{&tm_q, &tm_k, &tm_la, q, k, log_alpha, beta, ws_blobs, T, H, io_flags, l2_eps};
     PrepWorker<true> w;
     w.init(true);
-    prep_item<GATE>(w, a, slot, h, seq_span(cu, T, seq), n, pf, nullptr);
+    prep_item<GATE, L2>(w, a, slot, h, seq_span(cu, T, seq), n, pf, nullptr);
     w.release(nullptr);
 }
 
@@ -1281,8 +1283,8 @@ constexpr uint32_t C2_VNEW_COUNT = 32 * (CHAIN_EPI_WARPS + 1);
 // columns), run by threads 0 .. C2_NT-1 on shared memory `sm`. tm_o: the output as plain
 // 64 x 64 bf16 boxes.
 __device__ __forceinline__ void chain2_task(unsigned char *sm, const int tid, const ChainArgs &a,
-                                            const CUtensorMap *tm_o, const int seq, const int h,
-                                            const ChainWindow &win) {
+                                            const CUtensorMap *tm_o, const CUtensorMap *tm_g, const int seq,
+                                            const int h, const ChainWindow &win) {
     using Lay = Chain2Layout;
     const int warp = tid >> 5, lane = tid & 31;
     const bool epi = warp < CHAIN_EPI_WARPS;
@@ -1327,10 +1329,14 @@ __device__ __forceinline__ void chain2_task(unsigned char *sm, const int tid, co
         bulk_g2s(st + Lay::KTT, blob + BLOB_KTT, 16384, &bar_ld2[stage]);
         bulk_g2s(st + Lay::GAM, blob + BLOB_GAM, 512, &bar_ld2[stage]);
     };
-    auto prefetch = [&](int chunk) {  // warm L2 with a later chunk's blob and value tile
+    auto prefetch = [&](int chunk) {  // warm L2 with a later chunk's blob, value tile, output gate
         bulk_prefetch_l2(blob_of(chunk), BLOB_BYTES);
         tma_prefetch_l2_2d(&tm_v, h * D, chunk_y(chunk));
         tma_prefetch_l2_2d(&tm_v, h * D + 64, chunk_y(chunk));
+        if (a.out_gate) {
+            tma_prefetch_l2_2d(tm_g, h * D, chunk_y(chunk));
+            tma_prefetch_l2_2d(tm_g, h * D + 64, chunk_y(chunk));
+        }
     };
     // A chunk whose output goes through a staging tile: all 64 rows in the sequence.
     auto full_chunk = [&](int m) { return chunk_rows(span.len, (int64_t)(c0 + m) * CH) == CH; };
@@ -1480,12 +1486,28 @@ __device__ __forceinline__ void chain2_task(unsigned char *sm, const int tid, co
         // Output of chunk m (columns 0..63 of its D1 buffer): this thread's value column j,
         // tokens 32 half .. +31.
         const bool out_epi = a.out_gate != nullptr;
-        float ow[4] = {1.f, 1.f, 1.f, 1.f};  // RMSNorm weights of this lane's columns 4 lane .. +3
+        // Row pass layout: 16 lanes per row, lane l % 16 takes columns 8 (l % 16) .. +7;
+        // warp w takes rows 2w + l / 16 + 16 p for p = 0..3.
+        const int rc0 = 8 * (lane & 15);
+        float ow[8] = {1.f, 1.f, 1.f, 1.f, 1.f, 1.f, 1.f, 1.f};  // RMSNorm weights of those columns
         if (out_epi && a.out_w) {
-            const float4 w4 = *reinterpret_cast<const float4 *>(a.out_w + 4 * lane);
-            ow[0] = w4.x; ow[1] = w4.y; ow[2] = w4.z; ow[3] = w4.w;
+            const float4 w0 = *reinterpret_cast<const float4 *>(a.out_w + rc0);
+            const float4 w1 = *reinterpret_cast<const float4 *>(a.out_w + rc0 + 4);
+            ow[0] = w0.x; ow[1] = w0.y; ow[2] = w0.z; ow[3] = w0.w;
+            ow[4] = w1.x; ow[5] = w1.y; ow[6] = w1.z; ow[7] = w1.w;
         }
         auto store_output = [&](int m) {
+            // the output gate of this warp's 8 rows of the tile (row pass below) into L1,
+            // so that its loads there hit (the load warp has brought it into L2)
+            if (out_epi && (lane & 15) == 0) {
+                const int64_t g0 = span.start + (int64_t)(c0 + m) * CH;
+                const int glive = chunk_rows(span.len, (int64_t)(c0 + m) * CH);
+#pragma unroll
+                for (int rr = 0; rr < 8; ++rr) {
+                    const int r = 8 * warp + rr;
+                    if (r < glive) prefetch_l1(a.out_gate + ((g0 + r) * H + h) * (int64_t)D + 4 * lane);
+                }
+            }
             mbar_wait(&bar_o[m & 1], (uint32_t)(m >> 1) & 1u, dead, &g_kda_status);
             tc_fence_after();
             float ov[32];
@@ -1512,47 +1534,50 @@ __device__ __forceinline__ void chain2_task(unsigned char *sm, const int tid, co
                 fence_async_smem();
                 return;
             }
-            // Row pass over the staged tile: warp w takes rows 8w .. 8w+7, lane l columns
-            // 4l .. 4l+3. It applies the output epilogue, and writes the rows of a partial
-            // chunk straight to the output (a full chunk goes back to the tile, for TMA).
+            // Row pass over the staged tile (16 lanes per row, see rc0). It applies the
+            // output epilogue, and writes the rows of a partial chunk straight to the
+            // output (a full chunk goes back to the tile, for TMA).
             named_bar_sync(C2_BAR_OROWS, 32 * CHAIN_EPI_WARPS);
             const int64_t tok0 = span.start + m0;
+            uint4 graw[4];  // the output gate of this lane's four rows, loads in flight together
+            if (out_epi) {
 #pragma unroll
-            for (int half = 0; half < 2; ++half) {  // four rows at a time, gate loads first
-                uint2 graw[4];
+                for (int p = 0; p < 4; ++p) {
+                    const int r = 16 * p + 2 * warp + (lane >> 4);
+                    graw[p] = r < live ? *reinterpret_cast<const uint4 *>(a.out_gate + ((tok0 + r) * H + h) * (int64_t)D + rc0)
+                                       : make_uint4(0u, 0u, 0u, 0u);
+                }
+            }
+#pragma unroll
+            for (int p = 0; p < 4; ++p) {
+                const int r = 16 * p + 2 * warp + (lane >> 4);
+                unsigned char *cell = ost(m) + (rc0 >> 6) * 8192 + r * 128 + (rc0 & 63) * 2;
+                uint4 raw = *reinterpret_cast<const uint4 *>(cell);
                 if (out_epi) {
+                    const uint32_t ow32[4] = {raw.x, raw.y, raw.z, raw.w};
+                    const uint32_t gw32[4] = {graw[p].x, graw[p].y, graw[p].z, graw[p].w};
+                    float x[8], g[8];
 #pragma unroll
-                    for (int rr = 0; rr < 4; ++rr) {
-                        const int r = 8 * warp + 4 * half + rr;
-                        graw[rr] = r < live ? *reinterpret_cast<const uint2 *>(
-                                                  a.out_gate + ((tok0 + r) * H + h) * (int64_t)D + 4 * lane)
-                                            : make_uint2(0u, 0u);
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 xv = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&ow32[e]));
+                        const float2 gv = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&gw32[e]));
+                        x[2 * e] = xv.x; x[2 * e + 1] = xv.y;
+                        g[2 * e] = gv.x; g[2 * e + 1] = gv.y;
                     }
+                    float ss = 0.f;
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) ss += x[e] * x[e];
+#pragma unroll
+                    for (int off = 8; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+                    const float inv = rsqrtf(ss * (1.f / D) + a.out_eps);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) x[e] *= inv * ow[e] * __fdividef(1.f, 1.f + __expf(-g[e]));
+                    raw = make_uint4(pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]), pack_bf16x2(x[4], x[5]),
+                                     pack_bf16x2(x[6], x[7]));
                 }
-#pragma unroll
-                for (int rr = 0; rr < 4; ++rr) {
-                    const int r = 8 * warp + 4 * half + rr;
-                    unsigned char *cell = ost(m) + (lane >> 4) * 8192 + r * 128 + 8 * (lane & 15);
-                    uint2 raw = *reinterpret_cast<const uint2 *>(cell);
-                    if (out_epi) {
-                        const float2 lo = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&raw.x));
-                        const float2 hi = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&raw.y));
-                        float x[4] = {lo.x, lo.y, hi.x, hi.y};
-                        float ss = x[0] * x[0] + x[1] * x[1] + x[2] * x[2] + x[3] * x[3];
-#pragma unroll
-                        for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
-                        const float inv = rsqrtf(ss * (1.f / D) + a.out_eps);
-                        const float2 glo = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&graw[rr].x));
-                        const float2 ghi = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&graw[rr].y));
-                        const float g[4] = {glo.x, glo.y, ghi.x, ghi.y};
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) x[e] *= inv * ow[e] * sigmoid(g[e]);
-                        raw = make_uint2(pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]));
-                    }
-                    if (live == CH) *reinterpret_cast<uint2 *>(cell) = raw;
-                    else if (r < live)
-                        *reinterpret_cast<uint2 *>(a.o + ((tok0 + r) * H + h) * (int64_t)D + 4 * lane) = raw;
-                }
+                if (live == CH) *reinterpret_cast<uint4 *>(cell) = raw;
+                else if (r < live)
+                    *reinterpret_cast<uint4 *>(a.o + ((tok0 + r) * H + h) * (int64_t)D + rc0) = raw;
             }
             if (live == CH) fence_async_smem();
         };
@@ -1632,7 +1657,7 @@ __device__ __forceinline__ void chain2_task(unsigned char *sm, const int tid, co
 
 __global__ void __launch_bounds__(C2_NT, 1)
 kda_chain2_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
-                  const unsigned char *__restrict__ ws_blobs,
+                  const __grid_constant__ CUtensorMap tm_g, const unsigned char *__restrict__ ws_blobs,
                   const int32_t *__restrict__ chunk_off, const float *__restrict__ S0,
                   __nv_bfloat16 *__restrict__ o, float *__restrict__ S_T, const int32_t *__restrict__ cu,
                   int64_t T, int H, int nck, int wait_prior, const __nv_bfloat16 *__restrict__ out_gate,
@@ -1641,7 +1666,7 @@ kda_chain2_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constan
     if (chunk_off && !packed_offsets_ok(chunk_off, (int)gridDim.x)) return;
     const ChainArgs a{&tm_v, ws_blobs, chunk_off, S0, o, S_T, cu, T, H, nck, nullptr, wait_prior != 0,
                       out_gate, out_w, out_eps};
-    chain2_task(aligned_smem(smem_raw), threadIdx.x, a, &tm_o, blockIdx.x, blockIdx.y,
+    chain2_task(aligned_smem(smem_raw), threadIdx.x, a, &tm_o, &tm_g, blockIdx.x, blockIdx.y,
                 full_window(a, blockIdx.x, blockIdx.y));
 }
 
@@ -1864,7 +1889,7 @@ kda_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 y = (int)((int64_t)(pp / H) * T + (int64_t)(pit / P) * CH);
                 return true;
             };
-            prep_item<GATE>(w, pa, seq * nck + n, h, SeqSpan{(int64_t)seq * T, T}, n, pf, ready,
+            prep_item<GATE, false>(w, pa, seq * nck + n, h, SeqSpan{(int64_t)seq * T, T}, n, pf, ready,
                       ClaimAhead{claim_next, claim + ((j + 1) & 1), -1});
         }
         w.release(ready);
@@ -1955,8 +1980,8 @@ cudaError_t launch_chain(const CUtensorMap &mv, const unsigned char *blobs, cons
     return err != cudaSuccess ? err : cudaGetLastError();
 }
 
-cudaError_t launch_chain2(const CUtensorMap &mv, const CUtensorMap &mo, const unsigned char *blobs,
-                          const int32_t *chunk_off,
+cudaError_t launch_chain2(const CUtensorMap &mv, const CUtensorMap &mo, const CUtensorMap &mg,
+                          const unsigned char *blobs, const int32_t *chunk_off,
                           const float *S0, void *o, float *S_T, const int32_t *cu, int64_t T, int H,
                           int nck, int nseq, bool after_prep, const IoOpts &io, cudaStream_t stream) {
     using Lay = Chain2Layout;
@@ -1964,7 +1989,7 @@ cudaError_t launch_chain2(const CUtensorMap &mv, const CUtensorMap &mo, const un
                                            (int)Lay::BYTES);
     if (err != cudaSuccess) return err;
     err = launch_maybe_dependent(kda_chain2_kernel, dim3((unsigned)nseq, (unsigned)H), dim3(C2_NT), Lay::BYTES,
-                                 stream, after_prep, mv, mo, blobs, chunk_off, S0, (__nv_bfloat16 *)o, S_T, cu, T,
+                                 stream, after_prep, mv, mo, mg, blobs, chunk_off, S0, (__nv_bfloat16 *)o, S_T, cu, T,
                                  H, nck, after_prep ? 1 : 0, (const __nv_bfloat16 *)io.out_gate, io.out_w,
                                  io.out_eps);
     return err != cudaSuccess ? err : cudaGetLastError();
@@ -1976,7 +2001,7 @@ int prep_residency() {
     int dev = 0, n_sm = 0, per_sm = 0;
     if (cudaGetDevice(&dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kda_prep_kernel<KDA_GATE_CHANNEL>,
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kda_prep_kernel<KDA_GATE_CHANNEL, false>,
                                                       PREP_NT, PREP_SMEM) !=
             cudaSuccess)
         return 0;
@@ -2107,14 +2132,14 @@ int sm_count() {
 }
 
 // Kernels launch_prefill_tc launches for these arguments (its decisions, restated).
-int prefill_tc_launches(int B, int64_t T, int H, int n_seqs, bool out_epilogue) {
+int prefill_tc_launches(int B, int64_t T, int H, int n_seqs, bool out_epilogue, bool l2norm) {
     const bool packed = n_seqs > 0;
     const int64_t n_tok = packed ? T : (int64_t)B * T;
     const int nck = (int)((T + CH - 1) / CH);
     if (!packed && n_tok > 0 && !out_epilogue) {
         const BatchedPlan plan = batched_plan(B, H, nck, sm_count());
-        if (plan.kind == 1) return 1;  // the fused grid
-        if (plan.kind == 2) return 4;  // prep, pass 1, combine, pass 2
+        if (plan.kind == 1 && !l2norm) return 1;  // the fused grid
+        if (plan.kind == 2) return 4;             // prep, pass 1, combine, pass 2
     }
     const int64_t slots = packed ? T / CH + n_seqs : (int64_t)B * nck;
     return (packed ? 1 : 0) + (n_tok > 0 && slots > 0 ? 1 : 0) + 1;
@@ -2155,7 +2180,12 @@ cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, const
         chunk_offsets_kernel<<<1, 1024, 0, stream>>>(cu_seqlens, n_seqs, T, chunk_off);
     } else {
         blobs = ws + batched_head_bytes(B, nck, H);
-        plan = n_tok > 0 && !out_epi ? batched_plan(B, H, nck, n_sm) : BatchedPlan{0, 0, 0, 0};
+        // the fused grid's prep workers have no L2 normalisation: with it, or with an
+        // output epilogue, the call runs the prep and the chains
+        const bool two_kernels = out_epi || (io_flags & IO_QK_L2NORM) != 0;
+        plan = n_tok > 0 ? batched_plan(B, H, nck, n_sm) : BatchedPlan{0, 0, 0, 0};
+        if (two_kernels && plan.kind == 1) plan = BatchedPlan{0, 0, 0, 0};
+        if (out_epi) plan = BatchedPlan{0, 0, 0, 0};
         if (plan.kind == 1) {
             int32_t *ready = reinterpret_cast<int32_t *>(ws);
             FusedQueue *queue = reinterpret_cast<FusedQueue *>(ready + (size_t)B * nck * H);
@@ -2186,18 +2216,21 @@ cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, const
             !make_gate_map(&mla, log_alpha, gate, n_tok, H, mq))
             return cudaErrorInvalidValue;
         const int pf_dist = prep_residency();
-        err = with_gate(gate, [&](auto g) {
-            constexpr int G = decltype(g)::value;
-            cudaError_t e = cudaFuncSetAttribute(kda_prep_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                 (int)PREP_SMEM);
+        auto launch_prep = [&](auto kernel) {
+            cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)PREP_SMEM);
             if (e == cudaSuccess)  // three CTAs per SM need the largest shared-memory carveout
-                e = cudaFuncSetAttribute(kda_prep_kernel<G>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                e = cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
                                          (int)cudaSharedmemCarveoutMaxShared);
             if (e != cudaSuccess) return e;
-            kda_prep_kernel<G><<<dim3((unsigned)slots, (unsigned)H), PREP_NT, PREP_SMEM, stream>>>(
+            kernel<<<dim3((unsigned)slots, (unsigned)H), PREP_NT, PREP_SMEM, stream>>>(
                 mq, mk, mla, pf_dist, (const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k, log_alpha,
                 beta, blobs, chunk_off, cu_seqlens, T, H, n_seqs, nck, io_flags, l2_eps);
             return cudaGetLastError();
+        };
+        err = with_gate(gate, [&](auto g) {
+            constexpr int G = decltype(g)::value;
+            return (io_flags & IO_QK_L2NORM) ? launch_prep(kda_prep_kernel<G, true>)
+                                             : launch_prep(kda_prep_kernel<G, false>);
         });
         if (err != cudaSuccess) return err;
     }
@@ -2226,10 +2259,11 @@ cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, const
         return cudaGetLastError();
     }
     if (out_epi) {  // one full-head chain CTA per (sequence, head), with the output epilogue
-        CUtensorMap mo;
-        if (n_tok > 0 && !make_map(&mo, o, true, n_tok, H, false)) return cudaErrorInvalidValue;
-        if (n_tok == 0) mo = mv;  // no chunk: the map is never used
-        return launch_chain2(mv, mo, blobs, chunk_off, S0, o, S_T, cu_seqlens, T, H, nck, nseq,
+        CUtensorMap mo, mg;
+        if (n_tok > 0 && (!make_map(&mo, o, true, n_tok, H, false) || !make_map(&mg, io.out_gate, true, n_tok, H)))
+            return cudaErrorInvalidValue;
+        if (n_tok == 0) mo = mg = mv;  // no chunk: the maps are never used
+        return launch_chain2(mv, mo, mg, blobs, chunk_off, S0, o, S_T, cu_seqlens, T, H, nck, nseq,
                              prep_launched, io, stream);
     }
     // 128-column slices (one CTA per sequence-head) when there are enough pairs to fill

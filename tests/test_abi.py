@@ -187,7 +187,7 @@ def test_io_entry_points_validate_their_options(lib):
     assert chunk(Io(1, float("nan"), 0, None, None, 0.0)) == INVALID   # NaN eps
     assert chunk(Io(0, 0.0, 0, gate16, None, -1.0)) == INVALID          # negative output eps
     assert chunk(Io(0, 0.0, 0, gate16, None, 1e-6), dtype=F32) == UNSUPPORTED  # fp32: no epilogue
-    assert chunk(Io(0, 0.0, 0, gate16 + 2, None, 1e-6)) == INVALID     # bf16 gate: 8-byte aligned
+    assert chunk(Io(0, 0.0, 0, gate16 + 8, None, 1e-6)) == INVALID     # bf16 gate: 16-byte aligned
     assert chunk(Io(0, 0.0, 0, gate16, gate16 + 4, 1e-6)) == INVALID    # weights: 16-byte aligned
     assert decode(Io(1, -1.0, 0, None, None, 0.0)) == INVALID
     assert decode(Io(0, 0.0, 0, gate16 + 2, None, 1e-6)) == INVALID
