@@ -27,6 +27,7 @@ import subprocess
 import sys
 import time
 
+import numpy as np
 import torch
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -217,9 +218,13 @@ def time_steps(fn, steps, warmup, stream, flush=None, name="kda"):
     return times
 
 
-def cpu_oracle_sample(inp, min_s: float = 10.0, max_reps: int = 40):
+def cpu_oracle_sample(inp, o, S_T, min_s: float = 10.0, max_reps: int = 40):
     """Times the fp64 oracle on the whole prefill batch (every sequence and head),
-    repeated until at least ``min_s`` seconds of CPU time (at most ``max_reps`` passes)."""
+    repeated until at least ``min_s`` seconds of CPU time (at most ``max_reps`` passes).
+
+    The oracle's last result is also compared with the step's own outputs ``o`` and
+    ``S_T`` (the same inputs and S0), element by element over every output: relative L2
+    error and max-abs error, next to the bf16 bar the parity tests hold them to."""
     import oracle
 
     args = [oracle._f64(t) for t in (inp.q, inp.k, inp.v, inp.log_alpha, inp.beta, inp.S0)]
@@ -228,12 +233,24 @@ def cpu_oracle_sample(inp, min_s: float = 10.0, max_reps: int = 40):
     reps, total = 0, 0.0
     while total < min_s and reps < max_reps:
         t0 = time.perf_counter()
-        oracle.kda_fwd(*args, threads=threads)
+        ref = oracle.kda_fwd(*args, threads=threads)
         total += time.perf_counter() - t0
         reps += 1
-    return {"value": B * T * reps / total, "unit": "tokens/s", "cores": threads, "kind": "oracle",
-            "sample": f"the whole prefill batch ({B} sequences x {T} tokens x {H} heads, bf16 "
-                      f"inputs widened to fp64) {reps} times, {total:.1f} s on {threads} threads"}
+    cpu = {"value": B * T * reps / total, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+           "sample": f"the whole prefill batch ({B} sequences x {T} tokens x {H} heads, bf16 "
+                     f"inputs widened to fp64) {reps} times, {total:.1f} s on {threads} threads"}
+    parity = {"against": "the fp64 oracle on the same inputs, every element of o and S_T",
+              "bar": {"rel_l2": 1e-2, "max_abs_over_max_ref": 2e-2}}
+    for name, got, want in (("o", o, ref[0]), ("S_T", S_T, ref[1])):
+        x = got.detach().to("cpu", torch.float64).numpy()
+        diff = x - want
+        mref = float(np.max(np.abs(want)))
+        parity[name] = {"rel_l2": float(np.linalg.norm(diff) / np.linalg.norm(want)),
+                        "max_abs": float(np.max(np.abs(diff))), "max_ref": mref,
+                        "finite": bool(np.all(np.isfinite(x)))}
+    parity["pass"] = all(parity[n]["finite"] and parity[n]["rel_l2"] <= 1e-2
+                         and parity[n]["max_abs"] <= 2e-2 * parity[n]["max_ref"] for n in ("o", "S_T"))
+    return cpu, parity
 
 
 def prefill_config(world: int) -> dict:
@@ -576,6 +593,12 @@ def run_kda(args, rank, world, local_rank):
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e_ms}
     del host, dbuf
 
+    # ---------------- the gate layouts, next to the step they vary and before the decode
+    # graph (whose power draw would otherwise still hold the clocks down)
+    extra = {}
+    if not args.no_extra:
+        extra.update(gate_layout_workloads(kda, dev, stream, flush, pk, world, rank))
+
     # ---------------- decode (N=256, H=32, 1024 steps in one CUDA graph)
     decode = None
     if not args.no_decode:
@@ -615,16 +638,15 @@ def run_kda(args, rank, world, local_rank):
         del graph, dinp, S, od
 
     # ---------------- the other prefill workloads (reported beside the step, not the step)
-    extra = {}
-    if not args.no_extra:  # the gate layouts first, next to the step they vary
-        extra.update(gate_layout_workloads(kda, dev, stream, flush, pk, world, rank))
+    if not args.no_extra:
         extra.update(fused_io_workload(kda, dev, stream, flush, pk, world, rank))
         extra.update(backward_workload(kda, dev, stream, flush, pk, world, rank))
         extra.update(other_prefill_workloads(kda, dev, stream, flush, pk, world, rank))
 
-    cpu = None
+    cpu, parity = None, None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_oracle_sample(inp)
+        torch.cuda.synchronize()
+        cpu, parity = cpu_oracle_sample(inp, o, S_T)
 
     if rank == 0:
         line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
@@ -632,7 +654,7 @@ def run_kda(args, rank, world, local_rank):
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
                 "data": "synthetic",
                 "config": prefill_config(world),
-                "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+                "roofline": roofline, "cpu_baseline": cpu, "parity": parity, "e2e": e2e,
                 "gpu_launches": launches_per_call * args.steps, "clocks": clk, "decode": decode,
                 **extra}
         print(json.dumps(line), flush=True)

@@ -50,23 +50,25 @@ struct BwdSmem {
     float beta[CH];
     float v[CH][BW_J], dout[CH][BW_J];   // the slice's v and do
     float u[CH][BW_J], dd[CH][BW_J];     // u_t of the forward rerun; d_t (then reused)
-    float colsum[BW_NT / 32][BW_J];      // per-warp partial column sums
+    float colsum[2][BW_NT / 32][BW_J];   // per-warp partial column sums, two buffers
     float rows[BW_NT / 32][BW_ROWS][BW_J + 1];  // per-warp row-sum transposition
 };
 
 // Sum over the state's 128 rows of x (this thread's 16 rows, column lane), for every
-// column: the result is returned to all threads of column lane. Two CTA barriers.
-__device__ __forceinline__ float col_sum(const float (&x)[BW_ROWS], BwdSmem &sm) {
+// column: the result is returned to all threads of column lane. One CTA barrier: the
+// calls alternate between two buffers (`buf`, flipped here), so a buffer is written
+// again only after the barrier of the next call, when every thread has read it.
+__device__ __forceinline__ float col_sum(const float (&x)[BW_ROWS], BwdSmem &sm, int &buf) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     float s = 0.f;
 #pragma unroll
     for (int r = 0; r < BW_ROWS; ++r) s += x[r];
-    sm.colsum[warp][lane] = s;
+    sm.colsum[buf][warp][lane] = s;
     __syncthreads();
     float t = 0.f;
 #pragma unroll
-    for (int w = 0; w < BW_NT / 32; ++w) t += sm.colsum[w][lane];
-    __syncthreads();
+    for (int w = 0; w < BW_NT / 32; ++w) t += sm.colsum[buf][w][lane];
+    buf ^= 1;
     return t;
 }
 
@@ -138,6 +140,7 @@ kda_bwd_slice_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const
     float *cbase = chunk_states + ((size_t)slot0 * H + h) * BW_SLICES * BW_SLICE_STATE + slice * BW_SLICE_STATE;
     float *tstates = token_states + (size_t)slot * CH * BW_SLICE_STATE;
     auto st_off = [&](int r) { return (size_t)(r0 + r) * BW_J + lane; };
+    int cbuf = 0;  // col_sum's buffer
 
     // Loads a chunk's q, k, a and beta (rows >= L zero; a = 1 there) and the slice's v, do.
     auto load_chunk = [&](int64_t tok0, int L) {
@@ -192,7 +195,7 @@ kda_bwd_slice_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const
             s[r] *= sm.a[t][r0 + r];
             ka[r] = s[r] * sm.k[t][r0 + r];
         }
-        const float u = col_sum(ka, sm);
+        const float u = col_sum(ka, sm, cbuf);
         const float d = sm.beta[t] * (sm.v[t][lane] - u);
         if (warp == 0) {
             sm.u[t][lane] = u;
@@ -236,10 +239,20 @@ kda_bwd_slice_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const
         }
         __syncthreads();
         // s is the state after the chunk's last token; tokens in reverse
+        // S_{t-1} of the next token back is loaded while the current token is worked on
+        float nxt[BW_ROWS];
+        if (L > 0) {
+#pragma unroll
+            for (int r = 0; r < BW_ROWS; ++r) nxt[r] = tstates[(size_t)(L - 1) * BW_SLICE_STATE + st_off(r)];
+        }
         for (int t = L - 1; t >= 0; --t) {
             float prev[BW_ROWS];  // S_{t-1}
 #pragma unroll
-            for (int r = 0; r < BW_ROWS; ++r) prev[r] = tstates[(size_t)t * BW_SLICE_STATE + st_off(r)];
+            for (int r = 0; r < BW_ROWS; ++r) prev[r] = nxt[r];
+            if (t > 0) {
+#pragma unroll
+                for (int r = 0; r < BW_ROWS; ++r) nxt[r] = tstates[(size_t)(t - 1) * BW_SLICE_STATE + st_off(r)];
+            }
             const float do_j = sm.dout[t][lane];
             const float d_j = sm.dd[t][lane], u_j = sm.u[t][lane];
             float x[BW_ROWS];
@@ -253,7 +266,7 @@ kda_bwd_slice_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const
             // dd = G^T k
 #pragma unroll
             for (int r = 0; r < BW_ROWS; ++r) x[r] = G[r] * sm.k[t][r0 + r];
-            const float dd_j = col_sum(x, sm);
+            const float dd_j = col_sum(x, sm, cbuf);
             const float b = sm.beta[t];
             const float du_j = -b * dd_j;
             float* part = parts + ((size_t)(tok0 + t) * H + h) * (BW_SLICES * BW_PARTS) + (size_t)slice * BW_PARTS;

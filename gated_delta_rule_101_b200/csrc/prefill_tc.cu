@@ -247,6 +247,7 @@ struct PrepArgs {
     int H;
     int io_flags;   // IO_QK_L2NORM, IO_BETA_LOGITS
     float l2_eps;
+    int64_t n_rows;  // token-head rows of the call (tokens x H)
 };
 
 // One prep worker: 256 threads with their own shared-memory partition (PREP_SMEM
@@ -395,6 +396,19 @@ __device__ __forceinline__ void prep_item(Worker &w, const PrepArgs &a, int slot
             } else if constexpr (bf16_gate<GATE>()) {  // bf16 boxes of 64
                 tma_prefetch_l2_2d(a.tm_la, pf_x, pf_y);
                 tma_prefetch_l2_2d(a.tm_la, pf_x + 64, pf_y);
+            }
+        }
+    } else if (GATE == KDA_GATE_HEAD && tid < CH) {
+        // A head-wide gate (and beta) of that later item's rows: 4 bytes per token-head,
+        // one cache line every 128 / (4 H) rows, so each row's thread asks for its own.
+        // Only here does it pay: with per-channel gates the extra work costs more than
+        // the two scattered row reads it hides.
+        int pf_x, pf_y;
+        if (pf(pf_x, pf_y)) {
+            const int64_t prow = (int64_t)(pf_y + tid) * H + pf_x / D;
+            if (prow < a.n_rows) {
+                prefetch_l2(a.beta + prow);
+                prefetch_l2(static_cast<const float *>(a.log_alpha) + prow);
             }
         }
     }
@@ -852,7 +866,8 @@ kda_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         y = (int)(seq_span(cu, T, pseq).start + (int64_t)pn * CH);
         return true;
     };
-    const PrepArgs a{&tm_q, &tm_k, &tm_la, q, k, log_alpha, beta, ws_blobs, T, H, io_flags, l2_eps};
+    const int64_t n_tok = chunk_off ? T : (int64_t)(gridDim.x / nck) * T;  // packed: T tokens in all
+    const PrepArgs a{&tm_q, &tm_k, &tm_la, q, k, log_alpha, beta, ws_blobs, T, H, io_flags, l2_eps, n_tok * H};
     PrepWorker<true> w;
     w.init(true);
     prep_item<GATE, L2>(w, a, slot, h, seq_span(cu, T, seq), n, pf, nullptr);
@@ -1854,7 +1869,8 @@ kda_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     const int n_shared = n_first * P, n_total = nck * P;
     const bool chain_cta = (int)blockIdx.x < n_chain;
     {
-        const PrepArgs pa{&tm_q, &tm_k, &tm_la, q, k, log_alpha, beta, ws_blobs, T, H, io_flags, l2_eps};
+        const PrepArgs pa{&tm_q, &tm_k, &tm_la, q, k, log_alpha, beta, ws_blobs, T, H, io_flags, l2_eps,
+                          (int64_t)B * T * H};
         using Worker = PrepWorker<false>;
         Worker w;
         w.init(false);
