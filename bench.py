@@ -414,6 +414,49 @@ def gate_layout_workloads(kda, dev, stream, flush, pk, world, rank):
     return {"gate_layouts": out}
 
 
+def chunk_size_workloads(kda, dev, stream, flush, pk, world, rank):
+    """The step's workload at each chunk length the library takes (C = 32 and 64), for
+    bf16 and fp32 inputs. bf16 at C = 64 is the step itself (tensor cores); the other
+    three run on the CUDA-core kernel. Each call timed on the device, L2 flushed."""
+    from gated_delta_rule_101_b200.inputs import prefill_inputs
+
+    B, T, H = PREFILL["B"], PREFILL["T"], PREFILL["H"]
+    out = {}
+    for dtype, name, esize in ((torch.bfloat16, "bf16", 2), (torch.float32, "f32", 4)):
+        inp = prefill_inputs(B=B, T=T, H=H, dtype=dtype, s0_std=PREFILL["s0_std"],
+                             la_range=PREFILL["la_range"], seed=PREFILL["seed"] + 1000 * rank,
+                             device=dev)
+        o = torch.empty_like(inp.v)
+        S_T = torch.empty_like(inp.S0)
+        alg = (PREFILL_BYTES_PER_TOKEN_HEAD + 4 * 128 * (esize - 2)) * B * T * H + 2 * STATE_BYTES * B * H
+        for C in (32, 64):
+            ws = torch.empty(max(kda.workspace_size(B, T, H, 0, dtype, C), 16), dtype=torch.uint8, device=dev)
+            n_l = kda.chunk_fwd_launches(B, T, H, dtype=dtype, C=C)
+
+            def call():
+                kda.chunk_fwd(inp.q, inp.k, inp.v, inp.log_alpha, inp.beta, inp.S0, out=o, state_out=S_T,
+                              workspace=ws, stream=stream, C=C)
+
+            reps = 10 if (name == "bf16" and C == 64) else 3
+            barrier(world)
+            times = time_steps(call, reps, 3, stream, flush, name=f"kda.chunk{C}.{name}")
+            ms = max_over_ranks(sum(times), world, dev) / len(times)
+            kernel = "kda_prep_kernel + kda_chain_kernel (tensor cores)" if (name == "bf16" and C == 64) \
+                else "prefill_simt_kernel (CUDA cores, fp32)"
+            out[f"C{C}_{name}"] = {
+                "value": B * T * world / (ms * 1e-3), "unit": "tokens/s", "ms_per_call": ms,
+                "config": {"workload": f"KDA prefill B={B} T={T} H={H} d=128, {name} inputs, chunks of {C}",
+                           "l2": "flushed before every call"},
+                "roofline": {"bound": "hbm", "achieved": alg / (ms * 1e-3) / 1e9, "peak": pk["hbm_gbs"],
+                             "unit": "GB/s", "frac": alg / (ms * 1e-3) / 1e9 / pk["hbm_gbs"],
+                             "alg_bytes_per_launch": alg, "kernel": kernel},
+                "gpu_launches": n_l * len(times)}
+            del ws
+        del inp, o, S_T
+    torch.cuda.empty_cache()
+    return {"chunk_sizes": out}
+
+
 def fused_io_workload(kda, dev, stream, flush, pk, world, rank):
     """The step's shape through kda_chunk_fwd_io with every fused step of the layer:
     the gate's pre-activation z as bf16 logits (alpha = sigmoid(z)), q and k
@@ -640,6 +683,7 @@ def run_kda(args, rank, world, local_rank):
     # ---------------- the other prefill workloads (reported beside the step, not the step)
     if not args.no_extra:
         extra.update(fused_io_workload(kda, dev, stream, flush, pk, world, rank))
+        extra.update(chunk_size_workloads(kda, dev, stream, flush, pk, world, rank))
         extra.update(backward_workload(kda, dev, stream, flush, pk, world, rank))
         extra.update(other_prefill_workloads(kda, dev, stream, flush, pk, world, rank))
 

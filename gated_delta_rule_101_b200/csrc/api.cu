@@ -22,9 +22,13 @@ int check_gate_ptr(const void *log_alpha, int gate, bool tma) {
     return ((uintptr_t)log_alpha & (align - 1)) == 0 ? KDA_OK : KDA_ERR_INVALID_ARG;
 }
 
+// The tensor-core kernels take bf16 inputs in chunks of 64; everything else (fp32
+// inputs, and chunks of 32 in either dtype) runs on the CUDA-core kernel.
+bool tensor_core_path(int C, int dtype) { return dtype == KDA_BF16 && C == KDA_CHUNK; }
+
 // Validates the shape arguments shared by the size query and the call.
 int check_prefill_shape(int B, int64_t T, int H, int C, int n_seqs, int dtype) {
-    if (C != KDA_CHUNK) return KDA_ERR_UNSUPPORTED;
+    if (C != KDA_CHUNK && C != KDA_CHUNK_SMALL) return KDA_ERR_UNSUPPORTED;
     if (!valid_dtype(dtype)) return KDA_ERR_UNSUPPORTED;
     if (B <= 0 || T < 0 || H <= 0 || n_seqs < 0) return KDA_ERR_INVALID_ARG;
     if (n_seqs > 0 && B != 1) return KDA_ERR_INVALID_ARG;
@@ -83,7 +87,7 @@ int kda_chunk_fwd_workspace_size(int B, int64_t T, int H, int C, int n_seqs, int
     if (!bytes) return KDA_ERR_INVALID_ARG;
     const int st = check_prefill_shape(B, T, H, C, n_seqs, dtype);
     if (st != KDA_OK) return st;
-    *bytes = dtype == KDA_BF16 ? kda::prefill_tc_workspace(B, T, H, n_seqs) : 0;
+    *bytes = tensor_core_path(C, dtype) ? kda::prefill_tc_workspace(B, T, H, n_seqs) : 0;
     return KDA_OK;
 }
 
@@ -97,8 +101,9 @@ int kda_chunk_fwd_io_launches(int B, int64_t T, int H, int C, int n_seqs, int dt
     const int st = check_prefill_shape(B, T, H, C, n_seqs, dtype);
     if (st != KDA_OK) return st;
     const bool out_epi = io && io->out_gate;
-    if (out_epi && dtype != KDA_BF16) return KDA_ERR_UNSUPPORTED;
-    *n_kernels = dtype == KDA_BF16 ? kda::prefill_tc_launches(B, T, H, n_seqs, out_epi, io && io->qk_l2norm) : 1;
+    if (out_epi && !tensor_core_path(C, dtype)) return KDA_ERR_UNSUPPORTED;
+    *n_kernels = tensor_core_path(C, dtype)
+                     ? kda::prefill_tc_launches(B, T, H, n_seqs, out_epi, io && io->qk_l2norm) : 1;
     return KDA_OK;
 }
 
@@ -130,12 +135,13 @@ int kda_chunk_fwd_io(const void *q, const void *k, const void *v, const void *lo
     if (st != KDA_OK) return st;
     if (!valid_gate(gate)) return KDA_ERR_UNSUPPORTED;
     kda::IoOpts opts;
-    st = make_io(io, dtype == KDA_BF16, dtype == KDA_BF16 ? 2 : 4, &opts);
+    const bool tc = tensor_core_path(C, dtype);
+    st = make_io(io, tc, dtype == KDA_BF16 ? 2 : 4, &opts);
     if (st != KDA_OK) return st;
     const bool packed = n_seqs > 0;
     if (packed != (cu_seqlens != nullptr)) return KDA_ERR_INVALID_ARG;
     if (T > 0 && (!q || !k || !v || !beta || !o)) return KDA_ERR_INVALID_ARG;
-    if (T > 0 && check_gate_ptr(log_alpha, gate, dtype == KDA_BF16) != KDA_OK)
+    if (T > 0 && check_gate_ptr(log_alpha, gate, tc) != KDA_OK)
         return KDA_ERR_INVALID_ARG;
     if (cu_seqlens_host) {
         if (!packed || cu_seqlens_host[0] != 0 || cu_seqlens_host[n_seqs] != T)
@@ -152,7 +158,7 @@ int kda_chunk_fwd_io(const void *q, const void *k, const void *v, const void *lo
     const int nseq = packed ? n_seqs : B;
     cudaStream_t s = (cudaStream_t)stream;
     cudaError_t err;
-    if (dtype == KDA_BF16) {
+    if (tc) {
         // TMA requires 16-byte aligned tensor bases
         if (T > 0 && ((((uintptr_t)q | (uintptr_t)k | (uintptr_t)v) & 15u) != 0))
             return KDA_ERR_INVALID_ARG;
@@ -162,7 +168,7 @@ int kda_chunk_fwd_io(const void *q, const void *k, const void *v, const void *lo
                                      cu_seqlens, n_seqs, workspace, opts, s);
     } else {
         err = kda::launch_prefill_simt(q, k, v, log_alpha, gate, beta, S0, o, S_T, nseq, T, H,
-                                       cu_seqlens, dtype, opts, s);
+                                       cu_seqlens, dtype, C, opts, s);
     }
     if (err == cudaErrorInvalidValue) return KDA_ERR_INVALID_ARG;
     return err == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;

@@ -121,7 +121,7 @@ cudaError_t launch_decode(const void *q, const void *k, const void *v, const voi
 cudaError_t launch_prefill_simt(const void *q, const void *k, const void *v,
                                 const void *log_alpha, int gate, const float *beta, const float *S0,
                                 void *o, float *S_T, int n_seqs, int64_t T, int H,
-                                const int32_t *cu_seqlens, int dtype, const IoOpts &io,
+                                const int32_t *cu_seqlens, int dtype, int C, const IoOpts &io,
                                 cudaStream_t stream);
 
 // Tensor-core prefill (bf16 q/k/v): workspace bytes and launcher.

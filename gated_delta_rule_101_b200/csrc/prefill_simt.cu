@@ -1,11 +1,13 @@
 // KDA chunk-parallel prefill on CUDA cores, all arithmetic in fp32.
 //
 // This is the path for fp32 inputs, where tensor-core operand rounding would
-// exceed the fp32 error budget. It follows the chunked form of KDA
+// exceed the fp32 error budget, and for chunks of C = 32 tokens in either input
+// dtype (the chunk size is a template parameter, C = 32 or 64; mokono.cn section 4.1
+// names 32 to 128 as the useful range). It follows the chunked form of KDA
 // (mokono.cn "Kimi Linear：高效注意力机制在长序列处理中的创新应用" section 2.1,
 // S_r = P_r S_0 + H_r; blog.gzher.com "Kimi K3论文：Kimi Linear" section 4:
 // WY representation, UT transform, state passed from chunk to chunk). For a
-// chunk of L <= 64 tokens with start state S (dk x dv), per key channel c:
+// chunk of L <= C tokens with start state S (dk x dv), per key channel c:
 //
 //   g_r        = sum_{j<=r} log_alpha_j           (reset at every chunk)
 //   A_kk[r,i]  = beta_r sum_c k_rc k_ic exp(g_rc - g_ic)   for i < r
@@ -34,23 +36,26 @@ namespace {
 constexpr int NT = 256;           // threads per CTA
 constexpr int DVS = 32;           // value columns per CTA
 constexpr int LD = D + 4;         // row stride of the [64][128] buffers (floats)
-constexpr int LDA = CH + 1;       // row stride of the [64][64] buffers
 constexpr float SAFE_SPAN = 80.f; // max chunk log-decay for the factorised form
 
+// CK: chunk length (32 or 64). About 201 KB for 64, 100 KB for 32; 128 would need
+// about 400 KB and does not fit an SM.
+template <int CK>
 struct SimtSmem {
-    float q[CH * LD];    // q, then exp(g) * q
-    float k[CH * LD];    // k, then exp(g) * k, then W (solved in place)
-    float g[CH * LD];    // log_alpha, then g (high part), then exp(g_L - g) * k
-    float glo[CH * LD];  // low part of g
-    float akk[CH * LDA]; // beta-scaled strict-lower Gram
-    float aqk[CH * LDA]; // inclusive-lower Gram
-    float vu[CH * DVS];  // v slice, then U (solved in place)
-    float vn[CH * DVS];  // V_new
+    static constexpr int LDA = CK + 1;  // row stride of the [CK][CK] buffers
+    float q[CK * LD];    // q, then exp(g) * q
+    float k[CK * LD];    // k, then exp(g) * k, then W (solved in place)
+    float g[CK * LD];    // log_alpha, then g (high part), then exp(g_L - g) * k
+    float glo[CK * LD];  // low part of g
+    float akk[CK * LDA]; // beta-scaled strict-lower Gram
+    float aqk[CK * LDA]; // inclusive-lower Gram
+    float vu[CK * DVS];  // v slice, then U (solved in place)
+    float vn[CK * DVS];  // V_new
     float s[D * DVS];    // state slice S[c][j]
     float gl[D];         // g_L per channel (high part)
     float gllo[D];       // g_L per channel (low part)
     float einv[D];       // exp(-g_L) per channel
-    float beta[CH];
+    float beta[CK];
 };
 
 // Calls of a KDA_DEBUG build whose device offsets failed the checks (always 0 in the
@@ -63,7 +68,7 @@ __device__ __forceinline__ void load_row8(const TIn *src, float *dst) {
     for (int e = 0; e < 8; ++e) dst[e] = to_f32(src[e]);
 }
 
-template <typename TIn, int GATE>
+template <typename TIn, int GATE, int CK>
 __global__ void __launch_bounds__(NT, 1)
 prefill_simt_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k,
                     const TIn *__restrict__ v, const void *__restrict__ log_alpha,
@@ -71,7 +76,10 @@ prefill_simt_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k,
                     TIn *__restrict__ o, float *__restrict__ S_T, int64_t T, int H,
                     const int32_t *__restrict__ cu_seqlens, int io_flags, float l2_eps) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
-    SimtSmem &sm = *reinterpret_cast<SimtSmem *>(smem_raw);
+    using Smem = SimtSmem<CK>;
+    constexpr int LDA = Smem::LDA;
+    constexpr int NB = CK / 16;  // Gram blocks of 16 rows (columns) per thread
+    Smem &sm = *reinterpret_cast<Smem *>(smem_raw);
 
     const int seq = blockIdx.x, h = blockIdx.y, j0 = blockIdx.z * DVS;
     const int tid = threadIdx.x;
@@ -99,13 +107,13 @@ prefill_simt_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k,
         sm.s[e] = S0 ? S0[state_off + (int64_t)c * D + j0 + j] : 0.f;
     }
 
-    for (int64_t c0 = 0; c0 < span.len; c0 += CH) {
-        const int L = span.len - c0 < CH ? (int)(span.len - c0) : CH;
+    for (int64_t c0 = 0; c0 < span.len; c0 += CK) {
+        const int L = span.len - c0 < CK ? (int)(span.len - c0) : CK;
         const int64_t tok0 = span.start + c0;
         __syncthreads();  // previous chunk finished with every buffer
 
         // ---- load the chunk; rows >= L become k = q = 0, log_alpha = 0, beta = 0
-        for (int e = tid; e < CH * (D / 8); e += NT) {
+        for (int e = tid; e < CK * (D / 8); e += NT) {
             const int r = e / (D / 8), c8 = (e % (D / 8)) * 8;
             float *dq = sm.q + r * LD + c8, *dk = sm.k + r * LD + c8, *dg = sm.g + r * LD + c8;
             if (r < L) {
@@ -119,11 +127,11 @@ prefill_simt_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k,
                 for (int x = 0; x < 8; ++x) dq[x] = dk[x] = dg[x] = 0.f;
             }
         }
-        for (int e = tid; e < CH * DVS; e += NT) {
+        for (int e = tid; e < CK * DVS; e += NT) {
             const int r = e / DVS, j = e % DVS;
             sm.vu[e] = r < L ? to_f32(v[((tok0 + r) * H + h) * (int64_t)D + j0 + j]) : 0.f;
         }
-        if (tid < CH) {
+        if (tid < CK) {
             float b = tid < L ? beta[(tok0 + tid) * H + h] : 0.f;
             if ((io_flags & IO_BETA_LOGITS) && tid < L) b = sigmoid(b);
             sm.beta[tid] = b;
@@ -131,7 +139,7 @@ prefill_simt_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k,
         __syncthreads();
         if (io_flags & IO_QK_L2NORM) {  // q and k rows to unit length (rows >= L stay zero)
             const int warp = tid >> 5, lane = tid & 31;
-            for (int r = warp; r < CH; r += NT / 32) {
+            for (int r = warp; r < CK; r += NT / 32) {
                 float sq = 0.f, sk = 0.f;
                 for (int c = lane; c < D; c += 32) {
                     sq += sm.q[r * LD + c] * sm.q[r * LD + c];
@@ -156,7 +164,7 @@ prefill_simt_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k,
         bool unsafe = false;
         if (tid < D) {
             float hi = 0.f, lo = 0.f;
-            for (int r = 0; r < CH; ++r) {
+            for (int r = 0; r < CK; ++r) {
                 const float x = sm.g[r * LD + tid];
                 const float s = hi + x, bb = s - hi;  // two-sum: s + err == hi + x exactly
                 lo += (hi - (s - bb)) + (x - bb);
@@ -173,21 +181,21 @@ prefill_simt_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k,
 
         // ---- Grams. Thread (u, t) owns rows r = u + 16b and columns i = t + 16a.
         const int tu = tid / 16, tt = tid % 16;
-        float accq[4][4], acck[4][4];
+        float accq[NB][NB], acck[NB][NB];
 #pragma unroll
-        for (int b = 0; b < 4; ++b)
+        for (int b = 0; b < NB; ++b)
 #pragma unroll
-            for (int a = 0; a < 4; ++a) accq[b][a] = acck[b][a] = 0.f;
+            for (int a = 0; a < NB; ++a) accq[b][a] = acck[b][a] = 0.f;
         if (unsafe) {
             // pairwise exponentials from the raw q, k, g, only where i <= r
             for (int c = 0; c < D; ++c) {
 #pragma unroll
-                for (int b = 0; b < 4; ++b) {
+                for (int b = 0; b < NB; ++b) {
                     const int r = tu + 16 * b;
                     const float gr = sm.g[r * LD + c], grl = sm.glo[r * LD + c];
                     const float qv = sm.q[r * LD + c], kv = sm.k[r * LD + c];
 #pragma unroll
-                    for (int a = 0; a < 4; ++a) {
+                    for (int a = 0; a < NB; ++a) {
                         const int i = tt + 16 * a;
                         if (i <= r) {
                             const float d = (gr - sm.g[i * LD + c]) + (grl - sm.glo[i * LD + c]);
@@ -202,7 +210,7 @@ prefill_simt_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k,
         __syncthreads();
 
         // ---- rescale in place: q <- exp(g) q; k <- exp(g) k; g <- exp(g_L - g) k
-        for (int e = tid; e < CH * D; e += NT) {
+        for (int e = tid; e < CK * D; e += NT) {
             const int r = e / D, c = e % D;
             const float g = sm.g[r * LD + c], glo = sm.glo[r * LD + c], kv = sm.k[r * LD + c];
             const float eg = expf(g + glo);
@@ -217,28 +225,28 @@ prefill_simt_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k,
             // k_i exp(-g_i) = (exp(g_L - g_i) k_i) * exp(-g_L)
             for (int c = 0; c < D; ++c) {
                 const float ei = sm.einv[c];
-                float qr[4], kr[4], ki[4];
+                float qr[NB], kr[NB], ki[NB];
 #pragma unroll
-                for (int b = 0; b < 4; ++b) {
+                for (int b = 0; b < NB; ++b) {
                     const int r = tu + 16 * b;
                     qr[b] = sm.q[r * LD + c];
                     kr[b] = sm.k[r * LD + c];
                 }
 #pragma unroll
-                for (int a = 0; a < 4; ++a) ki[a] = sm.g[(tt + 16 * a) * LD + c] * ei;
+                for (int a = 0; a < NB; ++a) ki[a] = sm.g[(tt + 16 * a) * LD + c] * ei;
 #pragma unroll
-                for (int b = 0; b < 4; ++b)
+                for (int b = 0; b < NB; ++b)
 #pragma unroll
-                    for (int a = 0; a < 4; ++a) {
+                    for (int a = 0; a < NB; ++a) {
                         accq[b][a] += qr[b] * ki[a];
                         acck[b][a] += kr[b] * ki[a];
                     }
             }
         }
 #pragma unroll
-        for (int b = 0; b < 4; ++b)
+        for (int b = 0; b < NB; ++b)
 #pragma unroll
-            for (int a = 0; a < 4; ++a) {
+            for (int a = 0; a < NB; ++a) {
                 const int r = tu + 16 * b, i = tt + 16 * a;
                 sm.aqk[r * LDA + i] = i <= r ? accq[b][a] : 0.f;
                 sm.akk[r * LDA + i] = i < r ? sm.beta[r] * acck[b][a] : 0.f;
@@ -249,7 +257,7 @@ prefill_simt_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k,
         if (tid < D + DVS) {
             float *col = tid < D ? sm.k + tid : sm.vu + (tid - D);
             const int ld = tid < D ? LD : DVS;
-            for (int r = 0; r < CH; ++r) {
+            for (int r = 0; r < CK; ++r) {
                 float x = sm.beta[r] * col[r * ld];
                 for (int i = 0; i < r; ++i) x -= sm.akk[r * LDA + i] * col[i * ld];
                 col[r * ld] = x;
@@ -261,7 +269,7 @@ prefill_simt_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k,
         const int j = tid % DVS, rb = tid / DVS;
         {
 #pragma unroll
-            for (int m = 0; m < CH / 8; ++m) {
+            for (int m = 0; m < CK / 8; ++m) {
                 const int r = rb + 8 * m;
                 float acc = sm.vu[r * DVS + j];
                 for (int c = 0; c < D; ++c) acc -= sm.k[r * LD + c] * sm.s[c * DVS + j];
@@ -272,7 +280,7 @@ prefill_simt_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k,
 
         // ---- O = (exp(g) q) S + A_qk V_new
 #pragma unroll
-        for (int m = 0; m < CH / 8; ++m) {
+        for (int m = 0; m < CK / 8; ++m) {
             const int r = rb + 8 * m;
             if (r < L) {
                 float acc = 0.f;
@@ -300,16 +308,16 @@ prefill_simt_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k,
         }
 }
 
-template <typename TIn, int GATE>
+template <typename TIn, int GATE, int CK>
 cudaError_t launch_t(const void *q, const void *k, const void *v, const void *la,
                      const float *beta, const float *S0, void *o, float *S_T, int n_seqs,
                      int64_t T, int H, const int32_t *cu, const IoOpts &io, cudaStream_t stream) {
-    const size_t smem = sizeof(SimtSmem);
-    cudaError_t err = cudaFuncSetAttribute(prefill_simt_kernel<TIn, GATE>,
+    const size_t smem = sizeof(SimtSmem<CK>);
+    cudaError_t err = cudaFuncSetAttribute(prefill_simt_kernel<TIn, GATE, CK>,
                                            cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (err != cudaSuccess) return err;
     dim3 grid((unsigned)n_seqs, (unsigned)H, D / DVS);
-    prefill_simt_kernel<TIn, GATE><<<grid, NT, smem, stream>>>(
+    prefill_simt_kernel<TIn, GATE, CK><<<grid, NT, smem, stream>>>(
         (const TIn *)q, (const TIn *)k, (const TIn *)v, la, beta, S0, (TIn *)o, S_T, T, H, cu, io.flags,
         io.l2_eps);
     return cudaGetLastError();
@@ -320,15 +328,19 @@ cudaError_t launch_t(const void *q, const void *k, const void *v, const void *la
 cudaError_t launch_prefill_simt(const void *q, const void *k, const void *v,
                                 const void *log_alpha, int gate, const float *beta,
                                 const float *S0, void *o, float *S_T, int n_seqs, int64_t T,
-                                int H, const int32_t *cu_seqlens, int dtype, const IoOpts &io,
+                                int H, const int32_t *cu_seqlens, int dtype, int C, const IoOpts &io,
                                 cudaStream_t stream) {
     return with_gate(gate, [&](auto g) {
         constexpr int G = decltype(g)::value;
-        if (dtype == KDA_BF16)
-            return launch_t<__nv_bfloat16, G>(q, k, v, log_alpha, beta, S0, o, S_T, n_seqs, T, H,
-                                              cu_seqlens, io, stream);
-        return launch_t<float, G>(q, k, v, log_alpha, beta, S0, o, S_T, n_seqs, T, H,
-                                  cu_seqlens, io, stream);
+        auto run = [&](auto ck) {
+            constexpr int CK = decltype(ck)::value;
+            if (dtype == KDA_BF16)
+                return launch_t<__nv_bfloat16, G, CK>(q, k, v, log_alpha, beta, S0, o, S_T, n_seqs, T, H,
+                                                      cu_seqlens, io, stream);
+            return launch_t<float, G, CK>(q, k, v, log_alpha, beta, S0, o, S_T, n_seqs, T, H,
+                                          cu_seqlens, io, stream);
+        };
+        return C == 32 ? run(std::integral_constant<int, 32>{}) : run(std::integral_constant<int, 64>{});
     });
 }
 

@@ -55,7 +55,8 @@ extern "C" {
 #endif
 
 #define KDA_HEAD_DIM 128 /* dk = dv, fixed */
-#define KDA_CHUNK 64     /* the only chunk size accepted by kda_chunk_fwd */
+#define KDA_CHUNK 64       /* chunk length of the tensor-core prefill (bf16 inputs) */
+#define KDA_CHUNK_SMALL 32 /* the other chunk length kda_chunk_fwd accepts (CUDA cores) */
 
 typedef enum kda_dtype {
     KDA_BF16 = 0, /* q, k, v, o are bfloat16 */
@@ -89,7 +90,7 @@ typedef enum kda_gate {
 typedef enum kda_status {
     KDA_OK = 0,
     KDA_ERR_INVALID_ARG = -1, /* null pointer, bad size, bad offsets */
-    KDA_ERR_UNSUPPORTED = -2, /* C != 64, unknown dtype or unknown gate layout */
+    KDA_ERR_UNSUPPORTED = -2, /* C not 32 or 64, unknown dtype or unknown gate layout */
     KDA_ERR_WORKSPACE = -3,   /* workspace missing or smaller than required */
     KDA_ERR_CUDA = -4,        /* a kernel launch failed */
     KDA_ERR_TIMEOUT = -5,     /* a bounded device-side wait expired */
@@ -139,7 +140,13 @@ KDA_API int kda_chunk_fwd_launches(int B, int64_t T, int H, int C, int n_seqs, i
  *                               or NULL for zeros
  *   o          [B, T, H, 128]  dtype    output (written)
  *   S_T        [Nseq, H, 128, 128] fp32 final state (written), or NULL
- *   C          chunk length; must be 64
+ *   C          chunk length: 64 (KDA_CHUNK) or 32 (KDA_CHUNK_SMALL); the pages
+ *              name 32 to 128 as the useful range (mokono.cn section 4.1). bf16
+ *              inputs with C = 64 run on the tensor cores; fp32 inputs, and C = 32
+ *              in either dtype, run on the CUDA-core kernel (one launch, no
+ *              workspace, no output epilogue). C = 128 returns KDA_ERR_UNSUPPORTED:
+ *              the CUDA-core kernel's fp32 working set for one chunk (about 400 KB)
+ *              does not fit an SM, and the tensor-core kernels are built for 64.
  *   cu_seqlens device int32 [n_seqs + 1] token offsets of packed sequences
  *              (cu_seqlens[0] = 0, non-decreasing, cu_seqlens[n_seqs] = T),
  *              or NULL: then Nseq = B sequences of T tokens each.

@@ -258,7 +258,7 @@ def pin_varlen_equals_separate(fwd):
 
 def pin_chunked_form(fwd):
     """The chunked form (Proposition: S_r = P_r S_0 + H_r; WY/UT matrix form) equals the recurrence."""
-    for C, T in ((64, 150), (16, 37)):
+    for C, T in ((64, 150), (16, 37), (32, 100), (128, 300)):
         c = rand_case(53 + C, B=2, T=T, H=2, dk=32, dv=40, la_range=(0.001, 0.3))
         o, st = fwd(**c)
         o_c, st_c = kda_chunked_fp64(**c, C=C)

@@ -44,8 +44,8 @@ def _chunk(lib, *, q=FAKE, k=FAKE, v=FAKE, la=FAKE, beta=FAKE, S0=None, o=FAKE, 
 
 
 def test_chunk_fwd_rejects_bad_arguments(lib):
-    assert _chunk(lib, C=32) == UNSUPPORTED
-    assert _chunk(lib, C=128) == UNSUPPORTED
+    for C in (0, 16, 48, 128, 256):
+        assert _chunk(lib, C=C) == UNSUPPORTED, C
     assert _chunk(lib, dtype=7) == UNSUPPORTED
     assert _chunk(lib, B=0) == INVALID
     assert _chunk(lib, H=0) == INVALID
@@ -69,7 +69,12 @@ def test_chunk_fwd_rejects_bad_host_offsets(lib, offsets):
 def test_workspace_size_query(lib):
     out = ctypes.c_size_t(123)
     assert lib.kda_chunk_fwd_workspace_size(1, 64, 2, 64, 0, BF16, None) == INVALID
-    assert lib.kda_chunk_fwd_workspace_size(1, 64, 2, 32, 0, BF16, ctypes.byref(out)) == UNSUPPORTED
+    assert lib.kda_chunk_fwd_workspace_size(1, 64, 2, 128, 0, BF16, ctypes.byref(out)) == UNSUPPORTED
+    # C = 32 runs on the CUDA-core kernel, which needs no workspace in either dtype
+    for dtype in (BF16, F32):
+        out.value = 123
+        assert lib.kda_chunk_fwd_workspace_size(4, 4096, 16, 32, 0, dtype, ctypes.byref(out)) == 0
+        assert out.value == 0
     assert lib.kda_chunk_fwd_workspace_size(4, 4096, 16, 64, 0, BF16, ctypes.byref(out)) == 0
     assert lib.kda_chunk_fwd_workspace_size(1, 4096, 16, 64, 3, F32, ctypes.byref(out)) == 0
 
@@ -94,8 +99,12 @@ def test_launch_count_query_follows_the_plan():
     assert kda.chunk_fwd_launches(4, 4096, 16) == 2
     assert kda.chunk_fwd_launches(1, 1000, 2, n_seqs=3) == 3
     assert kda.chunk_fwd_launches(1, 256, 2, dtype=torch.float32) == 1
+    assert kda.chunk_fwd_launches(4, 4096, 16, C=32) == 1
+    assert kda.chunk_fwd_launches(1, 1000, 2, n_seqs=3, C=32) == 1
     with pytest.raises(kda.KDAError):
-        kda.chunk_fwd_launches(1, 256, 2, C=32)
+        kda.chunk_fwd_launches(1, 256, 2, C=128)
+    with pytest.raises(kda.KDAError):  # the output epilogue lives in the tensor-core chain
+        kda.chunk_fwd_launches(1, 256, 2, C=32, out_epilogue=True)
 
 
 def test_decode_rejects_bad_arguments(lib):
@@ -174,8 +183,8 @@ def test_io_entry_points_validate_their_options(lib):
     """kda_chunk_fwd_io / kda_decode_step_io check the fused options before launching."""
     Io = kda.KdaIo
 
-    def chunk(io, dtype=BF16, gate=kda.KDA_GATE_CHANNEL):
-        return lib.kda_chunk_fwd_io(FAKE, FAKE, FAKE, FAKE, gate, FAKE, None, FAKE, None, 1, 128, 2, 64,
+    def chunk(io, dtype=BF16, gate=kda.KDA_GATE_CHANNEL, C=64):
+        return lib.kda_chunk_fwd_io(FAKE, FAKE, FAKE, FAKE, gate, FAKE, None, FAKE, None, 1, 128, 2, C,
                                     None, 0, None, dtype, None, 0, ctypes.byref(io), None)
 
     def decode(io):
@@ -187,6 +196,7 @@ def test_io_entry_points_validate_their_options(lib):
     assert chunk(Io(1, float("nan"), 0, None, None, 0.0)) == INVALID   # NaN eps
     assert chunk(Io(0, 0.0, 0, gate16, None, -1.0)) == INVALID          # negative output eps
     assert chunk(Io(0, 0.0, 0, gate16, None, 1e-6), dtype=F32) == UNSUPPORTED  # fp32: no epilogue
+    assert chunk(Io(0, 0.0, 0, gate16, None, 1e-6), C=32) == UNSUPPORTED  # C = 32: no epilogue
     assert chunk(Io(0, 0.0, 0, gate16 + 8, None, 1e-6)) == INVALID     # bf16 gate: 16-byte aligned
     assert chunk(Io(0, 0.0, 0, gate16, gate16 + 4, 1e-6)) == INVALID    # weights: 16-byte aligned
     assert decode(Io(1, -1.0, 0, None, None, 0.0)) == INVALID
