@@ -54,7 +54,7 @@ int make_io(const kda_io *io, bool out_ok, int esize, kda::IoOpts *opts) {
         const uintptr_t align = esize == 2 ? 16u : (uintptr_t)esize;
         if (((uintptr_t)io->out_gate & (align - 1)) != 0) return KDA_ERR_INVALID_ARG;
         if (io->out_norm_weight && ((uintptr_t)io->out_norm_weight & 15u) != 0) return KDA_ERR_INVALID_ARG;
-        opts->out_gate = io->out_gate;
+        opts->out_gate = io->out_gate;  // (fp32 gates are read as float4 by the prefill epilogue)
         opts->out_w = io->out_norm_weight;
         opts->out_eps = io->out_norm_eps;
     }
@@ -101,9 +101,9 @@ int kda_chunk_fwd_io_launches(int B, int64_t T, int H, int C, int n_seqs, int dt
     const int st = check_prefill_shape(B, T, H, C, n_seqs, dtype);
     if (st != KDA_OK) return st;
     const bool out_epi = io && io->out_gate;
-    if (out_epi && !tensor_core_path(C, dtype)) return KDA_ERR_UNSUPPORTED;
-    *n_kernels = tensor_core_path(C, dtype)
-                     ? kda::prefill_tc_launches(B, T, H, n_seqs, out_epi, io && io->qk_l2norm) : 1;
+    const int64_t n_tok = n_seqs > 0 ? T : (int64_t)B * T;
+    *n_kernels = (tensor_core_path(C, dtype) ? kda::prefill_tc_launches(B, T, H, n_seqs, io && io->qk_l2norm) : 1) +
+                 (out_epi && n_tok > 0 ? 1 : 0);
     return KDA_OK;
 }
 
@@ -136,8 +136,10 @@ int kda_chunk_fwd_io(const void *q, const void *k, const void *v, const void *lo
     if (!valid_gate(gate)) return KDA_ERR_UNSUPPORTED;
     kda::IoOpts opts;
     const bool tc = tensor_core_path(C, dtype);
-    st = make_io(io, tc, dtype == KDA_BF16 ? 2 : 4, &opts);
+    st = make_io(io, true, dtype == KDA_BF16 ? 2 : 4, &opts);
     if (st != KDA_OK) return st;
+    if (opts.out_gate && ((uintptr_t)opts.out_gate & 15u) != 0) return KDA_ERR_INVALID_ARG;  // vector rows
+    if (opts.out_gate && ((uintptr_t)o & 15u) != 0) return KDA_ERR_INVALID_ARG;
     const bool packed = n_seqs > 0;
     if (packed != (cu_seqlens != nullptr)) return KDA_ERR_INVALID_ARG;
     if (T > 0 && (!q || !k || !v || !beta || !o)) return KDA_ERR_INVALID_ARG;
@@ -170,6 +172,8 @@ int kda_chunk_fwd_io(const void *q, const void *k, const void *v, const void *lo
         err = kda::launch_prefill_simt(q, k, v, log_alpha, gate, beta, S0, o, S_T, nseq, T, H,
                                        cu_seqlens, dtype, C, opts, s);
     }
+    if (err == cudaSuccess && opts.out_gate)
+        err = kda::launch_out_epilogue(o, opts, (packed ? T : (int64_t)B * T) * H, dtype, s);
     if (err == cudaErrorInvalidValue) return KDA_ERR_INVALID_ARG;
     return err == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }

@@ -126,13 +126,19 @@ cudaError_t launch_prefill_simt(const void *q, const void *k, const void *v,
 
 // Tensor-core prefill (bf16 q/k/v): workspace bytes and launcher.
 size_t prefill_tc_workspace(int B, int64_t T, int H, int n_seqs);
-// out_epilogue: the call applies an output gate and norm (runs prep and the full-head chain);
-// l2norm: q and k are normalised in the kernel (no fused grid).
-int prefill_tc_launches(int B, int64_t T, int H, int n_seqs, bool out_epilogue = false, bool l2norm = false);
+// l2norm: q and k are normalised in the kernel (no fused grid). The output epilogue is
+// not counted (launch_out_epilogue, one more launch).
+int prefill_tc_launches(int B, int64_t T, int H, int n_seqs, bool l2norm = false);
+// Runs every fused step of `io` except the output epilogue.
 cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, const void *log_alpha,
                               int gate, const float *beta, const float *S0, void *o, float *S_T, int B,
                               int64_t T, int H, const int32_t *cu_seqlens, int n_seqs,
                               void *workspace, const IoOpts &io, cudaStream_t stream);
+
+// Output epilogue (RMSNorm over each row's 128 channels, weights, sigmoid gate), in place
+// on the `rows` rows of o (dtype KDA_BF16 or KDA_F32). Nothing is launched without
+// io.out_gate or rows.
+cudaError_t launch_out_epilogue(void *o, const IoOpts &io, int64_t rows, int dtype, cudaStream_t stream);
 
 // Backward pass (kda_chunk_bwd): arguments of one call.
 struct BwdArgs {

@@ -436,11 +436,27 @@ __device__ __forceinline__ void prep_item(Worker &w, const PrepArgs &a, int slot
         }
     } else {
         const int64_t row0 = tok0 * H + h;  // token-head row of the chunk's first token
+        if constexpr (logit_gate<GATE>()) {
+            // all eight rows' loads first, then log sigmoid: the loads stay in flight together
+            constexpr int RAW = GATE == KDA_GATE_CHANNEL_LOGIT ? KDA_GATE_CHANNEL : KDA_GATE_CHANNEL_BF16;
+            constexpr float ZERO_LOGIT = 1e30f;  // rows >= L: log sigmoid(+big) = 0
 #pragma unroll
-        for (int v = 0; v < 8; ++v) {
-            const int r = 8 * warp + v;
-            g4[v] = r < L ? load_gate4<GATE>(a.log_alpha, row0 + (int64_t)r * H, 4 * f)
-                          : make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int v = 0; v < 8; ++v) {
+                const int r = 8 * warp + v;
+                g4[v] = r < L ? load_gate4<RAW>(a.log_alpha, row0 + (int64_t)r * H, 4 * f)
+                              : make_float4(ZERO_LOGIT, ZERO_LOGIT, ZERO_LOGIT, ZERO_LOGIT);
+            }
+#pragma unroll
+            for (int v = 0; v < 8; ++v)
+                g4[v] = make_float4(log_sigmoid(g4[v].x), log_sigmoid(g4[v].y), log_sigmoid(g4[v].z),
+                                    log_sigmoid(g4[v].w));
+        } else {
+#pragma unroll
+            for (int v = 0; v < 8; ++v) {
+                const int r = 8 * warp + v;
+                g4[v] = r < L ? load_gate4<GATE>(a.log_alpha, row0 + (int64_t)r * H, 4 * f)
+                              : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
         }
 #pragma unroll
         for (int v = 1; v < 8; ++v) {
@@ -913,11 +929,6 @@ struct ChainArgs {
     // Launched as a dependent of the prep kernel (which may still run): everything up
     // to the first blob load only touches the call's inputs, then griddep_wait.
     bool wait_prior = false;
-    // Output epilogue of the full-head chain (null: none): o <- RMSNorm(o) * w * sigmoid(gate)
-    // per (token, head) row, with w = out_w (null: ones) and eps = out_eps.
-    const __nv_bfloat16 *out_gate = nullptr;
-    const float *out_w = nullptr;
-    float out_eps = 0.f;
 };
 
 // The part of one (sequence, head, slice) recurrence a chain task runs: chunks [c0, c1)
@@ -1230,462 +1241,6 @@ kda_chain_kernel(const __grid_constant__ CUtensorMap tm_v,
 }
 
 // =====================================================================================
-// full-head chain: per (sequence, head) state recurrence, transposed onto TMEM lanes
-// =====================================================================================
-// One CTA per (sequence, head) walks the chunks in order with all 128 value columns.
-// Every product is formed transposed, so that TMEM lane j holds value column j:
-//   [Q~; W] S  -> (S^T [Q~; W]^T)[j][r']    A = S^T (TMEM), B = the [Q~; W] image (N = 128)
-//   K~^T V_new -> (V_new^T K~)[j][c]        A = V_new^T (TMEM), B = the K~ image (MN-major)
-//   A_qk V_new -> (V_new^T A_qk^T)[j][r]    A = V_new^T (TMEM), B = the A_qk image
-//   U          -> (V^T (T Diag b)^T)[j][r]  A = the value tile (shared, MN-major), B = T Diag(b)
-// The state's bf16 copy S^T and V_new^T are written to TMEM by the epilogue warps and used
-// there as the A operand, so no operand image of the recurrence goes through shared
-// memory, and the chunk's blob is read once per head. The blob layout is the one the prep
-// kernel writes for the 64-column chains.
-// The tensor pipe runs its MMAs in issue order at about one K = 16 instruction per 50 ns
-// for these shapes, whatever N is, so the chain is built around issuing few of them: 20
-// per chunk (8 for [Q~; W] S at N = 128, 4 each for the rest), with the recurrence's
-// critical path ([Q~; W] S -> V_new = U - W S -> K~^T V_new -> S_{n+1} = Diag(gamma) S_n +
-// K~^T V_new) issued first and the output MMA and U_{n+1} behind it.
-// Warps: 0-7 epilogue (warp w: TMEM lane quarter w % 4, i.e. value columns 32 (w % 4) ..
-// +31, and half w / 4 of the key channels / tokens); 8 issues the MMAs; 9 issues the stage
-// loads, the L2 prefetches and the output stores. Thread (j, half) keeps
-// S^T[j][64 half .. +63] in fp32 registers. The output of chunk n is staged in shared
-// memory by the epilogue right after the chunk ends, while [Q~; W] S of chunk n + 1 runs
-// (into the other D1 buffer), and stored by TMA (plain stores for the rows of a partial
-// last chunk, whose tile would run into the next sequence).
-constexpr int C2_NT = 32 * (CHAIN_EPI_WARPS + 2);
-constexpr int C2_ISSUER = CHAIN_EPI_WARPS, C2_LOADER = CHAIN_EPI_WARPS + 1;  // warp indices
-// TMEM columns (512): two D1 buffers of 128 ([Q~ S | W S], then the output Q~ S + A_qk V_new
-// in columns 0..63; V_new^T is written over the W S half once it has been read: tokens
-// 0..31 at +64, 32..63 at +96, inside the columns their writers read W S from), then
-// K~^T V_new, U and S^T as bf16 pairs.
-constexpr uint32_t C2_D1 = 0;
-constexpr uint32_t C2_D3 = 256;
-constexpr uint32_t C2_U = 384;
-constexpr uint32_t C2_ST = 448;
-constexpr uint32_t C2_TMEM_COLS = 512;
-__device__ __forceinline__ uint32_t c2_vn_col(int half) { return 64u + 32u * (uint32_t)half; }
-constexpr int C2_PF = 6;    // chunks ahead whose blob and value tile are prefetched into L2
-constexpr int C2_OBUF = 3;  // output staging tiles
-struct Chain2Layout {
-    // A stage mirrors the blob (A1, AQK, KTT, TB at the blob's offsets), then the value
-    // tile (two TMA boxes of 64 columns) and gamma_L.
-    static constexpr uint32_t A1 = 0;
-    static constexpr uint32_t AQK = 32768;
-    static constexpr uint32_t KTT = 40960;
-    static constexpr uint32_t TB = 57344;
-    static constexpr uint32_t V = 65536;
-    static constexpr uint32_t GAM = V + 16384;
-    static constexpr uint32_t STAGE = ((GAM + 512 + 1023) / 1024) * 1024;
-    // output staging tiles: 64 tokens x 128 columns bf16 as two plain 64 x 64 TMA boxes
-    static constexpr uint32_t OST = 2 * STAGE;
-    static constexpr uint32_t BAR = OST + C2_OBUF * 16384;  // 9 mbarriers
-    static constexpr uint32_t TMEM = BAR + 72;
-    static constexpr uint32_t BYTES = TMEM + 8 + 1024;
-    // part 1 (A1, TB, V) feeds [Q~; W] S and U; part 2 (AQK, KTT, GAM) the rest
-    static constexpr uint32_t LOAD1_BYTES = 32768 + 8192 + 16384;
-    static constexpr uint32_t LOAD2_BYTES = 8192 + 16384 + 512;
-};
-static_assert(Chain2Layout::BYTES <= 232448, "full-head chain exceeds the shared memory of an SM");
-// Named barriers: VNEW (epilogue arrives, MMA warp waits), END (every thread, once per
-// chunk; ORs the `dead` flags), CHAIN (every thread, prologue and end).
-constexpr uint32_t C2_BAR_VNEW = 1, C2_BAR_END = 2, C2_BAR_CHAIN = 3;
-constexpr uint32_t C2_BAR_OROWS = 4;  // epilogue warps: an output tile is fully staged
-constexpr uint32_t C2_VNEW_COUNT = 32 * (CHAIN_EPI_WARPS + 1);
-
-// The recurrence of one (sequence, head) over the window `win` (see ChainWindow; all 128
-// columns), run by threads 0 .. C2_NT-1 on shared memory `sm`. tm_o: the output as plain
-// 64 x 64 bf16 boxes.
-__device__ __forceinline__ void chain2_task(unsigned char *sm, const int tid, const ChainArgs &a,
-                                            const CUtensorMap *tm_o, const CUtensorMap *tm_g, const int seq,
-                                            const int h, const ChainWindow &win) {
-    using Lay = Chain2Layout;
-    const int warp = tid >> 5, lane = tid & 31;
-    const bool epi = warp < CHAIN_EPI_WARPS;
-    const int q4 = warp & 3, hf = (warp >> 2) & 1;
-    const CUtensorMap &tm_v = *a.tm_v;
-    const int64_t T = a.T;
-    const int H = a.H, nck = a.nck;
-    const SeqSpan span = seq_span(a.cu, T, seq);
-    const int c0 = win.c0;
-    const int seq_chunks = (int)((span.len + CH - 1) / CH);
-    const int c_end = win.c1 < 0 || win.c1 > seq_chunks ? seq_chunks : win.c1;
-    const int nchunks = c_end > c0 ? c_end - c0 : 0;
-    const int64_t slot0 = (a.chunk_off ? (int64_t)a.chunk_off[seq] : (int64_t)seq * nck) + c0;
-
-    uint64_t *bar_ld1 = reinterpret_cast<uint64_t *>(sm + Lay::BAR);  // [2] part 1, per stage
-    uint64_t *bar_ld2 = bar_ld1 + 2;                                  // [2] part 2, per stage
-    uint64_t *bar_u = bar_ld1 + 4;   // U done
-    uint64_t *bar_w = bar_ld1 + 5;   // [Q~; W] S done (part 1 of its stage fully read)
-    uint64_t *bar_d3 = bar_ld1 + 6;  // K~^T V_new done
-    uint64_t *bar_o = bar_ld1 + 7;   // [2] output complete, per D1 buffer
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + Lay::TMEM);
-    bool dead = false;
-
-    auto blob_of = [&](int chunk) {
-        return a.ws_blobs + ((size_t)(slot0 + chunk) * H + h) * BLOB_BYTES;
-    };
-    auto chunk_y = [&](int chunk) { return (int)(span.start + (int64_t)(c0 + chunk) * CH); };
-    auto issue_load1 = [&](int chunk, int stage) {
-        const unsigned char *blob = blob_of(chunk);
-        unsigned char *st = sm + stage * Lay::STAGE;
-        mbar_arrive_expect_tx(&bar_ld1[stage], Lay::LOAD1_BYTES);
-        bulk_g2s(st + Lay::A1, blob + BLOB_A1, 32768, &bar_ld1[stage]);
-        bulk_g2s(st + Lay::TB, blob + BLOB_TB, 8192, &bar_ld1[stage]);
-        tma_load_2d(st + Lay::V, &tm_v, h * D, chunk_y(chunk), &bar_ld1[stage]);
-        tma_load_2d(st + Lay::V + 8192, &tm_v, h * D + 64, chunk_y(chunk), &bar_ld1[stage]);
-    };
-    auto issue_load2 = [&](int chunk, int stage) {
-        const unsigned char *blob = blob_of(chunk);
-        unsigned char *st = sm + stage * Lay::STAGE;
-        mbar_arrive_expect_tx(&bar_ld2[stage], Lay::LOAD2_BYTES);
-        bulk_g2s(st + Lay::AQK, blob + BLOB_AQK, 8192, &bar_ld2[stage]);
-        bulk_g2s(st + Lay::KTT, blob + BLOB_KTT, 16384, &bar_ld2[stage]);
-        bulk_g2s(st + Lay::GAM, blob + BLOB_GAM, 512, &bar_ld2[stage]);
-    };
-    auto prefetch = [&](int chunk) {  // warm L2 with a later chunk's blob, value tile, output gate
-        bulk_prefetch_l2(blob_of(chunk), BLOB_BYTES);
-        tma_prefetch_l2_2d(&tm_v, h * D, chunk_y(chunk));
-        tma_prefetch_l2_2d(&tm_v, h * D + 64, chunk_y(chunk));
-        if (a.out_gate) {
-            tma_prefetch_l2_2d(tm_g, h * D, chunk_y(chunk));
-            tma_prefetch_l2_2d(tm_g, h * D + 64, chunk_y(chunk));
-        }
-    };
-    // A chunk whose output goes through a staging tile: all 64 rows in the sequence.
-    auto full_chunk = [&](int m) { return chunk_rows(span.len, (int64_t)(c0 + m) * CH) == CH; };
-    auto ost = [&](int m) { return sm + Lay::OST + (m % C2_OBUF) * 16384; };
-    // MMA warp, lane 0: TMA-stores the staged output of chunk m.
-    auto store_tile = [&](int m) {
-        tma_store_2d(tm_o, h * D, chunk_y(m), ost(m));
-        tma_store_2d(tm_o, h * D + 64, chunk_y(m), ost(m) + 8192);
-        bulk_commit();
-    };
-
-    if (tid == 0) {
-        for (int b = 0; b < 9; ++b) mbar_init(&bar_ld1[b], 1);
-        fence_mbar_init();
-    }
-    if (warp == 0) {
-        tmem_alloc(tmem_slot, C2_TMEM_COLS);
-        tmem_relinquish();
-    }
-    const int j = 32 * q4 + lane;  // value column of an epilogue thread
-    const int cb = 64 * hf;        // its first key channel
-    const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
-    float s_reg[64];
-    if (epi) {
-#pragma unroll
-        for (int e = 0; e < 64; ++e) {
-            const int c = cb + e;
-            float x = win.s0 ? win.s0[(int64_t)c * D + j] : 0.f;
-            if (win.s0_identity) x = c == j ? 1.f : 0.f;
-            s_reg[e] = x;
-        }
-    }
-    tc_fence_before();
-    named_bar_sync(C2_BAR_CHAIN, C2_NT);  // TMEM allocated, barriers initialised
-    tc_fence_after();
-    const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(tmem_slot);
-    if (epi) {  // S_0^T as bf16 pairs: this thread's 64 channels -> 32 columns
-#pragma unroll
-        for (int p = 0; p < 2; ++p) {
-            uint32_t r[16];
-#pragma unroll
-            for (int e = 0; e < 16; ++e) r[e] = pack_bf16x2(s_reg[32 * p + 2 * e], s_reg[32 * p + 2 * e + 1]);
-            tmem_st16(tmem + lane_off + C2_ST + 32 * hf + 16 * p, r);
-        }
-        tmem_wait_st();
-    }
-    if (a.wait_prior) {  // the blobs exist once the prep grid has completed
-        griddep_wait();
-        fence_proxy_async_global();
-    }
-    tc_fence_before();
-    named_bar_sync(C2_BAR_CHAIN, C2_NT);  // S_0^T is in TMEM
-    tc_fence_after();
-    const uint32_t sm_base = smem_u32(sm);
-
-    if (warp == C2_ISSUER) {
-        // ------------------------------------------------------------ MMA warp
-        const uint32_t id64 = idesc_bf16(128, 64, 0, 0), id128 = idesc_bf16(128, 128, 0, 0),
-                       id128_mn = idesc_bf16(128, 128, 0, 1), id_u = idesc_bf16(128, 64, 1, 0);
-        auto issue_u = [&](int m) {  // U_m = V_m^T (T Diag b)_m^T
-            const uint32_t st_base = sm_base + (m & 1) * Lay::STAGE;
-            mma_run<CH>(tmem + C2_U, mnmajor(st_base + Lay::V, 8192), kmajor(st_base + Lay::TB, 64), id_u, false);
-            mma_commit(bar_u);
-        };
-        // the 4 K steps of an MMA whose A is V_new^T (two 16-column halves, see c2_vn_col)
-        auto run_vn = [&](uint32_t d, uint32_t vn, Operand b, uint32_t idesc, bool acc) {
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-                mma_bf16_ts(d, vn + c2_vn_col(kk >> 1) + 8u * (uint32_t)(kk & 1), b.desc(kk), idesc,
-                            (acc || kk > 0) ? 1u : 0u);
-        };
-        if (lane == 0 && nchunks > 0 && mbar_wait(&bar_ld1[0], 0, dead, &g_kda_status)) {
-            tc_fence_after();
-            issue_u(0);
-        }
-#pragma unroll 1
-        for (int n = 0; n < nchunks; ++n) {
-            const int stage = n & 1;
-            const uint32_t st_base = sm_base + stage * Lay::STAGE;
-            const uint32_t lph = (uint32_t)(n >> 1) & 1u;
-            const uint32_t d1 = tmem + C2_D1 + 128u * (uint32_t)(n & 1);
-            if (lane == 0 && mbar_wait(&bar_ld1[stage], lph, dead, &g_kda_status)) {
-                tc_fence_after();
-                mma_run_ts<D>(d1, tmem + C2_ST, kmajor(st_base + Lay::A1, 128), id128, false);
-                mma_commit(bar_w);
-            }
-            __syncwarp();
-            named_bar_sync(C2_BAR_VNEW, C2_VNEW_COUNT);  // V_new^T of chunk n is in TMEM
-            if (lane == 0 && mbar_wait(&bar_ld2[stage], lph, dead, &g_kda_status)) {
-                tc_fence_after();
-                run_vn(tmem + C2_D3, d1, mnmajor(st_base + Lay::KTT, 8192), id128_mn, false);
-                mma_commit(bar_d3);
-                run_vn(d1, d1, kmajor(st_base + Lay::AQK, 64), id64, true);
-                mma_commit(&bar_o[n & 1]);
-                if (n + 1 < nchunks &&
-                    mbar_wait(&bar_ld1[(n + 1) & 1], (uint32_t)((n + 1) >> 1) & 1u, dead, &g_kda_status)) {
-                    tc_fence_after();
-                    issue_u(n + 1);
-                }
-            }
-            __syncwarp();
-            if (named_bar_or(C2_BAR_END, C2_NT, dead)) {
-                dead = true;
-                break;
-            }
-        }
-    } else if (warp == C2_LOADER) {
-        // ------------------------------------------------------------ load warp
-        if (lane == 0) {
-            for (int m = 0; m < 2 && m < nchunks; ++m) {
-                issue_load1(m, m);
-                issue_load2(m, m);
-            }
-            for (int m = 2; m < C2_PF && m < nchunks; ++m) prefetch(m);
-        }
-#pragma unroll 1
-        for (int n = 0; n < nchunks; ++n) {
-            const int stage = n & 1;
-            const uint32_t lph = (uint32_t)(n >> 1) & 1u;
-            // part 1 of the stage is free once [Q~; W] S has completed (U_n is done before
-            // it): refill it with chunk n + 2
-            if (lane == 0 && n + 2 < nchunks && mbar_wait(bar_w, (uint32_t)n & 1u, dead, &g_kda_status)) {
-                issue_load1(n + 2, stage);
-                if (n + C2_PF < nchunks) prefetch(n + C2_PF);
-            }
-            // the output of chunk n - 2, staged between the ends of chunks n - 2 and n - 1.
-            // Staging buffer m % 3 is staged again after the end of chunk m + 3, so before
-            // this chunk's end only the store of chunk n - 3 must have been read.
-            if (lane == 0 && win.write_o) {
-                if (n >= 2 && full_chunk(n - 2)) store_tile(n - 2);
-                else bulk_commit();  // an empty group keeps one group per chunk
-                bulk_wait_read_but<1>();
-            }
-            __syncwarp();
-            if (named_bar_or(C2_BAR_END, C2_NT, dead)) {
-                dead = true;
-                break;
-            }
-            // part 2 is free once the output MMA (the last reader of AQK and KTT) has
-            // completed and the state update (the reader of GAM) has passed C2_BAR_END
-            if (lane == 0 && n + 2 < nchunks && mbar_wait(&bar_o[stage], lph, dead, &g_kda_status))
-                issue_load2(n + 2, stage);
-            __syncwarp();
-        }
-    } else {
-        // ------------------------------------------------------------ epilogue warps
-        // Output of chunk m (columns 0..63 of its D1 buffer): this thread's value column j,
-        // tokens 32 half .. +31.
-        const bool out_epi = a.out_gate != nullptr;
-        // Row pass layout: 16 lanes per row, lane l % 16 takes columns 8 (l % 16) .. +7;
-        // warp w takes rows 2w + l / 16 + 16 p for p = 0..3.
-        const int rc0 = 8 * (lane & 15);
-        float ow[8] = {1.f, 1.f, 1.f, 1.f, 1.f, 1.f, 1.f, 1.f};  // RMSNorm weights of those columns
-        if (out_epi && a.out_w) {
-            const float4 w0 = *reinterpret_cast<const float4 *>(a.out_w + rc0);
-            const float4 w1 = *reinterpret_cast<const float4 *>(a.out_w + rc0 + 4);
-            ow[0] = w0.x; ow[1] = w0.y; ow[2] = w0.z; ow[3] = w0.w;
-            ow[4] = w1.x; ow[5] = w1.y; ow[6] = w1.z; ow[7] = w1.w;
-        }
-        auto store_output = [&](int m) {
-            // the output gate of this warp's 8 rows of the tile (row pass below) into L1,
-            // so that its loads there hit (the load warp has brought it into L2)
-            if (out_epi && (lane & 15) == 0) {
-                const int64_t g0 = span.start + (int64_t)(c0 + m) * CH;
-                const int glive = chunk_rows(span.len, (int64_t)(c0 + m) * CH);
-#pragma unroll
-                for (int rr = 0; rr < 8; ++rr) {
-                    const int r = 8 * warp + rr;
-                    if (r < glive) prefetch_l1(a.out_gate + ((g0 + r) * H + h) * (int64_t)D + 4 * lane);
-                }
-            }
-            mbar_wait(&bar_o[m & 1], (uint32_t)(m >> 1) & 1u, dead, &g_kda_status);
-            tc_fence_after();
-            float ov[32];
-            tmem_ld32(tmem + lane_off + C2_D1 + 128u * (uint32_t)(m & 1) + 32u * hf, ov);
-            const int64_t m0 = (int64_t)(c0 + m) * CH;
-            const int live = chunk_rows(span.len, m0);
-            {
-                // Into the staging tile (rows of 64 columns, two boxes), in 4-byte pairs of
-                // adjacent columns: lanes j and j ^ 1 swap one value per pair of tokens, so
-                // the even lane writes token e of columns (j, j + 1) and the odd lane token
-                // e + 1 of columns (j - 1, j).
-                const bool odd = lane & 1;
-                unsigned char *row0 = ost(m) + (j >> 6) * 8192 + (32 * hf) * 128 + ((j & 63) & ~1) * 2 +
-                                      (odd ? 128 : 0);
-#pragma unroll
-                for (int e = 0; e < 32; e += 2) {
-                    const float mine = odd ? ov[e + 1] : ov[e];
-                    const float other = __shfl_xor_sync(0xffffffffu, odd ? ov[e] : ov[e + 1], 1);
-                    *reinterpret_cast<uint32_t *>(row0 + e * 128) =
-                        odd ? pack_bf16x2(other, mine) : pack_bf16x2(mine, other);
-                }
-            }
-            if (!out_epi && live == CH) {  // a full chunk goes out by TMA as staged
-                fence_async_smem();
-                return;
-            }
-            // Row pass over the staged tile (16 lanes per row, see rc0). It applies the
-            // output epilogue, and writes the rows of a partial chunk straight to the
-            // output (a full chunk goes back to the tile, for TMA).
-            named_bar_sync(C2_BAR_OROWS, 32 * CHAIN_EPI_WARPS);
-            const int64_t tok0 = span.start + m0;
-            uint4 graw[4];  // the output gate of this lane's four rows, loads in flight together
-            if (out_epi) {
-#pragma unroll
-                for (int p = 0; p < 4; ++p) {
-                    const int r = 16 * p + 2 * warp + (lane >> 4);
-                    graw[p] = r < live ? *reinterpret_cast<const uint4 *>(a.out_gate + ((tok0 + r) * H + h) * (int64_t)D + rc0)
-                                       : make_uint4(0u, 0u, 0u, 0u);
-                }
-            }
-#pragma unroll
-            for (int p = 0; p < 4; ++p) {
-                const int r = 16 * p + 2 * warp + (lane >> 4);
-                unsigned char *cell = ost(m) + (rc0 >> 6) * 8192 + r * 128 + (rc0 & 63) * 2;
-                uint4 raw = *reinterpret_cast<const uint4 *>(cell);
-                if (out_epi) {
-                    const uint32_t ow32[4] = {raw.x, raw.y, raw.z, raw.w};
-                    const uint32_t gw32[4] = {graw[p].x, graw[p].y, graw[p].z, graw[p].w};
-                    float x[8], g[8];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float2 xv = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&ow32[e]));
-                        const float2 gv = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&gw32[e]));
-                        x[2 * e] = xv.x; x[2 * e + 1] = xv.y;
-                        g[2 * e] = gv.x; g[2 * e + 1] = gv.y;
-                    }
-                    float ss = 0.f;
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) ss += x[e] * x[e];
-#pragma unroll
-                    for (int off = 8; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
-                    const float inv = rsqrtf(ss * (1.f / D) + a.out_eps);
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) x[e] *= inv * ow[e] * __fdividef(1.f, 1.f + __expf(-g[e]));
-                    raw = make_uint4(pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]), pack_bf16x2(x[4], x[5]),
-                                     pack_bf16x2(x[6], x[7]));
-                }
-                if (live == CH) *reinterpret_cast<uint4 *>(cell) = raw;
-                else if (r < live)
-                    *reinterpret_cast<uint4 *>(a.o + ((tok0 + r) * H + h) * (int64_t)D + rc0) = raw;
-            }
-            if (live == CH) fence_async_smem();
-        };
-#pragma unroll 1
-        for (int n = 0; n < nchunks; ++n) {
-            const int stage = n & 1;
-            const uint32_t ph = (uint32_t)n & 1u;
-            const uint32_t lph = (uint32_t)(n >> 1) & 1u;
-            const uint32_t d1 = tmem + lane_off + C2_D1 + 128u * (uint32_t)(n & 1);
-            {  // V_new = U - W S for tokens 32 half .. +31, written over the W S it read
-                mbar_wait(bar_u, ph, dead, &g_kda_status);
-                mbar_wait(bar_w, ph, dead, &g_kda_status);
-                tc_fence_after();
-                float ws[32], us[32];
-                tmem_ld32x2(d1 + 64 + 32 * hf, tmem + lane_off + C2_U + 32 * hf, ws, us);
-                uint32_t r[16];
-#pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    const float v0 = (win.u_zero ? 0.f : us[2 * e]) - ws[2 * e];
-                    const float v1 = (win.u_zero ? 0.f : us[2 * e + 1]) - ws[2 * e + 1];
-                    r[e] = pack_bf16x2(v0, v1);
-                }
-                tmem_st16(d1 + c2_vn_col(hf), r);
-                tmem_wait_st();
-                tc_fence_before();
-                named_bar_arrive(C2_BAR_VNEW, C2_VNEW_COUNT);
-            }
-            {  // S^T <- S^T Diag(gamma_L) + (K~^T V_new)^T for channels cb .. cb+63
-                mbar_wait(&bar_ld2[stage], lph, dead, &g_kda_status);  // gamma_L
-                mbar_wait(bar_d3, ph, dead, &g_kda_status);  // also ends [Q~; W] S, the reader of S_n^T
-                tc_fence_after();
-                const float *gam = reinterpret_cast<const float *>(sm + stage * Lay::STAGE + Lay::GAM) + cb;
-                float dva[32], dvb[32];
-                tmem_ld32x2(tmem + lane_off + C2_D3 + cb, tmem + lane_off + C2_D3 + cb + 32, dva, dvb);
-#pragma unroll
-                for (int p = 0; p < 2; ++p) {
-                    const float *dv = p ? dvb : dva;
-                    uint32_t r[16];
-#pragma unroll
-                    for (int e = 0; e < 32; e += 4) {
-                        const float4 g4 = *reinterpret_cast<const float4 *>(gam + 32 * p + e);
-                        float *s = s_reg + 32 * p + e;
-                        s[0] = g4.x * s[0] + dv[e];
-                        s[1] = g4.y * s[1] + dv[e + 1];
-                        s[2] = g4.z * s[2] + dv[e + 2];
-                        s[3] = g4.w * s[3] + dv[e + 3];
-                        r[e / 2] = pack_bf16x2(s[0], s[1]);
-                        r[e / 2 + 1] = pack_bf16x2(s[2], s[3]);
-                    }
-                    tmem_st16(tmem + lane_off + C2_ST + 32 * hf + 16 * p, r);
-                }
-                tmem_wait_st();
-            }
-            tc_fence_before();
-            if (named_bar_or(C2_BAR_END, C2_NT, dead)) {
-                dead = true;
-                break;
-            }
-            // this chunk's output, while [Q~; W] S of the next one runs into the other D1
-            // buffer (this one is overwritten only after the next chunk's end)
-            if (win.write_o) store_output(n);
-        }
-        if (win.st) {
-#pragma unroll
-            for (int e = 0; e < 64; ++e) win.st[(int64_t)(cb + e) * D + j] = s_reg[e];
-        }
-    }
-    tc_fence_before();
-    named_bar_sync(C2_BAR_CHAIN, C2_NT);
-    if (warp == 0) tmem_dealloc(tmem, C2_TMEM_COLS);
-    if (warp == C2_LOADER && lane == 0 && win.write_o && !dead) {  // the last staged tiles
-        for (int m = nchunks - 2; m < nchunks; ++m)
-            if (m >= 0 && full_chunk(m)) store_tile(m);
-        bulk_wait_read();
-    }
-}
-
-__global__ void __launch_bounds__(C2_NT, 1)
-kda_chain2_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
-                  const __grid_constant__ CUtensorMap tm_g, const unsigned char *__restrict__ ws_blobs,
-                  const int32_t *__restrict__ chunk_off, const float *__restrict__ S0,
-                  __nv_bfloat16 *__restrict__ o, float *__restrict__ S_T, const int32_t *__restrict__ cu,
-                  int64_t T, int H, int nck, int wait_prior, const __nv_bfloat16 *__restrict__ out_gate,
-                  const float *__restrict__ out_w, float out_eps) {
-    extern __shared__ unsigned char smem_raw[];
-    if (chunk_off && !packed_offsets_ok(chunk_off, (int)gridDim.x)) return;
-    const ChainArgs a{&tm_v, ws_blobs, chunk_off, S0, o, S_T, cu, T, H, nck, nullptr, wait_prior != 0,
-                      out_gate, out_w, out_eps};
-    chain2_task(aligned_smem(smem_raw), threadIdx.x, a, &tm_o, &tm_g, blockIdx.x, blockIdx.y,
-                full_window(a, blockIdx.x, blockIdx.y));
-}
-
-// =====================================================================================
 // segment scan: long sequences with few sequence-heads (batched inputs)
 // =====================================================================================
 // The chunks of every sequence are cut into n_seg segments of seg_len chunks (the last
@@ -1947,10 +1502,9 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 }
 
 // [n_tok, H*128] row-major tensor; boxes of 64 rows x 64 bf16 or 128 fp32 columns. bf16
-// boxes use the 128-byte swizzle by default, so a box lands in shared memory as one
-// swizzled operand block; with swizzle = false (and for the fp32 log_alpha box) a box is
-// plain rows.
-bool make_map(CUtensorMap *m, const void *ptr, bool bf16, int64_t n_tok, int H, bool swizzle = true) {
+// boxes use the 128-byte swizzle, so a box lands in shared memory as one swizzled
+// operand block; the fp32 log_alpha box is plain rows.
+bool make_map(CUtensorMap *m, const void *ptr, bool bf16, int64_t n_tok, int H) {
     auto fn = encode_fn();
     if (!fn) return false;
     const int esize = bf16 ? 2 : 4;
@@ -1960,7 +1514,7 @@ bool make_map(CUtensorMap *m, const void *ptr, bool bf16, int64_t n_tok, int H, 
     cuuint32_t estr[2] = {1, 1};
     return fn(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2,
               const_cast<void *>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-              bf16 && swizzle ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+              bf16 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -1996,20 +1550,6 @@ cudaError_t launch_chain(const CUtensorMap &mv, const unsigned char *blobs, cons
     return err != cudaSuccess ? err : cudaGetLastError();
 }
 
-cudaError_t launch_chain2(const CUtensorMap &mv, const CUtensorMap &mo, const CUtensorMap &mg,
-                          const unsigned char *blobs, const int32_t *chunk_off,
-                          const float *S0, void *o, float *S_T, const int32_t *cu, int64_t T, int H,
-                          int nck, int nseq, bool after_prep, const IoOpts &io, cudaStream_t stream) {
-    using Lay = Chain2Layout;
-    cudaError_t err = cudaFuncSetAttribute(kda_chain2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           (int)Lay::BYTES);
-    if (err != cudaSuccess) return err;
-    err = launch_maybe_dependent(kda_chain2_kernel, dim3((unsigned)nseq, (unsigned)H), dim3(C2_NT), Lay::BYTES,
-                                 stream, after_prep, mv, mo, mg, blobs, chunk_off, S0, (__nv_bfloat16 *)o, S_T, cu, T,
-                                 H, nck, after_prep ? 1 : 0, (const __nv_bfloat16 *)io.out_gate, io.out_w,
-                                 io.out_eps);
-    return err != cudaSuccess ? err : cudaGetLastError();
-}
 
 // CTAs of the prep kernel resident on the whole GPU at once (its L2 prefetch
 // distance); 0 if it cannot be determined.
@@ -2148,11 +1688,11 @@ int sm_count() {
 }
 
 // Kernels launch_prefill_tc launches for these arguments (its decisions, restated).
-int prefill_tc_launches(int B, int64_t T, int H, int n_seqs, bool out_epilogue, bool l2norm) {
+int prefill_tc_launches(int B, int64_t T, int H, int n_seqs, bool l2norm) {
     const bool packed = n_seqs > 0;
     const int64_t n_tok = packed ? T : (int64_t)B * T;
     const int nck = (int)((T + CH - 1) / CH);
-    if (!packed && n_tok > 0 && !out_epilogue) {
+    if (!packed && n_tok > 0) {
         const BatchedPlan plan = batched_plan(B, H, nck, sm_count());
         if (plan.kind == 1 && !l2norm) return 1;  // the fused grid
         if (plan.kind == 2) return 4;             // prep, pass 1, combine, pass 2
@@ -2176,8 +1716,6 @@ cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, const
                               int64_t T, int H, const int32_t *cu_seqlens, int n_seqs,
                               void *workspace, const IoOpts &io, cudaStream_t stream) {
     const bool packed = n_seqs > 0;
-    // an output gate and norm run in the full-head chain, after the prep kernel
-    const bool out_epi = io.out_gate != nullptr;
     int io_flags = io.flags;
     float l2_eps = io.l2_eps;
     const int nseq = packed ? n_seqs : B;
@@ -2196,12 +1734,10 @@ cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, const
         chunk_offsets_kernel<<<1, 1024, 0, stream>>>(cu_seqlens, n_seqs, T, chunk_off);
     } else {
         blobs = ws + batched_head_bytes(B, nck, H);
-        // the fused grid's prep workers have no L2 normalisation: with it, or with an
-        // output epilogue, the call runs the prep and the chains
-        const bool two_kernels = out_epi || (io_flags & IO_QK_L2NORM) != 0;
+        // the fused grid's prep workers have no L2 normalisation: with it the call runs
+        // the prep and the chains
         plan = n_tok > 0 ? batched_plan(B, H, nck, n_sm) : BatchedPlan{0, 0, 0, 0};
-        if (two_kernels && plan.kind == 1) plan = BatchedPlan{0, 0, 0, 0};
-        if (out_epi) plan = BatchedPlan{0, 0, 0, 0};
+        if ((io_flags & IO_QK_L2NORM) != 0 && plan.kind == 1) plan = BatchedPlan{0, 0, 0, 0};
         if (plan.kind == 1) {
             int32_t *ready = reinterpret_cast<int32_t *>(ws);
             FusedQueue *queue = reinterpret_cast<FusedQueue *>(ready + (size_t)B * nck * H);
@@ -2273,14 +1809,6 @@ cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, const
         kda_seg_pass_kernel<64><<<dim3((unsigned)(2 * P), (unsigned)(plan.n_seg - 1)), CHAIN_NT,
                                   Lay::BYTES, stream>>>(mv, blobs, S0, ob, S_T, T, H, nck, sg, 2);
         return cudaGetLastError();
-    }
-    if (out_epi) {  // one full-head chain CTA per (sequence, head), with the output epilogue
-        CUtensorMap mo, mg;
-        if (n_tok > 0 && (!make_map(&mo, o, true, n_tok, H, false) || !make_map(&mg, io.out_gate, true, n_tok, H)))
-            return cudaErrorInvalidValue;
-        if (n_tok == 0) mo = mg = mv;  // no chunk: the maps are never used
-        return launch_chain2(mv, mo, mg, blobs, chunk_off, S0, o, S_T, cu_seqlens, T, H, nck, nseq,
-                             prep_launched, io, stream);
     }
     // 128-column slices (one CTA per sequence-head) when there are enough pairs to fill
     // the GPU; otherwise 64-column slices for twice the parallelism.

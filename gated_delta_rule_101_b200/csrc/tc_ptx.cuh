@@ -234,14 +234,8 @@ __device__ __forceinline__ void bulk_s2g(void *dst, const void *src, uint32_t by
 }
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
-// Waits until the shared-memory sources of all committed bulk stores have been read
-// (of all but the PENDING most recent bulk groups).
+// Waits until the shared-memory sources of all committed bulk stores have been read.
 __device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
-template <int PENDING>
-__device__ __forceinline__ void bulk_wait_read_but() {
-    asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(PENDING) : "memory");
-}
-
 // 2-D tiled tensor load (no multicast). x is the innermost coordinate.
 __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, int x, int y,
                                             uint64_t *bar) {
@@ -252,33 +246,10 @@ __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, i
         : "memory");
 }
 
-// 2-D tiled tensor store, shared -> global, completed as a bulk async-group (commit with
-// bulk_commit, wait with bulk_wait_read / bulk_wait_all). x is the innermost coordinate;
-// rows outside the tensor are not written.
-__device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, int x, int y, const void *src) {
-    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
-                     reinterpret_cast<uint64_t>(map)),
-                 "r"(x), "r"(y), "r"(smem_u32(src))
-                 : "memory");
-}
-
 // Brings the cache line of a global address into L2 without waiting for it.
 __device__ __forceinline__ void prefetch_l2(const void *p) {
     asm volatile("prefetch.global.L2 [%0];" ::"l"(reinterpret_cast<uint64_t>(p)));
 }
-// Brings the cache line of a global address into L1 without waiting for it.
-__device__ __forceinline__ void prefetch_l1(const void *p) {
-    asm volatile("prefetch.global.L1 [%0];" ::"l"(reinterpret_cast<uint64_t>(p)));
-}
-
-// Brings `bytes` (a multiple of 16, 16-byte aligned address) of global memory into L2
-// without waiting for it.
-__device__ __forceinline__ void bulk_prefetch_l2(const void *src, uint32_t bytes) {
-    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(src)),
-                 "r"(bytes)
-                 : "memory");
-}
-
 // Brings the box at (x, y) of a tiled tensor into L2 without waiting for it.
 __device__ __forceinline__ void tma_prefetch_l2_2d(const CUtensorMap *map, int x, int y) {
     asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(
@@ -333,19 +304,6 @@ __device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a_desc, uint6
         "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(0), "r"(0), "r"(0), "r"(0)
         : "memory");
 }
-// D[tmem] (+)= A[tmem] * B[smem], kind::f16. A sits in tensor memory: row m of A is
-// TMEM lane m, and its K elements are packed two per 32-bit column (element k in
-// column k / 2, the even one in the low half), so a K step of 16 spans 8 columns.
-__device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
-                                            uint32_t idesc, uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, {%5, %6, %7, %8}, p;\n\t}" ::"r"(
-            d_tmem),
-        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(0), "r"(0), "r"(0), "r"(0)
-        : "memory");
-}
 // Arrive once on `bar` when every MMA issued so far by this thread has completed.
 __device__ __forceinline__ void mma_commit(uint64_t *bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
@@ -375,29 +333,6 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float *v) {
     for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
-// Two loads of 32 consecutive columns each (taddr0, taddr1), then one wait: both
-// loads are in flight together.
-__device__ __forceinline__ void tmem_ld32x2(uint32_t taddr0, uint32_t taddr1, float *v0, float *v1) {
-    uint32_t r[64];
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
-        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
-        "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%64];\n\t"
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
-        "{%32, %33, %34, %35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47, "
-        "%48, %49, %50, %51, %52, %53, %54, %55, %56, %57, %58, %59, %60, %61, %62, %63}, [%65];\n\t"
-        "tcgen05.wait::ld.sync.aligned;"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]),
-          "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]), "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]), "=r"(r[48]), "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]), "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63])
-        : "r"(taddr0), "r"(taddr1)
-        : "memory");
-#pragma unroll
-    for (int i = 0; i < 32; ++i) {
-        v0[i] = __uint_as_float(r[i]);
-        v1[i] = __uint_as_float(r[32 + i]);
-    }
-}
-
 // 64 consecutive columns in one load, with the wait in the same statement.
 __device__ __forceinline__ void tmem_ld64(uint32_t taddr, float *v) {
     uint32_t r[64];
@@ -411,18 +346,6 @@ __device__ __forceinline__ void tmem_ld64(uint32_t taddr, float *v) {
 #pragma unroll
     for (int i = 0; i < 64; ++i) v[i] = __uint_as_float(r[i]);
 }
-
-// Stores 16 consecutive 32-bit TMEM columns of this thread's lane (lane = 32 * (warp %
-// 4) + lane id) starting at taddr. tmem_wait_st() waits until the warp's stores are done.
-__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
-    asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
-        "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
-        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
-        "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
-        : "memory");
-}
-__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 // ------------------------------------------------------------------ warp-level MMA
 // D (16x8, fp32) += A (16x8) * B (8x8), tf32 inputs. Used only for the 16- and
@@ -527,15 +450,6 @@ __device__ __forceinline__ Operand kmajor(uint32_t base, uint32_t rows) {
 }
 __device__ __forceinline__ Operand mnmajor(uint32_t base, uint32_t lbo) {
     return {sw128_desc(base, lbo), 0u};
-}
-
-// The K/16 MMAs of D (+)= A * B with A in tensor memory (a_tmem: its first column).
-template <int K>
-__device__ __forceinline__ void mma_run_ts(uint32_t d_tmem, uint32_t a_tmem, Operand b, uint32_t idesc,
-                                           bool accumulate) {
-#pragma unroll
-    for (int kk = 0; kk < K / 16; ++kk)
-        mma_bf16_ts(d_tmem, a_tmem + 8u * (uint32_t)kk, b.desc(kk), idesc, (accumulate || kk > 0) ? 1u : 0u);
 }
 
 // Issues the K/16 MMAs of D (+)= A * B (A: M x K, B: K x N as described by

@@ -199,8 +199,9 @@ KDA_API int kda_chunk_fwd_gated(const void *q, const void *k, const void *v,
  *                    need not be normalised
  *   beta_logits      nonzero: beta holds logits, the kernels use sigmoid(beta)
  *   out_gate         NULL, or the gate's input, shaped like o ([B, T, H, 128] or
- *                    [N, H, 128], q's dtype; 16-byte aligned for bf16): applies
- *                    the output epilogue above to o
+ *                    [N, H, 128], q's dtype; 16-byte aligned, and o too, for
+ *                    prefill; 16-byte aligned for bf16 decode): applies the
+ *                    output epilogue above to o
  *   out_norm_weight  [128] fp32, 16-byte aligned, or NULL for ones
  * eps values must be finite and >= 0. The gate's own pre-activation is a gate
  * layout (KDA_GATE_CHANNEL_LOGIT*), not a field here.
@@ -216,12 +217,11 @@ typedef struct kda_io {
 
 /*
  * kda_chunk_fwd_gated with the fused transformations of `io` (NULL: none, which
- * is kda_chunk_fwd_gated itself). The output epilogue is available for bf16
- * inputs (the fp32 path returns KDA_ERR_UNSUPPORTED for out_gate != NULL); it
- * runs the prep kernel and a chain kernel that holds whole output rows (one
- * CTA per sequence-head), whatever plan the call would otherwise take, in the
- * same workspace. With qk_l2norm a bf16 call that would take the fused grid
- * runs the prep and chain kernels instead. The other fields work on every path.
+ * is kda_chunk_fwd_gated itself). Every field works on every path (both dtypes,
+ * C = 32 and 64). The input steps run inside the prefill kernels; with qk_l2norm
+ * a bf16 call that would take the fused grid runs the prep and chain kernels
+ * instead. The output epilogue is one more kernel after the call's others (one
+ * read of o and out_gate, one write of o, in place), with the workspace unchanged.
  */
 KDA_API int kda_chunk_fwd_io(const void *q, const void *k, const void *v, const void *log_alpha,
                              int gate, const float *beta, const float *S0, void *o, float *S_T,

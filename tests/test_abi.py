@@ -103,8 +103,11 @@ def test_launch_count_query_follows_the_plan():
     assert kda.chunk_fwd_launches(1, 1000, 2, n_seqs=3, C=32) == 1
     with pytest.raises(kda.KDAError):
         kda.chunk_fwd_launches(1, 256, 2, C=128)
-    with pytest.raises(kda.KDAError):  # the output epilogue lives in the tensor-core chain
-        kda.chunk_fwd_launches(1, 256, 2, C=32, out_epilogue=True)
+    # the output epilogue is one more kernel after whichever plan the call takes
+    assert kda.chunk_fwd_launches(1, 256, 2, C=32, out_epilogue=True) == 2
+    assert kda.chunk_fwd_launches(1, 256, 2, dtype=torch.float32, out_epilogue=True) == 2
+    assert kda.chunk_fwd_launches(1, 3000, 2, out_epilogue=True) == 5
+    assert kda.chunk_fwd_launches(1, 1000, 2, n_seqs=3, out_epilogue=True) == 4
 
 
 def test_decode_rejects_bad_arguments(lib):
@@ -195,8 +198,7 @@ def test_io_entry_points_validate_their_options(lib):
     assert chunk(Io(1, -1.0, 0, None, None, 0.0)) == INVALID            # negative eps
     assert chunk(Io(1, float("nan"), 0, None, None, 0.0)) == INVALID   # NaN eps
     assert chunk(Io(0, 0.0, 0, gate16, None, -1.0)) == INVALID          # negative output eps
-    assert chunk(Io(0, 0.0, 0, gate16, None, 1e-6), dtype=F32) == UNSUPPORTED  # fp32: no epilogue
-    assert chunk(Io(0, 0.0, 0, gate16, None, 1e-6), C=32) == UNSUPPORTED  # C = 32: no epilogue
+    assert chunk(Io(0, 0.0, 0, gate16 + 4, None, 1e-6), dtype=F32) == INVALID  # rows read as float4
     assert chunk(Io(0, 0.0, 0, gate16 + 8, None, 1e-6)) == INVALID     # bf16 gate: 16-byte aligned
     assert chunk(Io(0, 0.0, 0, gate16, gate16 + 4, 1e-6)) == INVALID    # weights: 16-byte aligned
     assert decode(Io(1, -1.0, 0, None, None, 0.0)) == INVALID
@@ -204,8 +206,10 @@ def test_io_entry_points_validate_their_options(lib):
     # valid options go on to the next check (the missing workspace)
     assert chunk(Io(1, 1e-6, 1, gate16, gate16, 1e-6)) == WORKSPACE
     n = ctypes.c_int(0)
+    # fp32 inputs: the CUDA-core kernel, then the output epilogue
     assert lib.kda_chunk_fwd_io_launches(1, 128, 2, 64, 0, F32, ctypes.byref(Io(0, 0.0, 0, gate16, None, 0.0)),
-                                         ctypes.byref(n)) == UNSUPPORTED
+                                         ctypes.byref(n)) == 0
+    assert n.value == 2
 
 
 def test_backward_validates_before_launching(lib):

@@ -14,7 +14,7 @@ import torch
 import gated_delta_rule_101_b200 as kda
 import oracle
 from gated_delta_rule_101_b200.inputs import cu_from_lengths, prefill_inputs
-from io_ref import f64, l2norm_rows, log_sigmoid, sigmoid
+from io_ref import f64, l2norm_rows, log_sigmoid, rmsnorm_gate, sigmoid
 from parity import check, per_channel_gate
 
 pytestmark = pytest.mark.gpu
@@ -131,11 +131,15 @@ def test_chunk_lengths_agree():
     check(s32, s64, "f32", "C=32 vs C=64 S_T")
 
 
-def test_output_epilogue_is_refused():
-    inp = prefill_inputs(B=1, T=64, H=2, dtype=torch.bfloat16, seed=43, device=DEV)
-    with pytest.raises(kda.KDAError):
-        kda.chunk_fwd(inp.q, inp.k, inp.v, inp.log_alpha, inp.beta, None, C=32, out_gate=inp.v,
-                      out_norm_weight=torch.ones(128, device=DEV))
+def test_output_epilogue():
+    """The output epilogue (RMSNorm, weights, sigmoid gate) after the C = 32 kernel."""
+    inp = prefill_inputs(B=2, T=100, H=2, dtype=torch.bfloat16, s0_std=0.1, seed=43, device=DEV)
+    og = torch.randn(inp.v.shape, generator=torch.Generator().manual_seed(44)).to(torch.bfloat16).to(DEV)
+    w = torch.linspace(0.5, 1.5, 128, device=DEV)
+    o, st = run(inp, out_gate=og, out_norm_weight=w, out_eps=1e-6)
+    ro, rs = ref(inp)
+    check(o, rmsnorm_gate(ro, og, w, 1e-6), "bf16", "C=32 epilogue o")
+    check(st, rs, "f32", "C=32 epilogue S_T")
 
 
 def test_prefill_workload_b4_t4096_h16_sampled():

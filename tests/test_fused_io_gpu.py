@@ -51,11 +51,11 @@ def oracle_ref(x, cu=None, out_epi=True):
     return o, st
 
 
-def run_fused(x, cu=None, out_epi=True, gate_dtype=torch.float32):
+def run_fused(x, cu=None, out_epi=True, gate_dtype=torch.float32, **kw):
     return kda.chunk_fwd(x["q"], x["k"], x["v"], x["z"].to(gate_dtype).contiguous(), x["b"], x["S0"],
                          cu_seqlens=cu, gate_logits=True, qk_l2norm=True, qk_eps=EPS,
                          beta_logits=True, out_gate=x["og"] if out_epi else None,
-                         out_norm_weight=x["w"] if out_epi else None, out_eps=EPS)
+                         out_norm_weight=x["w"] if out_epi else None, out_eps=EPS, **kw)
 
 
 @pytest.mark.parametrize("T", [64, 200, 700])
@@ -80,12 +80,14 @@ def test_prefill_fused_packed_with_empty_and_ragged_sequences():
 
 
 @pytest.mark.parametrize("shape", [(1, 1000, 32), (1, 3000, 2)])
-def test_output_epilogue_replaces_the_fused_grid_and_segment_scan_plans(shape):
-    """Shapes that would take the fused grid or the segment scan run the prep and the
-    full-head chain when an output gate is given (2 kernels), and stay correct."""
+def test_output_epilogue_on_the_fused_grid_and_segment_scan_plans(shape):
+    """The output epilogue is one kernel after whichever plan the call takes: on the
+    fused grid's shape (whose L2Norm moves the call to prep and chains) and on the
+    segment scan's."""
     B, T, H = shape
-    assert kda.chunk_fwd_launches(B, T, H) in (1, 4)
-    assert kda.chunk_fwd_launches(B, T, H, out_epilogue=True) == 2
+    base = kda.chunk_fwd_launches(B, T, H)
+    assert base in (1, 4)
+    assert kda.chunk_fwd_launches(B, T, H, out_epilogue=True) == base + 1
     x = raw_inputs((B, T), H, torch.bfloat16, seed=T + H, n_seqs=B)
     o, st = run_fused(x)
     torch.cuda.synchronize()
@@ -112,10 +114,33 @@ def test_input_steps_on_every_dtype(dtype, gate_dtype):
     check(st, rs, KIND[dtype], "input steps S_T")
 
 
-def test_fp32_refuses_the_output_epilogue():
-    x = raw_inputs((1, 64), 2, torch.float32, seed=3, n_seqs=1)
-    with pytest.raises(kda.KDAError):
-        run_fused(x)
+@pytest.mark.parametrize("dtype,C", [(torch.float32, 64), (torch.float32, 32), (torch.bfloat16, 32)])
+def test_output_epilogue_on_the_cuda_core_kernel(dtype, C):
+    """fp32 inputs and chunks of 32 (the CUDA-core kernel) with every fused step."""
+    x = raw_inputs((2, 150), 2, dtype, seed=3 + C, n_seqs=2)
+    o, st = run_fused(x, C=C)
+    torch.cuda.synchronize()
+    ro, rs = oracle_ref(x)
+    check(o, ro, KIND[dtype], f"cuda-core fused o C={C}")
+    check(st, rs, KIND[dtype], f"cuda-core fused S_T C={C}")
+
+
+def test_segment_scan_plan_with_every_fused_step():
+    """The segment scan (few heads, long sequence) keeps its plan under the input steps
+    and adds the epilogue kernel (no RMSNorm weights: ones)."""
+    B, T, H = 1, 3000, 2
+    x = raw_inputs((B, T), H, torch.bfloat16, seed=77, n_seqs=B)
+    x["w"] = None
+    assert kda.chunk_fwd_launches(B, T, H, out_epilogue=True) == 5
+    o, st = kda.chunk_fwd(x["q"], x["k"], x["v"], x["z"], x["b"], x["S0"], gate_logits=True,
+                          qk_l2norm=True, qk_eps=EPS, beta_logits=True, out_gate=x["og"], out_eps=EPS)
+    torch.cuda.synchronize()
+    la, beta = log_sigmoid(x["z"]), sigmoid(x["b"])
+    ro, rs = oracle.kda_fwd(l2norm_rows(x["q"], EPS), l2norm_rows(x["k"], EPS), f64(x["v"]), la, beta,
+                            f64(x["S0"]))
+    ro = rmsnorm_gate(ro, x["og"], None, EPS)
+    check(o, ro, "bf16", "segment scan fused o")
+    check(st, rs, "bf16", "segment scan fused S_T")
 
 
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
