@@ -67,44 +67,46 @@ constexpr uint32_t BLOB_BYTES = 66048;
 
 // ---- prep kernel shared memory (offsets from a 1024-byte aligned base). Every
 // operand image is a 128-byte-swizzled tile of 128-byte rows (see tc_ptx.cuh).
-// The layout keeps a CTA under 68 KB so that three run on each SM.
+// The layout keeps a CTA under 52 KB so that four run on each SM.
+//   KINV rows = token i, two 64-channel blocks: (K e^-g)[i][c]; the Gram's K-major B.
 //   A1   K-major, rows r' = 0..127, K = key channel c (two 64-channel blocks of 16 KiB).
 //        TMA puts q in rows 0..63 and k in rows 64..127; they are scaled in place
 //        to Q e^g and K e^g. Rows 64..127 are later replaced by W.
-//   KT   rows = token i, two 64-channel blocks: (exp(g_L - g) K)[i][c]. The chain's
-//        MN-major A operand K~^T. Stored to the blob as soon as it is built.
-//   KINV rows = token i, two 64-channel blocks: (K e^-g)[i][c]; the Gram's K-major B.
-// Once the Gram MMA has completed and K~ has been stored, the 32 KiB of KT | KINV
-// take A_kk / T (fp32, rows padded to LDT floats), the solve's scratch and the
-// A_qk image, whose space then takes the T Diag(beta) image.
+// K~ = exp(g_L - g) K, the chain's MN-major A operand K~^T, goes from registers straight
+// to the blob. Once the Gram MMA has completed and the Q~ rows have been stored, KINV and
+// the Q rows of A1 take A_kk / T (fp32, rows padded to LDT floats, KINV and the first
+// 1 KiB of A1), the solve's scratch (in A1's first Q block) and the A_qk image (A1's
+// second Q block), whose space then takes the T Diag(beta) image.
 constexpr int PREP_NT = 256;
-constexpr uint32_t P_A1 = 0;          // 32768
-constexpr uint32_t P_KT = 32768;      // 16384
-constexpr uint32_t P_KINV = 49152;    // 16384 (dead after the Gram MMA)
-constexpr uint32_t P_GTOT = 49152;    // 8 x 128 fp32 per-warp log-decay totals (before KINV)
-constexpr uint32_t P_BADB = 49152;    // 8 x 3 x 64 fp32 bad-channel batch (after the Gram MMA)
-constexpr uint32_t P_AKK = 32768;     // 64 x 68 fp32 (17408): A_kk, then T in place
-constexpr uint32_t P_PBUF = 50176;    // 4608: solve scratch (2 x [16][20], then [32][36])
-constexpr uint32_t P_AQK = 55296;     // 8192: A_qk image, rows r, columns i
-constexpr uint32_t P_TB = 55296;      // 8192: T Diag(beta) image (after A_qk has been stored)
-constexpr uint32_t P_GAM = 65536;     // 128 fp32: exp(g_L)
-constexpr uint32_t P_GL = 66048;      // 128 fp32: g_L
-constexpr uint32_t P_BETA = 66560;    // 64 fp32
-constexpr uint32_t P_BADL = 66816;    // 128 int
-constexpr uint32_t P_BAR = 67328;     // 2 mbarriers
-constexpr uint32_t P_TMEM = 67344;
-constexpr uint32_t P_NBAD = 67348;    // number of listed bad channels
-constexpr uint32_t P_CLAIM = 67352;   // [2] item indices handed to the worker's threads
-constexpr uint32_t P_QN = 67360;      // 64 fp32: 1 / |q row| (rows L2-normalised in the kernel)
-constexpr uint32_t P_KN = 67616;      // 64 fp32: 1 / |k row|
-constexpr uint32_t PREP_SMEM = 67872 + 1024;
+constexpr uint32_t P_KINV = 0;        // 16384 (dead after the Gram MMA)
+constexpr uint32_t P_GTOT = 0;        // 8 x 128 fp32 per-warp log-decay totals (before KINV)
+constexpr uint32_t P_A1 = 16384;      // 32768
+constexpr uint32_t P_AKK = 0;         // 64 x 68 fp32 (17408): A_kk, then T in place
+constexpr uint32_t P_PBUF = 17408;    // 4608: solve scratch (2 x [16][20], then [32][36])
+constexpr uint32_t P_AQK = 32768;     // 8192: A_qk image, rows r, columns i
+constexpr uint32_t P_TB = 32768;      // 8192: T Diag(beta) image (after A_qk has been stored)
+constexpr uint32_t P_BADB = 17408;    // 8 x 3 x 64 fp32 bad-channel batch (Gram readout, before the solve)
+constexpr uint32_t P_GAM = 49152;     // 128 fp32: exp(g_L)
+constexpr uint32_t P_GL = 49664;      // 128 fp32: g_L
+constexpr uint32_t P_BETA = 50176;    // 64 fp32
+constexpr uint32_t P_BADL = 50432;    // 128 int
+constexpr uint32_t P_BAR = 50944;     // 2 mbarriers
+constexpr uint32_t P_TMEM = 50960;
+constexpr uint32_t P_NBAD = 50964;    // number of listed bad channels
+constexpr uint32_t P_CLAIM = 50968;   // [2] item indices handed to the worker's threads
+constexpr uint32_t P_QN = 50976;      // 64 fp32: 1 / |q row| (rows L2-normalised in the kernel)
+constexpr uint32_t P_KN = 51232;      // 64 fp32: 1 / |k row|
+constexpr uint32_t PREP_SMEM = 51488 + 1024;
 constexpr uint32_t PREP_TMEM_COLS = 128;  // Gram 64, then W 128
 constexpr uint32_t PREP_TMA_BYTES = 32768;  // q, k
-static_assert(P_AKK + 64 * 68 * 4 <= P_PBUF && P_PBUF + 4608 <= P_AQK && P_AQK + 8192 <= P_GAM,
-              "prep layout: A_kk, scratch and A_qk must fit in KT | KINV");
-static_assert(P_GTOT + 8 * 128 * 4 <= P_KINV + 16384 && P_BADB + 8 * 3 * 64 * 4 <= P_AQK + 8192,
-              "prep layout: scratch regions");
-static_assert(3 * (PREP_SMEM + 1024) <= 233472, "three prep CTAs per SM");
+static_assert(P_AKK + 64 * 68 * 4 <= P_PBUF && P_PBUF + 4608 <= P_A1 + 8192,
+              "prep layout: A_kk and the solve scratch must fit in KINV and A1's first Q block");
+static_assert(P_AQK == P_A1 + 16384 && P_AQK + 8192 <= P_A1 + 16384 + 8192,
+              "prep layout: the A_qk / T Diag(beta) image fills A1's second Q block");
+static_assert(P_GTOT + 8 * 128 * 4 <= P_KINV + 16384 && P_BADB >= P_AKK + 64 * 68 * 4 &&
+              P_BADB + 8 * 3 * 64 * 4 <= P_A1 + 8192 && P_A1 + 32768 <= P_GAM,
+              "prep layout: scratch regions (the bad-channel batch shares the solve scratch's space)");
+static_assert(4 * (PREP_SMEM + 1024) <= 233472, "four prep CTAs per SM");
 
 // A_kk / T rows are padded to 68 floats: float4 row segments stay aligned, and
 // 8 consecutive rows at the same column fall on distinct bank quads.
@@ -255,6 +257,7 @@ struct PrepArgs {
 // barrier. A CTA of kda_prep_kernel is one worker; a CTA of the fused kernel runs three.
 template <bool SINGLE>
 struct PrepWorker {
+    static constexpr bool kSingle = SINGLE;
     // Everything that identifies the worker is recomputed from threadIdx (its threads
     // are PREP_NT consecutive ones, worker g = threadIdx.x / PREP_NT), so that a loop
     // over items keeps few values live across the item's code. SINGLE: the worker is
@@ -510,6 +513,7 @@ __device__ __forceinline__ void prep_item(Worker &w, const PrepArgs &a, int slot
     //      channels whose chunk log-decay exceeds SAFE_SPAN (kept out of the unrolled
     //      common path so that it stays branch-free).
     constexpr bool l2 = L2;
+    unsigned char *blob = a.ws_blobs + ((size_t)slot * H + h) * BLOB_BYTES;
     float *sqn = reinterpret_cast<float *>(sm + P_QN);
     float *skn = reinterpret_cast<float *>(sm + P_KN);
     auto gate_rows = [&](auto bad_tag) {
@@ -564,9 +568,11 @@ __device__ __forceinline__ void prep_item(Worker &w, const PrepArgs &a, int slot
                 ke[e] = kk * eg;
                 // exp(-g) <= exp(80) for good channels
                 const float kin_ = kk * (ROW_GATE ? ein_row : __expf(-gs[e]));
-                if constexpr (BAD) {
-                    kin[e] = badc[e] ? 0.f : kin_;
-                    kt[e] = badc[e] ? kk * __expf(gls[e] - gs[e]) : kin_ * gams[e];
+                if constexpr (BAD) {  // g_L from shared memory: keeps gls and badc dead here
+                    const float gl_c = sgl[4 * f + e];
+                    const bool bad_c = -gl_c > SAFE_SPAN;
+                    kin[e] = bad_c ? 0.f : kin_;
+                    kt[e] = bad_c ? kk * __expf(gl_c - gs[e]) : kin_ * gams[e];
                 } else {
                     kin[e] = kin_;
                     kt[e] = kin_ * gams[e];  // exp(g_L - g) = exp(g_L) exp(-g)
@@ -576,7 +582,7 @@ __device__ __forceinline__ void prep_item(Worker &w, const PrepArgs &a, int slot
                 make_uint2(pack_bf16x2(qe[0], qe[1]), pack_bf16x2(qe[2], qe[3]));
             *reinterpret_cast<uint2 *>(blk + sw128_chunk_off(64 + r, fchunk, 128) + fhalf) =
                 make_uint2(pack_bf16x2(ke[0], ke[1]), pack_bf16x2(ke[2], ke[3]));
-            *reinterpret_cast<uint2 *>(sm + P_KT + fblk * 8192 + sw128_chunk_off(r, fchunk, 64) + fhalf) =
+            *reinterpret_cast<uint2 *>(blob + BLOB_KTT + fblk * 8192 + sw128_chunk_off(r, fchunk, 64) + fhalf) =
                 make_uint2(pack_bf16x2(kt[0], kt[1]), pack_bf16x2(kt[2], kt[3]));
             *reinterpret_cast<uint2 *>(sm + P_KINV + fblk * 8192 + sw128_chunk_off(r, fchunk, 64) + fhalf) =
                 make_uint2(pack_bf16x2(kin[0], kin[1]), pack_bf16x2(kin[2], kin[3]));
@@ -585,14 +591,15 @@ __device__ __forceinline__ void prep_item(Worker &w, const PrepArgs &a, int slot
     if (GATE != KDA_GATE_NONE && n_bad) gate_rows(std::true_type{});
     else gate_rows(std::false_type{});
     fence_async_smem();
+    // K~ went to the blob by ordinary stores; a worker of the fused grid publishes the
+    // blob to chains that read it with bulk copies, so order them for the async proxy
+    if constexpr (!Worker::kSingle) fence_proxy_async_global();
     tc_fence_before();
     w.sync();
 
     // Each blob image is stored as soon as it is final (bulk copies drain while the CTA
-    // keeps computing): K~, exp(g_L) and the Q~ rows of A1 are final now.
-    unsigned char *blob = a.ws_blobs + ((size_t)slot * H + h) * BLOB_BYTES;
+    // keeps computing): exp(g_L) and the Q~ rows of A1 are final now.
     if (tid == 0) {
-        bulk_s2g(blob + BLOB_KTT, sm + P_KT, 16384);
         bulk_s2g(blob + BLOB_GAM, sm + P_GAM, 512);
         bulk_s2g(blob + BLOB_A1, sm + P_A1, 8192);                   // Q~, channels 0..63
         bulk_s2g(blob + BLOB_A1 + 16384, sm + P_A1 + 16384, 8192);   // Q~, channels 64..127
@@ -604,7 +611,7 @@ __device__ __forceinline__ void prep_item(Worker &w, const PrepArgs &a, int slot
         tc_fence_after();
         mma_run<D>(tmem, kmajor(sm_base + P_A1, 128), kmajor(sm_base + P_KINV, 64), idesc_bf16(128, 64), false);
         mma_commit(bar_mma);
-        bulk_wait_read();  // K~ has left shared memory: its space takes A_kk after the MMA
+        bulk_wait_read();  // the Q~ rows have left shared memory: their space takes A_kk after the MMA
     }
     w.wait(bar_mma, 0);
     tc_fence_after();
@@ -614,13 +621,30 @@ __device__ __forceinline__ void prep_item(Worker &w, const PrepArgs &a, int slot
     const int m = 32 * (warp & 3) + lane, cb = 32 * (warp >> 2);
     const int r_own = m & 63;
     const bool kk_row = m >= 64;
+    // Output of Gram row r_own, columns i = cb + 8 cq .. +7 (8 values): A_qk (inclusive
+    // lower) to its bf16 image, or A_kk (strict lower, times beta_r) to fp32 for the solve.
+    auto store_gram8 = [&](int cq, const float *g8) {
+        const int r = r_own;
+        float v[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            const int i = cb + cq * 8 + e;
+            v[e] = kk_row ? (i < r ? sbeta[r] * g8[e] : 0.f) : ((i <= r && r < L) ? g8[e] : 0.f);
+        }
+        if (!kk_row) {
+            st_chunk(sm + P_AQK + sw128_chunk_off(r, (cb >> 3) + cq, 64), v);
+        } else {
+            float *akk = reinterpret_cast<float *>(sm + P_AKK) + r * LDT + cb + cq * 8;
+            *reinterpret_cast<float4 *>(akk) = make_float4(v[0], v[1], v[2], v[3]);
+            *reinterpret_cast<float4 *>(akk + 4) = make_float4(v[4], v[5], v[6], v[7]);
+        }
+    };
     auto gram_readout = [&](auto bad_tag) {
         constexpr bool BAD = decltype(bad_tag)::value;
-        float G[32];
-        if constexpr (BAD) {  // exact pairwise terms of the channels left out of the MMA
-            float acc[32];
-#pragma unroll
-            for (int e = 0; e < 32; ++e) acc[e] = 0.f;
+        if constexpr (BAD) {
+            // Exact pairwise terms of the key channels whose chunk log-decay exceeds
+            // SAFE_SPAN (left out of the MMA), added 8 columns at a time so that few
+            // registers are live: this path only runs for such chunks.
             int *nbad = reinterpret_cast<int *>(sm + P_NBAD);
             if (tid == 0) {
                 int cnt = 0;
@@ -631,76 +655,79 @@ __device__ __forceinline__ void prep_item(Worker &w, const PrepArgs &a, int slot
             w.sync();
             const int nb_total = *nbad;
             float *bb = reinterpret_cast<float *>(sm + P_BADB);  // [8][3][64]: q, k, g per row
-            for (int b0 = 0; b0 < nb_total; b0 += 8) {
-                for (int e = tid; e < 8 * 64; e += PREP_NT) {  // gather the batch's columns
-                    const int bi = e >> 6, r = e & 63;
-                    float qx = 0.f, kx = 0.f, gx = 0.f;
-                    if (b0 + bi < nb_total) {
-                        const int cc = badl[b0 + bi];
-                        const int64_t ccol = (int64_t)h * D + cc;
-                        float gsum = 0.f;
-                        for (int j = 0; j <= r; ++j)
-                            gsum += j < L ? gate_log<GATE>(a.log_alpha, (tok0 + j) * H + h, cc) : 0.f;
-                        gx = gsum;
-                        if (r < L) {
-                            qx = __bfloat162float(a.q[(tok0 + r) * H * D + ccol]);
-                            kx = __bfloat162float(a.k[(tok0 + r) * H * D + ccol]);
-                            if constexpr (L2) {  // the row norms gate_rows found
-                                qx *= sqn[r];
-                                kx *= skn[r];
+            for (int cq = 0; cq < 4; ++cq) {
+                float g8[8];
+                tmem_ld8(tmem + ((uint32_t)(32 * (warp & 3)) << 16) + cb + 8 * cq, g8);
+                for (int b0 = 0; b0 < nb_total; b0 += 8) {
+                    for (int e = tid; e < 8 * 64; e += PREP_NT) {  // gather the batch's columns
+                        const int bi = e >> 6, r = e & 63;
+                        float qx = 0.f, kx = 0.f, gx = 0.f;
+                        if (b0 + bi < nb_total) {
+                            const int cc = badl[b0 + bi];
+                            const int64_t ccol = (int64_t)h * D + cc;
+                            float gsum = 0.f;
+                            for (int j = 0; j <= r; ++j)
+                                gsum += j < L ? gate_log<GATE>(a.log_alpha, (tok0 + j) * H + h, cc) : 0.f;
+                            gx = gsum;
+                            if (r < L) {
+                                qx = __bfloat162float(a.q[(tok0 + r) * H * D + ccol]);
+                                kx = __bfloat162float(a.k[(tok0 + r) * H * D + ccol]);
+                                if constexpr (L2) {  // the row norms gate_rows found
+                                    qx *= sqn[r];
+                                    kx *= skn[r];
+                                }
                             }
                         }
+                        bb[(bi * 3 + 0) * 64 + r] = qx;
+                        bb[(bi * 3 + 1) * 64 + r] = kx;
+                        bb[(bi * 3 + 2) * 64 + r] = gx;
                     }
-                    bb[(bi * 3 + 0) * 64 + r] = qx;
-                    bb[(bi * 3 + 1) * 64 + r] = kx;
-                    bb[(bi * 3 + 2) * 64 + r] = gx;
-                }
-                w.sync();
-                const int nb = min(8, nb_total - b0);
-                for (int bi = 0; bi < nb; ++bi) {
-                    const float xr = bb[(bi * 3 + (kk_row ? 1 : 0)) * 64 + r_own];
-                    const float grr = bb[(bi * 3 + 2) * 64 + r_own];
+                    w.sync();
+                    const int nb = min(8, nb_total - b0);
+                    for (int bi = 0; bi < nb; ++bi) {
+                        const float xr = bb[(bi * 3 + (kk_row ? 1 : 0)) * 64 + r_own];
+                        const float grr = bb[(bi * 3 + 2) * 64 + r_own];
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) {
-                        const int i = cb + e;
-                        const float fi = i <= r_own ? bb[(bi * 3 + 1) * 64 + i] *
-                                                          expf(fminf(grr - bb[(bi * 3 + 2) * 64 + i], 0.f))
-                                                    : 0.f;
-                        acc[e] += xr * fi;
+                        for (int e = 0; e < 8; ++e) {
+                            const int i = cb + 8 * cq + e;
+                            const float fi = i <= r_own ? bb[(bi * 3 + 1) * 64 + i] *
+                                                              expf(fminf(grr - bb[(bi * 3 + 2) * 64 + i], 0.f))
+                                                        : 0.f;
+                            g8[e] += xr * fi;
+                        }
                     }
+                    w.sync();
                 }
-                w.sync();
+                store_gram8(cq, g8);
             }
-            tmem_ld32(tmem + ((uint32_t)(32 * (warp & 3)) << 16) + cb, G);
-#pragma unroll
-            for (int e = 0; e < 32; ++e) G[e] += acc[e];
         } else {
+            float G[32];
             tmem_ld32(tmem + ((uint32_t)(32 * (warp & 3)) << 16) + cb, G);
-        }
-        const int r = r_own;
-        if (!kk_row) {  // A_qk (inclusive lower) -> bf16 image, rows r, columns i
+            const int r = r_own;
+            if (!kk_row) {  // A_qk (inclusive lower) -> bf16 image, rows r, columns i
 #pragma unroll
-            for (int cq = 0; cq < 4; ++cq) {
-                float v[8];
+                for (int cq = 0; cq < 4; ++cq) {
+                    float v[8];
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const int i = cb + cq * 8 + e;
-                    v[e] = (i <= r && r < L) ? G[cq * 8 + e] : 0.f;
+                    for (int e = 0; e < 8; ++e) {
+                        const int i = cb + cq * 8 + e;
+                        v[e] = (i <= r && r < L) ? G[cq * 8 + e] : 0.f;
+                    }
+                    st_chunk(sm + P_AQK + sw128_chunk_off(r, (cb >> 3) + cq, 64), v);
                 }
-                st_chunk(sm + P_AQK + sw128_chunk_off(r, (cb >> 3) + cq, 64), v);
-            }
-        } else {  // A_kk (strict lower, times beta_r) -> fp32 for the solve
-            float *akk = reinterpret_cast<float *>(sm + P_AKK);
-            const float b = sbeta[r];
+            } else {  // A_kk (strict lower, times beta_r) -> fp32 for the solve
+                float *akk = reinterpret_cast<float *>(sm + P_AKK);
+                const float b = sbeta[r];
 #pragma unroll
-            for (int e4 = 0; e4 < 32; e4 += 4) {
-                float v[4];
+                for (int e4 = 0; e4 < 32; e4 += 4) {
+                    float v[4];
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int i = cb + e4 + e;
-                    v[e] = i < r ? b * G[e4 + e] : 0.f;
+                    for (int e = 0; e < 4; ++e) {
+                        const int i = cb + e4 + e;
+                        v[e] = i < r ? b * G[e4 + e] : 0.f;
+                    }
+                    *reinterpret_cast<float4 *>(akk + r * LDT + cb + e4) = make_float4(v[0], v[1], v[2], v[3]);
                 }
-                *reinterpret_cast<float4 *>(akk + r * LDT + cb + e4) = make_float4(v[0], v[1], v[2], v[3]);
             }
         }
     };
@@ -853,7 +880,7 @@ __device__ __forceinline__ void prep_item(Worker &w, const PrepArgs &a, int slot
 
 
 template <int GATE, bool L2>
-__global__ void __launch_bounds__(PREP_NT, 3)
+__global__ void __launch_bounds__(PREP_NT, 4)
 kda_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_la, int pf_dist,
                 const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
@@ -1553,13 +1580,13 @@ cudaError_t launch_chain(const CUtensorMap &mv, const unsigned char *blobs, cons
 
 // CTAs of the prep kernel resident on the whole GPU at once (its L2 prefetch
 // distance); 0 if it cannot be determined.
-int prep_residency() {
+// Prep CTAs resident at once on the device (the kernel's attributes must be set first).
+template <class K>
+int prep_residency(K kernel) {
     int dev = 0, n_sm = 0, per_sm = 0;
     if (cudaGetDevice(&dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kda_prep_kernel<KDA_GATE_CHANNEL, false>,
-                                                      PREP_NT, PREP_SMEM) !=
-            cudaSuccess)
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, PREP_NT, PREP_SMEM) != cudaSuccess)
         return 0;
     return n_sm * per_sm;
 }
@@ -1767,13 +1794,13 @@ cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, const
         if (!make_map(&mq, q, true, n_tok, H) || !make_map(&mk, k, true, n_tok, H) ||
             !make_gate_map(&mla, log_alpha, gate, n_tok, H, mq))
             return cudaErrorInvalidValue;
-        const int pf_dist = prep_residency();
         auto launch_prep = [&](auto kernel) {
             cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)PREP_SMEM);
-            if (e == cudaSuccess)  // three CTAs per SM need the largest shared-memory carveout
+            if (e == cudaSuccess)  // four CTAs per SM need the largest shared-memory carveout
                 e = cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
                                          (int)cudaSharedmemCarveoutMaxShared);
             if (e != cudaSuccess) return e;
+            const int pf_dist = prep_residency(kernel);
             kernel<<<dim3((unsigned)slots, (unsigned)H), PREP_NT, PREP_SMEM, stream>>>(
                 mq, mk, mla, pf_dist, (const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k, log_alpha,
                 beta, blobs, chunk_off, cu_seqlens, T, H, n_seqs, nck, io_flags, l2_eps);
