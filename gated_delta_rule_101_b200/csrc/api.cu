@@ -184,8 +184,7 @@ int kda_chunk_bwd_workspace_size(int B, int64_t T, int H, int n_seqs, size_t *by
     if (st != KDA_OK) return st;
     const bool packed = n_seqs > 0;
     const int64_t n_tok = packed ? T : (int64_t)B * T;
-    const int64_t slots = packed ? T / KDA_CHUNK + n_seqs : (int64_t)B * ((T + KDA_CHUNK - 1) / KDA_CHUNK);
-    *bytes = kda::bwd_workspace(n_tok, H, slots);
+    *bytes = kda::bwd_workspace(n_tok, H, kda::bwd_chunk_slots(B, T, n_seqs));
     return KDA_OK;
 }
 
@@ -220,7 +219,7 @@ int kda_chunk_bwd(const void *q, const void *k, const void *v, const void *log_a
     a.dS_T = dS_T; a.dq = dq; a.dk = dk; a.dv = dv; a.dgate = dgate; a.dbeta = dbeta; a.dS0 = dS0;
     a.B = B; a.T = T; a.H = H; a.cu = cu_seqlens; a.n_seqs = n_seqs;
     a.n_tok = packed ? T : (int64_t)B * T;
-    a.chunk_slots = packed ? T / KDA_CHUNK + n_seqs : (int64_t)B * ((T + KDA_CHUNK - 1) / KDA_CHUNK);
+    a.chunk_slots = kda::bwd_chunk_slots(B, T, n_seqs);
     a.workspace = workspace;
     a.io = opts;
     const cudaError_t err = kda::launch_bwd(a, gate, dtype, (cudaStream_t)stream);

@@ -23,7 +23,7 @@
 // kda_bwd_slice_kernel, grid (sequence, head, slice), 256 threads. Thread (warp w, lane
 // l) holds rows 16w .. 16w+15 of column l of the slice's state and gradient in
 // registers. Phase A runs the sequence forward once and keeps the state at every chunk
-// start (64 tokens) in the workspace. Phase B walks the chunks backwards: it reruns the
+// start (chunks of BW_CH = 32 tokens) in the workspace. Phase B walks the chunks backwards: it reruns the
 // chunk forward from its start state, keeping the state before each token in the
 // workspace and u, d in shared memory, then takes the chunk's tokens in reverse.
 #include "kda_internal.cuh"
@@ -39,17 +39,26 @@ constexpr int BW_PARTS = 3 * D + 1;         // per token and slice: dq, dk, dlog
 constexpr size_t BW_SLICE_STATE = (size_t)D * BW_J;  // floats of one state slice
 // Per-token states of the chunk being replayed live in one of BW_SM_SLOTS scratch slots.
 // A CTA claims a free slot at its start (atomic compare-and-swap on a per-slot word,
-// starting from its SM's index) and frees it at its end. At most one CTA of this kernel
-// is resident per SM (see BwdSmem), so with more slots than SMs a free slot always
-// exists; the claim does not depend on CTAs staying on one SM.
-constexpr int BW_SM_SLOTS = 256;
+// starting from its SM's index) and frees it at its end. At most two CTAs of this kernel
+// are resident per SM (shared memory and __launch_bounds__), so with more slots than
+// twice the SMs a free slot always exists; the claim does not depend on CTAs staying on
+// one SM.
+constexpr int BW_SM_SLOTS = 512;
+// Tokens per replayed chunk. 32 keeps a CTA's shared memory (the chunk's q, k, rates, v
+// and dout) small enough for two CTAs per SM.
+constexpr int BW_CH = 32;
+// Tokens of the replayed chunk starting at token c0 of a sequence of seq_len tokens.
+__device__ __forceinline__ int bw_chunk_rows(int64_t seq_len, int64_t c0) {
+    const int64_t left = seq_len - c0;
+    return left < BW_CH ? (int)left : BW_CH;
+}
 
-// About 146 KB: one CTA per SM (the per-SM scratch slots rely on it).
+// About 82 KB: two CTAs per SM.
 struct BwdSmem {
-    float q[CH][D], k[CH][D], a[CH][D];  // the chunk's q, k and per-channel rates a = exp(log_alpha)
-    float beta[CH];
-    float v[CH][BW_J], dout[CH][BW_J];   // the slice's v and do
-    float u[CH][BW_J], dd[CH][BW_J];     // u_t of the forward rerun; d_t (then reused)
+    float q[BW_CH][D], k[BW_CH][D], a[BW_CH][D];  // the chunk's q, k and per-channel rates a = exp(log_alpha)
+    float beta[BW_CH];
+    float v[BW_CH][BW_J], dout[BW_CH][BW_J];   // the slice's v and do
+    float u[BW_CH][BW_J], dd[BW_CH][BW_J];     // u_t of the forward rerun; d_t (then reused)
     float colsum[2][BW_NT / 32][BW_J];   // per-warp partial column sums, two buffers
     float rows[BW_NT / 32][BW_ROWS][BW_J + 1];  // per-warp row-sum transposition
 };
@@ -89,7 +98,7 @@ __device__ __forceinline__ float row_sum(const float (&x)[BW_ROWS], BwdSmem &sm)
 }
 
 template <typename TIn, int GATE>
-__global__ void __launch_bounds__(BW_NT, 1)
+__global__ void __launch_bounds__(BW_NT, 2)
 kda_bwd_slice_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const TIn *__restrict__ v,
                      const void *__restrict__ log_alpha, const float *__restrict__ beta,
                      const float *__restrict__ S0, const TIn *__restrict__ dout,
@@ -103,14 +112,14 @@ kda_bwd_slice_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const
     const int seq = blockIdx.x, h = blockIdx.y, slice = blockIdx.z, j0 = slice * BW_J;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, r0 = warp * BW_ROWS;
     const SeqSpan span = seq_span(cu, T, seq);
-    const int n_chunks = (int)((span.len + CH - 1) / CH);
+    const int n_chunks = (int)((span.len + BW_CH - 1) / BW_CH);
     const int64_t pair = (int64_t)seq * H + h;
     // the sequence's first chunk slot: seq * nck, or for packed sequences the chunks of
     // the sequences before it (sum of ceil(len / 64))
     int64_t slot0 = (int64_t)seq * nck;
     if (cu) {
         int64_t acc = 0;
-        for (int t = tid; t < seq; t += BW_NT) acc += (cu[t + 1] - cu[t] + CH - 1) / CH;
+        for (int t = tid; t < seq; t += BW_NT) acc += (cu[t + 1] - cu[t] + BW_CH - 1) / BW_CH;
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
         __shared__ long long chunk_acc[BW_NT / 32];
@@ -138,13 +147,13 @@ kda_bwd_slice_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const
     // this CTA's scratch: a state slice per chunk start, and per token of the current chunk
     const size_t cstride = (size_t)H * BW_SLICES * BW_SLICE_STATE;  // between chunk slots
     float *cbase = chunk_states + ((size_t)slot0 * H + h) * BW_SLICES * BW_SLICE_STATE + slice * BW_SLICE_STATE;
-    float *tstates = token_states + (size_t)slot * CH * BW_SLICE_STATE;
+    float *tstates = token_states + (size_t)slot * BW_CH * BW_SLICE_STATE;
     auto st_off = [&](int r) { return (size_t)(r0 + r) * BW_J + lane; };
     int cbuf = 0;  // col_sum's buffer
 
     // Loads a chunk's q, k, a and beta (rows >= L zero; a = 1 there) and the slice's v, do.
     auto load_chunk = [&](int64_t tok0, int L) {
-        for (int e = tid; e < CH * D; e += BW_NT) {
+        for (int e = tid; e < BW_CH * D; e += BW_NT) {
             const int r = e / D, c = e % D;
             const bool live = r < L;
             const int64_t row = (tok0 + r) * H + h;
@@ -152,20 +161,20 @@ kda_bwd_slice_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const
             sm.k[r][c] = live ? to_f32(k[row * D + c]) : 0.f;
             sm.a[r][c] = live ? expf(gate_log<GATE>(log_alpha, row, c)) : 1.f;
         }
-        for (int e = tid; e < CH * BW_J; e += BW_NT) {
+        for (int e = tid; e < BW_CH * BW_J; e += BW_NT) {
             const int r = e / BW_J, j = e % BW_J;
             const int64_t row = (tok0 + r) * H + h;
             sm.v[r][j] = r < L ? to_f32(v[row * D + j0 + j]) : 0.f;
             sm.dout[r][j] = r < L ? to_f32(dout[row * D + j0 + j]) : 0.f;
         }
-        if (tid < CH) {
+        if (tid < BW_CH) {
             float b = tid < L ? beta[(tok0 + tid) * H + h] : 0.f;
             if ((io_flags & IO_BETA_LOGITS) && tid < L) b = sigmoid(b);
             sm.beta[tid] = b;
         }
         __syncthreads();
         if (io_flags & IO_QK_L2NORM) {  // the rows the forward used
-            for (int r = warp; r < CH; r += BW_NT / 32) {
+            for (int r = warp; r < BW_CH; r += BW_NT / 32) {
                 float sq = 0.f, sk = 0.f;
                 for (int c = lane; c < D; c += 32) {
                     sq += sm.q[r][c] * sm.q[r][c];
@@ -210,8 +219,8 @@ kda_bwd_slice_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const
 #pragma unroll
     for (int r = 0; r < BW_ROWS; ++r) s[r] = S0 ? S0[pair * D * D + (int64_t)(r0 + r) * D + j0 + lane] : 0.f;
     for (int n = 0; n < n_chunks; ++n) {
-        const int64_t tok0 = span.start + (int64_t)n * CH;
-        const int L = chunk_rows(span.len, (int64_t)n * CH);
+        const int64_t tok0 = span.start + (int64_t)n * BW_CH;
+        const int L = bw_chunk_rows(span.len, (int64_t)n * BW_CH);
 #pragma unroll
         for (int r = 0; r < BW_ROWS; ++r) cbase[(size_t)n * cstride + st_off(r)] = s[r];
         if (n + 1 == n_chunks) break;  // the last chunk's tokens are replayed in phase B
@@ -225,8 +234,8 @@ kda_bwd_slice_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const
 #pragma unroll
     for (int r = 0; r < BW_ROWS; ++r) G[r] = dS_T ? dS_T[pair * D * D + (int64_t)(r0 + r) * D + j0 + lane] : 0.f;
     for (int n = n_chunks - 1; n >= 0; --n) {
-        const int64_t tok0 = span.start + (int64_t)n * CH;
-        const int L = chunk_rows(span.len, (int64_t)n * CH);
+        const int64_t tok0 = span.start + (int64_t)n * BW_CH;
+        const int L = bw_chunk_rows(span.len, (int64_t)n * BW_CH);
         __syncthreads();
         load_chunk(tok0, L);
         // rerun the chunk forward, keeping the state before each token
@@ -398,17 +407,23 @@ cudaError_t launch_bwd_t(const BwdArgs &a, int n_seqs, int nck, cudaStream_t str
 
 }  // namespace
 
+// Replayed chunks of a call: B * ceil(T / BW_CH), or for packed sequences at most
+// T / BW_CH + n_seqs (each sequence adds at most one partial chunk).
+int64_t bwd_chunk_slots(int B, int64_t T, int n_seqs) {
+    return n_seqs > 0 ? T / BW_CH + n_seqs : (int64_t)B * ((T + BW_CH - 1) / BW_CH);
+}
+
 // Workspace of kda_chunk_bwd: the replay slots' claim words, the slices' shares per
 // token-head, a state slice per chunk slot and head and slice, and the replay slots.
 size_t bwd_workspace(int64_t n_tok, int H, int64_t chunk_slots) {
     return (BW_SM_SLOTS + (size_t)n_tok * H * (BW_SLICES * BW_PARTS) +
-            (size_t)chunk_slots * H * BW_SLICES * BW_SLICE_STATE + (size_t)BW_SM_SLOTS * CH * BW_SLICE_STATE) *
+            (size_t)chunk_slots * H * BW_SLICES * BW_SLICE_STATE + (size_t)BW_SM_SLOTS * BW_CH * BW_SLICE_STATE) *
            sizeof(float);
 }
 
 cudaError_t launch_bwd(const BwdArgs &a, int gate, int dtype, cudaStream_t stream) {
     const int n_seqs = a.cu ? a.n_seqs : a.B;
-    const int nck = (int)((a.T + CH - 1) / CH);
+    const int nck = (int)((a.T + BW_CH - 1) / BW_CH);
     return with_gate(gate, [&](auto g) {
         constexpr int G = decltype(g)::value;
         if (dtype == KDA_BF16) return launch_bwd_t<__nv_bfloat16, G>(a, n_seqs, nck, stream);

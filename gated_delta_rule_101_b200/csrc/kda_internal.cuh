@@ -153,11 +153,12 @@ struct BwdArgs {
     const int32_t *cu;
     int n_seqs;
     int64_t n_tok;        // tokens in all (B * T, or T packed)
-    int64_t chunk_slots;  // chunks in all (B * ceil(T / 64), or T / 64 + n_seqs packed)
+    int64_t chunk_slots;  // replayed chunks in all (bwd_chunk_slots)
     void *workspace;
     IoOpts io;
 };
 size_t bwd_workspace(int64_t n_tok, int H, int64_t chunk_slots);
+int64_t bwd_chunk_slots(int B, int64_t T, int n_seqs);
 cudaError_t launch_bwd(const BwdArgs &a, int gate, int dtype, cudaStream_t stream);
 
 // Reads and clears the device status: *status is a mask of KDA_STATUS_TIMEOUT (a bounded

@@ -1331,20 +1331,24 @@ kda_seg_pass_kernel(const __grid_constant__ CUtensorMap tm_v,
 // products. Each step stages P_k in shared memory (rows padded to 129 floats, so that
 // the rows a warp reads at one column fall in distinct banks).
 constexpr int SEG_COMBINE_NT = 256;
-constexpr int SEG_PLD = D + 1;
-constexpr uint32_t SEG_COMBINE_SMEM = (D * 64 + D * SEG_PLD) * sizeof(float);
+constexpr int SEG_NJ = 16;       // state columns per CTA: (128 / SEG_NJ) CTAs per sequence-head
+constexpr int SEG_PLD = D + 1;   // row stride of P_k in shared memory (floats)
+constexpr uint32_t SEG_COMBINE_SMEM = (D * SEG_NJ + D * SEG_PLD) * sizeof(float);
+static_assert(D * SEG_NJ == 8 * SEG_COMBINE_NT, "one row and 8 columns per thread");
 __global__ void __launch_bounds__(SEG_COMBINE_NT)
 kda_seg_combine_kernel(SegScan sg) {
     extern __shared__ __align__(16) float seg_smem[];
-    float (*s)[64] = reinterpret_cast<float (*)[64]>(seg_smem);  // [128][64] current state slice
-    float *pm = seg_smem + D * 64;                                  // [128][SEG_PLD] P_k
-    const int pair = blockIdx.x >> 1, j0 = (blockIdx.x & 1) * 64;
-    const int tid = threadIdx.x, r0 = tid >> 2, jq = (tid & 3) * 4;
+    float (*s)[SEG_NJ] = reinterpret_cast<float (*)[SEG_NJ]>(seg_smem);  // [128][SEG_NJ] state slice
+    float *pm = seg_smem + D * SEG_NJ;                                    // [128][SEG_PLD] P_k
+    constexpr int SLICES = D / SEG_NJ;
+    const int pair = blockIdx.x / SLICES, j0 = (blockIdx.x % SLICES) * SEG_NJ;
+    // thread: state row r, columns jq .. jq + 7 of the slice
+    const int tid = threadIdx.x, r = tid >> 1, jq = (tid & 1) * 8;
     const float *s1 = sg.blk(sg.start, pair, 1);
-#pragma unroll
-    for (int i = 0; i < D * 16 / SEG_COMBINE_NT; ++i) {  // 16 float4 per row of the slice
-        const int e = tid + i * SEG_COMBINE_NT, row = e >> 4, c4 = (e & 15) * 4;
-        *reinterpret_cast<float4 *>(&s[row][c4]) = *reinterpret_cast<const float4 *>(s1 + row * D + j0 + c4);
+    {
+        const float4 *src = reinterpret_cast<const float4 *>(s1 + r * D + j0 + jq);
+        *reinterpret_cast<float4 *>(&s[r][jq]) = src[0];
+        *reinterpret_cast<float4 *>(&s[r][jq + 4]) = src[1];
     }
     for (int k = 1; k + 1 < sg.n_seg; ++k) {
         const float *pk = sg.blk(sg.p, pair, k);
@@ -1363,42 +1367,31 @@ kda_seg_combine_kernel(SegScan sg) {
                 dst[0] = v[i].x; dst[1] = v[i].y; dst[2] = v[i].z; dst[3] = v[i].w;
             }
         }
-        __syncthreads();  // P_k and the state are in shared memory
-        float acc[2][16];
-#pragma unroll
-        for (int h2 = 0; h2 < 2; ++h2) {
-            const float *hk = sg.blk(sg.hh, pair, k) + (size_t)(r0 + 64 * h2) * D + j0 + jq;
-#pragma unroll
-            for (int m = 0; m < 4; ++m) {
-                const float4 hv = *reinterpret_cast<const float4 *>(hk + 16 * m);
-                acc[h2][4 * m] = hv.x; acc[h2][4 * m + 1] = hv.y; acc[h2][4 * m + 2] = hv.z; acc[h2][4 * m + 3] = hv.w;
-            }
+        float acc[8];
+        {
+            const float4 *hk = reinterpret_cast<const float4 *>(sg.blk(sg.hh, pair, k) + (size_t)r * D + j0 + jq);
+            const float4 h0 = hk[0], h1 = hk[1];
+            acc[0] = h0.x; acc[1] = h0.y; acc[2] = h0.z; acc[3] = h0.w;
+            acc[4] = h1.x; acc[5] = h1.y; acc[6] = h1.z; acc[7] = h1.w;
         }
-        const float *p0 = pm + r0 * SEG_PLD, *p1 = pm + (r0 + 64) * SEG_PLD;
-#pragma unroll 4
+        __syncthreads();  // P_k and the state are in shared memory
+        const float *prow = pm + r * SEG_PLD;
+#pragma unroll 8
         for (int c = 0; c < D; ++c) {
-            const float a0 = p0[c], a1 = p1[c];
-#pragma unroll
-            for (int m = 0; m < 4; ++m) {
-                const float4 sv = *reinterpret_cast<const float4 *>(&s[c][jq + 16 * m]);
-                acc[0][4 * m] += a0 * sv.x; acc[0][4 * m + 1] += a0 * sv.y;
-                acc[0][4 * m + 2] += a0 * sv.z; acc[0][4 * m + 3] += a0 * sv.w;
-                acc[1][4 * m] += a1 * sv.x; acc[1][4 * m + 1] += a1 * sv.y;
-                acc[1][4 * m + 2] += a1 * sv.z; acc[1][4 * m + 3] += a1 * sv.w;
-            }
+            const float a = prow[c];
+            const float4 s0 = *reinterpret_cast<const float4 *>(&s[c][jq]);
+            const float4 s4 = *reinterpret_cast<const float4 *>(&s[c][jq + 4]);
+            acc[0] += a * s0.x; acc[1] += a * s0.y; acc[2] += a * s0.z; acc[3] += a * s0.w;
+            acc[4] += a * s4.x; acc[5] += a * s4.y; acc[6] += a * s4.z; acc[7] += a * s4.w;
         }
         __syncthreads();  // every thread has read the old state and P_k
-#pragma unroll
-        for (int h2 = 0; h2 < 2; ++h2) {
-            const int r = r0 + 64 * h2;
-            float *out = sg.blk(sg.start, pair, k + 1) + (size_t)r * D + j0 + jq;
-#pragma unroll
-            for (int m = 0; m < 4; ++m) {
-                const float4 v = make_float4(acc[h2][4 * m], acc[h2][4 * m + 1], acc[h2][4 * m + 2], acc[h2][4 * m + 3]);
-                *reinterpret_cast<float4 *>(&s[r][jq + 16 * m]) = v;
-                *reinterpret_cast<float4 *>(out + 16 * m) = v;
-            }
-        }
+        const float4 o0 = make_float4(acc[0], acc[1], acc[2], acc[3]);
+        const float4 o1 = make_float4(acc[4], acc[5], acc[6], acc[7]);
+        *reinterpret_cast<float4 *>(&s[r][jq]) = o0;
+        *reinterpret_cast<float4 *>(&s[r][jq + 4]) = o1;
+        float4 *out = reinterpret_cast<float4 *>(sg.blk(sg.start, pair, k + 1) + (size_t)r * D + j0 + jq);
+        out[0] = o0;
+        out[1] = o1;
     }
 }
 
@@ -1655,7 +1648,7 @@ size_t seg_bytes(int B, int H, int nck) {
 }
 BatchedPlan batched_plan(int B, int H, int nck, int n_sm) {
     constexpr double PREP_US_TWO = 14.4, PREP_US_FUSED = 16.5, CHAIN_US_64 = 1.45,
-                     CHAIN_US_128 = 2.3, COMBINE_US = 6.0, LAUNCH_US = 4.0;
+                     CHAIN_US_128 = 2.3, COMBINE_US = 2.0, LAUNCH_US = 4.0;
     constexpr int MIN_PREP_CTAS = 8;
     const int P = B * H;
     const double r2 = 3.0 / PREP_US_TWO, rf = 3.0 / PREP_US_FUSED;  // items per us per SM
@@ -1832,7 +1825,7 @@ cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, const
         err = cudaFuncSetAttribute(kda_seg_combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                    (int)SEG_COMBINE_SMEM);
         if (err != cudaSuccess) return err;
-        kda_seg_combine_kernel<<<2 * P, SEG_COMBINE_NT, SEG_COMBINE_SMEM, stream>>>(sg);
+        kda_seg_combine_kernel<<<(D / SEG_NJ) * P, SEG_COMBINE_NT, SEG_COMBINE_SMEM, stream>>>(sg);
         kda_seg_pass_kernel<64><<<dim3((unsigned)(2 * P), (unsigned)(plan.n_seg - 1)), CHAIN_NT,
                                   Lay::BYTES, stream>>>(mv, blobs, S0, ob, S_T, T, H, nck, sg, 2);
         return cudaGetLastError();

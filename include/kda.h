@@ -256,8 +256,8 @@ KDA_API int kda_chunk_fwd_io_launches(int B, int64_t T, int H, int C, int n_seqs
  *   dS0        [Nseq, H, 128, 128] fp32 (written), or NULL: dL/dS0
  *   workspace  device buffer of kda_chunk_bwd_workspace_size bytes, 16-byte
  *              aligned. It holds each token's per-slice gradient shares (6.2 KB
- *              per token-head), the state at every chunk start (64 KB per
- *              chunk-head) and a replay scratch of 256 x 1 MiB.
+ *              per token-head), the state every 32 tokens (64 KB per head) and
+ *              a replay scratch of 512 x 512 KiB.
  * The call launches two kernels; the result is bitwise reproducible.
  * Concurrent calls must not share a workspace.
  */

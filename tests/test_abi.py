@@ -234,5 +234,5 @@ def test_backward_validates_before_launching(lib):
     assert bwd() == WORKSPACE
     n = ctypes.c_size_t(0)
     assert lib.kda_chunk_bwd_workspace_size(4, 4096, 16, 0, ctypes.byref(n)) == 0
-    # slot words, shares 6.2 KB per token-head, 64 KB per chunk-head, 256 MiB replay scratch
-    assert n.value == (256 + 4 * 4096 * 16 * 4 * 385 + 4 * 64 * 16 * 4 * 4096 + 256 * 64 * 4096) * 4
+    # slot words, shares 6.2 KB per token-head, 64 KB per head every 32 tokens, 256 MiB replay scratch
+    assert n.value == (512 + 4 * 4096 * 16 * 4 * 385 + 4 * 128 * 16 * 4 * 4096 + 512 * 32 * 4096) * 4
