@@ -34,7 +34,9 @@ __device__ __forceinline__ float log_sigmoid(float z) {
     const float l = x < 1e-3f ? x * (1.f - 0.5f * x) : __logf(1.f + x);
     return fminf(z, 0.f) - l;
 }
-__device__ __forceinline__ float sigmoid(float z) { return 1.f / (1.f + __expf(-z)); }
+// Fast division (__fdividef: within 2 ulp; 0 once 1 + e^-z overflows) instead of the
+// correctly rounded one, whose multi-instruction sequence dominated the output epilogue.
+__device__ __forceinline__ float sigmoid(float z) { return __fdividef(1.f, 1.f + __expf(-z)); }
 
 // Fused input and output transformations of the layer around the operator
 // (blog.gzher.com "Kimi K3论文：Kimi Linear", section 3: q, k = L2Norm(...),
