@@ -1646,15 +1646,22 @@ size_t seg_bytes(int B, int H, int nck) {
     const int cap = seg_capacity(B, H, nck);
     return cap >= 3 ? (size_t)3 * B * H * cap * (size_t)(D * D) * sizeof(float) : 0;
 }
+constexpr double CHAIN_US_64 = 1.45, CHAIN_US_128 = 2.3;  // per chunk, B200
+// Whether P sequence-heads run faster as P 128-column chains than as 2 P 64-column ones:
+// a 128-column chain takes about CHAIN_US_128 per chunk, a 64-column one CHAIN_US_64,
+// one CTA per SM, in waves of n_sm CTAs.
+bool wide_chain(int64_t P, int n_sm) {
+    const int64_t w64 = (2 * P + n_sm - 1) / n_sm, w128 = (P + n_sm - 1) / n_sm;
+    return (double)w128 * CHAIN_US_128 < (double)w64 * CHAIN_US_64;
+}
 BatchedPlan batched_plan(int B, int H, int nck, int n_sm) {
-    constexpr double PREP_US_TWO = 14.4, PREP_US_FUSED = 16.5, CHAIN_US_64 = 1.45,
-                     CHAIN_US_128 = 2.3, COMBINE_US = 2.0, LAUNCH_US = 4.0;
+    constexpr double PREP_US_TWO = 14.4, PREP_US_FUSED = 16.5, COMBINE_US = 2.0, LAUNCH_US = 4.0;
     constexpr int MIN_PREP_CTAS = 8;
     const int P = B * H;
     const double r2 = 3.0 / PREP_US_TWO, rf = 3.0 / PREP_US_FUSED;  // items per us per SM
     const double t_prep = nck * (double)P / (n_sm * r2);
     // prep on every SM, then the chains in waves
-    const int n2 = P >= n_sm ? 128 : 64;
+    const int n2 = wide_chain(P, n_sm) ? 128 : 64;
     const double waves = (double)((P * (D / n2) + n_sm - 1) / n_sm);
     BatchedPlan best{0, 0, 0, 0};
     double t_best = t_prep + waves * nck * (n2 == 64 ? CHAIN_US_64 : CHAIN_US_128);
@@ -1830,9 +1837,10 @@ cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, const
                                   Lay::BYTES, stream>>>(mv, blobs, S0, ob, S_T, T, H, nck, sg, 2);
         return cudaGetLastError();
     }
-    // 128-column slices (one CTA per sequence-head) when there are enough pairs to fill
-    // the GPU; otherwise 64-column slices for twice the parallelism.
-    if ((int64_t)nseq * H >= n_sm)
+    // 128-column slices (one CTA per sequence-head) when twice as many 64-column chains
+    // would need more waves than that saves (about 75 sequence-heads and up on 148 SMs);
+    // otherwise 64-column slices for twice the parallelism.
+    if (wide_chain((int64_t)nseq * H, n_sm))
         return launch_chain<128>(mv, blobs, chunk_off, S0, o, S_T, cu_seqlens, T, H, nck, nseq,
                                  prep_launched, stream);
     return launch_chain<64>(mv, blobs, chunk_off, S0, o, S_T, cu_seqlens, T, H, nck, nseq,
