@@ -66,6 +66,9 @@ def _fake_cuda(monkeypatch):
         def wait_stream(self, other):
             pass
 
+        def wait_event(self, event):
+            pass
+
     class Graph:
         def replay(self):
             pass
