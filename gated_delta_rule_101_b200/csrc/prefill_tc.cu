@@ -1099,11 +1099,30 @@ __device__ __forceinline__ void chain_task(unsigned char *sm, const int tid, con
         __syncwarp();
     } else if (issuer) {
         // ------------------------------------------------------------ MMA / load warp
+        // DU = [.; T Diag(beta)] V does not depend on the state. With 128 columns, chunk m's
+        // is issued at the end of chunk m - 1 (after its V_new has been read from DU), so
+        // that the tensor pipe runs it while the epilogue updates the state, and chunk m
+        // starts with D1 alone; the next bar_a commit covers it. With 64 columns the
+        // product is short and issuing it early measured slower (A/B on one box: 0.2325
+        // against 0.2365 ms on B=4, T=4096, H=16; 0.4085 against 0.3932 ms at 128 columns
+        // on B=8), so there it follows D1 as before.
+        constexpr bool EARLY_DU = N == 128;
+        auto issue_du = [&](int m) {
+            const int sm_stage = m & 1;
+            mbar_wait(&bar_ld1[sm_stage], (uint32_t)(m >> 1) & 1u, dead, &g_kda_status);
+            if (!dead) {
+                const uint32_t sb = sm_base + sm_stage * Lay::STAGE;
+                tc_fence_after();
+                mma_run<CH>(du, kmajor(sb + Lay::TB - 8192, 128), mnmajor(sb + Lay::V, 8192),
+                            idesc_bf16(128, N, 0, 1), false);
+            }
+        };
         if (lane == 0) {
             for (int m = 0; m < 2 && m < nchunks; ++m) {
                 issue_load1(m, m);
                 issue_load2(m, m);
             }
+            if (EARLY_DU && nchunks > 0) issue_du(0);
         }
 #pragma unroll 1
         for (int n = 0; n < nchunks; ++n) {
@@ -1113,12 +1132,13 @@ __device__ __forceinline__ void chain_task(unsigned char *sm, const int tid, con
             const uint32_t lph = (uint32_t)(n >> 1) & 1u;
             if (lane == 0) {
                 mbar_wait(&bar_ld1[stage], lph, dead, &g_kda_status);
-                if (!dead) {  // D1 = [Q~; W] S, DU = [.; T Diag(beta)] V
+                if (!dead) {  // D1 = [Q~; W] S, then (unless issued early) DU
                     tc_fence_after();
                     mma_run<D>(d1, kmajor(st_base + Lay::A1, 128), mnmajor(sm_base + Lay::SIMG, 16384),
                                idesc_bf16(128, N, 0, 1), false);
-                    mma_run<CH>(du, kmajor(st_base + Lay::TB - 8192, 128), mnmajor(st_base + Lay::V, 8192),
-                                idesc_bf16(128, N, 0, 1), false);
+                    if constexpr (!EARLY_DU)
+                        mma_run<CH>(du, kmajor(st_base + Lay::TB - 8192, 128), mnmajor(st_base + Lay::V, 8192),
+                                    idesc_bf16(128, N, 0, 1), false);
                     mma_commit(bar_a);
                 }
             }
@@ -1134,6 +1154,7 @@ __device__ __forceinline__ void chain_task(unsigned char *sm, const int tid, con
                 mma_run<CH>(d1, kmajor(st_base + Lay::A2, 128), mnmajor(sm_base + Lay::VIMG, 8192),
                             idesc_bf16(128, N, 0, 1), true);
                 mma_commit(&bar_c[n & 1]);
+                if (EARLY_DU && n + 1 < nchunks) issue_du(n + 1);  // DU(n) has been read: V_new is written
             }
             __syncwarp();
             if (named_bar_or(BAR_END, CHAIN_NT, dead)) {
