@@ -1,10 +1,13 @@
-"""B200-native Kimi Delta Attention (KDA) forward: a thin binding over libkda.
+"""B200-native Kimi Delta Attention (KDA): a thin binding over libkda.
 
 libkda (``libkda.so`` next to this file, built by ``build.py`` from
-``csrc/``) implements the two entry points of ``include/kda.h``:
+``csrc/``) implements the entry points of ``include/kda.h``:
 
-* ``chunk_fwd``   -> ``kda_chunk_fwd``: chunk-parallel prefill, C = 64;
-* ``decode_step`` -> ``kda_decode_step``: one recurrent decode token.
+* ``chunk_fwd``   -> ``kda_chunk_fwd`` (``kda_chunk_fwd_io`` with fused steps):
+  chunk-parallel prefill, C = 64 (tensor cores for bf16) or C = 32 (CUDA cores);
+* ``decode_step`` -> ``kda_decode_step`` (``kda_decode_step_io``): one recurrent
+  decode token;
+* ``chunk_bwd``   -> ``kda_chunk_bwd``: the gradients of a prefill call.
 
 Both take the forget gate as ``log_alpha`` in any of the library's gate
 layouts (``kda_gate``), told apart by shape and dtype: ``[..., H, 128]``
