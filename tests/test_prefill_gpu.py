@@ -250,8 +250,10 @@ def test_long_context_1m_tokens_as_16_calls_sampled():
 
 
 def test_many_sequence_heads_take_full_width_chain():
-    """B*H >= the SM count selects one 128-column chain CTA per (sequence, head)."""
-    inp = prefill_inputs(B=2, T=130, H=80, dtype=torch.bfloat16, s0_std=0.1, seed=22, device=DEV)
+    """100 sequence-heads: two 64-column chains each would need two waves on 148 SMs, so
+    the call runs one 128-column chain CTA per (sequence, head) (chosen by wave count),
+    which also issues each chunk's U product one chunk early."""
+    inp = prefill_inputs(B=2, T=130, H=50, dtype=torch.bfloat16, s0_std=0.1, seed=22, device=DEV)
     o, st = run(inp)
     ro, rs = ref(inp)
     check(o, ro, "bf16", "128-column chain o")
@@ -328,10 +330,10 @@ def test_segment_scan_carries_state_across_calls():
 
 
 def test_wide_chain_all_outputs():
-    """Enough sequence-heads to fill the GPU: one 128-column chain CTA per sequence-head.
-    Ragged last chunk, carried state, every output."""
-    assert kda.chunk_fwd_launches(2, 200, 80) == 2
-    inp = prefill_inputs(B=2, T=200, H=80, dtype=torch.bfloat16, s0_std=0.1, seed=48, device=DEV)
+    """One 128-column chain CTA per sequence-head (100 of them, see above), 4 chunks with a
+    ragged last one, carried state, every output."""
+    assert kda.chunk_fwd_launches(2, 200, 50) == 2
+    inp = prefill_inputs(B=2, T=200, H=50, dtype=torch.bfloat16, s0_std=0.1, seed=48, device=DEV)
     o, st = run(inp)
     ro, rs = ref(inp)
     check(o, ro, "bf16", "wide chain o")
@@ -339,6 +341,7 @@ def test_wide_chain_all_outputs():
 
 
 def test_wide_chain_packed_with_empty_sequences():
+    """8 packed sequences x 40 heads (320 sequence-heads: 128-column chains)."""
     lengths = [0, 130, 64, 1, 257, 0, 65, 190]
     cu = cu_from_lengths(lengths)
     inp = prefill_inputs(T=int(cu[-1]), H=40, cu_seqlens=cu, dtype=torch.bfloat16, s0_std=0.1,
