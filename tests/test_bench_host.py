@@ -128,6 +128,13 @@ def test_gpu_arm_runs_end_to_end_on_fakes(monkeypatch):
         assert {"bound", "achieved", "peak", "unit", "frac", "traffic"} <= set(r)
     assert line["roofline"]["traffic"] is None  # captured at another shape
     assert {"kda_chunk_fwd", "kda_chunk_fwd_gated", "kda_decode_step"} <= set(rec.calls)
+    # the other legs: fused layer steps, chunk lengths, backward; parity only with the oracle leg
+    assert set(line["chunk_sizes"]) == {"C32_bf16", "C64_bf16", "C32_f32", "C64_f32"}
+    for leg in (line["fused_io"], line["backward"], *line["chunk_sizes"].values()):
+        assert {"value", "unit", "ms_per_call", "config", "roofline", "gpu_launches"} <= set(leg)
+    assert {"kda_chunk_fwd_io", "kda_chunk_bwd"} <= set(rec.calls)
+    assert line["parity"] is None and line["cpu_baseline"] is None
+    assert {"h2d_bytes_per_step", "d2h_bytes_per_step", "pipeline"} <= set(line["e2e"])
 
 
 def test_gpu_arm_remeasures_a_throttled_step(monkeypatch):
