@@ -144,7 +144,7 @@ KDA_API int kda_chunk_fwd_launches(int B, int64_t T, int H, int C, int n_seqs, i
  *              name 32 to 128 as the useful range (mokono.cn section 4.1). bf16
  *              inputs with C = 64 run on the tensor cores; fp32 inputs, and C = 32
  *              in either dtype, run on the CUDA-core kernel (one launch, no
- *              workspace, no output epilogue). C = 128 returns KDA_ERR_UNSUPPORTED:
+ *              workspace). C = 128 returns KDA_ERR_UNSUPPORTED:
  *              the CUDA-core kernel's fp32 working set for one chunk (about 400 KB)
  *              does not fit an SM, and the tensor-core kernels are built for 64.
  *   cu_seqlens device int32 [n_seqs + 1] token offsets of packed sequences
