@@ -152,7 +152,7 @@ def clock_rejected(clk: dict) -> bool:
 # from; otherwise the roofline's traffic is null.
 TRAFFIC_SOURCES = {"prefill": ("prefill_tc.cu", "tc_ptx.cuh", "kda_internal.cuh"),
                    "decode": ("decode.cu", "kda_internal.cuh")}
-TRAFFIC = {"prefill": {"source_hash": "4dfc008b23131578", "shape": (4, 4096, 16),  # prep + chain
+TRAFFIC = {"prefill": {"source_hash": "c6cc0cd03f29ccb3", "shape": (4, 4096, 16),  # prep + chain
                        "bytes": 271514240 + 220421120 + 341894443 + 52838272},
            "decode": {"source_hash": "2f2a24e4a98dd528", "shape": (256, 32),
                       "bytes": 547406592 + 480025216}}
